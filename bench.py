@@ -1,0 +1,602 @@
+"""Benchmark of the paged decode step on B200 (one JSON line on stdout).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl reference] [--no-extras]
+
+Step = one pass of the whole hot path over one batch: copy-on-write block
+copies (when the batch has shared partial blocks), the cache write of each
+sequence's new token through its slot, and the decode (plus the partition
+reduce) over every token.  ``value`` times that step on the device with every
+input already in HBM; ``e2e`` times the same step through the public Python
+API including, every step, the host block-manager append (one token per
+sequence), the table build, the host->device copies of q / new K,V / slots /
+tables / lengths from pinned memory and the device->host copy of the output.
+
+Metric: algorithmic KV bytes the decode reads (sum over sequences of
+context_len * num_kv_heads * head_dim * 2 bytes * 2 for K and V) per second;
+seq*layers/s is reported beside it.  Multi-GPU: one process per GPU, each an
+independent replica of the batch (the path has no exchange step), timed
+between barriers, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("paged decode KV GB/s and % of B200 HBM peak; "
+          "seq·layers/s at 1 GPU")
+SPEC_HBM_GBS = 8000.0          # the spec figure the target is quoted against
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--workload", default="llama3_70b_gqa8")
+    p.add_argument("--impl", default="native", choices=["native", "reference"])
+    p.add_argument("--kernel", default="auto")
+    p.add_argument("--partition-size", type=int, default=-1)
+    p.add_argument("--no-extras", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (timing only; the data path has no collective)
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "native" else "gloo"
+        if backend == "nccl":
+            import torch
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend,
+                                timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64,
+                     device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index),
+                 f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f[5], f[6], f[7], f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        sm = [r[0] for r in rows]
+        load = [r[0] for r in rows if r[0] > 0.5 * r[1]] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[2 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(load)), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# native arm
+
+def measured_hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("decode.cu", "device_utils.cuh"):
+        with open(os.path.join(ROOT, "paged_kv_cache_383_b200", "csrc",
+                               name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current decode source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"decode_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"source_hash:\s*([0-9a-f]+)", text)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not (m_hash and m_tr) or m_hash.group(1) != decode_source_hash():
+        return None
+    return float(m_tr.group(1))
+
+
+def kv_bytes(lengths, w) -> int:
+    return int(np.sum(lengths)) * w.num_kv_heads * w.head_dim * 2 * 2
+
+
+def run_native(args, rank, world, local):
+    import torch
+    import paged_kv_cache_383_b200 as pkv
+    from paged_kv_cache_383_b200 import flow
+    from paged_kv_cache_383_b200 import workloads as wl
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = wl.WORKLOADS[args.workload]
+    ps = w.partition_size if args.partition_size < 0 else args.partition_size
+
+    # CPU baseline inputs are gathered later from the same device tensors;
+    # start the oracle pool before any GPU work (spawn context).
+    pool = None
+    want_cpu = (rank == 0 and world == 1 and not args.no_cpu_baseline)
+    if want_cpu:
+        pool = start_oracle_pool()
+
+    inp = wl.make_paged(w, device=dev)
+    if inp.k_new is None:                   # every step writes a new token
+        g = torch.Generator(device=dev)
+        g.manual_seed(w.seed + 7)
+        shp = (w.num_seqs, w.num_kv_heads, w.head_dim)
+        inp.k_new = torch.randn(shp, generator=g, device=dev).to(inp.q.dtype)
+        inp.v_new = torch.randn(shp, generator=g, device=dev).to(inp.q.dtype)
+        pos = inp.lengths - 1
+        inp.new_slots = (inp.block_tables[np.arange(w.num_seqs),
+                                          pos // w.block_size]
+                         .astype(np.int64) * w.block_size
+                         + pos % w.block_size)
+    bt = torch.from_numpy(inp.block_tables).to(dev)
+    cl = torch.from_numpy(inp.lengths.astype(np.int32)).to(dev)
+    slots = torch.from_numpy(inp.new_slots).to(dev)
+    out = torch.empty_like(inp.q)
+    max_ctx = int(inp.lengths.max())
+    desc = pkv.make_desc(inp.q, inp.k_cache, bt, partition_size=ps,
+                         max_context_len=max_ctx, kernel=args.kernel)
+    ws_bytes = pkv.pa_decode_workspace_bytes(desc)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    step_bytes = kv_bytes(inp.lengths, w)
+
+    def step():
+        pkv.pa_cache_write(inp.k_cache, inp.v_cache, inp.k_new, inp.v_new,
+                           slots, dev_err=err, stream=stream)
+        pkv.pa_decode(out, inp.q, inp.k_cache, inp.v_cache, bt, cl,
+                      w.softmax_scale, desc=desc, workspace=ws, dev_err=err,
+                      stream=stream)
+
+    clocks = ClockSampler(local)
+    t_spin = time.time()
+    while time.time() - t_spin < 1.0:       # bring clocks up (untimed)
+        step()
+        torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    n_ev = args.steps
+    ev_dec = [(torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    launches0 = pkv.pa_launch_count()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(args.steps):
+        pkv.pa_cache_write(inp.k_cache, inp.v_cache, inp.k_new, inp.v_new,
+                           slots, dev_err=err, stream=stream)
+        ev_dec[i][0].record(stream)
+        pkv.pa_decode(out, inp.q, inp.k_cache, inp.v_cache, bt, cl,
+                      w.softmax_scale, desc=desc, workspace=ws, dev_err=err,
+                      stream=stream)
+        ev_dec[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = pkv.pa_launch_count() - launches0
+    clk = clocks.stop()
+    ms_local = t0.elapsed_time(t1)
+    ms_total = max_over_ranks(ms_local, world)
+    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_dec]))
+    if err.item() != 0:
+        raise RuntimeError(f"device error flag {err.item()} during bench")
+
+    ms_step = ms_total / args.steps
+    value = world * step_bytes / (ms_step * 1e-3) / 1e9
+    peak, peak_kind = measured_hbm_peak()
+    achieved = step_bytes / (dec_ms * 1e-3) / 1e9
+    res = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bfloat16" else "fp16",
+        "data": "synthetic (seeded N(0,1) q/K/V, shuffled physical blocks)",
+        "seq_layers_per_s": round(world * w.num_seqs / (ms_step * 1e-3), 1),
+        "pct_of_spec_8000": round(100 * value / world / SPEC_HBM_GBS, 2),
+        "pct_of_measured_copy": round(100 * value / world / peak, 2),
+        "config": {
+            "workload": w.name,
+            "num_seqs": w.num_seqs, "num_q_heads": w.num_q_heads,
+            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim,
+            "block_size": w.block_size, "total_tokens": int(inp.lengths.sum()),
+            "max_context_len": max_ctx,
+            "partition_size": pkv.pa_decode_partition_size(desc),
+            "kernel": args.kernel,
+            "kv_bytes_per_step": step_bytes,
+            "l2": "inputs larger than L2 (no flush): "
+                  f"{step_bytes / 1e9:.2f} GB of K/V read per step",
+            "parallelism": f"{world} independent replicas" if world > 1
+                           else "1 GPU",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "pa_decode (decode + partition reduce)",
+            "achieved": round(achieved, 2),
+            "peak": peak,
+            "peak_kind": f"{peak_kind} HBM copy bandwidth",
+            "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "frac_of_spec_8000": round(achieved / SPEC_HBM_GBS, 4),
+            "traffic": profiled_traffic(w.name),
+            "decode_ms": round(dec_ms, 5),
+        },
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_extras:
+        res["extras"] = extras(args, w, inp, dev, pkv)
+    res["e2e"] = run_e2e(args, w, inp, dev, pkv, flow, world, rank, ps)
+    if want_cpu:
+        res["cpu_baseline"] = cpu_baseline(pool, inp, w, dev)
+    if pool is not None:
+        pool.close()
+    return res
+
+
+def extras(args, w, inp, dev, pkv):
+    """Side measurements: the SIMT kernel on the same inputs, and a
+    read-only torch reduction over a 4 GB buffer (read bandwidth ref)."""
+    import torch
+    out = {}
+    bt = torch.from_numpy(inp.block_tables).to(dev)
+    cl = torch.from_numpy(inp.lengths.astype(np.int32)).to(dev)
+    o = torch.empty_like(inp.q)
+    max_ctx = int(inp.lengths.max())
+
+    def time_decode(kernel, ps):
+        desc = pkv.make_desc(inp.q, inp.k_cache, bt, partition_size=ps,
+                             max_context_len=max_ctx, kernel=kernel)
+        ws = torch.empty(max(pkv.pa_decode_workspace_bytes(desc), 16),
+                         dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            pkv.pa_decode(o, inp.q, inp.k_cache, inp.v_cache, bt, cl,
+                          w.softmax_scale, desc=desc, workspace=ws)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(20):
+            pkv.pa_decode(o, inp.q, inp.k_cache, inp.v_cache, bt, cl,
+                          w.softmax_scale, desc=desc, workspace=ws)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / 20
+        return round(kv_bytes(inp.lengths, w) / (ms * 1e-3) / 1e9, 1)
+
+    out["decode_gbs_simt"] = time_decode("simt", w.partition_size)
+    out["decode_gbs_mma"] = time_decode("mma", w.partition_size)
+    for ps in (256, 512, 1024, 2048):
+        out[f"decode_gbs_mma_ps{ps}"] = time_decode("mma", ps)
+    x = torch.empty(1 << 30, dtype=torch.float32, device=dev).fill_(1.0)
+    for _ in range(3):
+        x.sum()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(10):
+        x.sum()
+    b.record()
+    torch.cuda.synchronize()
+    out["torch_sum_read_gbs"] = round(4 * (1 << 30) / (a.elapsed_time(b) /
+                                                        10 * 1e-3) / 1e9, 1)
+    del x
+    return out
+
+
+def run_e2e(args, w, inp, dev, pkv, flow, world, rank, ps):
+    """Same step through the public API with host buffers: per step the
+    block manager appends one token to every sequence, the tables are
+    rebuilt, inputs go host->device from pinned memory, the output comes
+    back device->host."""
+    import torch
+    bm = pkv.BlockManager(inp.num_blocks, w.block_size,
+                          free_order=_free_order(inp))
+    ids = np.arange(w.num_seqs, dtype=np.int64)
+    for b in ids:
+        bm.add_seq(int(b))
+    bm.append_batch(ids, inp.lengths.astype(np.int32) - 1)
+    steps = args.steps
+    max_blocks = int(wl_blocks(inp.lengths + steps + args.warmup + 1,
+                               w.block_size).max())
+    pin = dict(
+        q=inp.q.cpu().pin_memory(), k=inp.k_new.cpu().pin_memory(),
+        v=inp.v_new.cpu().pin_memory(),
+        out=torch.empty(inp.q.shape, dtype=inp.q.dtype).pin_memory())
+    dq = torch.empty_like(inp.q)
+    dk = torch.empty_like(inp.k_new)
+    dv = torch.empty_like(inp.v_new)
+    dout = torch.empty_like(inp.q)
+    ones = np.ones(w.num_seqs, dtype=np.int32)
+    stream = torch.cuda.current_stream(dev)
+    t_slots = torch.empty(w.num_seqs, dtype=torch.int64).pin_memory()
+    t_table = torch.empty(w.num_seqs, max_blocks,
+                          dtype=torch.int32).pin_memory()
+    t_lens = torch.empty(w.num_seqs, dtype=torch.int32).pin_memory()
+    h2d = d2h = 0
+    tot_bytes = 0
+
+    def one(record):
+        nonlocal h2d, d2h, tot_bytes
+        stream.synchronize()          # pinned staging buffers are reused
+        slots, pairs = bm.append_batch(ids, ones, slots_out=t_slots.numpy())
+        table, lens = bm.block_table(ids, max_blocks,
+                                     table_out=t_table.numpy(),
+                                     lens_out=t_lens.numpy())
+        dq.copy_(pin["q"], non_blocking=True)
+        dk.copy_(pin["k"], non_blocking=True)
+        dv.copy_(pin["v"], non_blocking=True)
+        d_slots = t_slots.to(dev, non_blocking=True)
+        d_table = t_table.to(dev, non_blocking=True)
+        d_lens = t_lens.to(dev, non_blocking=True)
+        nb = 0
+        if len(pairs):
+            d_pairs = torch.from_numpy(pairs).pin_memory().to(
+                dev, non_blocking=True)
+            pkv.pa_copy_blocks(inp.k_cache, inp.v_cache, d_pairs)
+            nb += pairs.nbytes
+        pkv.pa_cache_write(inp.k_cache, inp.v_cache, dk, dv, d_slots)
+        pkv.pa_decode(dout, dq, inp.k_cache, inp.v_cache, d_table, d_lens,
+                      w.softmax_scale, partition_size=ps,
+                      max_context_len=int(lens.max()))
+        pin["out"].copy_(dout, non_blocking=True)
+        stream.synchronize()
+        if record:
+            h2d = (pin["q"].nbytes + pin["k"].nbytes + pin["v"].nbytes
+                   + slots.nbytes + table.nbytes + lens.nbytes + nb)
+            d2h = pin["out"].nbytes
+            tot_bytes += kv_bytes(lens, w)
+
+    for _ in range(args.warmup):
+        one(False)
+    barrier(world)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one(True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b), world)
+    bm.close()
+    return {"value": round(world * tot_bytes / (ms * 1e-3) / 1e9, 2),
+            "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(ms / steps, 4),
+            "includes": "host block-manager append + table build, pinned "
+                        "H2D of q/new K,V/slots/tables/lengths, cache write, "
+                        "decode, D2H of the output, one sync per step"}
+
+
+def wl_blocks(lengths, bs):
+    from paged_kv_cache_383_b200 import workloads as wl
+    return wl.blocks_needed(lengths, bs)
+
+
+def _free_order(inp):
+    """The pool order under which a fresh block manager hands out exactly
+    the workload's tables: their blocks in sequence order, then the rest."""
+    used = [inp.block_tables[b, : int(wl_blocks([L], inp.workload.block_size)
+                                      [0])]
+            for b, L in enumerate(inp.lengths)]
+    used = np.concatenate(used) if used else np.zeros(0, np.int32)
+    rest = np.setdiff1d(np.arange(inp.num_blocks), used, assume_unique=False)
+    return np.concatenate([used, rest]).astype(np.int32)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+
+def _oracle_task(task):
+    import numpy as _np
+    from oracle import attention as oa
+    q, kc, vc, L, scale = task
+    sub = _np.arange(kc.shape[0])[None, :]
+    return oa.paged_decode(q, kc, vc, sub, _np.array([L]), scale)
+
+
+POOL_SIZE = os.cpu_count() or 1
+
+
+def start_oracle_pool():
+    import multiprocessing as mp
+    os.environ.setdefault("OMP_NUM_THREADS", "1")
+    os.environ.setdefault("OPENBLAS_NUM_THREADS", "1")
+    os.environ.setdefault("MKL_NUM_THREADS", "1")
+    ctx = mp.get_context("spawn")
+    return ctx.Pool(POOL_SIZE)
+
+
+def _tasks_from_device(inp, w, seqs):
+    import torch
+    tasks = []
+    for b in seqs:
+        L = int(inp.lengths[b])
+        n = int(wl_blocks([L], w.block_size)[0])
+        idx = torch.from_numpy(inp.block_tables[b, :n].astype(np.int64)).to(
+            inp.k_cache.device)
+        tasks.append((inp.q[b:b + 1].float().cpu().numpy(),
+                      inp.k_cache.index_select(0, idx).float().cpu().numpy(),
+                      inp.v_cache.index_select(0, idx).float().cpu().numpy(),
+                      L, w.softmax_scale))
+    return tasks
+
+
+def time_oracle(pool, tasks, min_seconds):
+    t0 = time.time()
+    reps = 0
+    while True:
+        pool.map(_oracle_task, tasks, chunksize=1)
+        reps += 1
+        if time.time() - t0 >= min_seconds:
+            break
+    return time.time() - t0, reps
+
+
+def cpu_baseline(pool, inp, w, dev):
+    seqs = list(range(min(64, w.num_seqs)))
+    tasks = _tasks_from_device(inp, w, seqs)
+    secs, reps = time_oracle(pool, tasks, 10.0)
+    toks = int(inp.lengths[seqs].sum())
+    gbs = reps * kv_bytes(inp.lengths[seqs], w) / secs / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": POOL_SIZE,
+            "kind": "oracle",
+            "seq_layers_per_s": round(reps * len(seqs) / secs, 2),
+            "sample": f"first {len(seqs)} of {w.num_seqs} sequences of "
+                      f"{w.name} ({toks} tokens), fp64 oracle repeated "
+                      f"{reps}x over {secs:.1f} s, process pool of "
+                      f"{POOL_SIZE} (1 BLAS thread each)"}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 CPU oracle on this workload's shape, each
+    step a bounded sample of the batch (inputs drawn on the host)."""
+    from paged_kv_cache_383_b200 import workloads as wl
+    pool = start_oracle_pool()
+    w = wl.WORKLOADS[args.workload]
+    n = min(16, w.num_seqs)
+    ws = w.scaled(num_seqs=n) if w.lengths != "fixed" else w
+    inp = wl.make_paged(ws, device="cpu")
+    tasks = _tasks_from_device(inp, ws, range(ws.num_seqs))
+    for _ in range(args.warmup):
+        pool.map(_oracle_task, tasks, chunksize=1)
+    t0 = time.time()
+    for _ in range(args.steps):
+        pool.map(_oracle_task, tasks, chunksize=1)
+    secs = time.time() - t0
+    pool.close()
+    step_bytes = kv_bytes(inp.lengths, ws)
+    value = args.steps * step_bytes / secs / 1e9
+    cores = POOL_SIZE
+    sample = (f"{ws.num_seqs} sequences drawn with {w.name}'s length "
+              f"distribution ({int(inp.lengths.sum())} tokens) per step")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4),
+            "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(1e3 * secs / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "sample": sample},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s",
+                             "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s",
+                    "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_setup(args)
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    res = run_native(args, rank, world, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,267 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv.so: paged KV-cache decode attention for
+ * NVIDIA B200 (sm_100a), its cache-write and copy-on-write kernels, and the
+ * host-side block manager that produces block tables and slot mappings.
+ *
+ * Sources (cited by short name in the comments below):
+ *   [Taming the Tail]          "Taming the Tail: How PagedAttention Solves the
+ *                              KV-Cache Fragmentation Crisis in Multi-Tenant
+ *                              LLM Serving" (architects-blueprint.vercel.app)
+ *   [vLLM PagedAttention FAQ]  "vLLM PagedAttention: Eliminating KV Cache
+ *                              Memory Fragmentation & 4x Throughput"
+ *                              (tinycto.tv)
+ *   [KV-cache chapter]         the "g12s-kv-cache" chapter on KV-cache
+ *                              management (aicomputerinstitute.com)
+ *
+ * Conventions for every call:
+ *   - Tensor arguments are DEVICE pointers borrowed from the caller, who
+ *     allocates and frees them; the library never frees or keeps them.
+ *     Every tensor pointer must be 16-byte aligned and densely packed in the
+ *     layout stated for it.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Kernel calls are asynchronous on that stream; their return
+ *     value reports argument checks and launch errors only.
+ *   - `dev_err` (nullable) is a device int32.  A kernel that meets a
+ *     violation it can only see on the device (a block id outside the pool, a
+ *     slot outside the cache, a context length beyond the table) stores
+ *     PA_ERR_DEVICE_OOB there, skips the affected work and never touches an
+ *     out-of-range address; a bounded wait that gave up stores
+ *     PA_ERR_DEVICE_TIMEOUT.  The library never clears it: the caller zeroes
+ *     it and reads it after synchronising.
+ *   - Ordering on one stream: pa_copy_blocks, then pa_cache_write, then
+ *     pa_decode ([KV-cache chapter] "PagedAttention: borrowing virtual
+ *     memory...": a private copy is made before the first write into a shared
+ *     block).
+ *   - pa_last_error() returns a thread-local text describing the last
+ *     non-OK status produced on the calling thread.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID_ARG = 1,     /* null pointer, bad size, misaligned pointer */
+  PA_ERR_UNSUPPORTED = 2,     /* a shape the kernels are not built for      */
+  PA_ERR_NO_FREE_BLOCKS = 3,  /* block manager: the pool is exhausted       */
+  PA_ERR_CUDA = 4,            /* a CUDA runtime call or launch failed       */
+  PA_ERR_DEVICE_OOB = 5,      /* device-side index check failed (dev_err)   */
+  PA_ERR_WORKSPACE = 6,       /* workspace missing or too small             */
+  PA_ERR_DEVICE_TIMEOUT = 7   /* a bounded device-side wait gave up         */
+} pa_status;
+
+typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Which decode kernel runs.  Both compute the same result.
+ *   PA_KERNEL_AUTO  -- the tensor-core kernel.
+ *   PA_KERNEL_SIMT  -- fp32 CUDA-core dot products (kept for comparison).
+ *   PA_KERNEL_MMA   -- the grouped query heads of one KV head form the N=8
+ *                      side of warp-level bf16/fp16 tensor-core MMAs for
+ *                      both QK^T and PV, fp32 accumulation. */
+typedef enum { PA_KERNEL_AUTO = 0, PA_KERNEL_SIMT = 1, PA_KERNEL_MMA = 2 } pa_kernel;
+
+/* Shape of one decode call.
+ *   num_q_heads must be a multiple of num_kv_heads; G = num_q_heads /
+ *   num_kv_heads <= 8.  Query head h reads KV head h / G (consecutive
+ *   grouping; the pages name grouped-query attention but no mapping).
+ *   head_dim in {64, 128}; block_size in {16, 32} ([vLLM PagedAttention FAQ]
+ *   "Prevention & Safeguards": block size 16 or 32).
+ *   partition_size: tokens per split-context partition of one sequence; 0 =
+ *   choose automatically; otherwise a multiple of block_size in [block_size,
+ *   8192].  Sequences longer than one partition are computed as independent
+ *   partitions whose partial softmax statistics a second kernel combines.
+ *   max_context_len: host-side upper bound on every context_lens[] entry;
+ *   sizes the grid and the workspace.  0 means num_blocks_per_seq * block_size. */
+typedef struct {
+  int num_seqs;
+  int num_q_heads;
+  int num_kv_heads;
+  int head_dim;
+  int block_size;
+  int max_blocks_per_seq;
+  int num_blocks;
+  pa_dtype dtype;
+  int partition_size;
+  int max_context_len;
+  pa_kernel kernel;
+} pa_decode_desc;
+
+/* Library version string, and the text of a status code. */
+const char* pa_version(void);
+const char* pa_status_string(pa_status s);
+/* Description of the last non-OK status returned on this thread ("" if none). */
+const char* pa_last_error(void);
+
+/* ------------------------------------------------------------------------
+ * Decode attention over a paged KV cache.
+ *
+ * Defines ([Taming the Tail] "Under the Hood: The CUDA Kernel Engineering";
+ * [KV-cache chapter] "PagedAttention: borrowing virtual memory..." and
+ * "Common misconception..."; [vLLM PagedAttention FAQ] "Does PagedAttention
+ * change the mathematical attention output?"): for sequence b and query head
+ * h, with K_b / V_b the sequence's tokens gathered through its block table,
+ *     out[b,h,:] = softmax(scale * K_b q[b,h,:]) V_b
+ * exactly as contiguous multi-head attention would compute it.  A sequence
+ * with context length 0 gets a zero output row.
+ *
+ * Layouts (all dense, row-major):
+ *   out, q        [num_seqs, num_q_heads, head_dim]          dtype
+ *   k_cache,
+ *   v_cache       [num_blocks, num_kv_heads, block_size, head_dim]  dtype
+ *   block_tables  [num_seqs, max_blocks_per_seq] int32 physical block ids;
+ *                 entries past a sequence's last block are ignored
+ *   context_lens  [num_seqs] int32, tokens per sequence, the newest included
+ *   workspace     pa_decode_workspace_bytes(desc) bytes of device memory the
+ *                 caller owns (may be NULL when that size is 0); its contents
+ *                 need no initialisation and are scratch after the call.
+ * Computation: fp32 scores, fp32 online softmax, fp32 accumulation; the
+ * output is rounded once to dtype.
+ * Errors: PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED / PA_ERR_WORKSPACE before
+ * any launch; PA_ERR_CUDA if a launch fails.  Device-side: a context length
+ * outside [0, max_blocks_per_seq * block_size] or above max_context_len, or a
+ * block id outside [0, num_blocks), sets *dev_err = PA_ERR_DEVICE_OOB and the
+ * affected sequence's output rows are unspecified.
+ * ---------------------------------------------------------------------- */
+size_t pa_decode_workspace_bytes(const pa_decode_desc* desc);
+
+/* Partition size the call will use for this shape (resolves 0 = auto). */
+int pa_decode_partition_size(const pa_decode_desc* desc);
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache,
+                    const void* v_cache, const int32_t* block_tables,
+                    const int32_t* context_lens, float scale,
+                    const pa_decode_desc* desc, void* workspace,
+                    size_t workspace_bytes, int32_t* dev_err, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Write new tokens' K and V into their cache slots.
+ *
+ * Defines ([Taming the Tail] "How the Architecture Works"; [KV-cache
+ * chapter] "A one-paragraph recap": each step stores only the new token's K
+ * and V): for token t with s = slot_mapping[t] >= 0,
+ *     k_cache[s / block_size, :, s % block_size, :] = k[t, :, :]
+ *     v_cache[s / block_size, :, s % block_size, :] = v[t, :, :]
+ * a byte-exact copy.  slot_mapping[t] < 0 marks padding and is skipped.
+ * Layouts: k, v [num_tokens, num_kv_heads, head_dim]; slot_mapping
+ * [num_tokens] int64 on the device; caches as for pa_decode.
+ * Slots must be distinct (two tokens writing one slot race).  A slot >=
+ * num_blocks * block_size sets *dev_err = PA_ERR_DEVICE_OOB and is skipped.
+ * ---------------------------------------------------------------------- */
+pa_status pa_cache_write(void* k_cache, void* v_cache, const void* k,
+                         const void* v, const int64_t* slot_mapping,
+                         int num_tokens, int num_kv_heads, int head_dim,
+                         int block_size, int num_blocks, pa_dtype dtype,
+                         int32_t* dev_err, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Copy whole blocks for copy-on-write.
+ *
+ * Defines ([KV-cache chapter] "PagedAttention: borrowing virtual memory...";
+ * [Taming the Tail] "Complex Memory Sharing"): for each pair i,
+ *     k_cache[dst] = k_cache[src];  v_cache[dst] = v_cache[src]
+ * (all KV heads, all slots of the block), byte-exact, where
+ * (src, dst) = (pairs[2i], pairs[2i+1]).  pairs is device int32 [num_pairs][2]
+ * as produced by pa_bm_append.  Destinations must be distinct and no
+ * destination may also be a source in the same call.  An id outside
+ * [0, num_blocks) sets *dev_err = PA_ERR_DEVICE_OOB and that pair is skipped.
+ * ---------------------------------------------------------------------- */
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs,
+                         int num_pairs, int num_kv_heads, int head_dim,
+                         int block_size, int num_blocks, pa_dtype dtype,
+                         int32_t* dev_err, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Host block manager: free block pool, per-sequence logical->physical block
+ * tables, reference counts and copy-on-write ([Taming the Tail] "How the
+ * Architecture Works", "Complex Memory Sharing"; [vLLM PagedAttention FAQ]
+ * "Underlying Mechanism"; [KV-cache chapter] "PagedAttention: borrowing
+ * virtual memory..." and answer A6).  Pure host code: it touches no device
+ * memory and produces only integer arrays.  A handle is not thread-safe; its
+ * memory is owned by the handle and released by pa_bm_destroy.
+ * ---------------------------------------------------------------------- */
+
+/* Create a pool of num_blocks blocks of block_size tokens.  free_order
+ * (nullable, host int32[num_blocks]) is a permutation of 0..num_blocks-1
+ * giving the order in which a fresh pool hands blocks out (NULL = ascending).
+ * Blocks returned to the pool are handed out again before untouched ones
+ * (most recently freed first). */
+pa_status pa_bm_create(int num_blocks, int block_size,
+                       const int32_t* free_order, void** bm);
+void pa_bm_destroy(void* bm);
+
+/* Register an empty sequence.  INVALID_ARG if the id exists. */
+pa_status pa_bm_add_seq(void* bm, int64_t seq_id);
+
+/* The child shares every block of the parent (each reference count + 1) and
+ * starts with the parent's length ([vLLM PagedAttention FAQ] "Zero-Copy
+ * Forking & Parallel Sampling"). */
+pa_status pa_bm_fork(void* bm, int64_t parent_id, int64_t child_id);
+
+/* Reserve n_tokens new token slots at the end of seq_id.
+ * A new block is taken only when the last block is full; the first write
+ * into a block whose reference count is above one first moves the sequence
+ * to a private copy (count of the old block - 1).
+ *   slots_out      host int64[n_tokens]: slot = block * block_size + offset
+ *                  for each new token, in order (pass to pa_cache_write).
+ *   cow_pairs_out  host int32[2 * max_cow]: (src, dst) blocks to copy with
+ *                  pa_copy_blocks BEFORE writing the slots.  At most one pair
+ *                  per call.  Nullable only if max_cow == 0 and no copy is
+ *                  needed.
+ *   num_cow_out    number of pairs written.
+ * If the pool cannot supply every block the call needs, returns
+ * PA_ERR_NO_FREE_BLOCKS and changes nothing. */
+pa_status pa_bm_append(void* bm, int64_t seq_id, int n_tokens,
+                       int64_t* slots_out, int32_t* cow_pairs_out,
+                       int max_cow, int* num_cow_out);
+
+/* Batched form of pa_bm_append for one decode step: appends n_tokens[i]
+ * tokens to seq_ids[i] for i = 0..n-1, in order.
+ *   slots_out      host int64[sum(n_tokens)], the sequences' slots in order.
+ *   cow_pairs_out  host int32[2 * max_cow] (max_cow >= number of sequences
+ *                  whose last block is shared suffices); pairs in order.
+ *   num_cow_out    pairs written.   num_done_out  sequences fully appended.
+ * If the pool runs out at sequence i, returns PA_ERR_NO_FREE_BLOCKS with
+ * *num_done_out = i: appends 0..i-1 stand (their slots and pairs are
+ * written), sequence i and later are unchanged. */
+pa_status pa_bm_append_batch(void* bm, const int64_t* seq_ids,
+                             const int32_t* n_tokens, int n,
+                             int64_t* slots_out, int32_t* cow_pairs_out,
+                             int max_cow, int* num_cow_out, int* num_done_out);
+
+/* Drop the sequence: each of its blocks' counts - 1; blocks at zero return
+ * to the pool ([KV-cache chapter] answer A6). */
+pa_status pa_bm_free_seq(void* bm, int64_t seq_id);
+
+/* Keep the first new_len tokens and release the blocks past them, e.g. to
+ * discard rejected speculative tokens ([Taming the Tail] "The Future:
+ * Speculative Decoding and Beyond").  new_len <= current length. */
+pa_status pa_bm_truncate(void* bm, int64_t seq_id, int64_t new_len);
+
+/* Fill host table_out[n][max_blocks] (int32, unused entries -1) and
+ * lens_out[n] (int32) for the listed sequences.  INVALID_ARG if a sequence
+ * holds more than max_blocks blocks or is longer than INT32_MAX tokens. */
+pa_status pa_bm_block_table(void* bm, const int64_t* seq_ids, int n,
+                            int max_blocks, int32_t* table_out,
+                            int32_t* lens_out);
+
+/* Kernel launches this library has issued in this process (all devices,
+ * all threads): lets a caller count the GPU work a timed region contained. */
+int64_t pa_launch_count(void);
+
+/* Pool and sequence queries (-1 for an unknown handle / sequence / block). */
+int pa_bm_num_free(void* bm);
+int pa_bm_refcount(void* bm, int block);
+int64_t pa_bm_seq_len(void* bm, int64_t seq_id);
+int pa_bm_num_seq_blocks(void* bm, int64_t seq_id);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* PAGEDKV_H */

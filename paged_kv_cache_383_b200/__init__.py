@@ -1,0 +1,314 @@
+"""Paged KV-cache decode attention for NVIDIA B200 (sm_100a).
+
+Python binding of libpagedkv.so.  The functions keep the C ABI's names
+(``pa_decode``, ``pa_cache_write``, ``pa_copy_blocks``, ``pa_bm_*``) and only
+marshal arguments: they take torch tensors for device memory and streams,
+check dtypes / devices / contiguity, and pass raw pointers to the library.
+All computation happens in the library's CUDA kernels and C++ block manager;
+if the library is missing, every call raises.
+
+Layouts (see include/pagedkv.h for the full contract):
+  q, out            [num_seqs, num_q_heads, head_dim]            fp16 / bf16
+  k_cache, v_cache  [num_blocks, num_kv_heads, block_size, head_dim]
+  block_tables      [num_seqs, max_blocks_per_seq] int32
+  context_lens      [num_seqs] int32
+  k, v (new tokens) [num_tokens, num_kv_heads, head_dim]
+  slot_mapping      [num_tokens] int64
+  pairs             [num_pairs, 2] int32
+"""
+from __future__ import annotations
+
+import ctypes
+
+from . import _lib
+from ._lib import (PA_BF16, PA_F16, PA_KERNEL_AUTO, PA_KERNEL_MMA,
+                   PA_KERNEL_SIMT, PagedKVError, NoFreeBlocksError,
+                   pa_decode_desc)
+
+__all__ = [
+    "pa_decode", "pa_cache_write", "pa_copy_blocks",
+    "pa_decode_workspace_bytes", "pa_decode_partition_size", "make_desc",
+    "BlockManager", "PagedKVError", "NoFreeBlocksError", "library_path",
+    "pa_launch_count",
+    "PA_KERNEL_AUTO", "PA_KERNEL_MMA", "PA_KERNEL_SIMT",
+]
+
+_KERNELS = {"auto": PA_KERNEL_AUTO, "mma": PA_KERNEL_MMA,
+            "simt": PA_KERNEL_SIMT}
+
+
+def library_path() -> str:
+    return _lib.LIB_PATH
+
+
+def pa_launch_count() -> int:
+    """Kernel launches libpagedkv has issued in this process."""
+    return int(_lib.load().pa_launch_count())
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float16:
+        return PA_F16
+    if t.dtype == torch.bfloat16:
+        return PA_BF16
+    raise TypeError(f"expected float16 or bfloat16, got {t.dtype}")
+
+
+def _dev(t, name: str, dtype=None):
+    """Pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def make_desc(q, k_cache, block_tables, *, partition_size: int = 0,
+              max_context_len: int = 0, kernel: str = "auto") -> pa_decode_desc:
+    """Decode descriptor from tensor shapes."""
+    num_seqs, num_q_heads, head_dim = q.shape
+    num_blocks, num_kv_heads, block_size, hd2 = k_cache.shape
+    if hd2 != head_dim:
+        raise ValueError("q and k_cache disagree on head_dim")
+    if block_tables.shape[0] != num_seqs:
+        raise ValueError("block_tables rows != num_seqs")
+    return pa_decode_desc(
+        num_seqs=num_seqs, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
+        head_dim=head_dim, block_size=block_size,
+        max_blocks_per_seq=block_tables.shape[1], num_blocks=num_blocks,
+        dtype=_dtype_code(q), partition_size=partition_size,
+        max_context_len=max_context_len, kernel=_KERNELS[kernel])
+
+
+def pa_decode_workspace_bytes(desc: pa_decode_desc) -> int:
+    return int(_lib.load().pa_decode_workspace_bytes(ctypes.byref(desc)))
+
+
+def pa_decode_partition_size(desc: pa_decode_desc) -> int:
+    ps = _lib.load().pa_decode_partition_size(ctypes.byref(desc))
+    if ps < 0:
+        _lib.check(_lib.PA_ERR_INVALID_ARG, "pa_decode_partition_size")
+    return ps
+
+
+def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens,
+              scale: float, *, partition_size: int = 0,
+              max_context_len: int = 0, kernel: str = "auto",
+              workspace=None, dev_err=None, stream=None,
+              desc: pa_decode_desc | None = None):
+    """out[b, h] = softmax(scale * K_b q[b, h]) V_b over each sequence's
+    paged K/V.  ``workspace`` (uint8 CUDA tensor) is allocated with torch when
+    the call needs one and none is given.  Returns ``out``."""
+    import torch
+    lib = _lib.load()
+    if desc is None:
+        desc = make_desc(q, k_cache, block_tables,
+                         partition_size=partition_size,
+                         max_context_len=max_context_len, kernel=kernel)
+    dt = q.dtype
+    for name, t in (("out", out), ("k_cache", k_cache), ("v_cache", v_cache)):
+        if t.dtype != dt:
+            raise TypeError(f"{name} dtype {t.dtype} != q dtype {dt}")
+    need = int(lib.pa_decode_workspace_bytes(ctypes.byref(desc)))
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _dev(workspace, "workspace") if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() \
+        if workspace is not None else 0
+    st = lib.pa_decode(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32),
+        ctypes.c_float(scale), ctypes.byref(desc), ws_ptr, ws_bytes,
+        _dev(dev_err, "dev_err", torch.int32), _stream(stream))
+    _lib.check(st, "pa_decode")
+    return out
+
+
+def pa_cache_write(k_cache, v_cache, k, v, slot_mapping, *, dev_err=None,
+                   stream=None):
+    """Copy each new token's K and V rows into cache slot slot_mapping[t]
+    (negative slots are skipped)."""
+    import torch
+    lib = _lib.load()
+    num_blocks, num_kv_heads, block_size, head_dim = k_cache.shape
+    num_tokens = k.shape[0]
+    if k.shape != (num_tokens, num_kv_heads, head_dim) or v.shape != k.shape:
+        raise ValueError("k, v must be [num_tokens, num_kv_heads, head_dim]")
+    if slot_mapping.shape != (num_tokens,):
+        raise ValueError("slot_mapping must be [num_tokens]")
+    for name, t in (("v_cache", v_cache), ("k", k), ("v", v)):
+        if t.dtype != k_cache.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} != k_cache dtype")
+    st = lib.pa_cache_write(
+        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(k, "k"),
+        _dev(v, "v"), _dev(slot_mapping, "slot_mapping", torch.int64),
+        num_tokens, num_kv_heads, head_dim, block_size, num_blocks,
+        _dtype_code(k_cache), _dev(dev_err, "dev_err", torch.int32),
+        _stream(stream))
+    _lib.check(st, "pa_cache_write")
+
+
+def pa_copy_blocks(k_cache, v_cache, pairs, *, dev_err=None, stream=None):
+    """k_cache[dst] = k_cache[src] and v_cache[dst] = v_cache[src] for every
+    (src, dst) row of ``pairs`` (int32 [n, 2] on the device)."""
+    import torch
+    lib = _lib.load()
+    num_blocks, num_kv_heads, block_size, head_dim = k_cache.shape
+    if pairs.dim() != 2 or pairs.shape[1] != 2:
+        raise ValueError("pairs must be [num_pairs, 2]")
+    if v_cache.dtype != k_cache.dtype:
+        raise TypeError("k_cache and v_cache dtypes differ")
+    st = lib.pa_copy_blocks(
+        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(pairs, "pairs", torch.int32), pairs.shape[0], num_kv_heads,
+        head_dim, block_size, num_blocks, _dtype_code(k_cache),
+        _dev(dev_err, "dev_err", torch.int32), _stream(stream))
+    _lib.check(st, "pa_copy_blocks")
+
+
+class BlockManager:
+    """Host block manager of libpagedkv (pa_bm_* calls).
+
+    Free pool, per-sequence block tables, reference counts, fork and
+    copy-on-write.  Not thread-safe.
+    """
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        self._lib = _lib.load()
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        handle = ctypes.c_void_p()
+        order = None
+        if free_order is not None:
+            import numpy as np
+            arr = np.ascontiguousarray(free_order, dtype=np.int32)
+            if arr.shape != (num_blocks,):
+                raise ValueError("free_order must have num_blocks entries")
+            order = arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+        _lib.check(self._lib.pa_bm_create(num_blocks, block_size, order,
+                                          ctypes.byref(handle)),
+                   "pa_bm_create")
+        self._h = handle
+
+    def close(self):
+        if self._h:
+            self._lib.pa_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add_seq(self, seq_id: int):
+        _lib.check(self._lib.pa_bm_add_seq(self._h, seq_id), "pa_bm_add_seq")
+
+    def fork(self, parent: int, child: int):
+        _lib.check(self._lib.pa_bm_fork(self._h, parent, child), "pa_bm_fork")
+
+    def append(self, seq_id: int, n_tokens: int):
+        """Returns (slots int64 ndarray [n_tokens], cow_pairs int32 [k, 2])."""
+        import numpy as np
+        slots = np.empty(max(n_tokens, 0), dtype=np.int64)
+        pairs = np.empty(2, dtype=np.int32)
+        ncow = ctypes.c_int(0)
+        st = self._lib.pa_bm_append(
+            self._h, seq_id, n_tokens,
+            slots.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+            pairs.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), 1,
+            ctypes.byref(ncow))
+        _lib.check(st, "pa_bm_append")
+        return slots, pairs[: 2 * ncow.value].reshape(-1, 2).copy()
+
+    def append_batch(self, seq_ids, n_tokens, slots_out=None):
+        """One call for a whole decode step: appends n_tokens[i] tokens to
+        seq_ids[i].  Returns (slots int64 [sum], cow_pairs int32 [k, 2]).
+        ``slots_out`` (optional int64 ndarray, e.g. a view of pinned memory)
+        receives the slots.  Raises NoFreeBlocksError (with .num_done) if the
+        pool runs out."""
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        nt = np.ascontiguousarray(n_tokens, dtype=np.int32)
+        if nt.shape != ids.shape:
+            raise ValueError("seq_ids and n_tokens differ in length")
+        total = int(nt.sum())
+        if slots_out is not None:
+            if (slots_out.dtype != np.int64 or slots_out.shape != (total,)
+                    or not slots_out.flags.c_contiguous):
+                raise ValueError("slots_out must be contiguous int64 [sum]")
+            slots = slots_out
+        else:
+            slots = np.empty(total, dtype=np.int64)
+        pairs = np.empty(2 * max(len(ids), 1), dtype=np.int32)
+        ncow, ndone = ctypes.c_int(0), ctypes.c_int(0)
+        st = self._lib.pa_bm_append_batch(
+            self._h, ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+            nt.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), len(ids),
+            slots.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+            pairs.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), len(ids),
+            ctypes.byref(ncow), ctypes.byref(ndone))
+        try:
+            _lib.check(st, "pa_bm_append_batch")
+        except PagedKVError as e:
+            e.num_done = ndone.value
+            raise
+        return slots, pairs[: 2 * ncow.value].reshape(-1, 2).copy()
+
+    def free_seq(self, seq_id: int):
+        _lib.check(self._lib.pa_bm_free_seq(self._h, seq_id), "pa_bm_free_seq")
+
+    def truncate(self, seq_id: int, new_len: int):
+        _lib.check(self._lib.pa_bm_truncate(self._h, seq_id, new_len),
+                   "pa_bm_truncate")
+
+    def block_table(self, seq_ids, max_blocks: int, table_out=None,
+                    lens_out=None):
+        """Returns (table int32 [n, max_blocks] padded with -1, lens int32).
+        Optional contiguous int32 ``table_out`` / ``lens_out`` arrays receive
+        the result in place."""
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        table = table_out if table_out is not None else \
+            np.empty((len(ids), max_blocks), dtype=np.int32)
+        lens = lens_out if lens_out is not None else \
+            np.empty(len(ids), dtype=np.int32)
+        for arr, shp in ((table, (len(ids), max_blocks)), (lens, (len(ids),))):
+            if (arr.dtype != np.int32 or arr.shape != shp
+                    or not arr.flags.c_contiguous):
+                raise ValueError("block_table outputs: wrong dtype/shape")
+        st = self._lib.pa_bm_block_table(
+            self._h, ids.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+            len(ids), max_blocks,
+            table.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+            lens.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+        _lib.check(st, "pa_bm_block_table")
+        return table, lens
+
+    def num_free(self) -> int:
+        return self._lib.pa_bm_num_free(self._h)
+
+    def refcount(self, block: int) -> int:
+        return self._lib.pa_bm_refcount(self._h, block)
+
+    def seq_len(self, seq_id: int) -> int:
+        return self._lib.pa_bm_seq_len(self._h, seq_id)
+
+    def num_seq_blocks(self, seq_id: int) -> int:
+        return self._lib.pa_bm_num_seq_blocks(self._h, seq_id)

@@ -1,0 +1,57 @@
+"""Build libpagedkv.so in place with nvcc for sm_100a.
+
+Usage: python -m paged_kv_cache_383_b200.build_lib [--verbose]
+"""
+from __future__ import annotations
+
+import os
+import shutil
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(HERE, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+LIB = os.path.join(HERE, "libpagedkv.so")
+
+SOURCES = ["status.cpp", "block_manager.cpp", "cache_ops.cu", "decode.cu"]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), shutil.which("nvcc"),
+                 "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found")
+
+
+def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
+    """Compile every source into one shared library; returns its path."""
+    srcs = [os.path.join(CSRC, s) for s in SOURCES]
+    newest = max(os.path.getmtime(p) for p in
+                 srcs + [os.path.join(CSRC, f) for f in os.listdir(CSRC)] +
+                 [os.path.join(INCLUDE, "pagedkv.h"), __file__])
+    if (os.path.exists(LIB) and os.path.getmtime(LIB) >= newest
+            and not ptxas_verbose):
+        return LIB
+    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17",
+           "-Xcompiler", "-fPIC,-O3,-Wall", "-shared",
+           "-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp", *srcs]
+    if ptxas_verbose:
+        cmd.insert(1, "-Xptxas=-v")
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
+    if verbose or ptxas_verbose:
+        sys.stdout.write(res.stdout + res.stderr)
+    os.replace(LIB + ".tmp", LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(verbose="--verbose" in sys.argv,
+                ptxas_verbose="--ptxas" in sys.argv))

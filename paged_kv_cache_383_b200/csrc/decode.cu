@@ -1,0 +1,911 @@
+// Paged decode attention for sm_100a: pa_decode and its partition reduce.
+//
+// What is computed ([Taming the Tail] "Under the Hood: The CUDA Kernel
+// Engineering"; [KV-cache chapter] "PagedAttention: borrowing virtual memory
+// ..." and "Common misconception..."): for each sequence b and query head h,
+// softmax(scale * K_b q) V_b over the sequence's tokens, K_b / V_b gathered
+// block by block through the block table.  The pages ask three things of the
+// kernel: look the physical block up in the table, keep the accesses
+// coalesced despite the scattered blocks, and handle a partly filled last
+// block.  Their sketch (one fp32 element per thread) is prior art only.
+//
+// B200 design.
+//  * Work unit = (partition of <= partition_size tokens, KV head, sequence):
+//    one CTA.  All G = Hq/Hkv query heads of the KV head are served by the
+//    same CTA, so each K/V byte leaves HBM once.
+//  * Warp 0, lane 0 is the producer.  It stages the unit's slice of the block
+//    table in shared memory and issues 2-D TMA tile loads of whole pages
+//    (block_size rows x 128 B, 128-byte swizzle, no multicast) into an
+//    S-stage ring, each stage one K page + one V page, signalled by mbarriers
+//    with transaction counts.  Waits are bounded (1 s) and report
+//    PA_ERR_DEVICE_TIMEOUT instead of hanging.
+//  * Warps 1..4 are consumers; consumer w takes pages w, w+4, ... and keeps
+//    its own online-softmax state (running max m, sum l, accumulator o) for
+//    all G heads.  At the end the four states are merged through shared
+//    memory.
+//  * Compute variant MMA (default): S^T = K_page . Q^T and O^T += V^T . P^T as
+//    m16n8k16 tensor-core MMAs, N = 8 = the (padded) query-head group.  K
+//    fragments come from ldmatrix, V fragments from ldmatrix.trans, P moves
+//    from the score accumulator layout to the B-operand layout with
+//    movmatrix.  P is split into a rounded part and its residual (two
+//    16-bit operands) so PV keeps ~16 mantissa bits; accumulation is fp32.
+//  * Compute variant SIMT: fp32 FMA dot products on the CUDA cores (kept to
+//    show what the tensor-core mapping buys).
+//  * A sequence that needs more than one partition writes (m, l, o/l) per
+//    partition to the workspace; a second kernel combines them.  A sequence
+//    that fits one partition is written straight to `out`.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "device_utils.cuh"
+#include "pagedkv.h"
+#include "status.h"
+
+namespace pagedkv {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kConsumers = 4;                      // consumer warps per CTA
+constexpr int kThreads = (kConsumers + 1) * 32;    // + one producer warp
+constexpr int kMaxGroup = 8;                       // query heads per KV head
+constexpr int kMaxPartition = 8192;
+constexpr int kMaxParts = 16384;                   // partitions per sequence
+
+struct DecodeArgs {
+  void* out;
+  const void* q;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  float* ws_o;   // [num_seqs, num_q_heads, max_parts, head_dim]
+  float* ws_ml;  // [num_seqs, num_q_heads, max_parts, 2] = (max, sum), log2 units
+  int32_t* dev_err;
+  float scale_log2;  // scale * log2(e): scores are kept in base-2 units
+  int num_q_heads;
+  int num_kv_heads;
+  int group;
+  int max_blocks_per_seq;
+  int num_blocks;
+  int partition_size;
+  int max_parts;
+  int max_context_len;
+};
+
+// Shared-memory geometry of one (block_size, head_dim, stages) instance.
+// A page (one block, one KV head) is head_dim/64 TMA boxes of block_size
+// rows x 128 bytes; within a box, 16-byte chunk c of row r sits at chunk
+// c ^ (r % 8) (the TMA 128-byte swizzle), so eight consecutive rows read at
+// the same logical chunk hit eight different bank groups.
+template <int BS, int D, int S>
+struct Geometry {
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kBoxBytes = BS * 128;
+  static constexpr int kPageBytes = kBoxes * kBoxBytes;
+  static constexpr int kStageBytes = 2 * kPageBytes;  // K page then V page
+  static constexpr int kRingBytes = S * kStageBytes;
+  static constexpr int kBarBytes = 2 * S * 8;         // full[S], empty[S]
+  // Per consumer warp: o[8][D], m[8], l[8] (fp32); aliases the ring.
+  static constexpr int kEpiWarpFloats = kMaxGroup * D + 2 * kMaxGroup;
+  static_assert(kConsumers * kEpiWarpFloats * 4 <= kRingBytes,
+                "epilogue must fit in the ring");
+  // SIMT scratch: q in fp32 with a 4-float skew between the two halves of a
+  // row (bank spread), then per warp scores[BS][8], alpha[8], m_new[8].
+  static constexpr int kQRow = D + 8;
+  static constexpr int kSimtQFloats = kMaxGroup * kQRow;
+  static constexpr int kSimtWarpFloats = BS * kMaxGroup + 2 * kMaxGroup;
+  static constexpr int kSimtBytes =
+      (kSimtQFloats + kConsumers * kSimtWarpFloats) * 4;
+
+  // Byte offset of element (row, col) inside a page.
+  static __device__ __forceinline__ uint32_t offset(int row, int col) {
+    return (col >> 6) * kBoxBytes + row * 128 +
+           ((((col & 63) >> 3) ^ (row & 7)) << 4) + (col & 7) * 2;
+  }
+};
+
+// Bytes of the staged block-table slice, rounded to 16.
+__host__ __device__ constexpr int bt_bytes(int pages_per_part) {
+  return (pages_per_part * 4 + 15) & ~15;
+}
+
+// Dynamic shared memory of one CTA: alignment slack, ring, barriers, the
+// block-table slice and (SIMT only) the fp32 scratch.
+template <int BS, int D, int S, bool kMma>
+constexpr size_t smem_bytes_for(int pages_per_part) {
+  using G = Geometry<BS, D, S>;
+  return 1024 + G::kRingBytes + G::kBarBytes + bt_bytes(pages_per_part) +
+         (kMma ? 0 : G::kSimtBytes);
+}
+
+template <typename T>
+__device__ __forceinline__ T from_float(float x);
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_float(float x) {
+  return __float2bfloat16_rn(x);
+}
+template <>
+__device__ __forceinline__ __half from_float(float x) {
+  return __float2half_rn(x);
+}
+
+template <typename T>
+__device__ __forceinline__ float to_float(T x);
+template <>
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <>
+__device__ __forceinline__ float to_float(__half x) {
+  return __half2float(x);
+}
+
+__device__ __forceinline__ float warp_max_xor(float v, int lo_mask,
+                                              int hi_mask) {
+  for (int m = lo_mask; m <= hi_mask; m <<= 1)
+    v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// The decode kernel.
+template <typename T, int BS, int D, int S, bool kMma>
+__global__ void __launch_bounds__(kThreads)
+    decode_kernel(const __grid_constant__ CUtensorMap kmap,
+                  const __grid_constant__ CUtensorMap vmap,
+                  const DecodeArgs a) {
+  using Geo = Geometry<BS, D, S>;
+  extern __shared__ uint8_t smem_dyn[];
+  // The TMA swizzle is a function of shared-memory address bits, so the ring
+  // must start on a 1024-byte boundary of the shared window.
+  uint8_t* smem = smem_dyn + ((1024u - (dev::smem_u32(smem_dyn) & 1023u)) & 1023u);
+
+  const int part = blockIdx.x;
+  const int kvh = blockIdx.y;
+  const int b = blockIdx.z;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  const int ctx = a.context_lens[b];
+  if (ctx < 0 || ctx > a.max_blocks_per_seq * BS || ctx > a.max_context_len) {
+    if (part == 0 && kvh == 0 && tid == 0)
+      dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
+    return;
+  }
+  const int PS = a.partition_size;
+  const int n_parts = ctx > 0 ? (ctx + PS - 1) / PS : 1;
+  if (part >= n_parts) return;
+  const int tok0 = part * PS;
+  const int n_tok = min(ctx - tok0, PS);  // 0 only when ctx == 0
+  const int n_pages = (n_tok + BS - 1) / BS;
+  const int page0 = tok0 / BS;
+  const int G = a.group;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Geo::kRingBytes);
+  int32_t* bt_s = reinterpret_cast<int32_t*>(bars + 2 * S);
+  const uint32_t ring = dev::smem_u32(smem);
+  const uint32_t full0 = dev::smem_u32(bars);
+  const uint32_t empty0 = full0 + S * 8;
+
+  // Stage this partition's slice of the block table; check every id.
+  int bad = 0;
+  const int32_t* bt_row =
+      a.block_tables + static_cast<int64_t>(b) * a.max_blocks_per_seq + page0;
+  for (int i = tid; i < n_pages; i += kThreads) {
+    const int32_t p = bt_row[i];
+    bad |= (p < 0 || p >= a.num_blocks);
+    bt_s[i] = p;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      dev::mbar_init(full0 + s * 8, 1);
+      dev::mbar_init(empty0 + s * 8, 1);
+    }
+    dev::fence_mbar_init();
+  }
+  bad = __syncthreads_or(bad);
+  if (bad) {
+    if (tid == 0) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
+    if (n_parts > 1 && tid < G) {  // mark the partition empty for the reduce
+      const int64_t row =
+          (static_cast<int64_t>(b) * a.num_q_heads + kvh * G + tid) *
+              a.max_parts + part;
+      a.ws_ml[2 * row] = -INFINITY;
+      a.ws_ml[2 * row + 1] = 0.f;
+    }
+    return;
+  }
+
+  // ---------------- producer ----------------
+  if (warp == 0) {
+    if (lane == 0 && n_pages > 0) {
+      dev::prefetch_tmap(&kmap);
+      dev::prefetch_tmap(&vmap);
+      for (int i = 0; i < n_pages; ++i) {
+        const int s = i % S;
+        if (i >= S && !dev::mbar_wait(empty0 + s * 8, ((i / S) - 1) & 1)) {
+          dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
+          break;
+        }
+        const uint32_t full = full0 + s * 8;
+        dev::mbar_arrive_expect_tx(full, Geo::kStageBytes);
+        const int y = (bt_s[i] * a.num_kv_heads + kvh) * BS;
+        const uint32_t kdst = ring + s * Geo::kStageBytes;
+#pragma unroll
+        for (int bx = 0; bx < Geo::kBoxes; ++bx) {
+          dev::tma_load_2d(kdst + bx * Geo::kBoxBytes, &kmap, bx * 64, y, full);
+          dev::tma_load_2d(kdst + Geo::kPageBytes + bx * Geo::kBoxBytes, &vmap,
+                           bx * 64, y, full);
+        }
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int cw = warp - 1;
+  const int ctid = tid - 32;  // 0 .. kConsumers*32-1
+  const T* qrow = static_cast<const T*>(a.q) +
+                  (static_cast<int64_t>(b) * a.num_q_heads + kvh * G) * D;
+  float m_fin[2], l_fin[2];  // per-lane head state handed to the epilogue
+
+  if constexpr (kMma) {
+    using M = dev::Mma<T>;
+    const int g4 = lane >> 2;  // fragment row group
+    const int t4 = lane & 3;   // thread in group
+    // B fragments of Q^T (K = head_dim, N = 8 heads): head g4, dims
+    // kk*16 + 2*t4 (+1) and +8.  Heads past G are zero.
+    uint32_t qf[D / 16][2];
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        qf[kk][r] = 0u;
+        if (g4 < G)
+          qf[kk][r] = *reinterpret_cast<const uint32_t*>(
+              qrow + g4 * D + kk * 16 + r * 8 + 2 * t4);
+      }
+    }
+    float o[D / 16][4];
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+
+    // ldmatrix lane roles: matrix mi = lane/8, row j = lane%8.
+    const int mi = lane >> 3;
+    const int j = lane & 7;
+
+    for (int i = cw; i < n_pages; i += kConsumers) {
+      const int s = i % S;
+      if (!dev::mbar_wait(full0 + s * 8, (i / S) & 1)) {
+        dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
+        break;
+      }
+      const uint32_t kb = ring + s * Geo::kStageBytes;
+      const uint32_t vb = kb + Geo::kPageBytes;
+      const int nv = min(BS, n_tok - i * BS);
+
+      // S^T (tokens x heads) for each 16-token slice of the page.
+      float sc[BS / 16][4];
+#pragma unroll
+      for (int mt = 0; mt < BS / 16; ++mt) {
+        float acc0[4] = {0.f, 0.f, 0.f, 0.f};
+        float acc1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          uint32_t af[4];
+          dev::ldsm_x4(kb + Geo::offset(mt * 16 + j + (mi & 1) * 8,
+                                        kk * 16 + (mi >> 1) * 8),
+                       af);
+          if (kk & 1)
+            M::run(acc1, af, qf[kk][0], qf[kk][1]);
+          else
+            M::run(acc0, af, qf[kk][0], qf[kk][1]);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int tok = mt * 16 + g4 + (e >> 1) * 8;
+          const float x = (acc0[e] + acc1[e]) * a.scale_log2;
+          sc[mt][e] = tok < nv ? x : -INFINITY;
+        }
+      }
+      // Online softmax; this lane holds heads 2*t4 and 2*t4+1.
+      float alpha[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int mt = 0; mt < BS / 16; ++mt)
+          mx = fmaxf(mx, fmaxf(sc[mt][h], sc[mt][h + 2]));
+        mx = warp_max_xor(mx, 4, 16);
+        const float m_new = fmaxf(m_run[h], mx);
+        alpha[h] = dev::fast_exp2(m_run[h] - m_new);
+        float sum = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < BS / 16; ++mt) {
+          sc[mt][h] = dev::fast_exp2(sc[mt][h] - m_new);
+          sc[mt][h + 2] = dev::fast_exp2(sc[mt][h + 2] - m_new);
+          sum += sc[mt][h] + sc[mt][h + 2];
+        }
+        l_run[h] = l_run[h] * alpha[h] + sum;
+        m_run[h] = m_new;
+      }
+#pragma unroll
+      for (int dt = 0; dt < D / 16; ++dt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[dt][e] *= alpha[e & 1];
+
+      // P^T as B fragments (K = tokens, N = heads): rounded part and residual.
+      uint32_t bh[BS / 16][2], bl[BS / 16][2];
+#pragma unroll
+      for (int ks = 0; ks < BS / 16; ++ks) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float p0 = sc[ks][2 * r], p1 = sc[ks][2 * r + 1];
+          const uint32_t hi = M::pack(p0, p1);
+          const float2 hf = M::unpack(hi);
+          const uint32_t lo = M::pack(p0 - hf.x, p1 - hf.y);
+          bh[ks][r] = dev::movmatrix_trans(hi);
+          bl[ks][r] = dev::movmatrix_trans(lo);
+        }
+      }
+      // O^T (head_dim x heads) += V^T . P^T
+#pragma unroll
+      for (int dt = 0; dt < D / 16; ++dt) {
+#pragma unroll
+        for (int ks = 0; ks < BS / 16; ++ks) {
+          uint32_t af[4];
+          dev::ldsm_x4_trans(vb + Geo::offset(ks * 16 + j + (mi >> 1) * 8,
+                                              dt * 16 + (mi & 1) * 8),
+                             af);
+          M::run(o[dt], af, bh[ks][0], bh[ks][1]);
+          M::run(o[dt], af, bl[ks][0], bl[ks][1]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(empty0 + s * 8);
+    }
+
+    // Hand this warp's state to the epilogue area (aliases the ring).
+    dev::named_barrier(1, kConsumers * 32);
+    float* ep = reinterpret_cast<float*>(smem) + cw * Geo::kEpiWarpFloats;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float l = l_run[h];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      m_fin[h] = m_run[h];
+      l_fin[h] = l;
+    }
+#pragma unroll
+    for (int dt = 0; dt < D / 16; ++dt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        ep[(2 * t4 + (e & 1)) * D + dt * 16 + g4 + (e >> 1) * 8] = o[dt][e];
+    if (g4 == 0) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        ep[kMaxGroup * D + 2 * t4 + h] = m_fin[h];
+        ep[kMaxGroup * D + kMaxGroup + 2 * t4 + h] = l_fin[h];
+      }
+    }
+  } else {
+    // ---------------- SIMT variant ----------------
+    float* q_s = reinterpret_cast<float*>(
+        reinterpret_cast<uint8_t*>(bt_s) + bt_bytes(PS / BS));
+    float* wsp = q_s + Geo::kSimtQFloats + cw * Geo::kSimtWarpFloats;
+    float* sp = wsp;                      // scores / probabilities [BS][8]
+    float* alpha_s = wsp + BS * kMaxGroup;
+    float* mnew_s = alpha_s + kMaxGroup;
+
+    // q -> fp32 shared copy; half h of a row is skewed by 4h floats.
+    for (int idx = ctid; idx < kMaxGroup * D; idx += kConsumers * 32) {
+      const int g = idx / D, d = idx % D;
+      const float v = g < G ? to_float<T>(qrow[g * D + d]) : 0.f;
+      q_s[g * Geo::kQRow + d + (d >= D / 2 ? 4 : 0)] = v;
+    }
+    dev::named_barrier(1, kConsumers * 32);
+
+    // QK roles: BS=16 -> token lane%16, half lane/16; BS=32 -> token lane.
+    constexpr int kHalves = 32 / BS;       // 2 or 1
+    constexpr int kDPer = D / kHalves;     // dims per lane in QK
+    const int qtok = lane % BS;
+    const int qhalf = lane / BS;
+    // PV roles: lane owns dims [lane*D/32, +D/32).
+    constexpr int kDPV = D / 32;           // 4 or 2
+    const int d0 = lane * kDPV;
+
+    float acc_o[kMaxGroup][kDPV];
+#pragma unroll
+    for (int g = 0; g < kMaxGroup; ++g)
+#pragma unroll
+      for (int e = 0; e < kDPV; ++e) acc_o[g][e] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;  // lanes 0..7: head `lane`
+
+    for (int i = cw; i < n_pages; i += kConsumers) {
+      const int s = i % S;
+      if (!dev::mbar_wait(full0 + s * 8, (i / S) & 1)) {
+        dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
+        break;
+      }
+      const uint8_t* kpg = smem + s * Geo::kStageBytes;
+      const uint8_t* vpg = kpg + Geo::kPageBytes;
+      const int nv = min(BS, n_tok - i * BS);
+
+      float acc[kMaxGroup];
+#pragma unroll
+      for (int g = 0; g < kMaxGroup; ++g) acc[g] = 0.f;
+#pragma unroll 2
+      for (int c = 0; c < kDPer / 8; ++c) {
+        const int d = qhalf * kDPer + c * 8;
+        const uint4 raw = *reinterpret_cast<const uint4*>(
+            kpg + Geo::offset(qtok, d));
+        const T* kv = reinterpret_cast<const T*>(&raw);
+        float kf[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kf[e] = to_float<T>(kv[e]);
+        const float* qd = q_s + d + (d >= D / 2 ? 4 : 0);
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; ++g) {
+          const float4 qa = *reinterpret_cast<const float4*>(qd + g * Geo::kQRow);
+          const float4 qb =
+              *reinterpret_cast<const float4*>(qd + g * Geo::kQRow + 4);
+          acc[g] += qa.x * kf[0] + qa.y * kf[1] + qa.z * kf[2] + qa.w * kf[3] +
+                    qb.x * kf[4] + qb.y * kf[5] + qb.z * kf[6] + qb.w * kf[7];
+        }
+      }
+      if (kHalves == 2) {
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; ++g)
+          acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], 16);
+      }
+      if (qhalf == 0) {
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; ++g)
+          sp[qtok * kMaxGroup + g] =
+              qtok < nv ? acc[g] * a.scale_log2 : -INFINITY;
+      }
+      __syncwarp();
+      if (lane < kMaxGroup) {
+        float mx = -INFINITY;
+        for (int t = 0; t < BS; ++t) mx = fmaxf(mx, sp[t * kMaxGroup + lane]);
+        const float m_new = fmaxf(m_run, mx);
+        alpha_s[lane] = dev::fast_exp2(m_run - m_new);
+        mnew_s[lane] = m_new;
+        m_run = m_new;
+      }
+      __syncwarp();
+      for (int idx = lane; idx < BS * kMaxGroup; idx += 32)
+        sp[idx] = dev::fast_exp2(sp[idx] - mnew_s[idx % kMaxGroup]);
+      __syncwarp();
+      if (lane < kMaxGroup) {
+        float sum = 0.f;
+        for (int t = 0; t < BS; ++t) sum += sp[t * kMaxGroup + lane];
+        l_run = l_run * alpha_s[lane] + sum;
+      }
+#pragma unroll
+      for (int g = 0; g < kMaxGroup; ++g) {
+        const float al = alpha_s[g];
+#pragma unroll
+        for (int e = 0; e < kDPV; ++e) acc_o[g][e] *= al;
+      }
+      for (int t = 0; t < nv; ++t) {
+        float vf[kDPV];
+        if constexpr (kDPV == 4) {
+          const uint2 raw = *reinterpret_cast<const uint2*>(
+              vpg + Geo::offset(t, d0));
+          const T* vv = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) vf[e] = to_float<T>(vv[e]);
+        } else {
+          const uint32_t raw = *reinterpret_cast<const uint32_t*>(
+              vpg + Geo::offset(t, d0));
+          const T* vv = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+          for (int e = 0; e < 2; ++e) vf[e] = to_float<T>(vv[e]);
+        }
+        const float4 pa =
+            *reinterpret_cast<const float4*>(sp + t * kMaxGroup);
+        const float4 pb =
+            *reinterpret_cast<const float4*>(sp + t * kMaxGroup + 4);
+        const float p[8] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+#pragma unroll
+        for (int g = 0; g < kMaxGroup; ++g)
+#pragma unroll
+          for (int e = 0; e < kDPV; ++e) acc_o[g][e] += p[g] * vf[e];
+      }
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(empty0 + s * 8);
+    }
+
+    dev::named_barrier(1, kConsumers * 32);
+    float* ep = reinterpret_cast<float*>(smem) + cw * Geo::kEpiWarpFloats;
+#pragma unroll
+    for (int g = 0; g < kMaxGroup; ++g)
+#pragma unroll
+      for (int e = 0; e < kDPV; ++e) ep[g * D + d0 + e] = acc_o[g][e];
+    if (lane < kMaxGroup) {
+      ep[kMaxGroup * D + lane] = m_run;
+      ep[kMaxGroup * D + kMaxGroup + lane] = l_run;
+    }
+    (void)m_fin;
+    (void)l_fin;
+  }
+
+  // ---------------- merge the consumer warps, write the result -------------
+  dev::named_barrier(1, kConsumers * 32);
+  const float* ep0 = reinterpret_cast<const float*>(smem);
+  const bool split = n_parts > 1;
+  for (int idx = ctid; idx < G * D; idx += kConsumers * 32) {
+    const int g = idx / D, d = idx % D;
+    float mmax = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumers; ++w)
+      mmax = fmaxf(mmax, ep0[w * Geo::kEpiWarpFloats + kMaxGroup * D + g]);
+    float val = 0.f, wsum = 0.f;
+    if (mmax != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kConsumers; ++w) {
+        const float* e = ep0 + w * Geo::kEpiWarpFloats;
+        const float mw = e[kMaxGroup * D + g];
+        const float sc = mw == -INFINITY ? 0.f : dev::fast_exp2(mw - mmax);
+        wsum += e[kMaxGroup * D + kMaxGroup + g] * sc;
+        val += e[g * D + d] * sc;
+      }
+      val = wsum > 0.f ? val / wsum : 0.f;
+    }
+    const int qh = kvh * G + g;
+    if (!split) {
+      static_cast<T*>(a.out)[(static_cast<int64_t>(b) * a.num_q_heads + qh) * D +
+                             d] = from_float<T>(val);
+    } else {
+      const int64_t row =
+          (static_cast<int64_t>(b) * a.num_q_heads + qh) * a.max_parts + part;
+      a.ws_o[row * D + d] = val;
+      if (d == 0) {
+        a.ws_ml[2 * row] = mmax;
+        a.ws_ml[2 * row + 1] = wsum;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Partition reduce: out = sum_j w_j o_j / sum_j w_j, w_j = l_j 2^(m_j - M).
+template <typename T, int D>
+__global__ void __launch_bounds__(D)
+    reduce_kernel(const DecodeArgs a, int block_size) {
+  extern __shared__ float w_s[];  // [max_parts]
+  __shared__ float red[D / 32];
+  const int qh = blockIdx.x;
+  const int b = blockIdx.y;
+  const int tid = threadIdx.x;
+  const int ctx = a.context_lens[b];
+  if (ctx < 0 || ctx > a.max_blocks_per_seq * block_size ||
+      ctx > a.max_context_len)
+    return;  // flagged by the decode kernel
+  const int n_parts = ctx > 0 ? (ctx + a.partition_size - 1) / a.partition_size
+                              : 1;
+  if (n_parts <= 1) return;
+  const int64_t row0 =
+      (static_cast<int64_t>(b) * a.num_q_heads + qh) * a.max_parts;
+  const float* ml = a.ws_ml + 2 * row0;
+
+  float mx = -INFINITY;
+  for (int j = tid; j < n_parts; j += D) mx = fmaxf(mx, ml[2 * j]);
+  mx = warp_max_xor(mx, 1, 16);
+  if ((tid & 31) == 0) red[tid >> 5] = mx;
+  __syncthreads();
+  mx = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < D / 32; ++w) mx = fmaxf(mx, red[w]);
+  __syncthreads();
+
+  float ws = 0.f;
+  for (int j = tid; j < n_parts; j += D) {
+    const float mj = ml[2 * j];
+    const float w = (mj == -INFINITY || mx == -INFINITY)
+                        ? 0.f
+                        : ml[2 * j + 1] * dev::fast_exp2(mj - mx);
+    w_s[j] = w;
+    ws += w;
+  }
+  for (int m = 1; m < 32; m <<= 1) ws += __shfl_xor_sync(0xffffffffu, ws, m);
+  if ((tid & 31) == 0) red[tid >> 5] = ws;
+  __syncthreads();
+  ws = 0.f;
+#pragma unroll
+  for (int w = 0; w < D / 32; ++w) ws += red[w];
+
+  const float* o = a.ws_o + row0 * D + tid;
+  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+  int j = 0;
+  for (; j + 4 <= n_parts; j += 4) {
+    acc0 += w_s[j] * o[static_cast<int64_t>(j) * D];
+    acc1 += w_s[j + 1] * o[static_cast<int64_t>(j + 1) * D];
+    acc2 += w_s[j + 2] * o[static_cast<int64_t>(j + 2) * D];
+    acc3 += w_s[j + 3] * o[static_cast<int64_t>(j + 3) * D];
+  }
+  for (; j < n_parts; ++j) acc0 += w_s[j] * o[static_cast<int64_t>(j) * D];
+  const float acc = (acc0 + acc1) + (acc2 + acc3);
+  static_cast<T*>(a.out)[(static_cast<int64_t>(b) * a.num_q_heads + qh) * D +
+                         tid] = from_float<T>(ws > 0.f ? acc / ws : 0.f);
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+
+int device_sm_count() {
+  int dev = 0, count = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
+  return count;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                         cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// The cache viewed as a 2-D tensor of rows (block, kv head, slot) x head_dim;
+// one TMA box is block_size rows x 64 elements (128 bytes), swizzled.
+bool encode_cache_map(CUtensorMap* map, const void* base, uint64_t rows,
+                      int head_dim, int block_size, pa_dtype dtype) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), rows};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * 2};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(block_size)};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map,
+                   dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                    : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+constexpr int stages_for(int bs, int d) {
+  // 64 KB ring per CTA: three CTAs fit one SM's shared memory.
+  return 65536 / (2 * 2 * bs * d);
+}
+
+int resolve_partition(const pa_decode_desc* d, int max_ctx) {
+  if (d->partition_size > 0) return d->partition_size;
+  const int64_t pairs = static_cast<int64_t>(d->num_seqs) * d->num_kv_heads;
+  const int64_t target = 3LL * device_sm_count();
+  int ps = 512;
+  while (ps > 2 * d->block_size && ps > 64 &&
+         pairs * ((max_ctx + ps - 1) / ps) < target)
+    ps /= 2;
+  if (ps < d->block_size) ps = d->block_size;
+  return ps;
+}
+
+int resolve_max_ctx(const pa_decode_desc* d) {
+  return d->max_context_len > 0 ? d->max_context_len
+                                : d->max_blocks_per_seq * d->block_size;
+}
+
+pa_status check_desc(const pa_decode_desc* d) {
+  if (!d) return fail(PA_ERR_INVALID_ARG, "pa_decode: desc is NULL");
+  if (d->num_seqs < 0 || d->num_q_heads <= 0 || d->num_kv_heads <= 0 ||
+      d->max_blocks_per_seq <= 0 || d->num_blocks < 0 ||
+      d->max_context_len < 0 || d->partition_size < 0)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_decode: num_seqs=%d num_q_heads=%d num_kv_heads=%d "
+                "max_blocks_per_seq=%d num_blocks=%d max_context_len=%d "
+                "partition_size=%d", d->num_seqs, d->num_q_heads,
+                d->num_kv_heads, d->max_blocks_per_seq, d->num_blocks,
+                d->max_context_len, d->partition_size);
+  if (d->num_q_heads % d->num_kv_heads)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_decode: num_q_heads %d is not a multiple of num_kv_heads %d",
+                d->num_q_heads, d->num_kv_heads);
+  if (d->num_q_heads / d->num_kv_heads > kMaxGroup)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode: group size %d > %d",
+                d->num_q_heads / d->num_kv_heads, kMaxGroup);
+  if (d->head_dim != 64 && d->head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode: head_dim %d not in {64, 128}",
+                d->head_dim);
+  if (d->block_size != 16 && d->block_size != 32)
+    return fail(PA_ERR_UNSUPPORTED, "pa_decode: block_size %d not in {16, 32}",
+                d->block_size);
+  if (d->dtype != PA_F16 && d->dtype != PA_BF16)
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: dtype %d",
+                static_cast<int>(d->dtype));
+  if (d->kernel != PA_KERNEL_AUTO && d->kernel != PA_KERNEL_SIMT &&
+      d->kernel != PA_KERNEL_MMA)
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: kernel %d",
+                static_cast<int>(d->kernel));
+  if (d->partition_size > 0 &&
+      (d->partition_size % d->block_size || d->partition_size > kMaxPartition))
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_decode: partition_size %d must be a multiple of block_size "
+                "%d and <= %d", d->partition_size, d->block_size,
+                kMaxPartition);
+  if (static_cast<int64_t>(d->max_blocks_per_seq) * d->block_size >
+      0x7fffffffLL)
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: max_blocks_per_seq too large");
+  if (static_cast<int64_t>(d->num_blocks) * d->num_kv_heads * d->block_size >
+      0x7fffffffLL)
+    return fail(PA_ERR_UNSUPPORTED,
+                "pa_decode: num_blocks * num_kv_heads * block_size exceeds "
+                "2^31 rows");
+  if (d->num_seqs > 65535 || d->num_kv_heads > 65535)
+    return fail(PA_ERR_UNSUPPORTED,
+                "pa_decode: num_seqs and num_kv_heads must be <= 65535");
+  return PA_OK;
+}
+
+size_t workspace_bytes(const pa_decode_desc* d) {
+  const int max_ctx = resolve_max_ctx(d);
+  const int ps = resolve_partition(d, max_ctx);
+  const int64_t parts = max_ctx > 0 ? (max_ctx + ps - 1) / ps : 1;
+  if (parts <= 1) return 0;
+  return static_cast<size_t>(d->num_seqs) * d->num_q_heads * parts *
+         (d->head_dim + 2) * sizeof(float);
+}
+
+template <typename T, int BS, int D, bool kMma>
+pa_status launch(const pa_decode_desc* d, DecodeArgs& a, const CUtensorMap& km,
+                 const CUtensorMap& vm, cudaStream_t stream) {
+  constexpr int S = stages_for(BS, D);
+  auto kern = decode_kernel<T, BS, D, S, kMma>;
+  const size_t smem =
+      smem_bytes_for<BS, D, S, kMma>(a.partition_size / BS);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  static bool configured[64] = {false};
+  if (dev < 0 || dev >= 64 || !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(
+        kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        static_cast<int>(smem_bytes_for<BS, D, S, kMma>(kMaxPartition / BS)));
+    if (e != cudaSuccess)
+      return fail(PA_ERR_CUDA, "pa_decode: cudaFuncSetAttribute: %s",
+                  cudaGetErrorString(e));
+    if (dev >= 0 && dev < 64) configured[dev] = true;
+  }
+  dim3 grid(a.max_parts, d->num_kv_heads, d->num_seqs);
+  kern<<<grid, kThreads, smem, stream>>>(km, vm, a);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return fail(PA_ERR_CUDA, "pa_decode: decode launch failed: %s",
+                cudaGetErrorString(e));
+  if (a.max_parts > 1) {
+    reduce_kernel<T, D><<<dim3(d->num_q_heads, d->num_seqs), D,
+                          a.max_parts * sizeof(float), stream>>>(a, BS);
+    count_launch();
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+      return fail(PA_ERR_CUDA, "pa_decode: reduce launch failed: %s",
+                  cudaGetErrorString(e));
+  }
+  return PA_OK;
+}
+
+template <typename T, bool kMma>
+pa_status dispatch_shape(const pa_decode_desc* d, DecodeArgs& a,
+                         const CUtensorMap& km, const CUtensorMap& vm,
+                         cudaStream_t st) {
+  if (d->block_size == 16)
+    return d->head_dim == 128 ? launch<T, 16, 128, kMma>(d, a, km, vm, st)
+                              : launch<T, 16, 64, kMma>(d, a, km, vm, st);
+  return d->head_dim == 128 ? launch<T, 32, 128, kMma>(d, a, km, vm, st)
+                            : launch<T, 32, 64, kMma>(d, a, km, vm, st);
+}
+
+}  // namespace
+}  // namespace pagedkv
+
+using pagedkv::fail;
+
+extern "C" {
+
+size_t pa_decode_workspace_bytes(const pa_decode_desc* desc) {
+  pagedkv::clear_error();
+  if (pagedkv::check_desc(desc) != PA_OK) return 0;
+  return pagedkv::workspace_bytes(desc);
+}
+
+int pa_decode_partition_size(const pa_decode_desc* desc) {
+  pagedkv::clear_error();
+  if (pagedkv::check_desc(desc) != PA_OK) return -1;
+  return pagedkv::resolve_partition(desc, pagedkv::resolve_max_ctx(desc));
+}
+
+pa_status pa_decode(void* out, const void* q, const void* k_cache,
+                    const void* v_cache, const int32_t* block_tables,
+                    const int32_t* context_lens, float scale,
+                    const pa_decode_desc* desc, void* workspace,
+                    size_t workspace_bytes, int32_t* dev_err, void* stream) {
+  pagedkv::clear_error();
+  pa_status st = pagedkv::check_desc(desc);
+  if (st != PA_OK) return st;
+  if (!std::isfinite(scale))
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: scale is not finite");
+  if (desc->num_seqs == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: NULL tensor pointer");
+  if (!pagedkv::aligned16(out) || !pagedkv::aligned16(q) ||
+      !pagedkv::aligned16(k_cache) || !pagedkv::aligned16(v_cache))
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_decode: out, q and the caches must be 16-byte aligned");
+  if (desc->num_blocks == 0)
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: empty block pool");
+
+  const int max_ctx = pagedkv::resolve_max_ctx(desc);
+  const int ps = pagedkv::resolve_partition(desc, max_ctx);
+  const int parts = max_ctx > 0 ? (max_ctx + ps - 1) / ps : 1;
+  if (parts > pagedkv::kMaxParts)
+    return fail(PA_ERR_UNSUPPORTED,
+                "pa_decode: %d partitions of %d tokens exceed %d; use a "
+                "larger partition_size", parts, ps, pagedkv::kMaxParts);
+  const size_t need = pagedkv::workspace_bytes(desc);
+  if (need > 0 && (!workspace || workspace_bytes < need ||
+                   !pagedkv::aligned16(workspace)))
+    return fail(PA_ERR_WORKSPACE,
+                "pa_decode: workspace of %zu bytes (16-byte aligned) needed, "
+                "got %zu at %p", need, workspace_bytes, workspace);
+
+  CUtensorMap kmap, vmap;
+  const uint64_t rows = static_cast<uint64_t>(desc->num_blocks) *
+                        desc->num_kv_heads * desc->block_size;
+  if (!pagedkv::encode_cache_map(&kmap, k_cache, rows, desc->head_dim,
+                                 desc->block_size, desc->dtype) ||
+      !pagedkv::encode_cache_map(&vmap, v_cache, rows, desc->head_dim,
+                                 desc->block_size, desc->dtype))
+    return fail(PA_ERR_CUDA, "pa_decode: cuTensorMapEncodeTiled failed");
+
+  pagedkv::DecodeArgs a;
+  a.out = out;
+  a.q = q;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.ws_o = static_cast<float*>(workspace);
+  a.ws_ml = need > 0 ? static_cast<float*>(workspace) +
+                           static_cast<size_t>(desc->num_seqs) *
+                               desc->num_q_heads * parts * desc->head_dim
+                     : nullptr;
+  a.dev_err = dev_err;
+  a.scale_log2 = scale * pagedkv::kLog2e;
+  a.num_q_heads = desc->num_q_heads;
+  a.num_kv_heads = desc->num_kv_heads;
+  a.group = desc->num_q_heads / desc->num_kv_heads;
+  a.max_blocks_per_seq = desc->max_blocks_per_seq;
+  a.num_blocks = desc->num_blocks;
+  a.partition_size = ps;
+  a.max_parts = parts;
+  a.max_context_len = max_ctx;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool mma = desc->kernel != PA_KERNEL_SIMT;
+  if (desc->dtype == PA_BF16)
+    return mma ? pagedkv::dispatch_shape<__nv_bfloat16, true>(desc, a, kmap,
+                                                              vmap, s)
+               : pagedkv::dispatch_shape<__nv_bfloat16, false>(desc, a, kmap,
+                                                               vmap, s);
+  return mma ? pagedkv::dispatch_shape<__half, true>(desc, a, kmap, vmap, s)
+             : pagedkv::dispatch_shape<__half, false>(desc, a, kmap, vmap, s);
+}
+
+}  // extern "C"

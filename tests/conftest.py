@@ -19,3 +19,14 @@ def golden():
     with open(os.path.join(ROOT, "tests", "golden",
                            "worked_examples.json")) as f:
         return json.load(f)
+
+
+@pytest.fixture(scope="session")
+def pkv():
+    """The package with libpagedkv.so built (nvcc works without a GPU)."""
+    from paged_kv_cache_383_b200 import build_lib
+    build_lib.build()
+    import paged_kv_cache_383_b200 as pkv_mod
+    from paged_kv_cache_383_b200 import _lib
+    _lib.load()
+    return pkv_mod

@@ -1,0 +1,91 @@
+"""Shared helpers of the GPU parity tests: oracle calls on sampled sequences
+and the decode tolerance.
+
+Tolerance (decode output against the unrounded fp64 oracle): every element
+within 2e-3 absolute, and every element with |ref| >= 0.2 within 1e-2
+relative.  One carve-out, the output-rounding floor: where half a unit in the
+last place of the output dtype at |ref| is itself >= 2e-3 (|ref| >= 1 for
+bf16, >= 8 for fp16), no correctly rounded output can meet 2e-3, so such
+elements are held to the relative bound and to half an ulp + 2e-3.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import attention as oa
+
+ATOL = 2e-3
+RTOL = 1e-2
+REL_FLOOR = 0.2
+MANTISSA = {torch.bfloat16: 8, torch.float16: 11}   # incl. implicit bit
+
+
+def half_ulp(ref: np.ndarray, dtype) -> np.ndarray:
+    p = MANTISSA[dtype]
+    e = np.floor(np.log2(np.maximum(np.abs(ref), 1e-30)))
+    return 2.0 ** (e - p)          # ulp = 2^(e - p + 1)
+
+
+def check_decode(out, ref, dtype, what=""):
+    """Assert the tolerance; returns (max_abs, max_rel over |ref|>=0.2)."""
+    out = np.asarray(out, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert out.shape == ref.shape
+    assert np.isfinite(out).all(), f"{what}: non-finite output"
+    err = np.abs(out - ref)
+    hu = half_ulp(ref, dtype)
+    floor = hu >= ATOL
+    bad_abs = (~floor) & (err > ATOL)
+    bad_floor = floor & (err > hu + ATOL)
+    big = np.abs(ref) >= REL_FLOOR
+    rel = np.where(big, err / np.maximum(np.abs(ref), 1e-30), 0.0)
+    bad_rel = rel > RTOL
+    max_abs = float(err.max()) if err.size else 0.0
+    max_rel = float(rel.max()) if rel.size else 0.0
+    assert not bad_abs.any(), (
+        f"{what}: {int(bad_abs.sum())} elements over abs {ATOL}; "
+        f"max abs err {float(err[~floor].max()):.3e}")
+    assert not bad_floor.any(), f"{what}: rounding-floor elements too far"
+    assert not bad_rel.any(), f"{what}: max rel err {max_rel:.3e}"
+    return max_abs, max_rel
+
+
+def to_np(t) -> np.ndarray:
+    return t.detach().float().cpu().numpy()
+
+
+def oracle_paged_sample(q, k_cache, v_cache, tables, lengths, scale, seqs):
+    """fp64 oracle for the listed sequences; the sequences' own blocks are
+    copied to the host (a relabelled sub-pool: the oracle's result does not
+    depend on block ids) so full-size pools need not leave the device."""
+    out = {}
+    for b in seqs:
+        L = int(lengths[b])
+        nblk = -(-L // k_cache.shape[2])
+        ids = np.asarray(tables[b][:nblk], dtype=np.int64)
+        if nblk:
+            idx = torch.from_numpy(ids).to(k_cache.device)
+            kc = to_np(k_cache.index_select(0, idx))
+            vc = to_np(v_cache.index_select(0, idx))
+        else:
+            shp = (1,) + tuple(k_cache.shape[1:])
+            kc = vc = np.zeros(shp)
+        sub = np.arange(max(nblk, 1))[None, :]
+        out[b] = oa.paged_decode(to_np(q[b:b + 1]), kc, vc, sub,
+                                 np.array([L]), scale)[0]
+    return out
+
+
+def sample_seqs(lengths, k=6, seed=0):
+    """The shortest and longest sequences plus a few random ones."""
+    lengths = np.asarray(lengths)
+    order = np.argsort(lengths, kind="stable")
+    rng = np.random.default_rng(seed)
+    pick = {int(order[0]), int(order[-1])}
+    extra = rng.choice(len(lengths), size=min(k, len(lengths)), replace=False)
+    for b in extra:
+        if len(pick) >= k:
+            break
+        pick.add(int(b))
+    return sorted(pick)

@@ -1,0 +1,114 @@
+"""The C ABI: the library loads, exports every symbol include/pagedkv.h
+declares, and rejects bad arguments on the host (no GPU needed: argument
+checks run before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "pagedkv.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(pkv):
+    from paged_kv_cache_383_b200 import _lib
+    names = declared_functions()
+    assert len(names) >= 20
+    raw = ctypes.CDLL(_lib.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+    assert set(names) == set(_lib.SIGNATURES), \
+        set(names) ^ set(_lib.SIGNATURES)
+
+
+def test_version_and_status_strings(pkv):
+    from paged_kv_cache_383_b200 import _lib
+    lib = _lib.load()
+    assert b"sm_100a" in lib.pa_version()
+    assert lib.pa_status_string(_lib.PA_ERR_NO_FREE_BLOCKS) == b"no free blocks"
+
+
+def _desc(**kw):
+    from paged_kv_cache_383_b200 import pa_decode_desc
+    base = dict(num_seqs=2, num_q_heads=8, num_kv_heads=2, head_dim=128,
+                block_size=16, max_blocks_per_seq=4, num_blocks=16, dtype=1,
+                partition_size=0, max_context_len=0, kernel=0)
+    base.update(kw)
+    return pa_decode_desc(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(head_dim=96), 2),
+    (dict(block_size=8), 2),
+    (dict(num_q_heads=7), 1),
+    (dict(num_q_heads=32, num_kv_heads=2), 2),
+    (dict(partition_size=24), 1),
+    (dict(dtype=5), 1),
+    (dict(kernel=9), 1),
+    (dict(num_seqs=-1), 1),
+])
+def test_decode_rejects_bad_descriptors(pkv, kw, status):
+    from paged_kv_cache_383_b200 import _lib
+    lib = _lib.load()
+    d = _desc(**kw)
+    st = lib.pa_decode(None, None, None, None, None, None, ctypes.c_float(1.0),
+                       ctypes.byref(d), None, 0, None, None)
+    assert st == status
+    assert lib.pa_last_error()
+
+
+def test_decode_rejects_null_and_misaligned(pkv):
+    from paged_kv_cache_383_b200 import _lib
+    lib = _lib.load()
+    d = _desc()
+    st = lib.pa_decode(None, None, None, None, None, None, ctypes.c_float(1.0),
+                       ctypes.byref(d), None, 0, None, None)
+    assert st == _lib.PA_ERR_INVALID_ARG
+    fake = 0x1000
+    st = lib.pa_decode(fake + 2, fake, fake, fake, fake, fake,
+                       ctypes.c_float(1.0), ctypes.byref(d), None, 0, None,
+                       None)
+    assert st == _lib.PA_ERR_INVALID_ARG
+    assert b"aligned" in lib.pa_last_error()
+    st = lib.pa_decode(fake, fake, fake, fake, fake, fake,
+                       ctypes.c_float(float("nan")), ctypes.byref(d), None, 0,
+                       None, None)
+    assert st == _lib.PA_ERR_INVALID_ARG
+
+
+def test_decode_needs_workspace_for_split(pkv):
+    from paged_kv_cache_383_b200 import _lib
+    lib = _lib.load()
+    d = _desc(partition_size=16, max_blocks_per_seq=8)
+    need = lib.pa_decode_workspace_bytes(ctypes.byref(d))
+    # 2 seqs x 8 q heads x 8 partitions x (128 + 2) floats
+    assert need == 2 * 8 * 8 * 130 * 4
+    fake = 0x1000
+    st = lib.pa_decode(fake, fake, fake, fake, fake, fake,
+                       ctypes.c_float(1.0), ctypes.byref(d), None, 0, None,
+                       None)
+    assert st == _lib.PA_ERR_WORKSPACE
+    d1 = _desc(partition_size=64)
+    assert lib.pa_decode_workspace_bytes(ctypes.byref(d1)) == 0
+    assert lib.pa_decode_partition_size(ctypes.byref(d1)) == 64
+
+
+def test_zero_sized_calls_are_noops(pkv):
+    from paged_kv_cache_383_b200 import _lib
+    lib = _lib.load()
+    d = _desc(num_seqs=0)
+    assert lib.pa_decode(None, None, None, None, None, None,
+                         ctypes.c_float(1.0), ctypes.byref(d), None, 0, None,
+                         None) == 0
+    assert lib.pa_cache_write(None, None, None, None, None, 0, 8, 128, 16, 4,
+                              1, None, None) == 0
+    assert lib.pa_copy_blocks(None, None, None, 0, 8, 128, 16, 4, 1, None,
+                              None) == 0
+    assert lib.pa_cache_write(None, None, None, None, None, 3, 8, 128, 16, 4,
+                              1, None, None) == _lib.PA_ERR_INVALID_ARG
