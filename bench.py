@@ -52,6 +52,9 @@ def parse_args():
     p.add_argument("--partition-size", type=int, default=-1)
     p.add_argument("--no-extras", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-spinup", action="store_true",
+                   help="skip the 1 s untimed clock spin-up (profiling)")
     return p.parse_args()
 
 
@@ -235,7 +238,8 @@ def run_native(args, rank, world, local):
 
     clocks = ClockSampler(local)
     t_spin = time.time()
-    while time.time() - t_spin < 1.0:       # bring clocks up (untimed)
+    while not args.no_spinup and time.time() - t_spin < 1.0:
+        # bring clocks up (untimed)
         step()
         torch.cuda.synchronize()
     for _ in range(args.warmup):
@@ -321,7 +325,8 @@ def run_native(args, rank, world, local):
     }
     if rank == 0 and world == 1 and not args.no_extras:
         res["extras"] = extras(args, w, inp, dev, pkv)
-    res["e2e"] = run_e2e(args, w, inp, dev, pkv, flow, world, rank, ps)
+    if not args.no_e2e:
+        res["e2e"] = run_e2e(args, w, inp, dev, pkv, flow, world, rank, ps)
     if want_cpu:
         res["cpu_baseline"] = cpu_baseline(pool, inp, w, dev)
     if pool is not None:
@@ -360,7 +365,7 @@ def extras(args, w, inp, dev, pkv):
 
     out["decode_gbs_simt"] = time_decode("simt", w.partition_size)
     out["decode_gbs_mma"] = time_decode("mma", w.partition_size)
-    for ps in (256, 512, 1024, 2048):
+    for ps in (0, 256, 512, 1024, 2048):
         out[f"decode_gbs_mma_ps{ps}"] = time_decode("mma", ps)
     x = torch.empty(1 << 30, dtype=torch.float32, device=dev).fill_(1.0)
     for _ in range(3):

@@ -28,6 +28,7 @@ __global__ void cache_write_kernel(uint4* __restrict__ k_cache,
                                    int num_tokens, int head_chunks,
                                    int num_kv_heads, int block_size,
                                    int64_t num_slots, int32_t* dev_err) {
+  dev::pdl_trigger();  // a following decode may run its prologue now
   const int row_chunks = head_chunks * num_kv_heads;
   for (int64_t t = blockIdx.x; t < num_tokens; t += gridDim.x) {
     const int64_t slot = slot_mapping[t];
@@ -61,6 +62,7 @@ __global__ void copy_blocks_kernel(uint4* __restrict__ k_cache,
                                    const int32_t* __restrict__ pairs,
                                    int64_t block_chunks, int num_blocks,
                                    int32_t* dev_err) {
+  dev::pdl_trigger();
   const int pair = blockIdx.x;
   const int32_t src = pairs[2 * pair];
   const int32_t dst = pairs[2 * pair + 1];

@@ -87,8 +87,11 @@ struct Geometry {
   static constexpr int kStageBytes = 2 * kPageBytes;  // K page then V page
   static constexpr int kRingBytes = S * kStageBytes;
   static constexpr int kBarBytes = 2 * S * 8;         // full[S], empty[S]
-  // Per consumer warp: o[8][D], m[8], l[8] (fp32); aliases the ring.
-  static constexpr int kEpiWarpFloats = kMaxGroup * D + 2 * kMaxGroup;
+  // Per consumer warp: o[8][kORow], m[8], l[8] (fp32); aliases the ring.
+  // Rows are padded by 4 floats so the four head pairs a warp writes at
+  // once land in different banks.
+  static constexpr int kORow = D + 4;
+  static constexpr int kEpiWarpFloats = kMaxGroup * kORow + 2 * kMaxGroup;
   static_assert(kConsumers * kEpiWarpFloats * 4 <= kRingBytes,
                 "epilogue must fit in the ring");
   // SIMT scratch: q in fp32 with a 4-float skew between the two halves of a
@@ -169,6 +172,7 @@ __global__ void __launch_bounds__(kThreads)
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
+  dev::pdl_trigger();  // the reduce may start its prologue early
   const int ctx = a.context_lens[b];
   if (ctx < 0 || ctx > a.max_blocks_per_seq * BS || ctx > a.max_context_len) {
     if (part == 0 && kvh == 0 && tid == 0)
@@ -207,6 +211,9 @@ __global__ void __launch_bounds__(kThreads)
     dev::fence_mbar_init();
   }
   bad = __syncthreads_or(bad);
+  // Everything above reads only host-written inputs; the K/V pages and the
+  // outputs may belong to the previous kernel in the stream.
+  dev::pdl_wait();
   if (bad) {
     if (tid == 0) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
     if (n_parts > 1 && tid < G) {  // mark the partition empty for the reduce
@@ -388,12 +395,13 @@ __global__ void __launch_bounds__(kThreads)
     for (int dt = 0; dt < D / 16; ++dt)
 #pragma unroll
       for (int e = 0; e < 4; ++e)
-        ep[(2 * t4 + (e & 1)) * D + dt * 16 + g4 + (e >> 1) * 8] = o[dt][e];
+        ep[(2 * t4 + (e & 1)) * Geo::kORow + dt * 16 + g4 + (e >> 1) * 8] =
+            o[dt][e];
     if (g4 == 0) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        ep[kMaxGroup * D + 2 * t4 + h] = m_fin[h];
-        ep[kMaxGroup * D + kMaxGroup + 2 * t4 + h] = l_fin[h];
+        ep[kMaxGroup * Geo::kORow + 2 * t4 + h] = m_fin[h];
+        ep[kMaxGroup * Geo::kORow + kMaxGroup + 2 * t4 + h] = l_fin[h];
       }
     }
   } else {
@@ -530,10 +538,11 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int g = 0; g < kMaxGroup; ++g)
 #pragma unroll
-      for (int e = 0; e < kDPV; ++e) ep[g * D + d0 + e] = acc_o[g][e];
+      for (int e = 0; e < kDPV; ++e)
+        ep[g * Geo::kORow + d0 + e] = acc_o[g][e];
     if (lane < kMaxGroup) {
-      ep[kMaxGroup * D + lane] = m_run;
-      ep[kMaxGroup * D + kMaxGroup + lane] = l_run;
+      ep[kMaxGroup * Geo::kORow + lane] = m_run;
+      ep[kMaxGroup * Geo::kORow + kMaxGroup + lane] = l_run;
     }
     (void)m_fin;
     (void)l_fin;
@@ -548,16 +557,17 @@ __global__ void __launch_bounds__(kThreads)
     float mmax = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kConsumers; ++w)
-      mmax = fmaxf(mmax, ep0[w * Geo::kEpiWarpFloats + kMaxGroup * D + g]);
+      mmax = fmaxf(mmax,
+                   ep0[w * Geo::kEpiWarpFloats + kMaxGroup * Geo::kORow + g]);
     float val = 0.f, wsum = 0.f;
     if (mmax != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < kConsumers; ++w) {
         const float* e = ep0 + w * Geo::kEpiWarpFloats;
-        const float mw = e[kMaxGroup * D + g];
+        const float mw = e[kMaxGroup * Geo::kORow + g];
         const float sc = mw == -INFINITY ? 0.f : dev::fast_exp2(mw - mmax);
-        wsum += e[kMaxGroup * D + kMaxGroup + g] * sc;
-        val += e[g * D + d] * sc;
+        wsum += e[kMaxGroup * Geo::kORow + kMaxGroup + g] * sc;
+        val += e[g * Geo::kORow + d] * sc;
       }
       val = wsum > 0.f ? val / wsum : 0.f;
     }
@@ -578,65 +588,94 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ---------------------------------------------------------------------------
-// Partition reduce: out = sum_j w_j o_j / sum_j w_j, w_j = l_j 2^(m_j - M).
+// Partition reduce: out = sum_j w_j o_j / sum_j w_j, w_j = l_j 2^(m_j - M),
+// M = max_j m_j (all in base-2 units).  One CTA per (query head, sequence);
+// warp w folds partitions w, w+4, ... with a running max (one pass, four
+// partitions in flight per warp), then the four warp states are merged.
+constexpr int kReduceWarps = 4;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(D)
+__global__ void __launch_bounds__(kReduceWarps * 32)
     reduce_kernel(const DecodeArgs a, int block_size) {
-  extern __shared__ float w_s[];  // [max_parts]
-  __shared__ float red[D / 32];
+  constexpr int kPer = D / 32;  // dims per lane
+  __shared__ float s_m[kReduceWarps], s_w[kReduceWarps];
+  __shared__ float s_acc[kReduceWarps][D];
   const int qh = blockIdx.x;
   const int b = blockIdx.y;
-  const int tid = threadIdx.x;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  dev::pdl_trigger();
   const int ctx = a.context_lens[b];
   if (ctx < 0 || ctx > a.max_blocks_per_seq * block_size ||
       ctx > a.max_context_len)
     return;  // flagged by the decode kernel
   const int n_parts = ctx > 0 ? (ctx + a.partition_size - 1) / a.partition_size
                               : 1;
-  if (n_parts <= 1) return;
+  if (n_parts <= 1) return;  // the decode kernel wrote this row itself
+  dev::pdl_wait();           // partials of the decode kernel are visible
+
   const int64_t row0 =
       (static_cast<int64_t>(b) * a.num_q_heads + qh) * a.max_parts;
-  const float* ml = a.ws_ml + 2 * row0;
-
-  float mx = -INFINITY;
-  for (int j = tid; j < n_parts; j += D) mx = fmaxf(mx, ml[2 * j]);
-  mx = warp_max_xor(mx, 1, 16);
-  if ((tid & 31) == 0) red[tid >> 5] = mx;
-  __syncthreads();
-  mx = -INFINITY;
+  const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row0;
+  const float* o = a.ws_o + row0 * D + lane * kPer;
+  float M = -INFINITY, W = 0.f;
+  float acc[kPer];
 #pragma unroll
-  for (int w = 0; w < D / 32; ++w) mx = fmaxf(mx, red[w]);
-  __syncthreads();
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
 
-  float ws = 0.f;
-  for (int j = tid; j < n_parts; j += D) {
-    const float mj = ml[2 * j];
-    const float w = (mj == -INFINITY || mx == -INFINITY)
-                        ? 0.f
-                        : ml[2 * j + 1] * dev::fast_exp2(mj - mx);
-    w_s[j] = w;
-    ws += w;
-  }
-  for (int m = 1; m < 32; m <<= 1) ws += __shfl_xor_sync(0xffffffffu, ws, m);
-  if ((tid & 31) == 0) red[tid >> 5] = ws;
-  __syncthreads();
-  ws = 0.f;
+  constexpr int kBatch = 4;
+  for (int j0 = warp; j0 < n_parts; j0 += kBatch * kReduceWarps) {
+    float2 mlj[kBatch];
+    float oj[kBatch][kPer];
 #pragma unroll
-  for (int w = 0; w < D / 32; ++w) ws += red[w];
-
-  const float* o = a.ws_o + row0 * D + tid;
-  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-  int j = 0;
-  for (; j + 4 <= n_parts; j += 4) {
-    acc0 += w_s[j] * o[static_cast<int64_t>(j) * D];
-    acc1 += w_s[j + 1] * o[static_cast<int64_t>(j + 1) * D];
-    acc2 += w_s[j + 2] * o[static_cast<int64_t>(j + 2) * D];
-    acc3 += w_s[j + 3] * o[static_cast<int64_t>(j + 3) * D];
+    for (int u = 0; u < kBatch; ++u) {
+      const int j = j0 + u * kReduceWarps;
+      mlj[u] = j < n_parts ? __ldcg(ml + j) : make_float2(-INFINITY, 0.f);
+#pragma unroll
+      for (int e = 0; e < kPer; ++e)
+        oj[u][e] = j < n_parts ? __ldcg(o + static_cast<int64_t>(j) * D + e)
+                               : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (mlj[u].x == -INFINITY) continue;  // empty or skipped partition
+      if (mlj[u].x > M) {
+        const float sc = dev::fast_exp2(M - mlj[u].x);  // 0 when M = -inf
+        W *= sc;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[e] *= sc;
+        M = mlj[u].x;
+      }
+      const float w = mlj[u].y * dev::fast_exp2(mlj[u].x - M);
+      W += w;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) acc[e] += w * oj[u][e];
+    }
   }
-  for (; j < n_parts; ++j) acc0 += w_s[j] * o[static_cast<int64_t>(j) * D];
-  const float acc = (acc0 + acc1) + (acc2 + acc3);
-  static_cast<T*>(a.out)[(static_cast<int64_t>(b) * a.num_q_heads + qh) * D +
-                         tid] = from_float<T>(ws > 0.f ? acc / ws : 0.f);
+  if (lane == 0) {
+    s_m[warp] = M;
+    s_w[warp] = W;
+  }
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) s_acc[warp][lane * kPer + e] = acc[e];
+  __syncthreads();
+  for (int d = threadIdx.x; d < D; d += kReduceWarps * 32) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kReduceWarps; ++w) mx = fmaxf(mx, s_m[w]);
+    float tw = 0.f, tv = 0.f;
+    if (mx != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kReduceWarps; ++w) {
+        const float sc =
+            s_m[w] == -INFINITY ? 0.f : dev::fast_exp2(s_m[w] - mx);
+        tw += s_w[w] * sc;
+        tv += s_acc[w][d] * sc;
+      }
+    }
+    static_cast<T*>(a.out)[(static_cast<int64_t>(b) * a.num_q_heads + qh) *
+                               D + d] = from_float<T>(tw > 0.f ? tv / tw : 0.f);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -692,7 +731,7 @@ int resolve_partition(const pa_decode_desc* d, int max_ctx) {
   if (d->partition_size > 0) return d->partition_size;
   const int64_t pairs = static_cast<int64_t>(d->num_seqs) * d->num_kv_heads;
   const int64_t target = 3LL * device_sm_count();
-  int ps = 512;
+  int ps = 1024;
   while (ps > 2 * d->block_size && ps > 64 &&
          pairs * ((max_ctx + ps - 1) / ps) < target)
     ps /= 2;
@@ -784,18 +823,34 @@ pa_status launch(const pa_decode_desc* d, DecodeArgs& a, const CUtensorMap& km,
                   cudaGetErrorString(e));
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
-  dim3 grid(a.max_parts, d->num_kv_heads, d->num_seqs);
-  kern<<<grid, kThreads, smem, stream>>>(km, vm, a);
+  // Both kernels are launched with programmatic stream serialization: each
+  // may start while its predecessor drains and waits (griddepcontrol.wait)
+  // before touching memory the predecessor writes.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.max_parts, d->num_kv_heads, d->num_seqs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, km, vm, a);
   count_launch();
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return fail(PA_ERR_CUDA, "pa_decode: decode launch failed: %s",
                 cudaGetErrorString(e));
   if (a.max_parts > 1) {
-    reduce_kernel<T, D><<<dim3(d->num_q_heads, d->num_seqs), D,
-                          a.max_parts * sizeof(float), stream>>>(a, BS);
+    cudaLaunchConfig_t rcfg = {};
+    rcfg.gridDim = dim3(d->num_q_heads, d->num_seqs);
+    rcfg.blockDim = dim3(kReduceWarps * 32);
+    rcfg.dynamicSmemBytes = 0;
+    rcfg.stream = stream;
+    rcfg.attrs = attr;
+    rcfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&rcfg, reduce_kernel<T, D>, a, BS);
     count_launch();
-    e = cudaGetLastError();
     if (e != cudaSuccess)
       return fail(PA_ERR_CUDA, "pa_decode: reduce launch failed: %s",
                   cudaGetErrorString(e));

@@ -95,6 +95,18 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// ---- programmatic dependent launch --------------------------------------------
+// Let the next kernel in the stream (if launched with programmatic stream
+// serialization) start its prologue now.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Block until the kernels this grid depends on have completed and their
+// memory is visible (returns at once for a normally launched grid).
+__device__ __forceinline__ void pdl_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---- named barrier among a subset of warps ----------------------------------
 __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
