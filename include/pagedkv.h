@@ -66,6 +66,14 @@ typedef enum { PA_F16 = 0, PA_BF16 = 1 } pa_dtype;
  *                      both QK^T and PV, fp32 accumulation. */
 typedef enum { PA_KERNEL_AUTO = 0, PA_KERNEL_SIMT = 1, PA_KERNEL_MMA = 2 } pa_kernel;
 
+/* How the partitions of a split sequence are combined.  Both give the same
+ * result (out = sum_j w_j o_j / sum_j w_j with w_j = l_j exp(m_j - max m)).
+ *   PA_REDUCE_AUTO    -- up to 16 partitions per sequence: the partition
+ *                        CTA that finishes last combines them inside the
+ *                        decode kernel; more: the separate reduce kernel.
+ *   PA_REDUCE_KERNEL  -- always a second, separate reduce kernel. */
+typedef enum { PA_REDUCE_AUTO = 0, PA_REDUCE_KERNEL = 1 } pa_reduce;
+
 /* Shape of one decode call.
  *   num_q_heads must be a multiple of num_kv_heads; G = num_q_heads /
  *   num_kv_heads <= 8.  Query head h reads KV head h / G (consecutive
@@ -90,6 +98,7 @@ typedef struct {
   int partition_size;
   int max_context_len;
   pa_kernel kernel;
+  pa_reduce reduce;
 } pa_decode_desc;
 
 /* Library version string, and the text of a status code. */
@@ -118,8 +127,11 @@ const char* pa_last_error(void);
  *                 entries past a sequence's last block are ignored
  *   context_lens  [num_seqs] int32, tokens per sequence, the newest included
  *   workspace     pa_decode_workspace_bytes(desc) bytes of device memory the
- *                 caller owns (may be NULL when that size is 0); its contents
- *                 need no initialisation and are scratch after the call.
+ *                 caller owns, 16-byte aligned (may be NULL when that size is
+ *                 0): partition partials and per-(sequence, KV head)
+ *                 counters the call resets on its stream.  Its contents need
+ *                 no initialisation and are scratch after the call; calls
+ *                 that share a workspace must not overlap on the device.
  * Computation: fp32 scores, fp32 online softmax, fp32 accumulation; the
  * output is rounded once to dtype.
  * Errors: PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED / PA_ERR_WORKSPACE before

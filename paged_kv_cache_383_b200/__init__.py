@@ -35,6 +35,7 @@ __all__ = [
 
 _KERNELS = {"auto": PA_KERNEL_AUTO, "mma": PA_KERNEL_MMA,
             "simt": PA_KERNEL_SIMT}
+_REDUCES = {"auto": _lib.PA_REDUCE_AUTO, "kernel": _lib.PA_REDUCE_KERNEL}
 
 
 def library_path() -> str:
@@ -78,7 +79,8 @@ def _stream(stream) -> int:
 
 
 def make_desc(q, k_cache, block_tables, *, partition_size: int = 0,
-              max_context_len: int = 0, kernel: str = "auto") -> pa_decode_desc:
+              max_context_len: int = 0, kernel: str = "auto",
+              reduce: str = "auto") -> pa_decode_desc:
     """Decode descriptor from tensor shapes."""
     num_seqs, num_q_heads, head_dim = q.shape
     num_blocks, num_kv_heads, block_size, hd2 = k_cache.shape
@@ -91,7 +93,8 @@ def make_desc(q, k_cache, block_tables, *, partition_size: int = 0,
         head_dim=head_dim, block_size=block_size,
         max_blocks_per_seq=block_tables.shape[1], num_blocks=num_blocks,
         dtype=_dtype_code(q), partition_size=partition_size,
-        max_context_len=max_context_len, kernel=_KERNELS[kernel])
+        max_context_len=max_context_len, kernel=_KERNELS[kernel],
+        reduce=_REDUCES[reduce])
 
 
 def pa_decode_workspace_bytes(desc: pa_decode_desc) -> int:
@@ -108,8 +111,8 @@ def pa_decode_partition_size(desc: pa_decode_desc) -> int:
 def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens,
               scale: float, *, partition_size: int = 0,
               max_context_len: int = 0, kernel: str = "auto",
-              workspace=None, dev_err=None, stream=None,
-              desc: pa_decode_desc | None = None):
+              reduce: str = "auto", workspace=None, dev_err=None,
+              stream=None, desc: pa_decode_desc | None = None):
     """out[b, h] = softmax(scale * K_b q[b, h]) V_b over each sequence's
     paged K/V.  ``workspace`` (uint8 CUDA tensor) is allocated with torch when
     the call needs one and none is given.  Returns ``out``."""
@@ -118,7 +121,8 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens,
     if desc is None:
         desc = make_desc(q, k_cache, block_tables,
                          partition_size=partition_size,
-                         max_context_len=max_context_len, kernel=kernel)
+                         max_context_len=max_context_len, kernel=kernel,
+                         reduce=reduce)
     dt = q.dtype
     for name, t in (("out", out), ("k_cache", k_cache), ("v_cache", v_cache)):
         if t.dtype != dt:

@@ -26,6 +26,10 @@ PA_ERR_DEVICE_TIMEOUT = 7
 PA_F16 = 0
 PA_BF16 = 1
 
+# pa_reduce
+PA_REDUCE_AUTO = 0
+PA_REDUCE_KERNEL = 1
+
 # pa_kernel
 PA_KERNEL_AUTO = 0
 PA_KERNEL_SIMT = 1
@@ -45,6 +49,7 @@ class pa_decode_desc(ctypes.Structure):
         ("partition_size", ctypes.c_int),
         ("max_context_len", ctypes.c_int),
         ("kernel", ctypes.c_int),
+        ("reduce", ctypes.c_int),
     ]
 
 

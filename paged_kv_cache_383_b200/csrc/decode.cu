@@ -54,6 +54,7 @@ constexpr int kThreads = (kConsumers + 1) * 32;    // + one producer warp
 constexpr int kMaxGroup = 8;                       // query heads per KV head
 constexpr int kMaxPartition = 8192;
 constexpr int kMaxParts = 16384;                   // partitions per sequence
+constexpr int kFusedMaxParts = 16;  // up to this many: combine in the decode
 
 struct DecodeArgs {
   void* out;
@@ -62,6 +63,8 @@ struct DecodeArgs {
   const int32_t* context_lens;
   float* ws_o;   // [num_seqs, num_q_heads, max_parts, head_dim]
   float* ws_ml;  // [num_seqs, num_q_heads, max_parts, 2] = (max, sum), log2 units
+  int* counters; // [num_seqs, num_kv_heads] finished partitions (fused mode)
+  int fused;     // 1: the last partition CTA combines; 0: the reduce kernel
   int32_t* dev_err;
   float scale_log2;  // scale * log2(e): scores are kept in base-2 units
   int num_q_heads;
@@ -81,6 +84,11 @@ struct DecodeArgs {
 // the same logical chunk hit eight different bank groups.
 template <int BS, int D, int S>
 struct Geometry {
+  // Consumer warp w takes pages w, w+4, ... and page i sits in stage i % S.
+  // With S a multiple of the consumer count a warp owns its stages, so it
+  // waits on every use of them in order and a parity wait can never run two
+  // phases ahead (a parity test cannot tell phase m from m-2).
+  static_assert(S % kConsumers == 0, "stages must be a multiple of consumers");
   static constexpr int kBoxes = D / 64;
   static constexpr int kBoxBytes = BS * 128;
   static constexpr int kPageBytes = kBoxes * kBoxBytes;
@@ -153,6 +161,72 @@ __device__ __forceinline__ float warp_max_xor(float v, int lo_mask,
 }
 
 // ---------------------------------------------------------------------------
+// Fused combine of one (sequence, KV head)'s partitions, run by threads
+// [t, ...) step nt of the partition CTA that finished last:
+//   out = sum_j w_j o_j / sum_j w_j,  w_j = l_j 2^(m_j - M),  M = max_j m_j.
+// Thread item = (query head g, 16-lane slice of head_dim); four partitions
+// are loaded before they are folded.
+template <typename T, int D>
+__device__ __forceinline__ void combine_partials(const DecodeArgs& a, int b,
+                                                 int kvh, int n_parts, int t,
+                                                 int nt) {
+  constexpr int kDT = D / 16;  // dims per thread: 8 or 4
+  const int G = a.group;
+  const float2* ml2 = reinterpret_cast<const float2*>(a.ws_ml);
+  for (int item = t; item < G * 16; item += nt) {
+    const int g = item >> 4;
+    const int d0 = (item & 15) * kDT;
+    const int64_t row0 =
+        (static_cast<int64_t>(b) * a.num_q_heads + kvh * G + g) * a.max_parts;
+    float M = -INFINITY, W = 0.f;
+    float acc[kDT];
+#pragma unroll
+    for (int e = 0; e < kDT; ++e) acc[e] = 0.f;
+    for (int j0 = 0; j0 < n_parts; j0 += 4) {
+      float2 mlj[4];
+      float oj[4][kDT];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + u;
+        mlj[u] = j < n_parts ? __ldcg(ml2 + row0 + j)
+                             : make_float2(-INFINITY, 0.f);
+        const float4* src =
+            reinterpret_cast<const float4*>(a.ws_o + (row0 + j) * D + d0);
+#pragma unroll
+        for (int v = 0; v < kDT / 4; ++v) {
+          const float4 x = j < n_parts ? __ldcg(src + v)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+          oj[u][4 * v] = x.x;
+          oj[u][4 * v + 1] = x.y;
+          oj[u][4 * v + 2] = x.z;
+          oj[u][4 * v + 3] = x.w;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (mlj[u].x == -INFINITY) continue;  // empty or skipped partition
+        if (mlj[u].x > M) {
+          const float sc = dev::fast_exp2(M - mlj[u].x);  // 0 when M = -inf
+          W *= sc;
+#pragma unroll
+          for (int e = 0; e < kDT; ++e) acc[e] *= sc;
+          M = mlj[u].x;
+        }
+        const float w = mlj[u].y * dev::fast_exp2(mlj[u].x - M);
+        W += w;
+#pragma unroll
+        for (int e = 0; e < kDT; ++e) acc[e] += w * oj[u][e];
+      }
+    }
+    T* dst = static_cast<T*>(a.out) +
+             (static_cast<int64_t>(b) * a.num_q_heads + kvh * G + g) * D + d0;
+#pragma unroll
+    for (int e = 0; e < kDT; ++e)
+      dst[e] = from_float<T>(W > 0.f ? acc[e] / W : 0.f);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // The decode kernel.
 template <typename T, int BS, int D, int S, bool kMma>
 __global__ void __launch_bounds__(kThreads)
@@ -214,14 +288,29 @@ __global__ void __launch_bounds__(kThreads)
   // Everything above reads only host-written inputs; the K/V pages and the
   // outputs may belong to the previous kernel in the stream.
   dev::pdl_wait();
+  __shared__ int s_last;
   if (bad) {
     if (tid == 0) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
-    if (n_parts > 1 && tid < G) {  // mark the partition empty for the reduce
-      const int64_t row =
-          (static_cast<int64_t>(b) * a.num_q_heads + kvh * G + tid) *
-              a.max_parts + part;
-      a.ws_ml[2 * row] = -INFINITY;
-      a.ws_ml[2 * row + 1] = 0.f;
+    if (n_parts > 1) {
+      if (tid < G) {  // mark the partition empty for the combine
+        const int64_t row =
+            (static_cast<int64_t>(b) * a.num_q_heads + kvh * G + tid) *
+                a.max_parts + part;
+        a.ws_ml[2 * row] = -INFINITY;
+        a.ws_ml[2 * row + 1] = 0.f;
+      }
+      if (a.fused) {  // still counts as finished: the others may be fine
+        __threadfence();
+        __syncthreads();
+        if (tid == 0)
+          s_last = atomicAdd(a.counters + b * a.num_kv_heads + kvh, 1) ==
+                   n_parts - 1;
+        __syncthreads();
+        if (s_last) {
+          __threadfence();
+          combine_partials<T, D>(a, b, kvh, n_parts, tid, kThreads);
+        }
+      }
     }
     return;
   }
@@ -585,25 +674,43 @@ __global__ void __launch_bounds__(kThreads)
       }
     }
   }
+  if (split && a.fused) {
+    // Publish this partition; the partition CTA that finishes last combines
+    // all of them (fence + ticket: nobody waits for anybody).
+    __threadfence();
+    dev::named_barrier(1, kConsumers * 32);
+    if (ctid == 0)
+      s_last = atomicAdd(a.counters + b * a.num_kv_heads + kvh, 1) ==
+               n_parts - 1;
+    dev::named_barrier(1, kConsumers * 32);
+    if (s_last) {
+      __threadfence();
+      combine_partials<T, D>(a, b, kvh, n_parts, ctid, kConsumers * 32);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
 // Partition reduce: out = sum_j w_j o_j / sum_j w_j, w_j = l_j 2^(m_j - M),
-// M = max_j m_j (all in base-2 units).  One CTA per (query head, sequence);
-// warp w folds partitions w, w+4, ... with a running max (one pass, four
-// partitions in flight per warp), then the four warp states are merged.
-constexpr int kReduceWarps = 4;
+// M = max_j m_j (all in base-2 units).
+// One CTA per (KV head, sequence): warp w serves query head w % G and folds
+// partitions j = w / G, w / G + groups, ... with a running max, six to eight
+// partitions in flight per warp; the part-groups of a head are merged through
+// shared memory.  Few, fat CTAs: the cost of this kernel was the number of
+// CTAs the block scheduler had to start, not bytes.
+constexpr int kReduceMaxWarps = 32;
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kReduceWarps * 32)
-    reduce_kernel(const DecodeArgs a, int block_size) {
+__global__ void __launch_bounds__(kReduceMaxWarps * 32)
+    reduce_kernel(const DecodeArgs a, int block_size, int groups) {
   constexpr int kPer = D / 32;  // dims per lane
-  __shared__ float s_m[kReduceWarps], s_w[kReduceWarps];
-  __shared__ float s_acc[kReduceWarps][D];
-  const int qh = blockIdx.x;
+  __shared__ float s_m[kReduceMaxWarps], s_w[kReduceMaxWarps];
+  __shared__ float s_acc[kReduceMaxWarps][D];
+  const int kvh = blockIdx.x;
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int G = a.group;
   dev::pdl_trigger();
   const int ctx = a.context_lens[b];
   if (ctx < 0 || ctx > a.max_blocks_per_seq * block_size ||
@@ -611,45 +718,48 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
     return;  // flagged by the decode kernel
   const int n_parts = ctx > 0 ? (ctx + a.partition_size - 1) / a.partition_size
                               : 1;
-  if (n_parts <= 1) return;  // the decode kernel wrote this row itself
+  if (n_parts <= 1) return;  // the decode kernel wrote these rows itself
   dev::pdl_wait();           // partials of the decode kernel are visible
 
-  const int64_t row0 =
-      (static_cast<int64_t>(b) * a.num_q_heads + qh) * a.max_parts;
-  const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row0;
-  const float* o = a.ws_o + row0 * D + lane * kPer;
+  const int g = warp % G;
+  const int grp = warp / G;
   float M = -INFINITY, W = 0.f;
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-
-  constexpr int kBatch = 4;
-  for (int j0 = warp; j0 < n_parts; j0 += kBatch * kReduceWarps) {
-    float2 mlj[kBatch];
-    float oj[kBatch][kPer];
+  if (grp < groups) {
+    const int64_t row0 =
+        (static_cast<int64_t>(b) * a.num_q_heads + kvh * G + g) * a.max_parts;
+    const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row0;
+    const float* o = a.ws_o + row0 * D + lane * kPer;
+    constexpr int kBatch = kPer == 4 ? 6 : 8;  // partitions in flight (no spills)
+    for (int j0 = grp; j0 < n_parts; j0 += kBatch * groups) {
+      float2 mlj[kBatch];
+      float oj[kBatch][kPer];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int j = j0 + u * kReduceWarps;
-      mlj[u] = j < n_parts ? __ldcg(ml + j) : make_float2(-INFINITY, 0.f);
+      for (int u = 0; u < kBatch; ++u) {
+        const int j = j0 + u * groups;
+        mlj[u] = j < n_parts ? __ldcg(ml + j) : make_float2(-INFINITY, 0.f);
 #pragma unroll
-      for (int e = 0; e < kPer; ++e)
-        oj[u][e] = j < n_parts ? __ldcg(o + static_cast<int64_t>(j) * D + e)
-                               : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      if (mlj[u].x == -INFINITY) continue;  // empty or skipped partition
-      if (mlj[u].x > M) {
-        const float sc = dev::fast_exp2(M - mlj[u].x);  // 0 when M = -inf
-        W *= sc;
-#pragma unroll
-        for (int e = 0; e < kPer; ++e) acc[e] *= sc;
-        M = mlj[u].x;
+        for (int e = 0; e < kPer; ++e)
+          oj[u][e] =
+              j < n_parts ? __ldcg(o + static_cast<int64_t>(j) * D + e) : 0.f;
       }
-      const float w = mlj[u].y * dev::fast_exp2(mlj[u].x - M);
-      W += w;
 #pragma unroll
-      for (int e = 0; e < kPer; ++e) acc[e] += w * oj[u][e];
+      for (int u = 0; u < kBatch; ++u) {
+        if (mlj[u].x == -INFINITY) continue;  // empty or skipped partition
+        if (mlj[u].x > M) {
+          const float sc = dev::fast_exp2(M - mlj[u].x);  // 0 when M = -inf
+          W *= sc;
+#pragma unroll
+          for (int e = 0; e < kPer; ++e) acc[e] *= sc;
+          M = mlj[u].x;
+        }
+        const float w = mlj[u].y * dev::fast_exp2(mlj[u].x - M);
+        W += w;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[e] += w * oj[u][e];
+      }
     }
   }
   if (lane == 0) {
@@ -659,22 +769,22 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
 #pragma unroll
   for (int e = 0; e < kPer; ++e) s_acc[warp][lane * kPer + e] = acc[e];
   __syncthreads();
-  for (int d = threadIdx.x; d < D; d += kReduceWarps * 32) {
+  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+    const int h = idx / D, d = idx - (idx / D) * D;
     float mx = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kReduceWarps; ++w) mx = fmaxf(mx, s_m[w]);
+    for (int q = 0; q < groups; ++q) mx = fmaxf(mx, s_m[q * G + h]);
     float tw = 0.f, tv = 0.f;
     if (mx != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kReduceWarps; ++w) {
-        const float sc =
-            s_m[w] == -INFINITY ? 0.f : dev::fast_exp2(s_m[w] - mx);
-        tw += s_w[w] * sc;
-        tv += s_acc[w][d] * sc;
+      for (int q = 0; q < groups; ++q) {
+        const float mq = s_m[q * G + h];
+        const float sc = mq == -INFINITY ? 0.f : dev::fast_exp2(mq - mx);
+        tw += s_w[q * G + h] * sc;
+        tv += s_acc[q * G + h][d] * sc;
       }
     }
-    static_cast<T*>(a.out)[(static_cast<int64_t>(b) * a.num_q_heads + qh) *
-                               D + d] = from_float<T>(tw > 0.f ? tv / tw : 0.f);
+    static_cast<T*>(a.out)[(static_cast<int64_t>(b) * a.num_q_heads +
+                            kvh * G + h) * D + d] =
+        from_float<T>(tw > 0.f ? tv / tw : 0.f);
   }
 }
 
@@ -722,9 +832,13 @@ bool encode_cache_map(CUtensorMap* map, const void* base, uint64_t rows,
   return r == CUDA_SUCCESS;
 }
 
+#ifndef PAGEDKV_RING_BYTES
+#define PAGEDKV_RING_BYTES 65536
+#endif
 constexpr int stages_for(int bs, int d) {
-  // 64 KB ring per CTA: three CTAs fit one SM's shared memory.
-  return 65536 / (2 * 2 * bs * d);
+  // 64 KB ring per CTA: three CTAs fit one SM's shared memory.  Whole
+  // multiples of the consumer count (see Geometry).
+  return (PAGEDKV_RING_BYTES / (2 * 2 * bs * d)) / kConsumers * kConsumers;
 }
 
 int resolve_partition(const pa_decode_desc* d, int max_ctx) {
@@ -771,6 +885,9 @@ pa_status check_desc(const pa_decode_desc* d) {
   if (d->dtype != PA_F16 && d->dtype != PA_BF16)
     return fail(PA_ERR_INVALID_ARG, "pa_decode: dtype %d",
                 static_cast<int>(d->dtype));
+  if (d->reduce != PA_REDUCE_AUTO && d->reduce != PA_REDUCE_KERNEL)
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: reduce %d",
+                static_cast<int>(d->reduce));
   if (d->kernel != PA_KERNEL_AUTO && d->kernel != PA_KERNEL_SIMT &&
       d->kernel != PA_KERNEL_MMA)
     return fail(PA_ERR_INVALID_ARG, "pa_decode: kernel %d",
@@ -800,8 +917,18 @@ size_t workspace_bytes(const pa_decode_desc* d) {
   const int ps = resolve_partition(d, max_ctx);
   const int64_t parts = max_ctx > 0 ? (max_ctx + ps - 1) / ps : 1;
   if (parts <= 1) return 0;
-  return static_cast<size_t>(d->num_seqs) * d->num_q_heads * parts *
-         (d->head_dim + 2) * sizeof(float);
+  const size_t partials = static_cast<size_t>(d->num_seqs) * d->num_q_heads *
+                          parts * (d->head_dim + 2) * sizeof(float);
+  const size_t counters =
+      (static_cast<size_t>(d->num_seqs) * d->num_kv_heads * sizeof(int) + 15) &
+      ~size_t(15);
+  return partials + counters;
+}
+
+// Combine partitions inside the decode kernel (few partitions) or with the
+// separate reduce kernel.
+bool use_fused(const pa_decode_desc* d, int parts) {
+  return d->reduce == PA_REDUCE_AUTO && parts <= kFusedMaxParts;
 }
 
 template <typename T, int BS, int D, bool kMma>
@@ -829,6 +956,15 @@ pa_status launch(const pa_decode_desc* d, DecodeArgs& a, const CUtensorMap& km,
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  if (a.max_parts > 1 && a.fused) {
+    cudaError_t me = cudaMemsetAsync(
+        a.counters, 0,
+        static_cast<size_t>(d->num_seqs) * d->num_kv_heads * sizeof(int),
+        stream);
+    if (me != cudaSuccess)
+      return fail(PA_ERR_CUDA, "pa_decode: counter reset failed: %s",
+                  cudaGetErrorString(me));
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.max_parts, d->num_kv_heads, d->num_seqs);
   cfg.blockDim = dim3(kThreads);
@@ -841,15 +977,20 @@ pa_status launch(const pa_decode_desc* d, DecodeArgs& a, const CUtensorMap& km,
   if (e != cudaSuccess)
     return fail(PA_ERR_CUDA, "pa_decode: decode launch failed: %s",
                 cudaGetErrorString(e));
-  if (a.max_parts > 1) {
+  if (a.max_parts > 1 && !a.fused) {
+    // Part-groups per head: about 16 partitions per warp, at most 32 warps.
+    const int G = a.group;
+    int groups = (a.max_parts + 15) / 16;
+    if (groups > kReduceMaxWarps / G) groups = kReduceMaxWarps / G;
+    if (groups < 1) groups = 1;
     cudaLaunchConfig_t rcfg = {};
-    rcfg.gridDim = dim3(d->num_q_heads, d->num_seqs);
-    rcfg.blockDim = dim3(kReduceWarps * 32);
+    rcfg.gridDim = dim3(d->num_kv_heads, d->num_seqs);
+    rcfg.blockDim = dim3(32 * G * groups);
     rcfg.dynamicSmemBytes = 0;
     rcfg.stream = stream;
     rcfg.attrs = attr;
     rcfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&rcfg, reduce_kernel<T, D>, a, BS);
+    e = cudaLaunchKernelEx(&rcfg, reduce_kernel<T, D>, a, BS, groups);
     count_launch();
     if (e != cudaSuccess)
       return fail(PA_ERR_CUDA, "pa_decode: reduce launch failed: %s",
@@ -941,6 +1082,12 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache,
                            static_cast<size_t>(desc->num_seqs) *
                                desc->num_q_heads * parts * desc->head_dim
                      : nullptr;
+  a.counters = need > 0 ? reinterpret_cast<int*>(
+                               a.ws_ml + 2 * static_cast<size_t>(
+                                                 desc->num_seqs) *
+                                             desc->num_q_heads * parts)
+                         : nullptr;
+  a.fused = pagedkv::use_fused(desc, parts) ? 1 : 0;
   a.dev_err = dev_err;
   a.scale_log2 = scale * pagedkv::kLog2e;
   a.num_q_heads = desc->num_q_heads;

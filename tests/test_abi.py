@@ -51,6 +51,7 @@ def _desc(**kw):
     (dict(partition_size=24), 1),
     (dict(dtype=5), 1),
     (dict(kernel=9), 1),
+    (dict(reduce=4), 1),
     (dict(num_seqs=-1), 1),
 ])
 def test_decode_rejects_bad_descriptors(pkv, kw, status):
@@ -88,7 +89,8 @@ def test_decode_needs_workspace_for_split(pkv):
     d = _desc(partition_size=16, max_blocks_per_seq=8)
     need = lib.pa_decode_workspace_bytes(ctypes.byref(d))
     # 2 seqs x 8 q heads x 8 partitions x (128 + 2) floats
-    assert need == 2 * 8 * 8 * 130 * 4
+    # + 2 seqs x 2 kv heads int32 counters, rounded to 16 bytes
+    assert need == 2 * 8 * 8 * 130 * 4 + 16
     fake = 0x1000
     st = lib.pa_decode(fake, fake, fake, fake, fake, fake,
                        ctypes.c_float(1.0), ctypes.byref(d), None, 0, None,

@@ -22,7 +22,7 @@ pytestmark = pytest.mark.gpu
 
 
 def _run(pkv, inp, kernel="auto", partition_size=None, tables=None,
-         lens=None, dev_err=None):
+         lens=None, dev_err=None, reduce="auto"):
     w = inp.workload
     dev = inp.q.device
     bt = torch.from_numpy(inp.block_tables if tables is None else tables)
@@ -33,6 +33,7 @@ def _run(pkv, inp, kernel="auto", partition_size=None, tables=None,
     ps = w.partition_size if partition_size is None else partition_size
     pkv.pa_decode(out, inp.q, inp.k_cache, inp.v_cache, bt, cl,
                   w.softmax_scale, partition_size=ps, kernel=kernel,
+                  reduce=reduce,
                   max_context_len=int(inp.lengths.max()) if len(inp.lengths)
                   else 0, dev_err=dev_err)
     torch.cuda.synchronize()
@@ -82,14 +83,29 @@ def test_full_size_sampled(pkv, name):
     assert torch.isfinite(out.float()).all()
 
 
-def test_partition_size_invariance(pkv):
+@pytest.mark.parametrize("reduce", ["auto", "kernel"])
+def test_partition_size_invariance(pkv, reduce):
+    # 16-token partitions give up to 125 partitions per sequence (separate
+    # reduce kernel even in auto mode); 256 gives <= 8 (fused in auto mode).
     w = wl.WORKLOADS["llama3_70b_gqa8"].scaled(num_seqs=6, cap=2000)
     inp = wl.make_paged(w, device="cuda")
-    outs = {ps: _run(pkv, inp, partition_size=ps) for ps in (16, 64, 512, 0)}
+    outs = {ps: _run(pkv, inp, partition_size=ps, reduce=reduce)
+            for ps in (16, 64, 256, 512, 0)}
     for ps, out in outs.items():
-        _check_all(inp, out, f"partition {ps}")
+        _check_all(inp, out, f"partition {ps} / {reduce}")
     a, b = outs[16].float(), outs[512].float()
     assert (a - b).abs().max().item() <= 4e-3
+
+
+def test_fused_and_kernel_reduce_agree(pkv):
+    w = wl.WORKLOADS["long_context_split"].scaled(num_seqs=3, low=1500,
+                                                  high=4000)
+    inp = wl.make_paged(w, device="cuda")
+    fused = _run(pkv, inp, partition_size=512, reduce="auto")   # <= 8 parts
+    kern = _run(pkv, inp, partition_size=512, reduce="kernel")
+    _check_all(inp, fused, "fused")
+    _check_all(inp, kern, "kernel")
+    assert (fused.float() - kern.float()).abs().max().item() <= 2e-3
 
 
 def test_identity_vs_shuffled_tables(pkv):
@@ -173,8 +189,13 @@ def test_device_checks_flag_bad_inputs(pkv):
     lens[2] = 10_000                              # beyond the table
     _run(pkv, inp, lens=lens, dev_err=err)
     assert err.item() == 5
-    err.zero_()
-    tables = inp.block_tables.copy()
-    tables[0, 0] = -3
-    _run(pkv, inp, tables=tables, dev_err=err, partition_size=16)
-    assert err.item() == 5
+    for reduce in ("auto", "kernel"):   # split sequences, both combines
+        err.zero_()
+        tables = inp.block_tables.copy()
+        tables[0, 0] = -3
+        out = _run(pkv, inp, tables=tables, dev_err=err, partition_size=16,
+                   reduce=reduce)
+        assert err.item() == 5
+        for b in (1, 2):
+            check_decode(to_np(out[b]), ref[b], inp.q.dtype,
+                         f"split seq {b} / {reduce}")
