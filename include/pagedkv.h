@@ -152,6 +152,39 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache,
                     size_t workspace_bytes, int32_t* dev_err, void* stream);
 
 /* ------------------------------------------------------------------------
+ * pa_decode without a caller workspace.  (No counterpart in the pages: this
+ * is a convenience of this library, not part of the method.)
+ *
+ * For callers that cannot allocate device memory: for example a serving
+ * process that has handed nearly all of HBM to the KV-cache pool and allows
+ * no further device allocations while it decodes, or a host program that
+ * drives this library through the C ABI and has no device allocator of its
+ * own.  The call computes exactly what pa_decode computes, with the
+ * workspace taken from a fixed area of PA_NOALLOC_SCRATCH_BYTES inside the
+ * library (a file-scope device array: every GPU that loads the library keeps
+ * it until the process exits).  It allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
+ *   - A shape whose pa_decode_workspace_bytes() exceeds
+ *     PA_NOALLOC_SCRATCH_BYTES is rejected with PA_ERR_WORKSPACE and a
+ *     message naming both sizes (use a larger partition_size or pa_decode).
+ *   - The first call on a device looks up the area's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call uses the same area, which keeps the previous call's data;
+ *     what must start at zero (the per-sequence partition counters) is reset
+ *     on the call's stream.  Calls that overlap on the GPU (other streams,
+ *     other threads, the same device) race on the area and must be avoided.
+ * Arguments, layouts and errors are those of pa_decode.
+ * ---------------------------------------------------------------------- */
+#define PA_NOALLOC_SCRATCH_BYTES (32ull << 20) /* 32 MiB per device */
+
+pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* block_tables,
+                            const int32_t* context_lens, float scale,
+                            const pa_decode_desc* desc, int32_t* dev_err,
+                            void* stream);
+
+/* ------------------------------------------------------------------------
  * Write new tokens' K and V into their cache slots.
  *
  * Defines ([Taming the Tail] "How the Architecture Works"; [KV-cache

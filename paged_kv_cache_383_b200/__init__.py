@@ -26,7 +26,7 @@ from ._lib import (PA_BF16, PA_F16, PA_KERNEL_AUTO, PA_KERNEL_MMA,
                    pa_decode_desc)
 
 __all__ = [
-    "pa_decode", "pa_cache_write", "pa_copy_blocks",
+    "pa_decode", "pa_decode_noalloc", "pa_cache_write", "pa_copy_blocks",
     "pa_decode_workspace_bytes", "pa_decode_partition_size", "make_desc",
     "BlockManager", "PagedKVError", "NoFreeBlocksError", "library_path",
     "pa_launch_count",
@@ -141,6 +141,37 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens,
         ctypes.c_float(scale), ctypes.byref(desc), ws_ptr, ws_bytes,
         _dev(dev_err, "dev_err", torch.int32), _stream(stream))
     _lib.check(st, "pa_decode")
+    return out
+
+
+def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens,
+                      scale: float, *, partition_size: int = 0,
+                      max_context_len: int = 0, kernel: str = "auto",
+                      reduce: str = "auto", dev_err=None, stream=None,
+                      desc: pa_decode_desc | None = None):
+    """pa_decode for callers that cannot allocate device memory: the
+    workspace is the library's built-in scratch area
+    (PA_NOALLOC_SCRATCH_BYTES per device), so this wrapper allocates nothing
+    either.  Calls that overlap on one device race on that area.  Returns
+    ``out``."""
+    import torch
+    lib = _lib.load()
+    if desc is None:
+        desc = make_desc(q, k_cache, block_tables,
+                         partition_size=partition_size,
+                         max_context_len=max_context_len, kernel=kernel,
+                         reduce=reduce)
+    for name, t in (("out", out), ("k_cache", k_cache), ("v_cache", v_cache)):
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} != q dtype {q.dtype}")
+    st = lib.pa_decode_noalloc(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32),
+        ctypes.c_float(scale), ctypes.byref(desc),
+        _dev(dev_err, "dev_err", torch.int32), _stream(stream))
+    _lib.check(st, "pa_decode_noalloc")
     return out
 
 

@@ -22,6 +22,9 @@ PA_ERR_DEVICE_OOB = 5
 PA_ERR_WORKSPACE = 6
 PA_ERR_DEVICE_TIMEOUT = 7
 
+# bytes of the built-in scratch area behind pa_decode_noalloc
+PA_NOALLOC_SCRATCH_BYTES = 32 << 20
+
 # pa_dtype
 PA_F16 = 0
 PA_BF16 = 1
@@ -72,6 +75,8 @@ SIGNATURES = {
     "pa_decode": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
                         ctypes.POINTER(pa_decode_desc), _vp, ctypes.c_size_t,
                         _vp, _vp]),
+    "pa_decode_noalloc": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
+                                ctypes.POINTER(pa_decode_desc), _vp, _vp]),
     "pa_cache_write": (_st, [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int,
                              _int, _int, _vp, _vp]),
     "pa_copy_blocks": (_st, [_vp, _vp, _vp, _int, _int, _int, _int, _int, _int,

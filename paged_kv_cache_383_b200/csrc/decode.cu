@@ -45,6 +45,14 @@
 #include "pagedkv.h"
 #include "status.h"
 
+// Built-in scratch for pa_decode_noalloc: a fixed device array that lives in
+// this library's module on every GPU that loads it, for callers that cannot
+// allocate device memory.  In host code this name is only a stand-in, not a
+// device address: scratch_address() below asks the runtime for the address,
+// once per device.
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
 namespace pagedkv {
 namespace {
 
@@ -1010,12 +1018,59 @@ pa_status dispatch_shape(const pa_decode_desc* d, DecodeArgs& a,
                             : launch<T, 32, 64, kMma>(d, a, km, vm, st);
 }
 
+void* scratch_address(pa_status* st) {
+  constexpr int kMaxDevices = 64;
+  static void* addr[kMaxDevices] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *st = fail(PA_ERR_CUDA, "pa_decode_noalloc: no usable current device (%s)",
+               cudaGetErrorString(e));
+    return nullptr;
+  }
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, ::g_noalloc_scratch);
+    if (e != cudaSuccess || !p) {
+      *st = fail(PA_ERR_CUDA,
+                 "pa_decode_noalloc: cudaGetSymbolAddress of the built-in "
+                 "scratch failed: %s", cudaGetErrorString(e));
+      return nullptr;
+    }
+    addr[dev] = p;
+  }
+  *st = PA_OK;
+  return addr[dev];
+}
+
 }  // namespace
 }  // namespace pagedkv
 
 using pagedkv::fail;
 
 extern "C" {
+
+pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* block_tables,
+                            const int32_t* context_lens, float scale,
+                            const pa_decode_desc* desc, int32_t* dev_err,
+                            void* stream) {
+  pagedkv::clear_error();
+  pa_status st = pagedkv::check_desc(desc);
+  if (st != PA_OK) return st;
+  const size_t need = pagedkv::workspace_bytes(desc);
+  if (need > PA_NOALLOC_SCRATCH_BYTES)
+    return fail(PA_ERR_WORKSPACE,
+                "pa_decode_noalloc: this shape needs %zu bytes of scratch but "
+                "the built-in area holds %llu; use a larger partition_size, "
+                "fewer sequences, or pa_decode with a caller workspace", need,
+                static_cast<unsigned long long>(PA_NOALLOC_SCRATCH_BYTES));
+  void* scratch = pagedkv::scratch_address(&st);
+  if (st != PA_OK) return st;
+  return pa_decode(out, q, k_cache, v_cache, block_tables, context_lens,
+                   scale, desc, scratch, PA_NOALLOC_SCRATCH_BYTES, dev_err,
+                   stream);
+}
 
 size_t pa_decode_workspace_bytes(const pa_decode_desc* desc) {
   pagedkv::clear_error();
