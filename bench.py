@@ -204,21 +204,10 @@ def run_native(args, rank, world, local):
     if want_cpu:
         pool = start_oracle_pool()
 
-    inp = wl.make_paged(w, device=dev)
-    if inp.k_new is None:                   # every step writes a new token
-        g = torch.Generator(device=dev)
-        g.manual_seed(w.seed + 7)
-        shp = (w.num_seqs, w.num_kv_heads, w.head_dim)
-        inp.k_new = torch.randn(shp, generator=g, device=dev).to(inp.q.dtype)
-        inp.v_new = torch.randn(shp, generator=g, device=dev).to(inp.q.dtype)
-        pos = inp.lengths - 1
-        inp.new_slots = (inp.block_tables[np.arange(w.num_seqs),
-                                          pos // w.block_size]
-                         .astype(np.int64) * w.block_size
-                         + pos % w.block_size)
-    bt = torch.from_numpy(inp.block_tables).to(dev)
-    cl = torch.from_numpy(inp.lengths.astype(np.int32)).to(dev)
-    slots = torch.from_numpy(inp.new_slots).to(dev)
+    spec = setup_prefix(w, dev, pkv, flow, wl) if w.lengths == "prefix" \
+        else setup_paged(w, dev, wl)
+    inp = spec.inp
+    bt, cl, slots, pairs = spec.bt, spec.cl, spec.slots, spec.pairs
     out = torch.empty_like(inp.q)
     max_ctx = int(inp.lengths.max())
     desc = pkv.make_desc(inp.q, inp.k_cache, bt, partition_size=ps,
@@ -229,9 +218,15 @@ def run_native(args, rank, world, local):
     stream = torch.cuda.current_stream(dev)
     step_bytes = kv_bytes(inp.lengths, w)
 
+    def writes():
+        if pairs is not None:
+            pkv.pa_copy_blocks(inp.k_cache, inp.v_cache, pairs, dev_err=err,
+                               stream=stream)
+        pkv.pa_cache_write(inp.k_cache, inp.v_cache, spec.write_k,
+                           spec.write_v, slots, dev_err=err, stream=stream)
+
     def step():
-        pkv.pa_cache_write(inp.k_cache, inp.v_cache, inp.k_new, inp.v_new,
-                           slots, dev_err=err, stream=stream)
+        writes()
         pkv.pa_decode(out, inp.q, inp.k_cache, inp.v_cache, bt, cl,
                       w.softmax_scale, desc=desc, workspace=ws, dev_err=err,
                       stream=stream)
@@ -246,31 +241,35 @@ def run_native(args, rank, world, local):
         step()
     torch.cuda.synchronize()
 
-    n_ev = args.steps
-    ev_dec = [(torch.cuda.Event(enable_timing=True),
-               torch.cuda.Event(enable_timing=True)) for _ in range(n_ev)]
+    # Timed region: exactly K steps, events only at its two ends (an event
+    # between the kernels would break their programmatic-launch overlap).
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     launches0 = pkv.pa_launch_count()
     barrier(world)
     torch.cuda.synchronize()
     t0.record(stream)
-    for i in range(args.steps):
-        pkv.pa_cache_write(inp.k_cache, inp.v_cache, inp.k_new, inp.v_new,
-                           slots, dev_err=err, stream=stream)
-        ev_dec[i][0].record(stream)
-        pkv.pa_decode(out, inp.q, inp.k_cache, inp.v_cache, bt, cl,
-                      w.softmax_scale, desc=desc, workspace=ws, dev_err=err,
-                      stream=stream)
-        ev_dec[i][1].record(stream)
+    for _ in range(args.steps):
+        step()
     t1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     launches = pkv.pa_launch_count() - launches0
-    clk = clocks.stop()
     ms_local = t0.elapsed_time(t1)
     ms_total = max_over_ranks(ms_local, world)
-    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_dec]))
+    # The dominant kernel's launch duration: K back-to-back pa_decode calls on
+    # the same inputs, timed the same way on the same stream.
+    d0 = torch.cuda.Event(enable_timing=True)
+    d1 = torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for _ in range(args.steps):
+        pkv.pa_decode(out, inp.q, inp.k_cache, inp.v_cache, bt, cl,
+                      w.softmax_scale, desc=desc, workspace=ws, dev_err=err,
+                      stream=stream)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    dec_ms = max_over_ranks(d0.elapsed_time(d1), world) / args.steps
     if err.item() != 0:
         raise RuntimeError(f"device error flag {err.item()} during bench")
 
@@ -303,6 +302,7 @@ def run_native(args, rank, world, local):
             "partition_size": pkv.pa_decode_partition_size(desc),
             "kernel": args.kernel,
             "kv_bytes_per_step": step_bytes,
+            **spec.info,
             "l2": "inputs larger than L2 (no flush): "
                   f"{step_bytes / 1e9:.2f} GB of K/V read per step",
             "parallelism": f"{world} independent replicas" if world > 1
@@ -319,34 +319,173 @@ def run_native(args, rank, world, local):
             "frac_of_spec_8000": round(achieved / SPEC_HBM_GBS, 4),
             "traffic": profiled_traffic(w.name),
             "decode_ms": round(dec_ms, 5),
+            "decode_ms_how": "K back-to-back pa_decode calls on the step's "
+                             "inputs, CUDA events on the launch stream",
         },
         "gpu_launches": int(launches),
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_extras:
-        res["extras"] = extras(args, w, inp, dev, pkv)
+        res["extras"] = extras(args, w, inp, dev, pkv, bt, cl)
+        probe = res["extras"].get("read_probe_gbs")
+        if probe:
+            res["roofline"]["read_probe_gbs"] = probe
+            res["roofline"]["frac_of_read_probe"] = round(achieved / probe, 4)
     if not args.no_e2e:
-        res["e2e"] = run_e2e(args, w, inp, dev, pkv, flow, world, rank, ps)
-    if want_cpu:
+        if w.lengths == "prefix":
+            res["e2e"] = run_e2e_fixed(args, w, spec, dev, pkv, world, ps)
+        else:
+            res["e2e"] = run_e2e(args, w, inp, dev, pkv, flow, world, rank,
+                                 ps)
+    if want_cpu and w.lengths != "prefix":
         res["cpu_baseline"] = cpu_baseline(pool, inp, w, dev)
     if pool is not None:
         pool.close()
     return res
 
 
-def extras(args, w, inp, dev, pkv):
-    """Side measurements: the SIMT kernel on the same inputs, and a
-    read-only torch reduction over a 4 GB buffer (read bandwidth ref)."""
+class StepSpec:
+    """Device inputs of one step: the decode batch plus the writes that
+    precede it (new tokens' K/V and their slots, copy-on-write pairs)."""
+
+    def __init__(self, inp, bt, cl, write_k, write_v, slots, pairs, info):
+        self.inp, self.bt, self.cl = inp, bt, cl
+        self.write_k, self.write_v, self.slots = write_k, write_v, slots
+        self.pairs, self.info = pairs, info
+
+
+def setup_paged(w, dev, wl):
+    """Shuffled-pool batch; each step rewrites every sequence's newest token
+    (position L-1) through its slot, then decodes over all L tokens."""
     import torch
-    out = {}
+    inp = wl.make_paged(w, device=dev)
+    if inp.k_new is None:
+        g = torch.Generator(device=dev)
+        g.manual_seed(w.seed + 7)
+        shp = (w.num_seqs, w.num_kv_heads, w.head_dim)
+        inp.k_new = torch.randn(shp, generator=g, device=dev).to(inp.q.dtype)
+        inp.v_new = torch.randn(shp, generator=g, device=dev).to(inp.q.dtype)
+        pos = inp.lengths - 1
+        inp.new_slots = (inp.block_tables[np.arange(w.num_seqs),
+                                          pos // w.block_size]
+                         .astype(np.int64) * w.block_size
+                         + pos % w.block_size)
     bt = torch.from_numpy(inp.block_tables).to(dev)
     cl = torch.from_numpy(inp.lengths.astype(np.int32)).to(dev)
+    slots = torch.from_numpy(inp.new_slots).to(dev)
+    return StepSpec(inp, bt, cl, inp.k_new, inp.v_new, slots, None,
+                    {"step": "cache write of 1 token/seq + decode"})
+
+
+def setup_prefix(w, dev, pkv, flow, wl):
+    """Shared-prefix mix built through the block manager: sequence 0 takes
+    the prefix, the others fork from it (reference count = batch), then one
+    append per sequence gives the suffix slots and the copy-on-write pairs.
+    Each step copies the shared partial block for every writer but the last,
+    writes all suffix tokens, and decodes (idempotent: the same copies and
+    writes every step)."""
+    import torch
+    pin = wl.make_prefix(w, device=dev)
+    shape = (pin.num_blocks, w.num_kv_heads, w.block_size, w.head_dim)
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 1)
+    dt = wl.torch_dtype(w.dtype)
+    kc = torch.randn(shape, generator=g, device=dev).to(dt)
+    vc = torch.randn(shape, generator=g, device=dev).to(dt)
+    bm = pkv.BlockManager(pin.num_blocks, w.block_size,
+                          free_order=pin.free_order)
+    flow.shared_prefix_batch(bm, kc, vc, pin.prefix_k, pin.prefix_v,
+                             w.num_seqs)
+    ids = list(range(w.num_seqs))
+    slots, pairs = bm.append_batch(ids, pin.suffix_lens)
+    max_blocks = int(wl.blocks_needed(pin.lengths, w.block_size).max())
+    table, lens = bm.block_table(ids, max_blocks)
+    bm.close()
+    inp = wl.PagedInputs(w, pin.lengths, table, pin.num_blocks, pin.q, kc, vc)
+    unique = (w.prefix_len + int(pin.suffix_lens.sum())) * \
+        w.num_kv_heads * w.head_dim * 4
+    info = {"step": f"{len(pairs)} copy-on-write block copies + cache write "
+                    f"of {int(pin.suffix_lens.sum())} suffix tokens + decode",
+            "cow_pairs": int(len(pairs)),
+            "unique_kv_bytes_per_step": int(unique),
+            "note": "KV bytes are logical: the shared prefix is read once per "
+                    "sequence and stays L2-resident"}
+    return StepSpec(inp, torch.from_numpy(table).to(dev),
+                    torch.from_numpy(lens).to(dev), pin.suffix_k, pin.suffix_v,
+                    torch.from_numpy(slots).to(dev),
+                    torch.from_numpy(pairs).to(dev) if len(pairs) else None,
+                    info)
+
+
+def run_e2e_fixed(args, w, spec, dev, pkv, world, ps):
+    """End-to-end step of the shared-prefix mix through the public API: the
+    step's inputs (q, suffix K/V, slots, copy pairs, tables, lengths) go
+    host->device from pinned memory, then copies, writes and decode, then
+    the output comes back device->host; one sync per step."""
+    import torch
+    inp = spec.inp
+    host = {k: t.cpu().pin_memory() for k, t in (
+        ("q", inp.q), ("k", spec.write_k), ("v", spec.write_v),
+        ("slots", spec.slots), ("bt", spec.bt), ("cl", spec.cl))}
+    if spec.pairs is not None:
+        host["pairs"] = spec.pairs.cpu().pin_memory()
+    devt = {k: torch.empty_like(t, device=dev) for k, t in host.items()}
+    hout = torch.empty(inp.q.shape, dtype=inp.q.dtype).pin_memory()
+    dout = torch.empty_like(inp.q)
+    stream = torch.cuda.current_stream(dev)
+    max_ctx = int(inp.lengths.max())
+
+    def one():
+        for k in host:
+            devt[k].copy_(host[k], non_blocking=True)
+        if "pairs" in devt:
+            pkv.pa_copy_blocks(inp.k_cache, inp.v_cache, devt["pairs"])
+        pkv.pa_cache_write(inp.k_cache, inp.v_cache, devt["k"], devt["v"],
+                           devt["slots"])
+        pkv.pa_decode(dout, devt["q"], inp.k_cache, inp.v_cache, devt["bt"],
+                      devt["cl"], w.softmax_scale, partition_size=ps,
+                      max_context_len=max_ctx)
+        hout.copy_(dout, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(args.warmup):
+        one()
+    barrier(world)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(a.elapsed_time(b), world)
+    return {"value": round(world * args.steps * kv_bytes(inp.lengths, w) /
+                           (ms * 1e-3) / 1e9, 2),
+            "unit": "GB/s",
+            "h2d_bytes_per_step": int(sum(t.nbytes for t in host.values())),
+            "d2h_bytes_per_step": int(hout.nbytes),
+            "ms_per_step": round(ms / args.steps, 4),
+            "includes": "pinned H2D of the step's inputs, copy-on-write "
+                        "copies, cache write, decode, D2H of the output, one "
+                        "sync per step"}
+
+
+def extras(args, w, inp, dev, pkv, bt, cl):
+    """Side measurements on the same inputs: the SIMT kernel, a partition
+    size sweep, the separate reduce kernel, and the read bandwidth of the
+    library's streaming read probe over a 4 GiB buffer (the achievable read
+    roofline) beside a torch reduction."""
+    import torch
+    out = {}
     o = torch.empty_like(inp.q)
     max_ctx = int(inp.lengths.max())
 
-    def time_decode(kernel, ps):
+    def time_decode(kernel, ps, reduce="auto"):
         desc = pkv.make_desc(inp.q, inp.k_cache, bt, partition_size=ps,
-                             max_context_len=max_ctx, kernel=kernel)
+                             max_context_len=max_ctx, kernel=kernel,
+                             reduce=reduce)
         ws = torch.empty(max(pkv.pa_decode_workspace_bytes(desc), 16),
                          dtype=torch.uint8, device=dev)
         for _ in range(3):
@@ -365,9 +504,23 @@ def extras(args, w, inp, dev, pkv):
 
     out["decode_gbs_simt"] = time_decode("simt", w.partition_size)
     out["decode_gbs_mma"] = time_decode("mma", w.partition_size)
+    out["decode_gbs_mma_reduce_kernel"] = time_decode("mma", w.partition_size,
+                                                      "kernel")
     for ps in (0, 256, 512, 1024, 2048):
         out[f"decode_gbs_mma_ps{ps}"] = time_decode("mma", ps)
     x = torch.empty(1 << 30, dtype=torch.float32, device=dev).fill_(1.0)
+    sink = torch.zeros(4, dtype=torch.int32, device=dev)
+    for _ in range(3):
+        pkv.pa_read_probe(x, sink)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(10):
+        pkv.pa_read_probe(x, sink)
+    b.record()
+    torch.cuda.synchronize()
+    out["read_probe_gbs"] = round(4 * (1 << 30) / (a.elapsed_time(b) / 10 *
+                                                    1e-3) / 1e9, 1)
     for _ in range(3):
         x.sum()
     a = torch.cuda.Event(enable_timing=True)

@@ -299,6 +299,14 @@ pa_status pa_bm_block_table(void* bm, const int64_t* seq_ids, int n,
  * all threads): lets a caller count the GPU work a timed region contained. */
 int64_t pa_launch_count(void);
 
+/* Measurement helper (no counterpart in the pages): read `bytes` (rounded
+ * down to 16) of the device buffer `buf` once with streaming 128-bit loads
+ * on `stream`; `sink` is a device word the kernel may write.  Timed on a
+ * buffer far larger than L2 it gives the read bandwidth the GPU sustains,
+ * the roofline the decode's bandwidth is compared with. */
+pa_status pa_read_probe(const void* buf, size_t bytes, uint32_t* sink,
+                        void* stream);
+
 /* Pool and sequence queries (-1 for an unknown handle / sequence / block). */
 int pa_bm_num_free(void* bm);
 int pa_bm_refcount(void* bm, int block);

@@ -29,7 +29,7 @@ __all__ = [
     "pa_decode", "pa_decode_noalloc", "pa_cache_write", "pa_copy_blocks",
     "pa_decode_workspace_bytes", "pa_decode_partition_size", "make_desc",
     "BlockManager", "PagedKVError", "NoFreeBlocksError", "library_path",
-    "pa_launch_count",
+    "pa_launch_count", "pa_read_probe",
     "PA_KERNEL_AUTO", "PA_KERNEL_MMA", "PA_KERNEL_SIMT",
 ]
 
@@ -40,6 +40,16 @@ _REDUCES = {"auto": _lib.PA_REDUCE_AUTO, "kernel": _lib.PA_REDUCE_KERNEL}
 
 def library_path() -> str:
     return _lib.LIB_PATH
+
+
+def pa_read_probe(buf, sink, stream=None):
+    """Read the whole CUDA tensor ``buf`` once with streaming loads (a
+    bandwidth measurement helper); ``sink`` is an int32 CUDA tensor."""
+    import torch
+    st = _lib.load().pa_read_probe(
+        _dev(buf, "buf"), buf.numel() * buf.element_size(),
+        _dev(sink, "sink", torch.int32), _stream(stream))
+    _lib.check(st, "pa_read_probe")
 
 
 def pa_launch_count() -> int:

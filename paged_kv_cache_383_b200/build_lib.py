@@ -15,7 +15,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libpagedkv.so")
 
-SOURCES = ["status.cpp", "block_manager.cpp", "cache_ops.cu", "decode.cu"]
+SOURCES = ["status.cpp", "block_manager.cpp", "cache_ops.cu", "decode.cu",
+           "probe.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -17,9 +17,12 @@
 namespace pagedkv {
 namespace {
 
-// Grid-stride over tokens; the threads of a CTA walk the token's K row and V
-// row (num_kv_heads * head_dim elements each) in 16-byte chunks.  Chunk c of
-// head h lands in the (block, h, offset) page of the cache.
+// Grid-stride over groups of kTok tokens; thread c moves 16-byte chunk c of
+// each token's K row and V row (num_kv_heads * head_dim elements each), all
+// kTok loads issued before the stores so each thread keeps several chunks in
+// flight.  Chunk c of head h lands in the (block, h, offset) page.
+constexpr int kTok = 4;
+
 __global__ void cache_write_kernel(uint4* __restrict__ k_cache,
                                    uint4* __restrict__ v_cache,
                                    const uint4* __restrict__ k,
@@ -30,27 +33,40 @@ __global__ void cache_write_kernel(uint4* __restrict__ k_cache,
                                    int64_t num_slots, int32_t* dev_err) {
   dev::pdl_trigger();  // a following decode may run its prologue now
   const int row_chunks = head_chunks * num_kv_heads;
-  for (int64_t t = blockIdx.x; t < num_tokens; t += gridDim.x) {
-    const int64_t slot = slot_mapping[t];
-    if (slot < 0) continue;  // padding token
-    if (slot >= num_slots) {
-      if (threadIdx.x == 0) dev::set_error(dev_err, PA_ERR_DEVICE_OOB);
-      continue;
+  for (int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTok; t0 < num_tokens;
+       t0 += static_cast<int64_t>(gridDim.x) * kTok) {
+    int64_t base[kTok];  // first chunk of (block, head 0, offset), -1 = skip
+#pragma unroll
+    for (int u = 0; u < kTok; ++u) {
+      base[u] = -1;
+      const int64_t t = t0 + u;
+      if (t < num_tokens) {
+        const int64_t slot = slot_mapping[t];
+        if (slot >= num_slots) {
+          if (threadIdx.x == 0) dev::set_error(dev_err, PA_ERR_DEVICE_OOB);
+        } else if (slot >= 0) {  // negative: padding token
+          const int64_t blk = slot / block_size;
+          const int64_t off = slot - blk * block_size;
+          base[u] = (blk * num_kv_heads * block_size + off) * head_chunks;
+        }
+      }
     }
-    const int64_t blk = slot / block_size;
-    const int64_t off = slot - blk * block_size;
     for (int c = threadIdx.x; c < 2 * row_chunks; c += blockDim.x) {
       const int which = c >= row_chunks;  // 0 = K, 1 = V
       const int cc = c - which * row_chunks;
       const int h = cc / head_chunks;
       const int hc = cc - h * head_chunks;
-      const int64_t dst =
-          ((blk * num_kv_heads + h) * block_size + off) * head_chunks + hc;
-      const int64_t src = t * row_chunks + cc;
-      if (which == 0)
-        k_cache[dst] = k[src];
-      else
-        v_cache[dst] = v[src];
+      const uint4* src = which ? v : k;
+      uint4* dst = which ? v_cache : k_cache;
+      const int64_t head_off =
+          static_cast<int64_t>(h) * block_size * head_chunks + hc;
+      uint4 val[kTok];
+#pragma unroll
+      for (int u = 0; u < kTok; ++u)
+        if (base[u] >= 0) val[u] = src[(t0 + u) * row_chunks + cc];
+#pragma unroll
+      for (int u = 0; u < kTok; ++u)
+        if (base[u] >= 0) dst[base[u] + head_off] = val[u];
     }
   }
 }
@@ -134,8 +150,8 @@ pa_status pa_cache_write(void* k_cache, void* v_cache, const void* k,
   const int head_chunks = head_dim * 2 / 16;
   const int row2 = 2 * num_kv_heads * head_chunks;  // chunks per token (K+V)
   const int threads = row2 >= 256 ? 256 : ((row2 + 31) / 32) * 32;
-  int64_t blocks = num_tokens;
-  const int64_t cap = static_cast<int64_t>(pagedkv::sm_count()) * 32;
+  int64_t blocks = (num_tokens + pagedkv::kTok - 1) / pagedkv::kTok;
+  const int64_t cap = static_cast<int64_t>(pagedkv::sm_count()) * 16;
   if (blocks > cap) blocks = cap;
   pagedkv::cache_write_kernel<<<static_cast<unsigned>(blocks), threads, 0,
                                 static_cast<cudaStream_t>(stream)>>>(

@@ -255,36 +255,42 @@ __global__ void __launch_bounds__(kThreads)
   const int lane = tid & 31;
 
   dev::pdl_trigger();  // the reduce may start its prologue early
-  const int ctx = a.context_lens[b];
-  if (ctx < 0 || ctx > a.max_blocks_per_seq * BS || ctx > a.max_context_len) {
-    if (part == 0 && kvh == 0 && tid == 0)
-      dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
-    return;
-  }
   const int PS = a.partition_size;
-  const int n_parts = ctx > 0 ? (ctx + PS - 1) / PS : 1;
-  if (part >= n_parts) return;
-  const int tok0 = part * PS;
-  const int n_tok = min(ctx - tok0, PS);  // 0 only when ctx == 0
-  const int n_pages = (n_tok + BS - 1) / BS;
-  const int page0 = tok0 / BS;
-  const int G = a.group;
-
+  const int pages_per_part = PS / BS;
+  const int page0 = part * pages_per_part;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Geo::kRingBytes);
   int32_t* bt_s = reinterpret_cast<int32_t*>(bars + 2 * S);
   const uint32_t ring = dev::smem_u32(smem);
   const uint32_t full0 = dev::smem_u32(bars);
   const uint32_t empty0 = full0 + S * 8;
 
-  // Stage this partition's slice of the block table; check every id.
-  int bad = 0;
+  // The context length and this partition's slice of the block table are
+  // fetched together: the slice is read as if the partition were full (clipped
+  // to the table row) so the two loads do not wait on each other; entries past
+  // the sequence's end are never used.
   const int32_t* bt_row =
       a.block_tables + static_cast<int64_t>(b) * a.max_blocks_per_seq + page0;
-  for (int i = tid; i < n_pages; i += kThreads) {
-    const int32_t p = bt_row[i];
-    bad |= (p < 0 || p >= a.num_blocks);
-    bt_s[i] = p;
+  const int row_left = a.max_blocks_per_seq - page0;
+  const int ctx = a.context_lens[b];
+  for (int i = tid; i < pages_per_part && i < row_left; i += kThreads)
+    bt_s[i] = bt_row[i];
+  if (ctx < 0 || ctx > a.max_blocks_per_seq * BS || ctx > a.max_context_len) {
+    if (part == 0 && kvh == 0 && tid == 0)
+      dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
+    return;
   }
+  const int n_parts = ctx > 0 ? (ctx + PS - 1) / PS : 1;
+  if (part >= n_parts) return;
+  const int tok0 = part * PS;
+  const int n_tok = min(ctx - tok0, PS);  // 0 only when ctx == 0
+  const int n_pages = (n_tok + BS - 1) / BS;
+  const int G = a.group;
+
+  // Check every block id the partition uses (each thread the entries it
+  // staged itself).
+  int bad = 0;
+  for (int i = tid; i < n_pages; i += kThreads)
+    bad |= (bt_s[i] < 0 || bt_s[i] >= a.num_blocks);
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       dev::mbar_init(full0 + s * 8, 1);
@@ -699,26 +705,39 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ---------------------------------------------------------------------------
+// Zero the per-(sequence, KV head) partition counters before a decode that
+// combines in place.  Launched with programmatic stream serialization: it
+// lets the decode launch at once, waits for the previous kernel (which may
+// still read the counters), zeroes them, and the decode's own wait then
+// covers both.
+__global__ void zero_counters_kernel(int* counters, int n) {
+  dev::pdl_trigger();
+  dev::pdl_wait();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += gridDim.x * blockDim.x)
+    counters[i] = 0;
+}
+
+// ---------------------------------------------------------------------------
 // Partition reduce: out = sum_j w_j o_j / sum_j w_j, w_j = l_j 2^(m_j - M),
 // M = max_j m_j (all in base-2 units).
-// One CTA per (KV head, sequence): warp w serves query head w % G and folds
-// partitions j = w / G, w / G + groups, ... with a running max, six to eight
-// partitions in flight per warp; the part-groups of a head are merged through
-// shared memory.  Few, fat CTAs: the cost of this kernel was the number of
-// CTAs the block scheduler had to start, not bytes.
-constexpr int kReduceMaxWarps = 32;
+// One CTA per (query head, sequence); warp w folds partitions w, w+8, ...
+// with a running max, six to eight partitions in flight per warp, and the
+// eight warp states are merged through shared memory.  Used when a sequence
+// has many partitions (the fused combine handles few), so the work per CTA
+// is long enough to pay for the launch.
+constexpr int kReduceWarps = 8;
 
 template <typename T, int D>
-__global__ void __launch_bounds__(kReduceMaxWarps * 32)
-    reduce_kernel(const DecodeArgs a, int block_size, int groups) {
+__global__ void __launch_bounds__(kReduceWarps * 32)
+    reduce_kernel(const DecodeArgs a, int block_size) {
   constexpr int kPer = D / 32;  // dims per lane
-  __shared__ float s_m[kReduceMaxWarps], s_w[kReduceMaxWarps];
-  __shared__ float s_acc[kReduceMaxWarps][D];
-  const int kvh = blockIdx.x;
+  __shared__ float s_m[kReduceWarps], s_w[kReduceWarps];
+  __shared__ float s_acc[kReduceWarps][D];
+  const int qh = blockIdx.x;
   const int b = blockIdx.y;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int G = a.group;
   dev::pdl_trigger();
   const int ctx = a.context_lens[b];
   if (ctx < 0 || ctx > a.max_blocks_per_seq * block_size ||
@@ -726,48 +745,44 @@ __global__ void __launch_bounds__(kReduceMaxWarps * 32)
     return;  // flagged by the decode kernel
   const int n_parts = ctx > 0 ? (ctx + a.partition_size - 1) / a.partition_size
                               : 1;
-  if (n_parts <= 1) return;  // the decode kernel wrote these rows itself
+  if (n_parts <= 1) return;  // the decode kernel wrote this row itself
   dev::pdl_wait();           // partials of the decode kernel are visible
 
-  const int g = warp % G;
-  const int grp = warp / G;
+  const int64_t row0 =
+      (static_cast<int64_t>(b) * a.num_q_heads + qh) * a.max_parts;
+  const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row0;
+  const float* o = a.ws_o + row0 * D + lane * kPer;
   float M = -INFINITY, W = 0.f;
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-  if (grp < groups) {
-    const int64_t row0 =
-        (static_cast<int64_t>(b) * a.num_q_heads + kvh * G + g) * a.max_parts;
-    const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + row0;
-    const float* o = a.ws_o + row0 * D + lane * kPer;
-    constexpr int kBatch = kPer == 4 ? 6 : 8;  // partitions in flight (no spills)
-    for (int j0 = grp; j0 < n_parts; j0 += kBatch * groups) {
-      float2 mlj[kBatch];
-      float oj[kBatch][kPer];
+  constexpr int kBatch = kPer == 4 ? 6 : 8;  // partitions in flight
+  for (int j0 = warp; j0 < n_parts; j0 += kBatch * kReduceWarps) {
+    float2 mlj[kBatch];
+    float oj[kBatch][kPer];
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int j = j0 + u * groups;
-        mlj[u] = j < n_parts ? __ldcg(ml + j) : make_float2(-INFINITY, 0.f);
+    for (int u = 0; u < kBatch; ++u) {
+      const int j = j0 + u * kReduceWarps;
+      mlj[u] = j < n_parts ? __ldcg(ml + j) : make_float2(-INFINITY, 0.f);
 #pragma unroll
-        for (int e = 0; e < kPer; ++e)
-          oj[u][e] =
-              j < n_parts ? __ldcg(o + static_cast<int64_t>(j) * D + e) : 0.f;
+      for (int e = 0; e < kPer; ++e)
+        oj[u][e] =
+            j < n_parts ? __ldcg(o + static_cast<int64_t>(j) * D + e) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (mlj[u].x == -INFINITY) continue;  // empty or skipped partition
+      if (mlj[u].x > M) {
+        const float sc = dev::fast_exp2(M - mlj[u].x);  // 0 when M = -inf
+        W *= sc;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[e] *= sc;
+        M = mlj[u].x;
       }
+      const float w = mlj[u].y * dev::fast_exp2(mlj[u].x - M);
+      W += w;
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        if (mlj[u].x == -INFINITY) continue;  // empty or skipped partition
-        if (mlj[u].x > M) {
-          const float sc = dev::fast_exp2(M - mlj[u].x);  // 0 when M = -inf
-          W *= sc;
-#pragma unroll
-          for (int e = 0; e < kPer; ++e) acc[e] *= sc;
-          M = mlj[u].x;
-        }
-        const float w = mlj[u].y * dev::fast_exp2(mlj[u].x - M);
-        W += w;
-#pragma unroll
-        for (int e = 0; e < kPer; ++e) acc[e] += w * oj[u][e];
-      }
+      for (int e = 0; e < kPer; ++e) acc[e] += w * oj[u][e];
     }
   }
   if (lane == 0) {
@@ -777,22 +792,22 @@ __global__ void __launch_bounds__(kReduceMaxWarps * 32)
 #pragma unroll
   for (int e = 0; e < kPer; ++e) s_acc[warp][lane * kPer + e] = acc[e];
   __syncthreads();
-  for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-    const int h = idx / D, d = idx - (idx / D) * D;
+  for (int d = threadIdx.x; d < D; d += kReduceWarps * 32) {
     float mx = -INFINITY;
-    for (int q = 0; q < groups; ++q) mx = fmaxf(mx, s_m[q * G + h]);
+#pragma unroll
+    for (int w = 0; w < kReduceWarps; ++w) mx = fmaxf(mx, s_m[w]);
     float tw = 0.f, tv = 0.f;
     if (mx != -INFINITY) {
-      for (int q = 0; q < groups; ++q) {
-        const float mq = s_m[q * G + h];
-        const float sc = mq == -INFINITY ? 0.f : dev::fast_exp2(mq - mx);
-        tw += s_w[q * G + h] * sc;
-        tv += s_acc[q * G + h][d] * sc;
+#pragma unroll
+      for (int w = 0; w < kReduceWarps; ++w) {
+        const float sc =
+            s_m[w] == -INFINITY ? 0.f : dev::fast_exp2(s_m[w] - mx);
+        tw += s_w[w] * sc;
+        tv += s_acc[w][d] * sc;
       }
     }
-    static_cast<T*>(a.out)[(static_cast<int64_t>(b) * a.num_q_heads +
-                            kvh * G + h) * D + d] =
-        from_float<T>(tw > 0.f ? tv / tw : 0.f);
+    static_cast<T*>(a.out)[(static_cast<int64_t>(b) * a.num_q_heads + qh) *
+                               D + d] = from_float<T>(tw > 0.f ? tv / tw : 0.f);
   }
 }
 
@@ -843,6 +858,10 @@ bool encode_cache_map(CUtensorMap* map, const void* base, uint64_t rows,
 #ifndef PAGEDKV_RING_BYTES
 #define PAGEDKV_RING_BYTES 65536
 #endif
+#ifndef PAGEDKV_PDL
+#define PAGEDKV_PDL 1  // programmatic dependent launch between the kernels
+#endif
+constexpr int kUsePdl = PAGEDKV_PDL;
 constexpr int stages_for(int bs, int d) {
   // 64 KB ring per CTA: three CTAs fit one SM's shared memory.  Whole
   // multiples of the consumer count (see Geometry).
@@ -958,20 +977,27 @@ pa_status launch(const pa_decode_desc* d, DecodeArgs& a, const CUtensorMap& km,
                   cudaGetErrorString(e));
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
-  // Both kernels are launched with programmatic stream serialization: each
-  // may start while its predecessor drains and waits (griddepcontrol.wait)
-  // before touching memory the predecessor writes.
+  // Every kernel here (the counter reset, the decode, the reduce) is
+  // launched with programmatic stream serialization: each may start while
+  // its predecessor drains and waits (griddepcontrol.wait) before touching
+  // memory the predecessor writes.
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].val.programmaticStreamSerializationAllowed = kUsePdl;
   if (a.max_parts > 1 && a.fused) {
-    cudaError_t me = cudaMemsetAsync(
-        a.counters, 0,
-        static_cast<size_t>(d->num_seqs) * d->num_kv_heads * sizeof(int),
-        stream);
-    if (me != cudaSuccess)
+    const int n = d->num_seqs * d->num_kv_heads;
+    cudaLaunchConfig_t zcfg = {};
+    zcfg.gridDim = dim3((n + 1023) / 1024 < 64 ? (n + 1023) / 1024 : 64);
+    zcfg.blockDim = dim3(1024);
+    zcfg.stream = stream;
+    zcfg.attrs = attr;
+    zcfg.numAttrs = 1;
+    const cudaError_t ze =
+        cudaLaunchKernelEx(&zcfg, zero_counters_kernel, a.counters, n);
+    count_launch();
+    if (ze != cudaSuccess)
       return fail(PA_ERR_CUDA, "pa_decode: counter reset failed: %s",
-                  cudaGetErrorString(me));
+                  cudaGetErrorString(ze));
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.max_parts, d->num_kv_heads, d->num_seqs);
@@ -986,19 +1012,14 @@ pa_status launch(const pa_decode_desc* d, DecodeArgs& a, const CUtensorMap& km,
     return fail(PA_ERR_CUDA, "pa_decode: decode launch failed: %s",
                 cudaGetErrorString(e));
   if (a.max_parts > 1 && !a.fused) {
-    // Part-groups per head: about 16 partitions per warp, at most 32 warps.
-    const int G = a.group;
-    int groups = (a.max_parts + 15) / 16;
-    if (groups > kReduceMaxWarps / G) groups = kReduceMaxWarps / G;
-    if (groups < 1) groups = 1;
     cudaLaunchConfig_t rcfg = {};
-    rcfg.gridDim = dim3(d->num_kv_heads, d->num_seqs);
-    rcfg.blockDim = dim3(32 * G * groups);
+    rcfg.gridDim = dim3(d->num_q_heads, d->num_seqs);
+    rcfg.blockDim = dim3(kReduceWarps * 32);
     rcfg.dynamicSmemBytes = 0;
     rcfg.stream = stream;
     rcfg.attrs = attr;
     rcfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&rcfg, reduce_kernel<T, D>, a, BS, groups);
+    e = cudaLaunchKernelEx(&rcfg, reduce_kernel<T, D>, a, BS);
     count_launch();
     if (e != cudaSuccess)
       return fail(PA_ERR_CUDA, "pa_decode: reduce launch failed: %s",
