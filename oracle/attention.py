@@ -138,3 +138,47 @@ def contiguous_decode(q: np.ndarray, K_seqs, V_seqs, scale: float,
             kvh = kv_head_of(h, num_q_heads, num_kv_heads)
             out[b, h] = attend(q[b, h], Kb[:, kvh, :], Vb[:, kvh, :], scale)
     return out
+
+
+def paged_prefill(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
+                  block_tables: np.ndarray, context_lens: np.ndarray,
+                  query_start: np.ndarray, scale: float,
+                  seqs=None) -> np.ndarray:
+    """Causal attention of each sequence's newest tokens over its paged K/V.
+
+    Sequence b holds ``context_lens[b]`` = L tokens in the cache, of which the
+    last ``q_len = query_start[b+1] - query_start[b]`` are new and have query
+    vectors ``q[query_start[b] + i]`` (i = 0 .. q_len-1).  New token i sits
+    at position ``p = L - q_len + i`` and attends to positions 0 .. p (the
+    tokens before it and itself), with the same scores and softmax as
+    contiguous attention.  Decode is the case q_len = 1; prefilling a whole
+    prompt is q_len = L; anything between is a chunk of a longer prompt, or
+    several speculative tokens checked at once ([Taming the Tail] "The
+    Future: Speculative Decoding and Beyond": the verifying model processes
+    the draft tokens in one pass).
+
+    ``q`` is ``[total_q, num_q_heads, head_dim]``; returns the same shape in
+    float64 (NaN rows for sequences not in ``seqs``).
+    """
+    total_q, num_q_heads, head_dim = q.shape
+    num_kv_heads = k_cache.shape[1]
+    block_size = k_cache.shape[2]
+    out = np.full((total_q, num_q_heads, head_dim), np.nan)
+    B = len(context_lens)
+    for b in (range(B) if seqs is None else seqs):
+        L = int(context_lens[b])
+        q0, q1 = int(query_start[b]), int(query_start[b + 1])
+        q_len = q1 - q0
+        if q_len > L:
+            raise ValueError("more new tokens than the context holds")
+        for kvh in range(num_kv_heads):
+            K = depage(k_cache, block_tables[b], L, kvh, block_size)
+            V = depage(v_cache, block_tables[b], L, kvh, block_size)
+            for h in range(num_q_heads):
+                if kv_head_of(h, num_q_heads, num_kv_heads) != kvh:
+                    continue
+                for i in range(q_len):
+                    p = L - q_len + i
+                    out[q0 + i, h] = attend(q[q0 + i, h], K[:p + 1],
+                                            V[:p + 1], scale)
+    return out
