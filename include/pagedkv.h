@@ -185,6 +185,51 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,
                             void* stream);
 
 /* ------------------------------------------------------------------------
+ * Causal attention of new tokens over the paged cache (chunked prefill,
+ * several speculative tokens at once).
+ *
+ * Defines ([vLLM PagedAttention FAQ] "Does PagedAttention change the
+ * mathematical attention output?"; [Taming the Tail] "The Future:
+ * Speculative Decoding and Beyond"; [KV-cache chapter] "Common
+ * misconception...": serving kernels run FlashAttention-style tiles over the
+ * paged layout): sequence b holds L = context_lens[b] tokens in the cache
+ * (the new ones already written with pa_cache_write); its last
+ * q_len = query_start[b+1] - query_start[b] tokens are new, with query rows
+ * q[query_start[b] + i].  New token i sits at position p = L - q_len + i and
+ *     out[query_start[b] + i, h, :] = softmax(scale * K_b[0..p] q) V_b[0..p]
+ * with query head h reading KV head h / G.  q_len = 1 is decode; q_len = L a
+ * whole prompt.
+ * Layouts: q, out [total_q, num_q_heads, 128] dtype; query_start [num_seqs+1]
+ * int32 on the device, non-decreasing, query_start[0] = 0 and
+ * query_start[num_seqs] <= total_q; the rest as for pa_decode.
+ * Supported: head_dim 128, block_size 16 or 32, G = 1, 2, 4 or 8 (else
+ * PA_ERR_UNSUPPORTED).  Runs on the tcgen05 tensor cores with fp32
+ * accumulation in tensor memory; output rounded once to dtype.
+ * Device-side: a context or query range outside the table, or a block id
+ * outside the pool, sets *dev_err = PA_ERR_DEVICE_OOB and the affected
+ * rows are unspecified.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int num_seqs;
+  int num_q_heads;
+  int num_kv_heads;
+  int head_dim;
+  int block_size;
+  int max_blocks_per_seq;
+  int num_blocks;
+  pa_dtype dtype;
+  int total_q;          /* rows of q and out */
+  int max_q_len;        /* host bound on any sequence's new-token count */
+  int max_context_len;  /* host bound on context_lens[] (0: table capacity) */
+} pa_prefill_desc;
+
+pa_status pa_prefill(void* out, const void* q, const void* k_cache,
+                     const void* v_cache, const int32_t* block_tables,
+                     const int32_t* context_lens, const int32_t* query_start,
+                     float scale, const pa_prefill_desc* desc,
+                     int32_t* dev_err, void* stream);
+
+/* ------------------------------------------------------------------------
  * Write new tokens' K and V into their cache slots.
  *
  * Defines ([Taming the Tail] "How the Architecture Works"; [KV-cache

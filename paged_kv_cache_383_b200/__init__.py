@@ -26,7 +26,8 @@ from ._lib import (PA_BF16, PA_F16, PA_KERNEL_AUTO, PA_KERNEL_MMA,
                    pa_decode_desc)
 
 __all__ = [
-    "pa_decode", "pa_decode_noalloc", "pa_cache_write", "pa_copy_blocks",
+    "pa_decode", "pa_decode_noalloc", "pa_prefill", "pa_cache_write",
+    "pa_copy_blocks",
     "pa_decode_workspace_bytes", "pa_decode_partition_size", "make_desc",
     "BlockManager", "PagedKVError", "NoFreeBlocksError", "library_path",
     "pa_launch_count", "pa_read_probe",
@@ -182,6 +183,40 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens,
         ctypes.c_float(scale), ctypes.byref(desc),
         _dev(dev_err, "dev_err", torch.int32), _stream(stream))
     _lib.check(st, "pa_decode_noalloc")
+    return out
+
+
+def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens,
+               query_start, scale: float, *, max_q_len: int,
+               max_context_len: int = 0, dev_err=None, stream=None):
+    """Causal attention of each sequence's new tokens (rows
+    query_start[b] .. query_start[b+1]-1 of ``q``) over its paged K/V, the
+    new tokens being the last ones of the context.  ``max_q_len`` bounds
+    every sequence's new-token count (sizes the grid).  Returns ``out``."""
+    import torch
+    lib = _lib.load()
+    total_q, num_q_heads, head_dim = q.shape
+    num_blocks, num_kv_heads, block_size, hd2 = k_cache.shape
+    if hd2 != head_dim or out.shape != q.shape:
+        raise ValueError("q, out and the caches disagree on shape")
+    for name, t in (("out", out), ("k_cache", k_cache), ("v_cache", v_cache)):
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} dtype {t.dtype} != q dtype {q.dtype}")
+    desc = _lib.pa_prefill_desc(
+        num_seqs=block_tables.shape[0], num_q_heads=num_q_heads,
+        num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=block_size,
+        max_blocks_per_seq=block_tables.shape[1], num_blocks=num_blocks,
+        dtype=_dtype_code(q), total_q=total_q, max_q_len=max_q_len,
+        max_context_len=max_context_len)
+    st = lib.pa_prefill(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32),
+        _dev(query_start, "query_start", torch.int32),
+        ctypes.c_float(scale), ctypes.byref(desc),
+        _dev(dev_err, "dev_err", torch.int32), _stream(stream))
+    _lib.check(st, "pa_prefill")
     return out
 
 

@@ -56,6 +56,22 @@ class pa_decode_desc(ctypes.Structure):
     ]
 
 
+class pa_prefill_desc(ctypes.Structure):
+    _fields_ = [
+        ("num_seqs", ctypes.c_int),
+        ("num_q_heads", ctypes.c_int),
+        ("num_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int),
+        ("block_size", ctypes.c_int),
+        ("max_blocks_per_seq", ctypes.c_int),
+        ("num_blocks", ctypes.c_int),
+        ("dtype", ctypes.c_int),
+        ("total_q", ctypes.c_int),
+        ("max_q_len", ctypes.c_int),
+        ("max_context_len", ctypes.c_int),
+    ]
+
+
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int32
 _i64 = ctypes.c_int64
@@ -77,6 +93,8 @@ SIGNATURES = {
                         _vp, _vp]),
     "pa_decode_noalloc": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
                                 ctypes.POINTER(pa_decode_desc), _vp, _vp]),
+    "pa_prefill": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
+                         ctypes.POINTER(pa_prefill_desc), _vp, _vp]),
     "pa_cache_write": (_st, [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int,
                              _int, _int, _vp, _vp]),
     "pa_copy_blocks": (_st, [_vp, _vp, _vp, _int, _int, _int, _int, _int, _int,

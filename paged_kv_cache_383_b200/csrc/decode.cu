@@ -400,6 +400,18 @@ __global__ void __launch_bounds__(kThreads)
       const uint32_t kb = ring + s * Geo::kStageBytes;
       const uint32_t vb = kb + Geo::kPageBytes;
       const int nv = min(BS, n_tok - i * BS);
+      if (nv < BS) {
+        // Slots past the context get P = 0, but 0 * NaN is NaN in the MMA:
+        // clear the V rows the sequence never wrote (last page only).
+        for (int idx = lane; idx < (BS - nv) * Geo::kBoxes * 8; idx += 32) {
+          const int row = nv + idx / (Geo::kBoxes * 8);
+          const int c = idx % (Geo::kBoxes * 8);
+          dev::st_shared_zero16(vb + (c >> 3) * Geo::kBoxBytes + row * 128 +
+                                (c & 7) * 16);
+        }
+        dev::fence_proxy_async_smem();  // before TMA reuses the stage
+        __syncwarp();
+      }
 
       // S^T (tokens x heads) for each 16-token slice of the page.
       float sc[BS / 16][4];

@@ -1,0 +1,603 @@
+// pa_prefill: causal attention of each sequence's new tokens over its paged
+// K/V cache, on the 5th-generation tensor cores (tcgen05, tensor memory).
+//
+// What is computed: for sequence b with L = context_lens[b] tokens cached, of
+// which the last q_len are new (query rows query_start[b] .. +q_len), new
+// token i at position p = L - q_len + i attends to positions 0 .. p with the
+// scores and softmax of contiguous attention ([vLLM PagedAttention FAQ] "Does
+// PagedAttention change the mathematical attention output?").  q_len = L is a
+// whole prompt, q_len < L a chunk of one; a few new tokens at once is how a
+// target model checks speculative draft tokens ([Taming the Tail] "The
+// Future: Speculative Decoding and Beyond"); the attention is tiled as
+// [KV-cache chapter] "Common misconception..." describes serving kernels
+// doing: FlashAttention-style tiles over paged memory.
+//
+// B200 design.  Work unit = (tile of 128 query rows, KV head, sequence); a
+// row is a (new token, query head of this KV head) pair, so with G query heads
+// per KV head a tile holds 128/G tokens and each K/V byte serves all G heads.
+//   * Warp 0, lane 0 loads the Q tile with one 3-D TMA box per half of
+//     head_dim, then streams 64-key K and V tiles page by page (2-D TMA boxes
+//     of block_size rows x 128 B, 128-byte swizzle, no multicast) into a
+//     3-stage ring.  Pages are placed so that a tile is the canonical
+//     128-byte-swizzled layout the tensor core reads.
+//   * Warp 1 allocates 256 tensor-memory columns; its lane 0 issues
+//     S = Q K^T (M=128, N=64) and O += P V (M=128, N=128, V read MN-major)
+//     as tcgen05.mma with fp32 accumulators in tensor memory, and signals
+//     completion with tcgen05.commit.
+//   * Warps 2..5 own one tensor-memory row each (thread = query row): they
+//     read S with tcgen05.ld, apply the causal mask, keep the online softmax
+//     in registers (no shuffles: a row is one thread), rescale O in tensor
+//     memory only when the running maximum grows by more than 2^8 (the final
+//     division uses the same reference, so the result is unchanged), and
+//     write P to shared memory as a 16-bit rounded part plus its residual so
+//     P . V keeps ~16 mantissa bits.
+//   * Every wait is bounded (1 s) and reports PA_ERR_DEVICE_TIMEOUT; tensor
+//     memory is always released.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "device_utils.cuh"
+#include "pagedkv.h"
+#include "status.h"
+
+namespace pagedkv {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kRows = 128;      // query rows per tile (tensor memory lanes)
+constexpr int kKeys = 64;       // keys per K/V tile
+constexpr int kD = 128;         // head_dim
+constexpr int kStages = 3;      // K/V ring depth
+constexpr int kThreads = 192;   // producer, MMA, 4 softmax warps
+constexpr int kTmemCols = 256;  // S: cols [0, 64), O: cols [128, 256)
+constexpr float kRescaleLog2 = 8.f;
+
+struct PrefillArgs {
+  void* out;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  const int32_t* query_start;
+  int32_t* dev_err;
+  float scale_log2;
+  int num_q_heads;
+  int num_kv_heads;
+  int max_blocks_per_seq;
+  int num_blocks;
+  int max_context_len;
+  int total_q;
+};
+
+// Shared memory (offsets from a 1024-byte aligned base).
+constexpr int kQBytes = kRows * kD * 2;                 // 32 KB, two halves
+constexpr int kHalfQ = kRows * 128;                     // 16 KB
+constexpr int kTileHalf = kKeys * 128;                  // 8 KB: 64 keys x 64 d
+constexpr int kKVTile = 2 * kTileHalf;                  // 16 KB per K or V
+constexpr int kStageBytes = 2 * kKVTile;                // K + V
+constexpr int kPBytes = kRows * kKeys * 2;              // 16 KB per P part
+constexpr int kOffQ = 0;
+constexpr int kOffRing = kOffQ + kQBytes;
+constexpr int kOffP = kOffRing + kStages * kStageBytes;  // hi, then lo
+constexpr int kOffBars = kOffP + 2 * kPBytes;
+// barriers: q_full, kv_full[S], kv_empty[S], s_full, s_free, p_full, o_ready,
+// done, then the tensor-memory base address word.
+constexpr int kNumBars = 1 + 2 * kStages + 5;
+constexpr int kOffTable = kOffBars + kNumBars * 8 + 16;
+
+size_t prefill_smem_bytes(int max_pages) {
+  return 1024 + kOffTable + ((static_cast<size_t>(max_pages) * 4 + 15) & ~15);
+}
+
+template <typename T, int BS, int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap qmap,
+                   const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap,
+                   const PrefillArgs a) {
+  constexpr int kTok = kRows / G;         // new tokens per tile
+  constexpr int kPagesPerTile = kKeys / BS;
+  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
+  using M = dev::Mma<T>;
+  extern __shared__ uint8_t smem_dyn[];
+  uint8_t* smem =
+      smem_dyn + ((1024u - (dev::smem_u32(smem_dyn) & 1023u)) & 1023u);
+  const uint32_t base = dev::smem_u32(smem);
+  const uint32_t q_s = base + kOffQ;
+  const uint32_t ring = base + kOffRing;
+  const uint32_t p_s = base + kOffP;
+  const uint32_t bars = base + kOffBars;
+  const uint32_t q_full = bars;
+  const uint32_t kv_full0 = bars + 8;
+  const uint32_t kv_empty0 = kv_full0 + kStages * 8;
+  const uint32_t s_full = kv_empty0 + kStages * 8;
+  const uint32_t s_free = s_full + 8;
+  const uint32_t p_full = s_free + 8;
+  const uint32_t o_ready = p_full + 8;
+  const uint32_t done = o_ready + 8;
+  uint32_t* tmem_slot =
+      reinterpret_cast<uint32_t*>(smem + kOffBars + kNumBars * 8);
+  int32_t* bt_s = reinterpret_cast<int32_t*>(smem + kOffTable);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int L = a.context_lens[b];
+  const int q0 = a.query_start[b];
+  const int q_len = a.query_start[b + 1] - q0;
+  if (L < 0 || L > a.max_blocks_per_seq * BS || L > a.max_context_len ||
+      q_len < 0 || q_len > L || q0 < 0 || q0 + q_len > a.total_q) {
+    if (qt == 0 && kvh == 0 && tid == 0)
+      dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
+    return;
+  }
+  const int tok0 = qt * kTok;
+  if (qt == gridDim.x - 1 && q_len > tok0 + kTok) {
+    // max_q_len was below this sequence's new-token count: the grid misses
+    // rows, which are left unwritten.
+    if (kvh == 0 && tid == 0) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
+  }
+  if (tok0 >= q_len) return;
+  const int n_q = min(kTok, q_len - tok0);
+  const int kv_end = L - q_len + tok0 + n_q;     // keys this tile may see
+  const int n_tiles = (kv_end + kKeys - 1) / kKeys;
+  const int n_pages = (kv_end + BS - 1) / BS;
+
+  // Block ids of the pages the tile reads; every one is checked.
+  int bad = 0;
+  const int32_t* row = a.block_tables +
+                       static_cast<int64_t>(b) * a.max_blocks_per_seq;
+  for (int i = tid; i < n_pages; i += kThreads) {
+    const int32_t p = row[i];
+    bad |= (p < 0 || p >= a.num_blocks);
+    bt_s[i] = p;
+  }
+  if (tid == 0) {
+    dev::mbar_init(q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      dev::mbar_init(kv_full0 + 8 * s, 1);
+      dev::mbar_init(kv_empty0 + 8 * s, 1);
+    }
+    dev::mbar_init(s_full, 1);
+    dev::mbar_init(s_free, 4);
+    dev::mbar_init(p_full, 4);
+    dev::mbar_init(o_ready, 1);
+    dev::mbar_init(done, 4);
+    dev::fence_mbar_init();
+  }
+  bad = __syncthreads_or(bad);
+  if (bad) {
+    if (tid == 0) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
+    return;
+  }
+  if (warp == 1) {  // the whole warp allocates tensor memory
+    dev::tmem_alloc(dev::smem_u32(tmem_slot), kTmemCols);
+    dev::tmem_relinquish();
+  }
+  dev::tc_fence_before();
+  __syncthreads();
+  dev::tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t s_tmem = tbase;        // columns [0, 64)
+  const uint32_t o_tmem = tbase + 128;  // columns [128, 256)
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      dev::prefetch_tmap(&qmap);
+      dev::prefetch_tmap(&kmap);
+      dev::prefetch_tmap(&vmap);
+      dev::mbar_arrive_expect_tx(q_full, kQBytes);
+      dev::tma_load_3d(q_s, &qmap, 0, kvh * G, q0 + tok0, q_full);
+      dev::tma_load_3d(q_s + kHalfQ, &qmap, 64, kvh * G, q0 + tok0, q_full);
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % kStages;
+        if (j >= kStages &&
+            !dev::mbar_wait(kv_empty0 + 8 * s, ((j / kStages) - 1) & 1)) {
+          dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
+          break;
+        }
+        const uint32_t full = kv_full0 + 8 * s;
+        dev::mbar_arrive_expect_tx(full, kStageBytes);
+        const uint32_t kt = ring + s * kStageBytes;
+        const uint32_t vt = kt + kKVTile;
+#pragma unroll
+        for (int p = 0; p < kPagesPerTile; ++p) {
+          const int page = j * kPagesPerTile + p;
+          // Pages past the sequence are masked; read a valid one instead.
+          const int32_t phys = page < n_pages ? bt_s[page] : bt_s[0];
+          const int y = (phys * a.num_kv_heads + kvh) * BS;
+          const uint32_t off = p * BS * 128;
+          dev::tma_load_2d(kt + off, &kmap, 0, y, full);
+          dev::tma_load_2d(kt + kTileHalf + off, &kmap, 64, y, full);
+          dev::tma_load_2d(vt + off, &vmap, 0, y, full);
+          dev::tma_load_2d(vt + kTileHalf + off, &vmap, 64, y, full);
+        }
+      }
+    }
+    return;
+  }
+
+  if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    bool ok = true;
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = dev::umma_idesc_f16(kBf16, kRows, kKeys,
+                                                        false, false);
+      constexpr uint32_t idesc_pv = dev::umma_idesc_f16(kBf16, kRows, kD,
+                                                        false, true);
+      auto issue_pv = [&](int t) -> bool {
+        if (!dev::mbar_wait(p_full, t & 1)) return false;
+        dev::tc_fence_after();
+        const uint32_t vt = ring + (t % kStages) * kStageBytes + kKVTile;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {  // P rounded part, residual
+#pragma unroll
+          for (int kk = 0; kk < kKeys / 16; ++kk) {
+            const uint64_t ad =
+                dev::sw128_desc(p_s + part * kPBytes + kk * 32, 16, 1024);
+            // V as the MN-major B operand: 64-wide d halves kTileHalf apart,
+            // 8-key groups 1024 bytes apart.
+            const uint64_t bd =
+                dev::sw128_desc(vt + kk * 2048, kTileHalf, 1024);
+            dev::umma_f16(o_tmem, ad, bd, idesc_pv,
+                          (t > 0 || part > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        dev::umma_commit(o_ready);
+        dev::umma_commit(kv_empty0 + 8 * (t % kStages));
+        return true;
+      };
+      ok = dev::mbar_wait(q_full, 0);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int s = j % kStages;
+        if (!dev::mbar_wait(kv_full0 + 8 * s, (j / kStages) & 1) ||
+            (j >= 1 && !dev::mbar_wait(s_free, (j - 1) & 1))) {
+          ok = false;
+          break;
+        }
+        dev::tc_fence_after();
+        const uint32_t kt = ring + s * kStageBytes;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const int h = kk >> 2, k4 = kk & 3;
+          const uint64_t ad = dev::sw128_desc(q_s + h * kHalfQ + k4 * 32, 16,
+                                              1024);
+          const uint64_t bd = dev::sw128_desc(kt + h * kTileHalf + k4 * 32,
+                                              16, 1024);
+          dev::umma_f16(s_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        dev::umma_commit(s_full);
+        if (j >= 1 && !issue_pv(j - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok) ok = issue_pv(n_tiles - 1);
+      if (ok) ok = dev::mbar_wait(o_ready, (n_tiles - 1) & 1);
+      if (!ok) dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
+      // Release tensor memory only after the softmax warps are done with it.
+      if (!dev::mbar_wait(done, 0)) dev::set_error(a.dev_err,
+                                                   PA_ERR_DEVICE_TIMEOUT);
+    }
+    __syncwarp();
+    dev::tc_fence_after();
+    dev::tmem_dealloc(tbase, kTmemCols);
+    return;
+  }
+
+  // ---------------- softmax warps (thread = query row) ----------------
+  const int quarter = warp & 3;  // tensor-memory lane quarter of this warp
+  const int r = quarter * 32 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+  const int t_loc = r / G;
+  const int g = r - t_loc * G;
+  const int tok = tok0 + t_loc;
+  const bool valid = t_loc < n_q;
+  // Padding rows (no query) see every key the tile loads; never stored.
+  const int qpos = valid ? L - q_len + tok : kv_end - 1;
+  float m_ref = -INFINITY, l = 0.f;
+  bool ok = true;
+  // Wait results are made warp-uniform: the tcgen05 loads and stores below
+  // are warp-collective.
+  for (int j = 0; j < n_tiles && ok; ++j) {
+    ok = __all_sync(0xffffffffu, dev::mbar_wait(s_full, j & 1));
+    if (!ok) break;
+    dev::tc_fence_after();
+    float sv[kKeys];
+    {
+      float (&lo)[32] = *reinterpret_cast<float(*)[32]>(sv);
+      float (&hi)[32] = *reinterpret_cast<float(*)[32]>(sv + 32);
+      dev::tmem_ld32(s_tmem + lane_off, lo);
+      dev::tmem_ld32(s_tmem + lane_off + 32, hi);
+      dev::tmem_ld_wait();
+    }
+    dev::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) dev::mbar_arrive(s_free);
+    float mx = -INFINITY;
+    const int k0 = j * kKeys;
+    if (k0 + kKeys > L) {
+      // Keys past the context get P = 0, but 0 * NaN is NaN in the MMA:
+      // clear the V rows of slots the sequence never wrote (and of pages
+      // past it).  Warp q clears rows 16q .. 16q+15 of the last tile.
+      const uint32_t vt = ring + (j % kStages) * kStageBytes + kKVTile;
+      for (int idx = lane; idx < 16 * 16; idx += 32) {
+        const int krow = quarter * 16 + (idx >> 4), c = idx & 15;
+        if (k0 + krow >= L)
+          dev::st_shared_zero16(vt + (c >> 3) * kTileHalf + krow * 128 +
+                                (c & 7) * 16);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < kKeys; ++c) {
+      const float x = (k0 + c <= qpos) ? sv[c] * a.scale_log2 : -INFINITY;
+      sv[c] = x;
+      mx = fmaxf(mx, x);
+    }
+    // P smem and O are busy until the previous P.V has finished.
+    if (j >= 1) {
+      ok = __all_sync(0xffffffffu, dev::mbar_wait(o_ready, (j - 1) & 1));
+      if (!ok) break;
+    }
+    dev::tc_fence_after();
+    float factor = 1.f;
+    if (j == 0) {
+      m_ref = mx;  // O is still empty: the first P.V overwrites it
+    } else if (mx > m_ref + kRescaleLog2) {
+      factor = dev::fast_exp2(m_ref - mx);
+      m_ref = mx;
+      l *= factor;
+    }
+    if (__any_sync(0xffffffffu, factor != 1.f)) {
+#pragma unroll
+      for (int c = 0; c < kD; c += 32) {
+        float ov[32];
+        dev::tmem_ld32(o_tmem + lane_off + c, ov);
+        dev::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ov[e] *= factor;
+        dev::tmem_st32(o_tmem + lane_off + c, ov);
+      }
+      dev::tmem_st_wait();
+    }
+    // P = 2^(s - m_ref) as a rounded part plus its residual, row r of the
+    // K-major 128-byte-swizzled A operand (16-byte chunk c at c ^ (r % 8)).
+    uint8_t* prow_hi = smem + kOffP + r * 128;
+    uint8_t* prow_lo = prow_hi + kPBytes;
+#pragma unroll
+    for (int c = 0; c < kKeys / 8; ++c) {
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float p0 = dev::fast_exp2(sv[8 * c + 2 * e] - m_ref);
+        const float p1 = dev::fast_exp2(sv[8 * c + 2 * e + 1] - m_ref);
+        l += p0 + p1;
+        hw[e] = M::pack(p0, p1);
+        const float2 hf = M::unpack(hw[e]);
+        lw[e] = M::pack(p0 - hf.x, p1 - hf.y);
+      }
+      const int sw = (c ^ (r & 7)) * 16;
+      *reinterpret_cast<uint4*>(prow_hi + sw) =
+          make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(prow_lo + sw) =
+          make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    dev::fence_proxy_async_smem();
+    dev::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) dev::mbar_arrive(p_full);
+  }
+  // Epilogue: O / l -> out[token, query head].
+  if (ok) ok = __all_sync(0xffffffffu,
+                          dev::mbar_wait(o_ready, (n_tiles - 1) & 1));
+  if (ok) {
+    dev::tc_fence_after();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    T* dst = static_cast<T*>(a.out) +
+             (static_cast<int64_t>(q0 + tok) * a.num_q_heads + kvh * G + g) *
+                 kD;
+#pragma unroll
+    for (int c = 0; c < kD; c += 32) {
+      float ov[32];
+      dev::tmem_ld32(o_tmem + lane_off + c, ov);
+      dev::tmem_ld_wait();
+      if (valid) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          uint4 w;
+          w.x = M::pack(ov[e] * inv, ov[e + 1] * inv);
+          w.y = M::pack(ov[e + 2] * inv, ov[e + 3] * inv);
+          w.z = M::pack(ov[e + 4] * inv, ov[e + 5] * inv);
+          w.w = M::pack(ov[e + 6] * inv, ov[e + 7] * inv);
+          *reinterpret_cast<uint4*>(dst + c + e) = w;
+        }
+      }
+    }
+  } else {
+    dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
+  }
+  dev::tc_fence_before();
+  __syncwarp();
+  if (lane == 0) dev::mbar_arrive(done);
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                         cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+CUtensorMapDataType tma_type(pa_dtype t) {
+  return t == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+}
+
+// q [total_q, Hq, 128] as a 3-D tensor; box = 64 dims x G heads x tokens.
+bool encode_q(CUtensorMap* m, const void* q, int total_q, int hq, int g,
+              int tok, pa_dtype dt) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD),
+                        static_cast<cuuint64_t>(hq),
+                        static_cast<cuuint64_t>(total_q)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * 2,
+                           static_cast<cuuint64_t>(hq) * kD * 2};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(g),
+                       static_cast<cuuint32_t>(tok)};
+  cuuint32_t es[3] = {1u, 1u, 1u};
+  return enc(m, tma_type(dt), 3, const_cast<void*>(q), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_cache(CUtensorMap* m, const void* cache, uint64_t rows, int bs,
+                  pa_dtype dt) {
+  auto enc = encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), rows};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+  cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(bs)};
+  cuuint32_t es[2] = {1u, 1u};
+  return enc(m, tma_type(dt), 2, const_cast<void*>(cache), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int BS, int G>
+pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
+                 const CUtensorMap& qm, const CUtensorMap& km,
+                 const CUtensorMap& vm, int max_pages, cudaStream_t st) {
+  auto kern = prefill_kernel<T, BS, G>;
+  const size_t smem = prefill_smem_bytes(max_pages);
+  cudaError_t e = cudaFuncSetAttribute(
+      kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      static_cast<int>(smem));
+  if (e != cudaSuccess)
+    return fail(PA_ERR_CUDA, "pa_prefill: cudaFuncSetAttribute(%zu): %s",
+                smem, cudaGetErrorString(e));
+  constexpr int kTok = kRows / G;
+  dim3 grid((d->max_q_len + kTok - 1) / kTok, d->num_kv_heads, d->num_seqs);
+  kern<<<grid, kThreads, smem, st>>>(qm, km, vm, a);
+  count_launch();
+  e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return fail(PA_ERR_CUDA, "pa_prefill: launch failed: %s",
+                cudaGetErrorString(e));
+  return PA_OK;
+}
+
+template <typename T, int BS>
+pa_status dispatch_group(const pa_prefill_desc* d, const PrefillArgs& a,
+                         const CUtensorMap& qm, const CUtensorMap& km,
+                         const CUtensorMap& vm, int max_pages, cudaStream_t st) {
+  switch (d->num_q_heads / d->num_kv_heads) {
+    case 1: return launch<T, BS, 1>(d, a, qm, km, vm, max_pages, st);
+    case 2: return launch<T, BS, 2>(d, a, qm, km, vm, max_pages, st);
+    case 4: return launch<T, BS, 4>(d, a, qm, km, vm, max_pages, st);
+    default: return launch<T, BS, 8>(d, a, qm, km, vm, max_pages, st);
+  }
+}
+
+}  // namespace
+}  // namespace pagedkv
+
+using pagedkv::fail;
+
+extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
+                                const void* v_cache,
+                                const int32_t* block_tables,
+                                const int32_t* context_lens,
+                                const int32_t* query_start, float scale,
+                                const pa_prefill_desc* d, int32_t* dev_err,
+                                void* stream) {
+  pagedkv::clear_error();
+  if (!d) return fail(PA_ERR_INVALID_ARG, "pa_prefill: desc is NULL");
+  if (d->num_seqs < 0 || d->num_q_heads <= 0 || d->num_kv_heads <= 0 ||
+      d->max_blocks_per_seq <= 0 || d->num_blocks < 0 || d->total_q < 0 ||
+      d->max_q_len < 0 || d->max_context_len < 0 ||
+      d->num_q_heads % d->num_kv_heads ||
+      (d->dtype != PA_F16 && d->dtype != PA_BF16) || !std::isfinite(scale))
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_prefill: num_seqs=%d num_q_heads=%d num_kv_heads=%d "
+                "max_blocks_per_seq=%d total_q=%d max_q_len=%d dtype=%d",
+                d->num_seqs, d->num_q_heads, d->num_kv_heads,
+                d->max_blocks_per_seq, d->total_q, d->max_q_len,
+                static_cast<int>(d->dtype));
+  const int G = d->num_q_heads / d->num_kv_heads;
+  if (d->head_dim != 128 || (d->block_size != 16 && d->block_size != 32) ||
+      (G != 1 && G != 2 && G != 4 && G != 8))
+    return fail(PA_ERR_UNSUPPORTED,
+                "pa_prefill: needs head_dim 128 (got %d), block_size 16 or 32 "
+                "(got %d) and a query group of 1, 2, 4 or 8 (got %d)",
+                d->head_dim, d->block_size, G);
+  if (d->num_seqs == 0 || d->total_q == 0 || d->max_q_len == 0) return PA_OK;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens ||
+      !query_start)
+    return fail(PA_ERR_INVALID_ARG, "pa_prefill: NULL tensor pointer");
+  if (!pagedkv::aligned16(out) || !pagedkv::aligned16(q) ||
+      !pagedkv::aligned16(k_cache) || !pagedkv::aligned16(v_cache))
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_prefill: out, q and the caches must be 16-byte aligned");
+  if (d->num_blocks == 0 || d->num_seqs > 65535 || d->num_kv_heads > 65535)
+    return fail(PA_ERR_INVALID_ARG, "pa_prefill: bad pool or batch size");
+  if (static_cast<int64_t>(d->num_blocks) * d->num_kv_heads * d->block_size >
+      0x7fffffffLL)
+    return fail(PA_ERR_UNSUPPORTED, "pa_prefill: pool exceeds 2^31 rows");
+  const int max_ctx = d->max_context_len > 0
+                          ? d->max_context_len
+                          : d->max_blocks_per_seq * d->block_size;
+  const int max_pages = (max_ctx + d->block_size - 1) / d->block_size;
+  if (pagedkv::prefill_smem_bytes(max_pages) > 227 * 1024)
+    return fail(PA_ERR_UNSUPPORTED,
+                "pa_prefill: context of %d tokens needs a block-table slice "
+                "beyond shared memory", max_ctx);
+  const int tok = pagedkv::kRows / G;
+  CUtensorMap qm, km, vm;
+  const uint64_t rows = static_cast<uint64_t>(d->num_blocks) *
+                        d->num_kv_heads * d->block_size;
+  if (!pagedkv::encode_q(&qm, q, d->total_q, d->num_q_heads, G, tok,
+                         d->dtype) ||
+      !pagedkv::encode_cache(&km, k_cache, rows, d->block_size, d->dtype) ||
+      !pagedkv::encode_cache(&vm, v_cache, rows, d->block_size, d->dtype))
+    return fail(PA_ERR_CUDA, "pa_prefill: cuTensorMapEncodeTiled failed");
+  pagedkv::PrefillArgs a;
+  a.out = out;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.query_start = query_start;
+  a.dev_err = dev_err;
+  a.scale_log2 = scale * pagedkv::kLog2e;
+  a.num_q_heads = d->num_q_heads;
+  a.num_kv_heads = d->num_kv_heads;
+  a.max_blocks_per_seq = d->max_blocks_per_seq;
+  a.num_blocks = d->num_blocks;
+  a.max_context_len = max_ctx;
+  a.total_q = d->total_q;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d->dtype == PA_BF16)
+    return d->block_size == 16
+               ? pagedkv::dispatch_group<__nv_bfloat16, 16>(d, a, qm, km, vm,
+                                                            max_pages, s)
+               : pagedkv::dispatch_group<__nv_bfloat16, 32>(d, a, qm, km, vm,
+                                                            max_pages, s);
+  return d->block_size == 16
+             ? pagedkv::dispatch_group<__half, 16>(d, a, qm, km, vm, max_pages,
+                                                   s)
+             : pagedkv::dispatch_group<__half, 32>(d, a, qm, km, vm, max_pages,
+                                                   s);
+}

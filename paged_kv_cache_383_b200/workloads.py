@@ -256,3 +256,33 @@ def make_prefix(w: Workload, device="cpu") -> PrefixInputs:
     sv = _randn((total, H, D), g, device, dt)
     return PrefixInputs(w, lengths, suffix, num_blocks, free_order, q, pk, pv,
                         sk, sv)
+
+
+@dataclass
+class PrefillInputs:
+    """A paged batch plus query rows for each sequence's newest tokens."""
+    paged: PagedInputs
+    q_lens: np.ndarray         # int64 [B]: new tokens per sequence (<= L)
+    query_start: np.ndarray    # int32 [B+1]
+    q: object                  # torch [sum(q_lens), Hq, D]
+
+
+def make_prefill(w: Workload, q_lens, device="cpu",
+                 seed_offset: int = 17) -> PrefillInputs:
+    """``make_paged`` for the cache, plus N(0, 1) query rows for the last
+    ``q_lens[b]`` tokens of every sequence (clipped to its length)."""
+    import torch
+    inp = make_paged(w, device=device)
+    q_lens = np.minimum(np.asarray(q_lens, dtype=np.int64), inp.lengths)
+    start = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed + seed_offset)
+    q = torch.randn(int(start[-1]), w.num_q_heads, w.head_dim, generator=g,
+                    device=device, dtype=torch.float32).to(
+                        torch_dtype(w.dtype))
+    return PrefillInputs(inp, q_lens, start, q)
+
+
+WORKLOADS["chunked_prefill_gqa8"] = Workload(
+    "chunked_prefill_gqa8", 383006, 16, 64, 8, 128, 16, "bfloat16",
+    "uniform", low=2048, high=8192)

@@ -89,3 +89,21 @@ def sample_seqs(lengths, k=6, seed=0):
             break
         pick.add(int(b))
     return sorted(pick)
+
+
+def poison_unwritten(inp) -> None:
+    """Fill every cache slot no sequence has written (the tail of each last
+    block and every block no table references) with NaN, in place.  Keys
+    past a context are masked, so the result must not change."""
+    bs = inp.workload.block_size
+    used = np.zeros(inp.num_blocks, dtype=bool)
+    for b, L in enumerate(inp.lengths):
+        n = (int(L) + bs - 1) // bs
+        used[inp.block_tables[b, :n]] = True
+        if L % bs:
+            last = int(inp.block_tables[b, n - 1])
+            inp.k_cache[last, :, L % bs:] = float("nan")
+            inp.v_cache[last, :, L % bs:] = float("nan")
+    free = torch.from_numpy(np.flatnonzero(~used)).to(inp.k_cache.device)
+    inp.k_cache[free] = float("nan")
+    inp.v_cache[free] = float("nan")

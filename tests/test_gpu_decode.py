@@ -7,6 +7,7 @@
 * invariances: partition size, identity vs shuffled block tables;
 * edge cases: empty batch, empty and one-token sequences, full tables, group
   sizes 1..8, head_dim 64/128, both dtypes;
+* NaN in slots no sequence wrote does not reach the output;
 * device-side index checks set the error word instead of faulting.
 """
 import numpy as np
@@ -16,7 +17,8 @@ import torch
 from oracle import attention as oa
 from paged_kv_cache_383_b200 import workloads as wl
 
-from helpers import check_decode, oracle_paged_sample, sample_seqs, to_np
+from helpers import (check_decode, oracle_paged_sample, poison_unwritten,
+                     sample_seqs, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -199,3 +201,18 @@ def test_device_checks_flag_bad_inputs(pkv):
         for b in (1, 2):
             check_decode(to_np(out[b]), ref[b], inp.q.dtype,
                          f"split seq {b} / {reduce}")
+
+
+@pytest.mark.parametrize("kernel", ["mma", "simt"])
+@pytest.mark.parametrize("bs", [16, 32])
+def test_unwritten_slots_hold_nan(pkv, kernel, bs):
+    w = wl.Workload("nan_tail", 21, 6, 32, 8, 128, bs, "bfloat16", "fixed",
+                    fixed_lengths=(1, 15, 17, 100, 333, 1000))
+    inp = wl.make_paged(w, device="cuda")
+    ref = oa.paged_decode(to_np(inp.q), to_np(inp.k_cache),
+                          to_np(inp.v_cache), inp.block_tables, inp.lengths,
+                          w.softmax_scale)
+    poison_unwritten(inp)
+    for ps in (0, 64):
+        out = _run(pkv, inp, kernel=kernel, partition_size=ps)
+        check_decode(to_np(out), ref, inp.q.dtype, f"{kernel} ps={ps}")

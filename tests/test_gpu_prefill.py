@@ -1,0 +1,185 @@
+"""GPU parity of pa_prefill (causal attention of new tokens over the paged
+cache, tcgen05 tensor cores) against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as oa
+from paged_kv_cache_383_b200 import workloads as wl
+
+from helpers import check_decode, poison_unwritten, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(pkv, pin, tables=None, err=None):
+    inp = pin.paged
+    w = inp.workload
+    out = torch.full_like(pin.q, float("nan"))
+    bt = torch.from_numpy(inp.block_tables if tables is None
+                          else tables).cuda()
+    cl = torch.from_numpy(inp.lengths.astype(np.int32)).cuda()
+    qs = torch.from_numpy(pin.query_start).cuda()
+    pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl, qs,
+                   w.softmax_scale, max_q_len=int(max(pin.q_lens.max(), 1)),
+                   max_context_len=int(inp.lengths.max()), dev_err=err)
+    torch.cuda.synchronize()
+    return out
+
+
+def _check(pin, out, what, seqs=None):
+    inp = pin.paged
+    ref = oa.paged_prefill(to_np(pin.q), to_np(inp.k_cache),
+                           to_np(inp.v_cache), inp.block_tables, inp.lengths,
+                           pin.query_start, inp.workload.softmax_scale,
+                           seqs=seqs)
+    rows = np.concatenate([np.arange(pin.query_start[b],
+                                     pin.query_start[b + 1])
+                           for b in (seqs if seqs is not None
+                                     else range(len(pin.q_lens)))])
+    return check_decode(to_np(out)[rows], ref[rows], pin.q.dtype, what)
+
+
+@pytest.mark.parametrize("dtype", ["bfloat16", "float16"])
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (32, 8), (64, 8)])
+@pytest.mark.parametrize("bs", [16, 32])
+def test_mixed_chunks(pkv, dtype, hq, hkv, bs):
+    # whole prompts, chunks, single tokens and a few speculative tokens
+    lens = (1, 17, 130, 300, 520, 64, 700, 33)
+    qlens = (1, 17, 130, 57, 1, 4, 200, 33)
+    w = wl.Workload("prefill", 11, len(lens), hq, hkv, 128, bs, dtype,
+                    "fixed", fixed_lengths=lens)
+    pin = wl.make_prefill(w, qlens, device="cuda")
+    out = _run(pkv, pin)
+    _check(pin, out, f"{dtype}/{hq}:{hkv}/bs{bs}")
+
+
+def test_single_token_matches_decode(pkv):
+    w = wl.WORKLOADS["llama3_70b_gqa8"].scaled(num_seqs=8, cap=2000)
+    pin = wl.make_prefill(w, np.ones(8), device="cuda")
+    out = _run(pkv, pin)
+    inp = pin.paged
+    dec = torch.empty_like(pin.q)
+    pkv.pa_decode(dec, pin.q, inp.k_cache, inp.v_cache,
+                  torch.from_numpy(inp.block_tables).cuda(),
+                  torch.from_numpy(inp.lengths.astype(np.int32)).cuda(),
+                  w.softmax_scale, max_context_len=int(inp.lengths.max()))
+    torch.cuda.synchronize()
+    _check(pin, out, "prefill q_len=1")
+    assert (out.float() - dec.float()).abs().max().item() <= 4e-3
+
+
+def test_sequences_without_new_tokens(pkv):
+    w = wl.Workload("prefill0", 12, 3, 32, 8, 128, 16, "bfloat16", "fixed",
+                    fixed_lengths=(100, 50, 80))
+    pin = wl.make_prefill(w, (0, 50, 0), device="cuda")
+    out = _run(pkv, pin)
+    _check(pin, out, "middle sequence only")
+    assert out.shape[0] == 50
+
+
+def test_chunked_prefill_full_size_sampled(pkv):
+    w = wl.WORKLOADS["chunked_prefill_gqa8"]
+    pin = wl.make_prefill(w, np.full(w.num_seqs, 512), device="cuda")
+    out = _run(pkv, pin)
+    _check(pin, out, "chunked prefill", seqs=[0, 7, 15])
+    assert torch.isfinite(out.float()).all()
+
+
+def test_bad_block_id_is_flagged(pkv):
+    w = wl.Workload("prefillbad", 13, 3, 16, 8, 128, 16, "bfloat16", "fixed",
+                    fixed_lengths=(90, 90, 90))
+    pin = wl.make_prefill(w, (30, 30, 30), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tables = pin.paged.block_tables.copy()
+    tables[1, 2] = pin.paged.num_blocks + 3
+    out = _run(pkv, pin, tables=tables, err=err)
+    assert err.item() == 5
+    _check(pin, out, "other sequences intact", seqs=[0, 2])
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+def test_unwritten_slots_hold_nan(pkv, bs):
+    lens = (1, 15, 17, 100, 333, 1000)
+    w = wl.Workload("prefill_nan", 14, len(lens), 32, 8, 128, bs,
+                    "bfloat16", "fixed", fixed_lengths=lens)
+    pin = wl.make_prefill(w, (1, 15, 5, 100, 40, 300), device="cuda")
+    _check(pin, _run(pkv, pin), "clean pool")
+    poison_unwritten(pin.paged)
+    _check(pin, _run(pkv, pin), "poisoned pool")
+
+
+def _contiguous_pool(K_seqs, V_seqs, bs):
+    """Host pool holding each sequence's K/V in consecutive blocks, and the
+    identity tables that reach them (built from inputs only)."""
+    nblk = [(len(k) + bs - 1) // bs for k in K_seqs]
+    hkv, d = K_seqs[0].shape[1:]
+    kp = np.zeros((sum(nblk), hkv, bs, d))
+    vp = np.zeros_like(kp)
+    tables = np.full((len(K_seqs), max(nblk)), -1, dtype=np.int32)
+    base = 0
+    for b, (k, v) in enumerate(zip(K_seqs, V_seqs)):
+        for t in range(len(k)):
+            kp[base + t // bs, :, t % bs] = k[t]
+            vp[base + t // bs, :, t % bs] = v[t]
+        tables[b, :nblk[b]] = np.arange(base, base + nblk[b])
+        base += nblk[b]
+    return kp, vp, tables
+
+
+def test_speculative_verify_and_rollback(pkv):
+    """Prompt prefill -> 4 draft tokens verified in one pass -> rejected
+    drafts rolled back with truncate -> next token written over the freed
+    slots and decoded; every step against the oracle on input K/V."""
+    from paged_kv_cache_383_b200 import flow
+    hq, hkv, d, bs, draft = 32, 8, 128, 16, 4
+    prompts, accept = [37, 64, 100, 5], [0, 1, 3, 4]
+    B = len(prompts)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(383007)
+    rnd = lambda *s: torch.randn(*s, generator=g, device="cuda").to(
+        torch.bfloat16)
+    kc, vc = rnd(64, hkv, bs, d), rnd(64, hkv, bs, d)
+    bm = pkv.BlockManager(64, bs)
+    ids = list(range(B))
+    for s in ids:
+        bm.add_seq(s)
+    K = [np.zeros((0, hkv, d)) for _ in ids]
+    V = [np.zeros((0, hkv, d)) for _ in ids]
+    scale = d ** -0.5
+
+    def step(n_new):
+        """Write n_new[b] tokens, attend their queries causally, check."""
+        kn, vn = rnd(sum(n_new), hkv, d), rnd(sum(n_new), hkv, d)
+        q = rnd(sum(n_new), hq, d)
+        flow.write_tokens(bm, kc, vc, ids, n_new, kn, vn)
+        qs = np.concatenate([[0], np.cumsum(n_new)]).astype(np.int32)
+        for b in ids:
+            K[b] = np.concatenate([K[b], to_np(kn[qs[b]:qs[b + 1]])])
+            V[b] = np.concatenate([V[b], to_np(vn[qs[b]:qs[b + 1]])])
+        bt, cl, lens = flow.tables_on_device(bm, ids, 16, "cuda")
+        assert list(lens) == [len(k) for k in K]
+        out = torch.empty_like(q)
+        pkv.pa_prefill(out, q, kc, vc, bt, cl, torch.from_numpy(qs).cuda(),
+                       scale, max_q_len=max(n_new),
+                       max_context_len=int(lens.max()))
+        kp, vp, tables = _contiguous_pool(K, V, bs)
+        ref = oa.paged_prefill(to_np(q), kp, vp, tables, lens, qs, scale)
+        torch.cuda.synchronize()
+        check_decode(to_np(out), ref, q.dtype, f"step {n_new}")
+        return q, bt, cl, lens, out
+
+    step(prompts)                      # whole prompts
+    step([draft] * B)                  # verify the drafts in one pass
+    for b in ids:                      # keep the accepted drafts only
+        keep = prompts[b] + accept[b]
+        bm.truncate(b, keep)
+        K[b], V[b] = K[b][:keep], V[b][:keep]
+    q, bt, cl, lens, out = step([1] * B)   # next token over freed slots
+    dec = torch.empty_like(q)
+    pkv.pa_decode(dec, q, kc, vc, bt, cl, scale,
+                  max_context_len=int(lens.max()))
+    torch.cuda.synchronize()
+    kp, vp, tables = _contiguous_pool(K, V, bs)
+    check_decode(to_np(dec), oa.paged_decode(to_np(q), kp, vp, tables, lens,
+                                             scale), q.dtype, "decode")
