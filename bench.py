@@ -39,6 +39,7 @@ METRIC = ("paged decode KV GB/s and % of B200 HBM peak; "
           "seq·layers/s at 1 GPU")
 SPEC_HBM_GBS = 8000.0          # the spec figure the target is quoted against
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse_args():
@@ -55,6 +56,9 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-spinup", action="store_true",
                    help="skip the 1 s untimed clock spin-up (profiling)")
+    p.add_argument("--prefill-only", action="store_true",
+                   help="time only pa_prefill on the two prefill workloads "
+                        "and print their line (tuning and profiling)")
     return p.parse_args()
 
 
@@ -533,7 +537,91 @@ def extras(args, w, inp, dev, pkv, bt, cl):
     out["torch_sum_read_gbs"] = round(4 * (1 << 30) / (a.elapsed_time(b) /
                                                         10 * 1e-3) / 1e9, 1)
     del x
+    from paged_kv_cache_383_b200 import workloads as wl
+    out["prefill"] = [time_prefill(pkv, wl, n, c, dev)
+                      for n, c in PREFILL_CASES]
     return out
+
+
+def measured_bf16_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def prefill_flops(lengths, q_lens, num_q_heads, head_dim) -> int:
+    """Algorithmic FLOPs of causal attention of the new tokens: per query
+    head, new token and key it attends to, 2*D for q.k and 2*D for p*v."""
+    keys = 0
+    for L, n in zip(lengths, q_lens):
+        L, n = int(L), int(n)
+        keys += n * (L - n) + n * (n + 1) // 2
+    return 4 * head_dim * num_q_heads * keys
+
+
+PREFILL_CASES = (
+    # (workload, new tokens per sequence or None for the whole prompt)
+    ("chunked_prefill_gqa8", 512),
+    ("prompt_prefill_gqa8", None),
+)
+
+
+def time_prefill(pkv, wl, name, chunk, dev, iters=10):
+    """pa_prefill on a prefill workload: CUDA events around ``iters``
+    back-to-back launches on the launch stream (inputs > L2)."""
+    import torch
+    w = wl.WORKLOADS[name]
+    rng_lens = wl.make_paged(w, values=False).lengths
+    q_lens = rng_lens if chunk is None else np.minimum(rng_lens, chunk)
+    pin = wl.make_prefill(w, q_lens, device=dev)
+    inp = pin.paged
+    out = torch.empty_like(pin.q)
+    bt = torch.from_numpy(inp.block_tables).to(dev)
+    cl = torch.from_numpy(inp.lengths.astype(np.int32)).to(dev)
+    qs = torch.from_numpy(pin.query_start).to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    kw = dict(max_q_len=int(pin.q_lens.max()),
+              max_context_len=int(inp.lengths.max()), dev_err=err)
+    for _ in range(3):
+        pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl, qs,
+                       w.softmax_scale, **kw)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl, qs,
+                       w.softmax_scale, **kw)
+    b.record()
+    torch.cuda.synchronize()
+    if err.item():
+        raise RuntimeError(f"pa_prefill device error {err.item()}")
+    ms = a.elapsed_time(b) / iters
+    flops = prefill_flops(inp.lengths, pin.q_lens, w.num_q_heads, w.head_dim)
+    peak, kind = measured_bf16_peak()
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": name, "seqs": w.num_seqs,
+            "new_tokens": int(pin.q_lens.sum()),
+            "context_tokens": int(inp.lengths.sum()), "ms": round(ms, 4),
+            "tflops": round(tf, 1), "peak_tflops": peak,
+            "peak_kind": f"{kind} bf16 dense (cuBLAS GEMM)",
+            "frac": round(tf / peak, 4),
+            "note": "P.V runs twice (rounded P and its residual): the tensor "
+                    "cores do 1.5x the algorithmic FLOPs"}
+
+
+def run_prefill_only(args):
+    import torch
+    import paged_kv_cache_383_b200 as pkv
+    from paged_kv_cache_383_b200 import workloads as wl
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    res = [time_prefill(pkv, wl, n, c, dev, iters=max(args.steps, 1))
+           for n, c in PREFILL_CASES]
+    return {"metric": "prefill attention TFLOP/s (algorithmic)",
+            "unit": "TFLOP/s", "cases": res,
+            "gpu_launches": pkv.pa_launch_count()}
 
 
 def run_e2e(args, w, inp, dev, pkv, flow, world, rank, ps):
@@ -747,6 +835,9 @@ def main():
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
+        return
+    if args.prefill_only:
+        print(json.dumps(run_prefill_only(args)), flush=True)
         return
     res = run_native(args, rank, world, local)
     if rank == 0:

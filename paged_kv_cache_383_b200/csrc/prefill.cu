@@ -23,16 +23,22 @@
 //   * Warp 1 allocates 256 tensor-memory columns; its lane 0 issues
 //     S = Q K^T (M=128, N=64) and O += P V (M=128, N=128, V read MN-major)
 //     as tcgen05.mma with fp32 accumulators in tensor memory, and signals
-//     completion with tcgen05.commit.
+//     completion with tcgen05.commit.  S and P are double-buffered, so the
+//     tensor cores compute S(j+1) and P(j-1).V while the softmax warps work
+//     on tile j.
 //   * Warps 2..5 own one tensor-memory row each (thread = query row): they
-//     read S with tcgen05.ld, apply the causal mask, keep the online softmax
-//     in registers (no shuffles: a row is one thread), rescale O in tensor
-//     memory only when the running maximum grows by more than 2^8 (the final
-//     division uses the same reference, so the result is unchanged), and
-//     write P to shared memory as a 16-bit rounded part plus its residual so
-//     P . V keeps ~16 mantissa bits.
+//     read S with tcgen05.ld, apply the causal mask (diagonal tiles only),
+//     keep the online softmax in registers (no shuffles: a row is one
+//     thread), compute the exponentials before waiting for the previous P.V,
+//     rescale O in tensor memory only when the running maximum grows by more
+//     than 2^8 (the final division uses the same reference, so the result is
+//     unchanged), and write P to shared memory as a 16-bit rounded part plus
+//     its residual so P . V keeps ~16 mantissa bits.
 //   * Every wait is bounded (1 s) and reports PA_ERR_DEVICE_TIMEOUT; tensor
-//     memory is always released.
+//     memory is always released.  A barrier that is waited on by parity is
+//     never allowed to run two phases ahead of its waiter: each double
+//     buffer has its own barriers, and a buffer is refilled only after its
+//     consumer has observed the previous fill.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -78,13 +84,14 @@ constexpr int kTileHalf = kKeys * 128;                  // 8 KB: 64 keys x 64 d
 constexpr int kKVTile = 2 * kTileHalf;                  // 16 KB per K or V
 constexpr int kStageBytes = 2 * kKVTile;                // K + V
 constexpr int kPBytes = kRows * kKeys * 2;              // 16 KB per P part
+constexpr int kPBuf = 2 * kPBytes;                      // rounded + residual
 constexpr int kOffQ = 0;
 constexpr int kOffRing = kOffQ + kQBytes;
-constexpr int kOffP = kOffRing + kStages * kStageBytes;  // hi, then lo
-constexpr int kOffBars = kOffP + 2 * kPBytes;
-// barriers: q_full, kv_full[S], kv_empty[S], s_full, s_free, p_full, o_ready,
-// done, then the tensor-memory base address word.
-constexpr int kNumBars = 1 + 2 * kStages + 5;
+constexpr int kOffP = kOffRing + kStages * kStageBytes;  // 2 P buffers
+constexpr int kOffBars = kOffP + 2 * kPBuf;
+// barriers: q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2],
+// p_full[2], o_ready[2], done, then the tensor-memory base address word.
+constexpr int kNumBars = 1 + 2 * kStages + 4 * 2 + 1;
 constexpr int kOffTable = kOffBars + kNumBars * 8 + 16;
 
 size_t prefill_smem_bytes(int max_pages) {
@@ -112,11 +119,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t q_full = bars;
   const uint32_t kv_full0 = bars + 8;
   const uint32_t kv_empty0 = kv_full0 + kStages * 8;
-  const uint32_t s_full = kv_empty0 + kStages * 8;
-  const uint32_t s_free = s_full + 8;
-  const uint32_t p_full = s_free + 8;
-  const uint32_t o_ready = p_full + 8;
-  const uint32_t done = o_ready + 8;
+  // Double-buffer barriers: tile t uses element t & 1, phase t >> 1.
+  const uint32_t s_full0 = kv_empty0 + kStages * 8;
+  const uint32_t s_free0 = s_full0 + 16;
+  const uint32_t p_full0 = s_free0 + 16;
+  const uint32_t o_ready0 = p_full0 + 16;
+  const uint32_t done = o_ready0 + 16;
   uint32_t* tmem_slot =
       reinterpret_cast<uint32_t*>(smem + kOffBars + kNumBars * 8);
   int32_t* bt_s = reinterpret_cast<int32_t*>(smem + kOffTable);
@@ -159,10 +167,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_init(kv_full0 + 8 * s, 1);
       dev::mbar_init(kv_empty0 + 8 * s, 1);
     }
-    dev::mbar_init(s_full, 1);
-    dev::mbar_init(s_free, 4);
-    dev::mbar_init(p_full, 4);
-    dev::mbar_init(o_ready, 1);
+    for (int i = 0; i < 2; ++i) {
+      dev::mbar_init(s_full0 + 8 * i, 1);
+      dev::mbar_init(s_free0 + 8 * i, 4);
+      dev::mbar_init(p_full0 + 8 * i, 4);
+      dev::mbar_init(o_ready0 + 8 * i, 1);
+    }
     dev::mbar_init(done, 4);
     dev::fence_mbar_init();
   }
@@ -179,8 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   dev::tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t s_tmem = tbase;        // columns [0, 64)
-  const uint32_t o_tmem = tbase + 128;  // columns [128, 256)
+  const uint32_t s_tmem = tbase;        // S buffers: columns [0, 64), [64, 128)
+  const uint32_t o_tmem = tbase + 128;  // O: columns [128, 256)
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -228,15 +238,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_pv = dev::umma_idesc_f16(kBf16, kRows, kD,
                                                         false, true);
       auto issue_pv = [&](int t) -> bool {
-        if (!dev::mbar_wait(p_full, t & 1)) return false;
+        if (!dev::mbar_wait(p_full0 + 8 * (t & 1), (t >> 1) & 1)) return false;
         dev::tc_fence_after();
         const uint32_t vt = ring + (t % kStages) * kStageBytes + kKVTile;
+        const uint32_t pb = p_s + (t & 1) * kPBuf;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {  // P rounded part, residual
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk) {
             const uint64_t ad =
-                dev::sw128_desc(p_s + part * kPBytes + kk * 32, 16, 1024);
+                dev::sw128_desc(pb + part * kPBytes + kk * 32, 16, 1024);
             // V as the MN-major B operand: 64-wide d halves kTileHalf apart,
             // 8-key groups 1024 bytes apart.
             const uint64_t bd =
@@ -245,20 +256,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                           (t > 0 || part > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        dev::umma_commit(o_ready);
+        dev::umma_commit(o_ready0 + 8 * (t & 1));
         dev::umma_commit(kv_empty0 + 8 * (t % kStages));
         return true;
       };
       ok = dev::mbar_wait(q_full, 0);
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int s = j % kStages;
+        // S buffer j & 1 is free once the softmax warps have read S(j-2).
         if (!dev::mbar_wait(kv_full0 + 8 * s, (j / kStages) & 1) ||
-            (j >= 1 && !dev::mbar_wait(s_free, (j - 1) & 1))) {
+            (j >= 2 &&
+             !dev::mbar_wait(s_free0 + 8 * (j & 1), ((j >> 1) - 1) & 1))) {
           ok = false;
           break;
         }
         dev::tc_fence_after();
         const uint32_t kt = ring + s * kStageBytes;
+        const uint32_t sd = s_tmem + (j & 1) * kKeys;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const int h = kk >> 2, k4 = kk & 3;
@@ -266,16 +280,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                                               1024);
           const uint64_t bd = dev::sw128_desc(kt + h * kTileHalf + k4 * 32,
                                               16, 1024);
-          dev::umma_f16(s_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          dev::umma_f16(sd, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        dev::umma_commit(s_full);
+        dev::umma_commit(s_full0 + 8 * (j & 1));
         if (j >= 1 && !issue_pv(j - 1)) {
           ok = false;
           break;
         }
       }
-      if (ok) ok = issue_pv(n_tiles - 1);
-      if (ok) ok = dev::mbar_wait(o_ready, (n_tiles - 1) & 1);
+      const int last = n_tiles - 1;
+      if (ok) ok = issue_pv(last);
+      if (ok) ok = dev::mbar_wait(o_ready0 + 8 * (last & 1), (last >> 1) & 1);
       if (!ok) dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
       // Release tensor memory only after the softmax warps are done with it.
       if (!dev::mbar_wait(done, 0)) dev::set_error(a.dev_err,
@@ -297,26 +312,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool valid = t_loc < n_q;
   // Padding rows (no query) see every key the tile loads; never stored.
   const int qpos = valid ? L - q_len + tok : kv_end - 1;
+  const float c = a.scale_log2;
   float m_ref = -INFINITY, l = 0.f;
   bool ok = true;
   // Wait results are made warp-uniform: the tcgen05 loads and stores below
   // are warp-collective.
+  auto wait_pv = [&](int t) {  // P(t).V has completed
+    return __all_sync(0xffffffffu, dev::mbar_wait(o_ready0 + 8 * (t & 1),
+                                                  (t >> 1) & 1));
+  };
   for (int j = 0; j < n_tiles && ok; ++j) {
-    ok = __all_sync(0xffffffffu, dev::mbar_wait(s_full, j & 1));
+    ok = __all_sync(0xffffffffu,
+                    dev::mbar_wait(s_full0 + 8 * (j & 1), (j >> 1) & 1));
     if (!ok) break;
     dev::tc_fence_after();
     float sv[kKeys];
     {
+      const uint32_t sa = s_tmem + (j & 1) * kKeys + lane_off;
       float (&lo)[32] = *reinterpret_cast<float(*)[32]>(sv);
       float (&hi)[32] = *reinterpret_cast<float(*)[32]>(sv + 32);
-      dev::tmem_ld32(s_tmem + lane_off, lo);
-      dev::tmem_ld32(s_tmem + lane_off + 32, hi);
+      dev::tmem_ld32(sa, lo);
+      dev::tmem_ld32(sa + 32, hi);
       dev::tmem_ld_wait();
     }
     dev::tc_fence_before();
     __syncwarp();
-    if (lane == 0) dev::mbar_arrive(s_free);
-    float mx = -INFINITY;
+    if (lane == 0) dev::mbar_arrive(s_free0 + 8 * (j & 1));
     const int k0 = j * kKeys;
     if (k0 + kKeys > L) {
       // Keys past the context get P = 0, but 0 * NaN is NaN in the MMA:
@@ -324,24 +345,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // past it).  Warp q clears rows 16q .. 16q+15 of the last tile.
       const uint32_t vt = ring + (j % kStages) * kStageBytes + kKVTile;
       for (int idx = lane; idx < 16 * 16; idx += 32) {
-        const int krow = quarter * 16 + (idx >> 4), c = idx & 15;
+        const int krow = quarter * 16 + (idx >> 4), ch = idx & 15;
         if (k0 + krow >= L)
-          dev::st_shared_zero16(vt + (c >> 3) * kTileHalf + krow * 128 +
-                                (c & 7) * 16);
+          dev::st_shared_zero16(vt + (ch >> 3) * kTileHalf + krow * 128 +
+                                (ch & 7) * 16);
       }
     }
+    // Causal mask: only tiles that reach past this row's position.
+    const int lim = qpos - k0;
+    if (lim < kKeys - 1) {
 #pragma unroll
-    for (int c = 0; c < kKeys; ++c) {
-      const float x = (k0 + c <= qpos) ? sv[c] * a.scale_log2 : -INFINITY;
-      sv[c] = x;
-      mx = fmaxf(mx, x);
+      for (int k = 0; k < kKeys; ++k)
+        if (k > lim) sv[k] = -INFINITY;
     }
-    // P smem and O are busy until the previous P.V has finished.
-    if (j >= 1) {
-      ok = __all_sync(0xffffffffu, dev::mbar_wait(o_ready, (j - 1) & 1));
-      if (!ok) break;
-    }
-    dev::tc_fence_after();
+    float mx = sv[0];
+#pragma unroll
+    for (int k = 1; k < kKeys; ++k) mx = fmaxf(mx, sv[k]);
+    mx *= c;  // the scale is positive: max commutes with it
     float factor = 1.f;
     if (j == 0) {
       m_ref = mx;  // O is still empty: the first P.V overwrites it
@@ -350,35 +370,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       m_ref = mx;
       l *= factor;
     }
-    if (__any_sync(0xffffffffu, factor != 1.f)) {
+    // P = 2^(s * c - m_ref), before waiting for the tensor cores.
 #pragma unroll
-      for (int c = 0; c < kD; c += 32) {
+    for (int k = 0; k < kKeys; ++k) {
+      sv[k] = dev::fast_exp2(fmaf(sv[k], c, -m_ref));
+      l += sv[k];
+    }
+    if (__any_sync(0xffffffffu, factor != 1.f)) {
+      // O must hold P(j-1).V before it is rescaled (P(j).V is not issued
+      // until this warp arrives on p_full below).
+      ok = wait_pv(j - 1);
+      if (!ok) break;
+      dev::tc_fence_after();
+#pragma unroll
+      for (int col = 0; col < kD; col += 32) {
         float ov[32];
-        dev::tmem_ld32(o_tmem + lane_off + c, ov);
+        dev::tmem_ld32(o_tmem + lane_off + col, ov);
         dev::tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) ov[e] *= factor;
-        dev::tmem_st32(o_tmem + lane_off + c, ov);
+        dev::tmem_st32(o_tmem + lane_off + col, ov);
       }
       dev::tmem_st_wait();
     }
-    // P = 2^(s - m_ref) as a rounded part plus its residual, row r of the
-    // K-major 128-byte-swizzled A operand (16-byte chunk c at c ^ (r % 8)).
-    uint8_t* prow_hi = smem + kOffP + r * 128;
+    // P buffer j & 1 was last read by P(j-2).V.
+    if (j >= 2) {
+      ok = wait_pv(j - 2);
+      if (!ok) break;
+    }
+    // Row r of the K-major 128-byte-swizzled A operand (16-byte chunk ch at
+    // ch ^ (r % 8)): rounded part, then the residual.
+    uint8_t* prow_hi = smem + kOffP + (j & 1) * kPBuf + r * 128;
     uint8_t* prow_lo = prow_hi + kPBytes;
 #pragma unroll
-    for (int c = 0; c < kKeys / 8; ++c) {
+    for (int ch = 0; ch < kKeys / 8; ++ch) {
       uint32_t hw[4], lw[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float p0 = dev::fast_exp2(sv[8 * c + 2 * e] - m_ref);
-        const float p1 = dev::fast_exp2(sv[8 * c + 2 * e + 1] - m_ref);
-        l += p0 + p1;
+        const float p0 = sv[8 * ch + 2 * e], p1 = sv[8 * ch + 2 * e + 1];
         hw[e] = M::pack(p0, p1);
         const float2 hf = M::unpack(hw[e]);
         lw[e] = M::pack(p0 - hf.x, p1 - hf.y);
       }
-      const int sw = (c ^ (r & 7)) * 16;
+      const int sw = (ch ^ (r & 7)) * 16;
       *reinterpret_cast<uint4*>(prow_hi + sw) =
           make_uint4(hw[0], hw[1], hw[2], hw[3]);
       *reinterpret_cast<uint4*>(prow_lo + sw) =
@@ -387,11 +421,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     dev::fence_proxy_async_smem();
     dev::tc_fence_before();
     __syncwarp();
-    if (lane == 0) dev::mbar_arrive(p_full);
+    if (lane == 0) dev::mbar_arrive(p_full0 + 8 * (j & 1));
   }
   // Epilogue: O / l -> out[token, query head].
-  if (ok) ok = __all_sync(0xffffffffu,
-                          dev::mbar_wait(o_ready, (n_tiles - 1) & 1));
+  if (ok) ok = wait_pv(n_tiles - 1);
   if (ok) {
     dev::tc_fence_after();
     const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -399,9 +432,9 @@ __global__ void __launch_bounds__(kThreads, 1)
              (static_cast<int64_t>(q0 + tok) * a.num_q_heads + kvh * G + g) *
                  kD;
 #pragma unroll
-    for (int c = 0; c < kD; c += 32) {
+    for (int col = 0; col < kD; col += 32) {
       float ov[32];
-      dev::tmem_ld32(o_tmem + lane_off + c, ov);
+      dev::tmem_ld32(o_tmem + lane_off + col, ov);
       dev::tmem_ld_wait();
       if (valid) {
 #pragma unroll
@@ -411,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           w.y = M::pack(ov[e + 2] * inv, ov[e + 3] * inv);
           w.z = M::pack(ov[e + 4] * inv, ov[e + 5] * inv);
           w.w = M::pack(ov[e + 6] * inv, ov[e + 7] * inv);
-          *reinterpret_cast<uint4*>(dst + c + e) = w;
+          *reinterpret_cast<uint4*>(dst + col + e) = w;
         }
       }
     }

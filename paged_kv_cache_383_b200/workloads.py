@@ -283,6 +283,13 @@ def make_prefill(w: Workload, q_lens, device="cpu",
     return PrefillInputs(inp, q_lens, start, q)
 
 
+# Prefill workloads (tensor-core bound): Llama-3-70B heads, block 16, bf16.
+# chunked: the last 512 tokens of 16 contexts uniform in [2048, 8192]
+# (a chunk of a long prompt appended to what is cached); prompt: 8 whole
+# prompts uniform in [1024, 8192] (every token new).
 WORKLOADS["chunked_prefill_gqa8"] = Workload(
     "chunked_prefill_gqa8", 383006, 16, 64, 8, 128, 16, "bfloat16",
     "uniform", low=2048, high=8192)
+WORKLOADS["prompt_prefill_gqa8"] = Workload(
+    "prompt_prefill_gqa8", 383007, 8, 64, 8, 128, 16, "bfloat16",
+    "uniform", low=1024, high=8192)
