@@ -540,6 +540,7 @@ def extras(args, w, inp, dev, pkv, bt, cl):
     from paged_kv_cache_383_b200 import workloads as wl
     out["prefill"] = [time_prefill(pkv, wl, n, c, dev)
                       for n, c in PREFILL_CASES]
+    out["prefix_cache"] = prefix_cache_measure(pkv, dev)
     return out
 
 
@@ -611,6 +612,74 @@ def time_prefill(pkv, wl, name, chunk, dev, iters=10):
                     "cores do 1.5x the algorithmic FLOPs"}
 
 
+def prefix_cache_measure(pkv, dev, requests=128, prompt_len=2048,
+                         q_low=64, q_high=512, seed=383009):
+    """A shared system prompt: ``requests`` requests of one 2048-token prompt
+    plus a question of U[64, 512] tokens (Llama-3-70B heads, block 16,
+    bf16).  Host: microseconds per request of match + append + cache insert
+    through the C ABI.  GPU: one pa_prefill over the whole batch when every
+    request prefills its full prompt, against the suffix-only prefill the
+    cache leaves (the tokens of the first request's prompt are computed
+    once, in an earlier pass that is not timed).  Also the blocks held."""
+    import time
+    import torch
+    bs, hq, hkv, d = 16, 64, 8, 128
+    rng = np.random.default_rng(seed)
+    qlens = rng.integers(q_low, q_high + 1, size=requests)
+    prompt = np.arange(prompt_len, dtype=np.int32) + 1_000_000
+    toks = [np.concatenate([prompt, rng.integers(0, 100_000, size=n)
+                            .astype(np.int32)]) for n in qlens]
+    need = int(sum(-(-len(t) // bs) for t in toks))
+    bm = pkv.BlockManager(need + 64, bs)
+    hits = np.zeros(requests, dtype=np.int64)
+    t0 = time.perf_counter()
+    for r in range(requests):
+        bm.add_seq(r)
+        hits[r] = bm.match_prefix(r, toks[r])
+        bm.append(r, len(toks[r]) - int(hits[r]))
+        bm.cache_insert(r, toks[r])
+    host_us = (time.perf_counter() - t0) / requests * 1e6
+    blocks_cached = need + 64 - bm.num_free()
+    max_blocks = max(-(-len(t) // bs) for t in toks)
+    table, lens = bm.block_table(list(range(requests)), max_blocks)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    shape = (need + 64, hkv, bs, d)
+    kc = torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+    vc = torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+    bt = torch.from_numpy(table).to(dev)
+    cl = torch.from_numpy(lens).to(dev)
+    res = {"requests": requests, "prompt_tokens": prompt_len,
+           "question_tokens_mean": float(qlens.mean()),
+           "host_us_per_request": round(host_us, 2),
+           "blocks_with_cache": int(blocks_cached), "blocks_without": need,
+           "matched_tokens_mean": float(hits[1:].mean())}
+    for mode, q_lens in (("full", lens.astype(np.int64)),
+                         ("cached", lens.astype(np.int64) - hits)):
+        qs = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+        q = torch.randn(int(qs[-1]), hq, d, generator=g,
+                        device=dev).to(torch.bfloat16)
+        out = torch.empty_like(q)
+        qsd = torch.from_numpy(qs).to(dev)
+        kw = dict(max_q_len=int(q_lens.max()),
+                  max_context_len=int(lens.max()))
+        for _ in range(2):
+            pkv.pa_prefill(out, q, kc, vc, bt, cl, qsd, d ** -0.5, **kw)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(5):
+            pkv.pa_prefill(out, q, kc, vc, bt, cl, qsd, d ** -0.5, **kw)
+        b.record()
+        torch.cuda.synchronize()
+        res[f"prefill_ms_{mode}"] = round(a.elapsed_time(b) / 5, 3)
+        res[f"prefill_tokens_{mode}"] = int(qs[-1])
+    res["prefill_speedup"] = round(res["prefill_ms_full"] /
+                                   res["prefill_ms_cached"], 2)
+    bm.close()
+    return res
+
+
 def run_prefill_only(args):
     import torch
     import paged_kv_cache_383_b200 as pkv
@@ -621,6 +690,7 @@ def run_prefill_only(args):
            for n, c in PREFILL_CASES]
     return {"metric": "prefill attention TFLOP/s (algorithmic)",
             "unit": "TFLOP/s", "cases": res,
+            "prefix_cache": prefix_cache_measure(pkv, dev),
             "gpu_launches": pkv.pa_launch_count()}
 
 

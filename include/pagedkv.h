@@ -340,6 +340,56 @@ pa_status pa_bm_block_table(void* bm, const int64_t* seq_ids, int n,
                             int max_blocks, int32_t* table_out,
                             int32_t* lens_out);
 
+/* ---- Prefix cache ([KV-cache chapter] "RadixAttention: caching, not just
+ * packing, the prefix") ------------------------------------------------------
+ * Cached token sequences form a radix tree with one node per FULL block,
+ * keyed by that block's block_size tokens under its parent; the partly filled
+ * last block of a sequence is never cached.  The cache holds one reference
+ * on every block it stores (pa_bm_refcount counts it).  A cached block that
+ * only the cache references and that has no cached children is an evictable
+ * leaf.  A logical clock stamps every node on the path of each match and
+ * insert; when pa_bm_append / pa_bm_append_batch need more blocks than the
+ * pool has free, evictable leaves are evicted oldest stamp first (a parent
+ * can become an evictable leaf in turn).  If even evicting all of them would
+ * not supply the append, the append fails with PA_ERR_NO_FREE_BLOCKS and the
+ * cache is left exactly as it was.  Blocks a sequence uses are never
+ * evicted.  Token ids are opaque int32 values compared for equality. */
+
+/* Attach to the new, EMPTY sequence seq_id the longest run of cached full
+ * blocks that starts tokens[0 .. n_tokens) (host int32): those blocks are
+ * referenced, not copied, and the sequence's length becomes *matched_out,
+ * a multiple of block_size.  Only tokens past it need a prefill; append them
+ * with pa_bm_append (which opens a fresh block: no copy-on-write).
+ * INVALID_ARG if the sequence is unknown or not empty. */
+pa_status pa_bm_match_prefix(void* bm, int64_t seq_id, const int32_t* tokens,
+                             int64_t n_tokens, int64_t* matched_out);
+
+/* Cache the full blocks among the first n_tokens tokens of seq_id, whose
+ * token ids are tokens[0 .. n_tokens) (host int32; n_tokens <= the
+ * sequence's length).  Call it once their K/V are written.  A block whose
+ * tokens are already cached at that place keeps the cached node (the
+ * sequence's duplicate stays outside the cache).  INVALID_ARG, changing
+ * nothing, if one of the sequence's blocks is cached under different
+ * tokens. */
+pa_status pa_bm_cache_insert(void* bm, int64_t seq_id, const int32_t* tokens,
+                             int64_t n_tokens);
+
+/* Evict up to max_blocks evictable leaves, oldest stamp first; their blocks
+ * return to the pool.  *evicted_out = how many. */
+pa_status pa_bm_cache_evict(void* bm, int max_blocks, int* evicted_out);
+
+/* Number of cached blocks (-1 for a NULL handle). */
+int pa_bm_num_cached(void* bm);
+
+/* Dump the tree breadth-first (every parent before its children):
+ * parent_out[i] = index of node i's parent in this dump (-1 under the root),
+ * block_out[i] = its physical block, tokens_out[i * block_size ..] = its
+ * tokens (host arrays sized max_nodes, max_nodes * block_size).  INVALID_ARG
+ * if more than max_nodes blocks are cached. */
+pa_status pa_bm_cache_nodes(void* bm, int max_nodes, int32_t* parent_out,
+                            int32_t* block_out, int32_t* tokens_out,
+                            int* n_out);
+
 /* Kernel launches this library has issued in this process (all devices,
  * all threads): lets a caller count the GPU work a timed region contained. */
 int64_t pa_launch_count(void);

@@ -392,3 +392,61 @@ class BlockManager:
 
     def num_seq_blocks(self, seq_id: int) -> int:
         return self._lib.pa_bm_num_seq_blocks(self._h, seq_id)
+
+    # -- prefix cache -------------------------------------------------------
+    def match_prefix(self, seq_id: int, tokens) -> int:
+        """Attach the longest cached run of full blocks that starts
+        ``tokens`` to the new, empty ``seq_id``; returns the tokens matched
+        (only the rest needs a prefill)."""
+        import numpy as np
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        out = ctypes.c_int64(0)
+        _lib.check(self._lib.pa_bm_match_prefix(
+            self._h, seq_id, t.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+            len(t), ctypes.byref(out)), "pa_bm_match_prefix")
+        return out.value
+
+    def cache_insert(self, seq_id: int, tokens):
+        """Cache the full blocks of the first len(tokens) tokens of
+        ``seq_id`` (call once their K/V are written)."""
+        import numpy as np
+        t = np.ascontiguousarray(tokens, dtype=np.int32)
+        _lib.check(self._lib.pa_bm_cache_insert(
+            self._h, seq_id, t.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+            len(t)), "pa_bm_cache_insert")
+
+    def cache_evict(self, max_blocks: int) -> int:
+        out = ctypes.c_int(0)
+        _lib.check(self._lib.pa_bm_cache_evict(self._h, max_blocks,
+                                               ctypes.byref(out)),
+                   "pa_bm_cache_evict")
+        return out.value
+
+    def num_cached(self) -> int:
+        return self._lib.pa_bm_num_cached(self._h)
+
+    def cache_nodes(self):
+        """The cached tree as (parent_index int32 [n], block int32 [n],
+        tokens int32 [n, block_size]), parents before children."""
+        import numpy as np
+        n = max(self.num_cached(), 0)
+        parent = np.empty(max(n, 1), dtype=np.int32)
+        block = np.empty(max(n, 1), dtype=np.int32)
+        toks = np.empty((max(n, 1), self.block_size), dtype=np.int32)
+        got = ctypes.c_int(0)
+        p32 = ctypes.POINTER(ctypes.c_int32)
+        _lib.check(self._lib.pa_bm_cache_nodes(
+            self._h, n, parent.ctypes.data_as(p32), block.ctypes.data_as(p32),
+            toks.ctypes.data_as(p32), ctypes.byref(got)), "pa_bm_cache_nodes")
+        k = got.value
+        return parent[:k], block[:k], toks[:k]
+
+    def cached_paths(self):
+        """Every cached block as the tuple of its token keys from the root
+        (the same form as the oracle model's ``cached_paths``)."""
+        parent, _, toks = self.cache_nodes()
+        paths = []
+        for i in range(len(parent)):
+            key = tuple(int(t) for t in toks[i])
+            paths.append((key,) if parent[i] < 0 else paths[parent[i]] + (key,))
+        return set(paths)

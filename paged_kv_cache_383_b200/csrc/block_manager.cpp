@@ -1,5 +1,5 @@
 // Host block manager: free pool, per-sequence block tables, reference counts,
-// fork and copy-on-write.
+// fork, copy-on-write, and a radix-tree prefix cache.
 //
 // Semantics follow [Taming the Tail] "How the Architecture Works" (free block
 // pool; a new block only when the last one is full), [vLLM PagedAttention FAQ]
@@ -8,14 +8,32 @@
 // memory..." and answer A6 (reference counts; a block rejoins the pool only at
 // count zero; a private copy before the first write into a shared block).
 //
+// Prefix cache ([KV-cache chapter] "RadixAttention: caching, not just packing,
+// the prefix"): cached token sequences form a tree with one node per full
+// block, keyed by that block's tokens under its parent.  A request walks the
+// tree and references every matched block instead of recomputing it.  The
+// cache holds one reference per cached block; a cached block that only the
+// cache references and that has no cached children is an evictable leaf.
+// When an append needs more blocks than the pool has, evictable leaves go
+// least recently used first (a logical clock stamps each match / insert
+// walk), and a leaf's parent may become evictable in turn.  Reference counts
+// keep every block a sequence still uses out of reach.
+//
 // Design: everything is flat integer arrays.  The pool is a LIFO stack so a
 // block freed a moment ago (likely still in L2) is reused first; the first
 // fill follows the caller's free_order.  Appends are all-or-nothing: the
-// number of blocks an append needs is computed before anything changes.
+// number of blocks an append needs is computed before anything changes, and
+// an append that eviction cannot satisfy puts back what it evicted.  Cache
+// nodes live in one array; children are found through a hash map keyed by
+// (parent node, block tokens); evictable leaves sit in an ordered set by
+// stamp, kept current whenever a count, a stamp or a child count changes.
 #include <cstdint>
+#include <cstring>
 #include <limits>
 #include <new>
+#include <set>
 #include <unordered_map>
+#include <utility>
 #include <vector>
 
 #include "pagedkv.h"
@@ -29,12 +47,48 @@ struct Sequence {
   int64_t len = 0;              // tokens stored
 };
 
+struct Node {
+  int32_t block = -1;   // -1: the root, or a released node
+  int32_t parent = -1;
+  int32_t n_children = 0;
+  int64_t last = 0;     // stamp of the last walk through this node
+  uint64_t hash = 0;    // of (parent, tokens)
+  bool in_lru = false;
+  int64_t lru_stamp = 0;
+  std::vector<int32_t> tokens;
+};
+
+uint64_t mix(uint64_t h, uint64_t v) {
+  // splitmix64 finaliser over the running value
+  h ^= v + 0x9e3779b97f4a7c15ull + (h << 6) + (h >> 2);
+  h ^= h >> 30;
+  h *= 0xbf58476d1ce4e5b9ull;
+  h ^= h >> 27;
+  h *= 0x94d049bb133111ebull;
+  return h ^ (h >> 31);
+}
+
+uint64_t key_hash(int32_t parent, const int32_t* tokens, int n) {
+  uint64_t h = mix(0x2545f4914f6cdd1dull, static_cast<uint32_t>(parent));
+  for (int i = 0; i < n; ++i) h = mix(h, static_cast<uint32_t>(tokens[i]));
+  return h;
+}
+
 struct BlockManager {
   int num_blocks = 0;
   int block_size = 0;
   std::vector<int32_t> free_stack;  // top = back()
-  std::vector<int32_t> ref;         // tables pointing at each block
+  std::vector<int32_t> ref;         // tables (+1 if cached) per block
   std::unordered_map<int64_t, Sequence> seqs;
+
+  // prefix cache
+  std::vector<Node> nodes{Node{}};  // [0] = root
+  std::vector<int32_t> free_nodes;
+  std::vector<int32_t> node_of;     // block -> cache node or -1
+  std::unordered_multimap<uint64_t, int32_t> children;
+  std::set<std::pair<int64_t, int32_t>> lru;  // evictable leaves by stamp
+  int64_t clock = 0;
+  int num_cached = 0;
 
   int32_t take() {
     int32_t b = free_stack.back();
@@ -43,10 +97,130 @@ struct BlockManager {
     return b;
   }
   void drop(int32_t b) {
-    if (--ref[b] == 0) free_stack.push_back(b);
+    if (--ref[b] == 0)
+      free_stack.push_back(b);
+    else if (node_of[b] >= 0)
+      refresh(node_of[b]);
+  }
+  void add_ref(int32_t b) {
+    ++ref[b];
+    if (node_of[b] >= 0) refresh(node_of[b]);
   }
   int64_t blocks_for(int64_t len) const {
     return (len + block_size - 1) / block_size;
+  }
+
+  // Keep node n's membership of the evictable-leaf set current.
+  void refresh(int32_t n) {
+    Node& x = nodes[n];
+    const bool want = x.block >= 0 && x.n_children == 0 && ref[x.block] == 1;
+    if (x.in_lru && (!want || x.lru_stamp != x.last)) {
+      lru.erase({x.lru_stamp, n});
+      x.in_lru = false;
+    }
+    if (want && !x.in_lru) {
+      lru.insert({x.last, n});
+      x.lru_stamp = x.last;
+      x.in_lru = true;
+    }
+  }
+  void touch(int32_t n, int64_t now) {
+    nodes[n].last = now;
+    refresh(n);
+  }
+
+  int32_t find_child(int32_t parent, const int32_t* tokens) const {
+    const uint64_t h = key_hash(parent, tokens, block_size);
+    auto range = children.equal_range(h);
+    for (auto it = range.first; it != range.second; ++it) {
+      const Node& c = nodes[it->second];
+      if (c.parent == parent &&
+          std::memcmp(c.tokens.data(), tokens, sizeof(int32_t) * block_size) ==
+              0)
+        return it->second;
+    }
+    return -1;
+  }
+
+  // New node for block b (the cache takes a reference) under parent.
+  int32_t add_node(int32_t parent, const int32_t* tokens, int32_t b,
+                   int64_t now) {
+    int32_t n;
+    if (!free_nodes.empty()) {
+      n = free_nodes.back();
+      free_nodes.pop_back();
+    } else {
+      n = static_cast<int32_t>(nodes.size());
+      nodes.emplace_back();
+    }
+    Node& x = nodes[n];
+    x.block = b;
+    x.parent = parent;
+    x.n_children = 0;
+    x.last = now;
+    x.in_lru = false;
+    x.tokens.assign(tokens, tokens + block_size);
+    x.hash = key_hash(parent, tokens, block_size);
+    children.emplace(x.hash, n);
+    ++nodes[parent].n_children;
+    if (parent != 0) refresh(parent);
+    node_of[b] = n;
+    ++num_cached;
+    add_ref(b);
+    return n;
+  }
+
+  // Remove evictable leaf n from the tree; its block returns to the pool.
+  // The node keeps its fields so relink() can undo this.
+  void unlink(int32_t n) {
+    Node& x = nodes[n];
+    lru.erase({x.lru_stamp, n});
+    x.in_lru = false;
+    auto range = children.equal_range(x.hash);
+    for (auto it = range.first; it != range.second; ++it)
+      if (it->second == n) {
+        children.erase(it);
+        break;
+      }
+    --nodes[x.parent].n_children;
+    if (x.parent != 0) refresh(x.parent);
+    node_of[x.block] = -1;
+    --num_cached;
+    drop(x.block);  // 1 -> 0: back to the pool
+  }
+  void relink(int32_t n) {  // exact inverse of the last unlink()
+    Node& x = nodes[n];
+    free_stack.pop_back();  // x.block, pushed by unlink
+    ref[x.block] = 1;
+    node_of[x.block] = n;
+    ++num_cached;
+    children.emplace(x.hash, n);
+    ++nodes[x.parent].n_children;
+    if (x.parent != 0) refresh(x.parent);
+    refresh(n);
+  }
+  void release_node(int32_t n) {
+    nodes[n].block = -1;
+    nodes[n].tokens.clear();
+    free_nodes.push_back(n);
+  }
+
+  // Make at least `need` blocks free by evicting leaves, oldest first.  All
+  // or nothing: if the cache cannot supply enough, nothing is evicted.
+  bool ensure_free(int64_t need) {
+    if (need <= static_cast<int64_t>(free_stack.size())) return true;
+    std::vector<int32_t> evicted;
+    while (static_cast<int64_t>(free_stack.size()) < need && !lru.empty()) {
+      const int32_t n = lru.begin()->second;
+      unlink(n);
+      evicted.push_back(n);
+    }
+    if (static_cast<int64_t>(free_stack.size()) >= need) {
+      for (int32_t n : evicted) release_node(n);
+      return true;
+    }
+    for (auto it = evicted.rbegin(); it != evicted.rend(); ++it) relink(*it);
+    return false;
   }
 };
 
@@ -56,6 +230,7 @@ BlockManager* as_bm(void* p) { return static_cast<BlockManager*>(p); }
 }  // namespace pagedkv
 
 using pagedkv::BlockManager;
+using pagedkv::Node;
 using pagedkv::Sequence;
 using pagedkv::as_bm;
 using pagedkv::fail;
@@ -76,6 +251,7 @@ pa_status pa_bm_create(int num_blocks, int block_size,
   bm->num_blocks = num_blocks;
   bm->block_size = block_size;
   bm->ref.assign(num_blocks, 0);
+  bm->node_of.assign(num_blocks, -1);
   bm->free_stack.resize(num_blocks);
   if (free_order) {
     std::vector<uint8_t> seen(num_blocks, 0);
@@ -122,7 +298,7 @@ pa_status pa_bm_fork(void* p, int64_t parent_id, int64_t child_id) {
     return fail(PA_ERR_INVALID_ARG, "pa_bm_fork: child %lld exists",
                 static_cast<long long>(child_id));
   Sequence child = it->second;  // copy of table and length
-  for (int32_t b : child.blocks) ++bm->ref[b];
+  for (int32_t b : child.blocks) bm->add_ref(b);
   bm->seqs.emplace(child_id, std::move(child));
   return PA_OK;
 }
@@ -157,11 +333,12 @@ pa_status pa_bm_append(void* p, int64_t seq_id, int n_tokens,
     return fail(PA_ERR_INVALID_ARG,
                 "pa_bm_append: sequence %lld needs a copy-on-write pair but "
                 "max_cow=%d", static_cast<long long>(seq_id), max_cow);
-  if (need > static_cast<int64_t>(bm->free_stack.size()))
+  if (!bm->ensure_free(need))
     return fail(PA_ERR_NO_FREE_BLOCKS,
-                "pa_bm_append: sequence %lld needs %lld blocks, %zu free",
+                "pa_bm_append: sequence %lld needs %lld blocks, %zu free "
+                "after evicting every evictable cached block",
                 static_cast<long long>(seq_id), static_cast<long long>(need),
-                bm->free_stack.size());
+                bm->free_stack.size() + bm->lru.size());
 
   if (shared_partial) {  // private copy of the shared, partly filled block
     int32_t src = s.blocks.back();
@@ -297,6 +474,149 @@ int pa_bm_num_seq_blocks(void* p, int64_t seq_id) {
   if (!bm) return -1;
   auto it = bm->seqs.find(seq_id);
   return it == bm->seqs.end() ? -1 : static_cast<int>(it->second.blocks.size());
+}
+
+pa_status pa_bm_match_prefix(void* p, int64_t seq_id, const int32_t* tokens,
+                             int64_t n_tokens, int64_t* matched_out) {
+  pagedkv::clear_error();
+  BlockManager* bm = as_bm(p);
+  if (!bm || n_tokens < 0 || (n_tokens > 0 && !tokens) || !matched_out)
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_match_prefix: bad arguments");
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end())
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_match_prefix: no sequence %lld",
+                static_cast<long long>(seq_id));
+  Sequence& s = it->second;
+  if (s.len != 0 || !s.blocks.empty())
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_bm_match_prefix: sequence %lld is not empty",
+                static_cast<long long>(seq_id));
+  const int bs = bm->block_size;
+  const int64_t now = ++bm->clock;
+  int32_t node = 0;
+  for (int64_t i = 0; i < n_tokens / bs; ++i) {
+    const int32_t c = bm->find_child(node, tokens + i * bs);
+    if (c < 0) break;
+    bm->touch(c, now);
+    s.blocks.push_back(bm->nodes[c].block);
+    bm->add_ref(bm->nodes[c].block);
+    node = c;
+  }
+  s.len = static_cast<int64_t>(s.blocks.size()) * bs;
+  *matched_out = s.len;
+  return PA_OK;
+}
+
+pa_status pa_bm_cache_insert(void* p, int64_t seq_id, const int32_t* tokens,
+                             int64_t n_tokens) {
+  pagedkv::clear_error();
+  BlockManager* bm = as_bm(p);
+  if (!bm || n_tokens < 0 || (n_tokens > 0 && !tokens))
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_cache_insert: bad arguments");
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end())
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_cache_insert: no sequence %lld",
+                static_cast<long long>(seq_id));
+  const Sequence& s = it->second;
+  if (n_tokens > s.len)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_bm_cache_insert: %lld tokens, sequence %lld holds %lld",
+                static_cast<long long>(n_tokens),
+                static_cast<long long>(seq_id), static_cast<long long>(s.len));
+  const int bs = bm->block_size;
+  const int64_t n_full = n_tokens / bs;
+  // Check first, so a refused insert changes nothing: a block may sit in the
+  // tree only under its own tokens.
+  int32_t node = 0;
+  bool creating = false;
+  for (int64_t i = 0; i < n_full; ++i) {
+    const int32_t c = creating ? -1 : bm->find_child(node, tokens + i * bs);
+    const int32_t placed = bm->node_of[s.blocks[i]];
+    if (c < 0) {
+      creating = true;
+      if (placed >= 0)
+        return fail(PA_ERR_INVALID_ARG,
+                    "pa_bm_cache_insert: block %d of sequence %lld is cached "
+                    "under other tokens", s.blocks[i],
+                    static_cast<long long>(seq_id));
+    } else {
+      if (placed >= 0 && placed != c)
+        return fail(PA_ERR_INVALID_ARG,
+                    "pa_bm_cache_insert: block %d of sequence %lld is cached "
+                    "under other tokens", s.blocks[i],
+                    static_cast<long long>(seq_id));
+      node = c;
+    }
+  }
+  const int64_t now = ++bm->clock;
+  node = 0;
+  for (int64_t i = 0; i < n_full; ++i) {
+    int32_t c = bm->find_child(node, tokens + i * bs);
+    if (c < 0)
+      c = bm->add_node(node, tokens + i * bs, s.blocks[i], now);
+    else
+      bm->touch(c, now);
+    node = c;
+  }
+  return PA_OK;
+}
+
+pa_status pa_bm_cache_evict(void* p, int max_blocks, int* evicted_out) {
+  pagedkv::clear_error();
+  BlockManager* bm = as_bm(p);
+  if (!bm || max_blocks < 0 || !evicted_out)
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_cache_evict: bad arguments");
+  int done = 0;
+  while (done < max_blocks && !bm->lru.empty()) {
+    const int32_t n = bm->lru.begin()->second;
+    bm->unlink(n);
+    bm->release_node(n);
+    ++done;
+  }
+  *evicted_out = done;
+  return PA_OK;
+}
+
+int pa_bm_num_cached(void* p) {
+  BlockManager* bm = as_bm(p);
+  return bm ? bm->num_cached : -1;
+}
+
+pa_status pa_bm_cache_nodes(void* p, int max_nodes, int32_t* parent_out,
+                            int32_t* block_out, int32_t* tokens_out,
+                            int* n_out) {
+  pagedkv::clear_error();
+  BlockManager* bm = as_bm(p);
+  if (!bm || max_nodes < 0 || !n_out ||
+      (max_nodes > 0 && (!parent_out || !block_out || !tokens_out)))
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_cache_nodes: bad arguments");
+  if (bm->num_cached > max_nodes)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_bm_cache_nodes: %d cached blocks, room for %d",
+                bm->num_cached, max_nodes);
+  // Breadth-first from the root, so every parent precedes its children.
+  std::vector<std::vector<int32_t>> kids(bm->nodes.size());
+  for (size_t n = 1; n < bm->nodes.size(); ++n)
+    if (bm->nodes[n].block >= 0 && bm->node_of[bm->nodes[n].block] ==
+                                       static_cast<int32_t>(n))
+      kids[bm->nodes[n].parent].push_back(static_cast<int32_t>(n));
+  std::vector<int32_t> index(bm->nodes.size(), -1);
+  std::vector<int32_t> queue{0};
+  int out = 0;
+  for (size_t q = 0; q < queue.size(); ++q) {
+    for (int32_t c : kids[queue[q]]) {
+      const Node& x = bm->nodes[c];
+      index[c] = out;
+      parent_out[out] = x.parent == 0 ? -1 : index[x.parent];
+      block_out[out] = x.block;
+      std::memcpy(tokens_out + static_cast<int64_t>(out) * bm->block_size,
+                  x.tokens.data(), sizeof(int32_t) * bm->block_size);
+      ++out;
+      queue.push_back(c);
+    }
+  }
+  *n_out = out;
+  return PA_OK;
 }
 
 }  // extern "C"
