@@ -56,9 +56,9 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-spinup", action="store_true",
                    help="skip the 1 s untimed clock spin-up (profiling)")
-    p.add_argument("--prefill-only", action="store_true",
-                   help="time only pa_prefill on the two prefill workloads "
-                        "and print their line (tuning and profiling)")
+    p.add_argument("--extras-only", action="store_true",
+                   help="time only the side measurements (prefill, prefix "
+                        "cache, swap) and print them (tuning and profiling)")
     return p.parse_args()
 
 
@@ -541,6 +541,7 @@ def extras(args, w, inp, dev, pkv, bt, cl):
     out["prefill"] = [time_prefill(pkv, wl, n, c, dev)
                       for n, c in PREFILL_CASES]
     out["prefix_cache"] = prefix_cache_measure(pkv, dev)
+    out["swap"] = swap_measure(pkv, dev)
     return out
 
 
@@ -680,7 +681,100 @@ def prefix_cache_measure(pkv, dev, requests=128, prompt_len=2048,
     return res
 
 
-def run_prefill_only(args):
+def swap_measure(pkv, dev, group_size=64, seed=383010):
+    """Preempting ``group_size`` of the 256 Llama-3-70B-shaped sequences
+    (log-normal lengths, block 16, bf16): block-manager swap-out / swap-in
+    (host microseconds) and pa_swap_blocks moving their K/V to a pinned host
+    pool and back (GB/s), beside torch's own pinned copy of the same bytes
+    in one piece (the host link's copy bandwidth)."""
+    import time
+    import torch
+    from paged_kv_cache_383_b200 import workloads as wl
+    w = wl.WORKLOADS["llama3_70b_gqa8"]
+    lengths = wl.make_paged(w, values=False).lengths
+    bs, hkv, d = w.block_size, w.num_kv_heads, w.head_dim
+    need = int(sum(-(-int(L) // bs) for L in lengths))
+    nb = need + 64
+    bm = pkv.BlockManager(nb, bs)
+    for b, L in enumerate(lengths):
+        bm.add_seq(b)
+        bm.append(b, int(L))
+    rng = np.random.default_rng(seed)
+    group = sorted(rng.choice(len(lengths), group_size, replace=False)
+                   .tolist())
+    host_blocks = int(sum(-(-int(lengths[b]) // bs) for b in group))
+    bm.set_host_blocks(host_blocks)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    shape = (nb, hkv, bs, d)
+    kc = torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+    vc = torch.randn(shape, generator=g, device=dev).to(torch.bfloat16)
+    hk = torch.empty((host_blocks, hkv, bs, d), dtype=torch.bfloat16,
+                     pin_memory=True)
+    hv = torch.empty_like(hk, pin_memory=True)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    block_bytes = hkv * bs * d * 2 * 2          # K and V
+    res = {"group": group_size, "blocks": host_blocks,
+           "bytes": host_blocks * block_bytes}
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    t_out = t_in = 0.0
+    ms_out, ms_in, reps = [], [], 3
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        pairs = bm.swap_out(group)
+        t_out += time.perf_counter() - t0
+        pd = torch.from_numpy(pairs).to(dev)
+        a, b = ev(), ev()
+        a.record()
+        pkv.pa_swap_blocks(hk, hv, kc, vc, pd, dev_err=err)
+        b.record()
+        torch.cuda.synchronize()
+        ms_out.append(a.elapsed_time(b))
+        t0 = time.perf_counter()
+        pairs = bm.swap_in(group)
+        t_in += time.perf_counter() - t0
+        pd = torch.from_numpy(pairs).to(dev)
+        a, b = ev(), ev()
+        a.record()
+        pkv.pa_swap_blocks(kc, vc, hk, hv, pd, dev_err=err)
+        b.record()
+        torch.cuda.synchronize()
+        ms_in.append(a.elapsed_time(b))
+    if err.item():
+        raise RuntimeError(f"pa_swap_blocks device error {err.item()}")
+    gbs = lambda ms: round(res["bytes"] / (ms * 1e-3) / 1e9, 2)
+    res["host_us_swap_out"] = round(t_out / reps * 1e6, 1)
+    res["host_us_swap_in"] = round(t_in / reps * 1e6, 1)
+    res["d2h_ms"] = round(min(ms_out[1:]), 3)
+    res["h2d_ms"] = round(min(ms_in[1:]), 3)
+    res["d2h_gbs"] = gbs(res["d2h_ms"])
+    res["h2d_gbs"] = gbs(res["h2d_ms"])
+    # torch's pinned copy of the same number of bytes, one contiguous piece
+    n = host_blocks * hkv * bs * d
+    dflat = kc.view(-1)[:n]
+    hflat = hk.view(-1)
+    for direction in ("d2h", "h2d"):
+        best = None
+        for _ in range(3):
+            a, b = ev(), ev()
+            a.record()
+            for _ in range(2):  # K and V
+                if direction == "d2h":
+                    hflat.copy_(dflat, non_blocking=True)
+                else:
+                    dflat.copy_(hflat, non_blocking=True)
+            b.record()
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b)
+            best = ms if best is None else min(best, ms)
+        res[f"torch_copy_{direction}_gbs"] = gbs(best)
+        res[f"frac_{direction}"] = round(res[f"{direction}_gbs"] /
+                                         res[f"torch_copy_{direction}_gbs"], 3)
+    bm.close()
+    return res
+
+
+def run_extras_only(args):
     import torch
     import paged_kv_cache_383_b200 as pkv
     from paged_kv_cache_383_b200 import workloads as wl
@@ -688,9 +782,11 @@ def run_prefill_only(args):
     torch.cuda.set_device(dev)
     res = [time_prefill(pkv, wl, n, c, dev, iters=max(args.steps, 1))
            for n, c in PREFILL_CASES]
-    return {"metric": "prefill attention TFLOP/s (algorithmic)",
-            "unit": "TFLOP/s", "cases": res,
+    return {"metric": "side measurements: prefill attention TFLOP/s "
+                      "(algorithmic), prefix cache, swap",
+            "prefill": res,
             "prefix_cache": prefix_cache_measure(pkv, dev),
+            "swap": swap_measure(pkv, dev),
             "gpu_launches": pkv.pa_launch_count()}
 
 
@@ -906,8 +1002,8 @@ def main():
             import torch.distributed as dist
             dist.destroy_process_group()
         return
-    if args.prefill_only:
-        print(json.dumps(run_prefill_only(args)), flush=True)
+    if args.extras_only:
+        print(json.dumps(run_extras_only(args)), flush=True)
         return
     res = run_native(args, rank, world, local)
     if rank == 0:

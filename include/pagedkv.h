@@ -267,6 +267,32 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs,
                          int32_t* dev_err, void* stream);
 
 /* ------------------------------------------------------------------------
+ * pa_swap_blocks -- move whole blocks between two pools for preemption by
+ * swapping a request's KV cache to CPU RAM and back ([Taming the Tail]
+ * "Infrastructure Scale"; the pairs come from pa_bm_swap_out / _swap_in).
+ *   dst_*_cache, src_*_cache  [num_dst_blocks | num_src_blocks, num_kv_heads,
+ *                 block_size, head_dim] of `dtype`, 16-byte aligned.  Each
+ *                 may be memory of the current device or page-locked host
+ *                 memory mapped into the device address space (e.g. from
+ *                 cudaHostAlloc / cudaMallocHost, or registered); the kernel
+ *                 reads and writes host pages directly over the host link.
+ *                 Pageable memory or another device's memory -> INVALID_ARG.
+ *   pairs         int32 [num_pairs][2] (source block, destination block),
+ *                 device or mapped page-locked host memory.
+ * One launch; K and V of every pair.  A pair outside [0, num_src_blocks) x
+ * [0, num_dst_blocks) sets *dev_err = PA_ERR_DEVICE_OOB and is skipped.
+ * Stream-ordered: run it before anything reuses the source blocks (swap-out
+ * frees device blocks; swap-in frees host blocks).  The caller keeps host
+ * buffers alive until the stream has passed the copy.
+ * ---------------------------------------------------------------------- */
+pa_status pa_swap_blocks(void* dst_k_cache, void* dst_v_cache,
+                         const void* src_k_cache, const void* src_v_cache,
+                         const int32_t* pairs, int num_pairs,
+                         int num_kv_heads, int head_dim, int block_size,
+                         int num_src_blocks, int num_dst_blocks,
+                         pa_dtype dtype, int32_t* dev_err, void* stream);
+
+/* ------------------------------------------------------------------------
  * Host block manager: free block pool, per-sequence logical->physical block
  * tables, reference counts and copy-on-write ([Taming the Tail] "How the
  * Architecture Works", "Complex Memory Sharing"; [vLLM PagedAttention FAQ]
@@ -389,6 +415,50 @@ int pa_bm_num_cached(void* bm);
 pa_status pa_bm_cache_nodes(void* bm, int max_nodes, int32_t* parent_out,
                             int32_t* block_out, int32_t* tokens_out,
                             int* n_out);
+
+/* ---- Swapping to a host pool ([Taming the Tail] "Infrastructure Scale":
+ * pause a request and move its KV cache to CPU RAM) --------------------------
+ * A second pool of host blocks; a swapped-out sequence keeps its table but
+ * its entries name host blocks.  A group of sequences is swapped at once so
+ * blocks the group shares cross the link once: each distinct block of the
+ * group's tables (in order of first use: sequences as listed, logical blocks
+ * in order) gets one block in the other pool holding the group's references
+ * to it; the old block keeps the references other tables or the prefix cache
+ * hold and returns to its pool when none are left.  pairs_out receives the
+ * (source, destination) copies for pa_swap_blocks, which must run before the
+ * freed blocks are written again.  All or nothing: PA_ERR_NO_FREE_BLOCKS (the
+ * target pool, after evicting cache leaves for a swap-in, cannot supply every
+ * block) or INVALID_ARG (unknown / repeated sequence, wrong swap state,
+ * max_pairs too small: the distinct block count suffices) change nothing.
+ * A swapped-out sequence can only be swapped in or freed: append, fork,
+ * truncate, block_table, match_prefix and cache_insert refuse it. */
+
+/* Size the host pool (ids 0..num_host_blocks-1).  INVALID_ARG while any host
+ * block is in use. */
+pa_status pa_bm_set_host_blocks(void* bm, int num_host_blocks);
+
+/* Swap the n sequences out: pairs_out (host int32 [2 * max_pairs]) gets
+ * (device block, host block) pairs, *num_pairs_out their number. */
+pa_status pa_bm_swap_out(void* bm, const int64_t* seq_ids, int n,
+                         int32_t* pairs_out, int max_pairs,
+                         int* num_pairs_out);
+
+/* Swap the n sequences back in: (host block, device block) pairs. */
+pa_status pa_bm_swap_in(void* bm, const int64_t* seq_ids, int n,
+                        int32_t* pairs_out, int max_pairs,
+                        int* num_pairs_out);
+
+/* Free host blocks; a host block's reference count (-1 if out of range);
+ * 1 if the sequence is swapped out, 0 if not, -1 if unknown. */
+int pa_bm_num_free_host(void* bm);
+int pa_bm_host_refcount(void* bm, int host_block);
+int pa_bm_is_swapped(void* bm, int64_t seq_id);
+
+/* The sequence's table entries in logical order (device block ids, or host
+ * block ids while it is swapped out) into blocks_out (host int32
+ * [max_blocks]); *n_out = how many. */
+pa_status pa_bm_seq_blocks(void* bm, int64_t seq_id, int32_t* blocks_out,
+                           int max_blocks, int* n_out);
 
 /* Kernel launches this library has issued in this process (all devices,
  * all threads): lets a caller count the GPU work a timed region contained. */

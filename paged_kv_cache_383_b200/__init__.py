@@ -220,6 +220,44 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens,
     return out
 
 
+def _reachable(t, name: str, dtype=None):
+    """Pointer of a contiguous CUDA tensor or pinned (page-locked) CPU
+    tensor; the library checks that the device can reach it."""
+    if not (t.is_cuda or t.is_pinned()):
+        raise ValueError(f"{name} must be a CUDA tensor or pinned CPU memory")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def pa_swap_blocks(dst_k, dst_v, src_k, src_v, pairs, *, dev_err=None,
+                   stream=None):
+    """Copy block pairs[i, 0] of (src_k, src_v) to block pairs[i, 1] of
+    (dst_k, dst_v); any of the pools (and ``pairs``) may be pinned CPU
+    tensors, e.g. a host pool for swapped-out sequences."""
+    import torch
+    lib = _lib.load()
+    ns, hkv, bs, d = src_k.shape
+    nd = dst_k.shape[0]
+    for name, t, n in (("dst_k", dst_k, nd), ("dst_v", dst_v, nd),
+                       ("src_v", src_v, ns)):
+        if t.shape != (n, hkv, bs, d):
+            raise ValueError(f"{name} shape {tuple(t.shape)} does not match")
+        if t.dtype != src_k.dtype:
+            raise TypeError(f"{name} dtype differs from src_k")
+    if pairs.ndim != 2 or pairs.shape[1] != 2:
+        raise ValueError("pairs must be [n, 2]")
+    st = lib.pa_swap_blocks(
+        _reachable(dst_k, "dst_k"), _reachable(dst_v, "dst_v"),
+        _reachable(src_k, "src_k"), _reachable(src_v, "src_v"),
+        _reachable(pairs, "pairs", torch.int32), pairs.shape[0], hkv, d, bs,
+        ns, nd, _dtype_code(src_k), _dev(dev_err, "dev_err", torch.int32),
+        _stream(stream))
+    _lib.check(st, "pa_swap_blocks")
+
+
 def pa_cache_write(k_cache, v_cache, k, v, slot_mapping, *, dev_err=None,
                    stream=None):
     """Copy each new token's K and V rows into cache slot slot_mapping[t]
@@ -450,3 +488,61 @@ class BlockManager:
             key = tuple(int(t) for t in toks[i])
             paths.append((key,) if parent[i] < 0 else paths[parent[i]] + (key,))
         return set(paths)
+
+    # -- swapping to a host pool ------------------------------------------------
+    def set_host_blocks(self, num_host_blocks: int):
+        _lib.check(self._lib.pa_bm_set_host_blocks(self._h, num_host_blocks),
+                   "pa_bm_set_host_blocks")
+        self.num_host_blocks = num_host_blocks
+
+    def _swap(self, fn, name, seq_ids, pairs_out):
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        cap = sum(max(self.num_seq_blocks(int(s)), 0) for s in ids)
+        if pairs_out is None:
+            pairs = np.empty((max(cap, 1), 2), dtype=np.int32)
+        else:
+            if (pairs_out.dtype != np.int32 or pairs_out.ndim != 2
+                    or pairs_out.shape[1] != 2
+                    or not pairs_out.flags.c_contiguous):
+                raise ValueError("pairs_out must be contiguous int32 [k, 2]")
+            pairs, cap = pairs_out, pairs_out.shape[0]
+        n = ctypes.c_int(0)
+        _lib.check(fn(self._h, ids.ctypes.data_as(ctypes.POINTER(
+            ctypes.c_int64)), len(ids), pairs.ctypes.data_as(
+                ctypes.POINTER(ctypes.c_int32)), cap, ctypes.byref(n)), name)
+        return pairs[:n.value]
+
+    def swap_out(self, seq_ids, pairs_out=None):
+        """Swap the group out; returns (device, host) block pairs int32
+        [k, 2] (a view of ``pairs_out`` if given, e.g. pinned memory)."""
+        return self._swap(self._lib.pa_bm_swap_out, "pa_bm_swap_out",
+                          seq_ids, pairs_out)
+
+    def swap_in(self, seq_ids, pairs_out=None):
+        """Swap the group back in; returns (host, device) block pairs."""
+        return self._swap(self._lib.pa_bm_swap_in, "pa_bm_swap_in", seq_ids,
+                          pairs_out)
+
+    def num_free_host(self) -> int:
+        return self._lib.pa_bm_num_free_host(self._h)
+
+    def host_refcount(self, block: int) -> int:
+        return self._lib.pa_bm_host_refcount(self._h, block)
+
+    def is_swapped(self, seq_id: int) -> bool:
+        r = self._lib.pa_bm_is_swapped(self._h, seq_id)
+        if r < 0:
+            raise KeyError(seq_id)
+        return bool(r)
+
+    def seq_blocks(self, seq_id: int):
+        """Table entries in logical order (host ids while swapped out)."""
+        import numpy as np
+        n = max(self.num_seq_blocks(seq_id), 0)
+        out = np.empty(max(n, 1), dtype=np.int32)
+        got = ctypes.c_int(0)
+        _lib.check(self._lib.pa_bm_seq_blocks(
+            self._h, seq_id, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+            n, ctypes.byref(got)), "pa_bm_seq_blocks")
+        return out[:got.value]

@@ -99,6 +99,8 @@ SIGNATURES = {
                              _int, _int, _vp, _vp]),
     "pa_copy_blocks": (_st, [_vp, _vp, _vp, _int, _int, _int, _int, _int, _int,
                              _vp, _vp]),
+    "pa_swap_blocks": (_st, [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int,
+                             _int, _int, _int, _vp, _vp]),
     "pa_bm_create": (_st, [_int, _int, _pi32, ctypes.POINTER(_vp)]),
     "pa_bm_destroy": (None, [_vp]),
     "pa_bm_add_seq": (_st, [_vp, _i64]),
@@ -122,6 +124,15 @@ SIGNATURES = {
     "pa_bm_num_cached": (_int, [_vp]),
     "pa_bm_cache_nodes": (_st, [_vp, _int, _pi32, _pi32, _pi32,
                                 ctypes.POINTER(_int)]),
+    "pa_bm_set_host_blocks": (_st, [_vp, _int]),
+    "pa_bm_swap_out": (_st, [_vp, _pi64, _int, _pi32, _int,
+                             ctypes.POINTER(_int)]),
+    "pa_bm_swap_in": (_st, [_vp, _pi64, _int, _pi32, _int,
+                            ctypes.POINTER(_int)]),
+    "pa_bm_num_free_host": (_int, [_vp]),
+    "pa_bm_host_refcount": (_int, [_vp, _int]),
+    "pa_bm_is_swapped": (_int, [_vp, _i64]),
+    "pa_bm_seq_blocks": (_st, [_vp, _i64, _pi32, _int, ctypes.POINTER(_int)]),
 }
 
 _lib = None

@@ -16,7 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libpagedkv.so")
 
 SOURCES = ["status.cpp", "block_manager.cpp", "cache_ops.cu", "decode.cu",
-           "prefill.cu", "probe.cu"]
+           "prefill.cu", "probe.cu", "swap.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -19,6 +19,15 @@
 // walk), and a leaf's parent may become evictable in turn.  Reference counts
 // keep every block a sequence still uses out of reach.
 //
+// Swap ([Taming the Tail] "Infrastructure Scale", preemption by moving a
+// request's KV cache to CPU RAM): a second pool of host blocks.  A group of
+// sequences is swapped at once, so a block the group shares crosses the link
+// once: each distinct device block of the group gets one host block carrying
+// the group's references, and the device block keeps the references other
+// tables (or the cache) hold.  Swap-in is the mirror image and allocates
+// device blocks like an append (evicting cache leaves).  Both are all or
+// nothing and return the (source, destination) pairs pa_swap_blocks copies.
+//
 // Design: everything is flat integer arrays.  The pool is a LIFO stack so a
 // block freed a moment ago (likely still in L2) is reused first; the first
 // fill follows the caller's free_order.  Appends are all-or-nothing: the
@@ -27,6 +36,7 @@
 // nodes live in one array; children are found through a hash map keyed by
 // (parent node, block tokens); evictable leaves sit in an ordered set by
 // stamp, kept current whenever a count, a stamp or a child count changes.
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <limits>
@@ -45,6 +55,7 @@ namespace {
 struct Sequence {
   std::vector<int32_t> blocks;  // logical block i -> physical block
   int64_t len = 0;              // tokens stored
+  bool swapped = false;         // blocks name host-pool blocks
 };
 
 struct Node {
@@ -89,6 +100,11 @@ struct BlockManager {
   std::set<std::pair<int64_t, int32_t>> lru;  // evictable leaves by stamp
   int64_t clock = 0;
   int num_cached = 0;
+
+  // host pool for swapped-out sequences
+  int num_host_blocks = 0;
+  std::vector<int32_t> host_free;  // top = back()
+  std::vector<int32_t> host_ref;
 
   int32_t take() {
     int32_t b = free_stack.back();
@@ -297,6 +313,9 @@ pa_status pa_bm_fork(void* p, int64_t parent_id, int64_t child_id) {
   if (bm->seqs.count(child_id))
     return fail(PA_ERR_INVALID_ARG, "pa_bm_fork: child %lld exists",
                 static_cast<long long>(child_id));
+  if (it->second.swapped)
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_fork: parent %lld is swapped out",
+                static_cast<long long>(parent_id));
   Sequence child = it->second;  // copy of table and length
   for (int32_t b : child.blocks) bm->add_ref(b);
   bm->seqs.emplace(child_id, std::move(child));
@@ -321,6 +340,10 @@ pa_status pa_bm_append(void* p, int64_t seq_id, int n_tokens,
   Sequence& s = it->second;
   const int bs = bm->block_size;
   *num_cow_out = 0;
+  if (s.swapped)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_bm_append: sequence %lld is swapped out",
+                static_cast<long long>(seq_id));
   if (n_tokens == 0) return PA_OK;
 
   // Blocks this append takes from the pool, decided before any change.
@@ -394,7 +417,12 @@ pa_status pa_bm_free_seq(void* p, int64_t seq_id) {
   if (it == bm->seqs.end())
     return fail(PA_ERR_INVALID_ARG, "pa_bm_free_seq: no sequence %lld",
                 static_cast<long long>(seq_id));
-  for (int32_t b : it->second.blocks) bm->drop(b);
+  if (it->second.swapped) {
+    for (int32_t h : it->second.blocks)
+      if (--bm->host_ref[h] == 0) bm->host_free.push_back(h);
+  } else {
+    for (int32_t b : it->second.blocks) bm->drop(b);
+  }
   bm->seqs.erase(it);
   return PA_OK;
 }
@@ -408,6 +436,10 @@ pa_status pa_bm_truncate(void* p, int64_t seq_id, int64_t new_len) {
     return fail(PA_ERR_INVALID_ARG, "pa_bm_truncate: no sequence %lld",
                 static_cast<long long>(seq_id));
   Sequence& s = it->second;
+  if (s.swapped)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_bm_truncate: sequence %lld is swapped out",
+                static_cast<long long>(seq_id));
   if (new_len < 0 || new_len > s.len)
     return fail(PA_ERR_INVALID_ARG,
                 "pa_bm_truncate: new_len %lld outside [0, %lld]",
@@ -436,6 +468,10 @@ pa_status pa_bm_block_table(void* p, const int64_t* seq_ids, int n,
       return fail(PA_ERR_INVALID_ARG, "pa_bm_block_table: no sequence %lld",
                   static_cast<long long>(seq_ids[i]));
     const Sequence& s = it->second;
+    if (s.swapped)
+      return fail(PA_ERR_INVALID_ARG,
+                  "pa_bm_block_table: sequence %lld is swapped out",
+                  static_cast<long long>(seq_ids[i]));
     if (static_cast<int64_t>(s.blocks.size()) > max_blocks ||
         s.len > std::numeric_limits<int32_t>::max())
       return fail(PA_ERR_INVALID_ARG,
@@ -487,9 +523,10 @@ pa_status pa_bm_match_prefix(void* p, int64_t seq_id, const int32_t* tokens,
     return fail(PA_ERR_INVALID_ARG, "pa_bm_match_prefix: no sequence %lld",
                 static_cast<long long>(seq_id));
   Sequence& s = it->second;
-  if (s.len != 0 || !s.blocks.empty())
+  if (s.len != 0 || !s.blocks.empty() || s.swapped)
     return fail(PA_ERR_INVALID_ARG,
-                "pa_bm_match_prefix: sequence %lld is not empty",
+                "pa_bm_match_prefix: sequence %lld is not empty or is "
+                "swapped out",
                 static_cast<long long>(seq_id));
   const int bs = bm->block_size;
   const int64_t now = ++bm->clock;
@@ -518,6 +555,10 @@ pa_status pa_bm_cache_insert(void* p, int64_t seq_id, const int32_t* tokens,
     return fail(PA_ERR_INVALID_ARG, "pa_bm_cache_insert: no sequence %lld",
                 static_cast<long long>(seq_id));
   const Sequence& s = it->second;
+  if (s.swapped)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_bm_cache_insert: sequence %lld is swapped out",
+                static_cast<long long>(seq_id));
   if (n_tokens > s.len)
     return fail(PA_ERR_INVALID_ARG,
                 "pa_bm_cache_insert: %lld tokens, sequence %lld holds %lld",
@@ -616,6 +657,192 @@ pa_status pa_bm_cache_nodes(void* p, int max_nodes, int32_t* parent_out,
     }
   }
   *n_out = out;
+  return PA_OK;
+}
+
+pa_status pa_bm_set_host_blocks(void* p, int num_host_blocks) {
+  pagedkv::clear_error();
+  BlockManager* bm = as_bm(p);
+  if (!bm || num_host_blocks < 0)
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_set_host_blocks: bad arguments");
+  if (static_cast<int>(bm->host_free.size()) != bm->num_host_blocks)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_bm_set_host_blocks: %d host blocks are in use",
+                bm->num_host_blocks -
+                    static_cast<int>(bm->host_free.size()));
+  bm->num_host_blocks = num_host_blocks;
+  bm->host_ref.assign(num_host_blocks, 0);
+  bm->host_free.resize(num_host_blocks);
+  for (int i = 0; i < num_host_blocks; ++i)
+    bm->host_free[num_host_blocks - 1 - i] = i;  // first handed out = 0
+  return PA_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Distinct blocks of the group's tables in order of first use, with the
+// group's reference count of each.  `seen` is indexed by block id.
+void group_uses(const std::vector<Sequence*>& group, int pool_size,
+                std::vector<int32_t>* order, std::vector<int32_t>* count) {
+  count->assign(pool_size, 0);
+  order->clear();
+  for (const Sequence* s : group)
+    for (int32_t b : s->blocks)
+      if ((*count)[b]++ == 0) order->push_back(b);
+}
+
+// Validate the group: known, distinct, and swapped (or not) as required.
+pa_status collect_group(BlockManager* bm, const int64_t* seq_ids, int n,
+                        bool want_swapped, const char* fn,
+                        std::vector<Sequence*>* group) {
+  group->clear();
+  for (int i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seq_ids[i]);
+    if (it == bm->seqs.end())
+      return fail(PA_ERR_INVALID_ARG, "%s: no sequence %lld", fn,
+                  static_cast<long long>(seq_ids[i]));
+    if (it->second.swapped != want_swapped)
+      return fail(PA_ERR_INVALID_ARG, "%s: sequence %lld is %s", fn,
+                  static_cast<long long>(seq_ids[i]),
+                  want_swapped ? "not swapped out" : "already swapped out");
+    for (const Sequence* g : *group)
+      if (g == &it->second)
+        return fail(PA_ERR_INVALID_ARG, "%s: sequence %lld listed twice", fn,
+                    static_cast<long long>(seq_ids[i]));
+    group->push_back(&it->second);
+  }
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_status pa_bm_swap_out(void* p, const int64_t* seq_ids, int n,
+                         int32_t* pairs_out, int max_pairs,
+                         int* num_pairs_out) {
+  pagedkv::clear_error();
+  BlockManager* bm = as_bm(p);
+  if (!bm || n < 0 || (n > 0 && !seq_ids) || !num_pairs_out ||
+      max_pairs < 0 || (max_pairs > 0 && !pairs_out))
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_swap_out: bad arguments");
+  *num_pairs_out = 0;
+  std::vector<Sequence*> group;
+  pa_status st = collect_group(bm, seq_ids, n, false, "pa_bm_swap_out",
+                               &group);
+  if (st != PA_OK) return st;
+  std::vector<int32_t> order, count;
+  group_uses(group, bm->num_blocks, &order, &count);
+  const int distinct = static_cast<int>(order.size());
+  if (distinct > max_pairs)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_bm_swap_out: %d pairs, room for %d", distinct, max_pairs);
+  if (distinct > static_cast<int>(bm->host_free.size()))
+    return fail(PA_ERR_NO_FREE_BLOCKS,
+                "pa_bm_swap_out: %d host blocks needed, %zu free", distinct,
+                bm->host_free.size());
+  std::vector<int32_t> to_host(bm->num_blocks, -1);
+  for (int i = 0; i < distinct; ++i) {
+    const int32_t d = order[i];
+    const int32_t h = bm->host_free.back();
+    bm->host_free.pop_back();
+    bm->host_ref[h] = count[d];
+    to_host[d] = h;
+    pairs_out[2 * i] = d;
+    pairs_out[2 * i + 1] = h;
+  }
+  for (int32_t d : order)
+    for (int r = 0; r < count[d]; ++r) bm->drop(d);
+  for (Sequence* s : group) {
+    for (int32_t& b : s->blocks) b = to_host[b];
+    s->swapped = true;
+  }
+  *num_pairs_out = distinct;
+  return PA_OK;
+}
+
+pa_status pa_bm_swap_in(void* p, const int64_t* seq_ids, int n,
+                        int32_t* pairs_out, int max_pairs,
+                        int* num_pairs_out) {
+  pagedkv::clear_error();
+  BlockManager* bm = as_bm(p);
+  if (!bm || n < 0 || (n > 0 && !seq_ids) || !num_pairs_out ||
+      max_pairs < 0 || (max_pairs > 0 && !pairs_out))
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_swap_in: bad arguments");
+  *num_pairs_out = 0;
+  std::vector<Sequence*> group;
+  pa_status st = collect_group(bm, seq_ids, n, true, "pa_bm_swap_in",
+                               &group);
+  if (st != PA_OK) return st;
+  std::vector<int32_t> order, count;
+  group_uses(group, bm->num_host_blocks, &order, &count);
+  const int distinct = static_cast<int>(order.size());
+  if (distinct > max_pairs)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_bm_swap_in: %d pairs, room for %d", distinct, max_pairs);
+  if (!bm->ensure_free(distinct))
+    return fail(PA_ERR_NO_FREE_BLOCKS,
+                "pa_bm_swap_in: %d device blocks needed, %zu free after "
+                "evicting every evictable cached block", distinct,
+                bm->free_stack.size() + bm->lru.size());
+  std::vector<int32_t> to_dev(bm->num_host_blocks, -1);
+  for (int i = 0; i < distinct; ++i) {
+    const int32_t h = order[i];
+    const int32_t d = bm->take();
+    bm->ref[d] = count[h];
+    to_dev[h] = d;
+    pairs_out[2 * i] = h;
+    pairs_out[2 * i + 1] = d;
+  }
+  for (int32_t h : order) {
+    bm->host_ref[h] -= count[h];
+    if (bm->host_ref[h] == 0) bm->host_free.push_back(h);
+  }
+  for (Sequence* s : group) {
+    for (int32_t& b : s->blocks) b = to_dev[b];
+    s->swapped = false;
+  }
+  *num_pairs_out = distinct;
+  return PA_OK;
+}
+
+int pa_bm_num_free_host(void* p) {
+  BlockManager* bm = as_bm(p);
+  return bm ? static_cast<int>(bm->host_free.size()) : -1;
+}
+
+int pa_bm_host_refcount(void* p, int block) {
+  BlockManager* bm = as_bm(p);
+  if (!bm || block < 0 || block >= bm->num_host_blocks) return -1;
+  return bm->host_ref[block];
+}
+
+int pa_bm_is_swapped(void* p, int64_t seq_id) {
+  BlockManager* bm = as_bm(p);
+  if (!bm) return -1;
+  auto it = bm->seqs.find(seq_id);
+  return it == bm->seqs.end() ? -1 : (it->second.swapped ? 1 : 0);
+}
+
+pa_status pa_bm_seq_blocks(void* p, int64_t seq_id, int32_t* blocks_out,
+                           int max_blocks, int* n_out) {
+  pagedkv::clear_error();
+  BlockManager* bm = as_bm(p);
+  if (!bm || !n_out || max_blocks < 0 || (max_blocks > 0 && !blocks_out))
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_seq_blocks: bad arguments");
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end())
+    return fail(PA_ERR_INVALID_ARG, "pa_bm_seq_blocks: no sequence %lld",
+                static_cast<long long>(seq_id));
+  const std::vector<int32_t>& b = it->second.blocks;
+  if (static_cast<int64_t>(b.size()) > max_blocks)
+    return fail(PA_ERR_INVALID_ARG,
+                "pa_bm_seq_blocks: %zu blocks, room for %d", b.size(),
+                max_blocks);
+  std::copy(b.begin(), b.end(), blocks_out);
+  *n_out = static_cast<int>(b.size());
   return PA_OK;
 }
 
