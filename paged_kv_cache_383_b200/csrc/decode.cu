@@ -884,6 +884,13 @@ int resolve_partition(const pa_decode_desc* d, int max_ctx) {
   if (d->partition_size > 0) return d->partition_size;
   const int64_t pairs = static_cast<int64_t>(d->num_seqs) * d->num_kv_heads;
   const int64_t target = 3LL * device_sm_count();
+  // Plenty of work units even at 2048 tokens each (at least 8 per SM if every
+  // sequence were max_ctx long): fewer, longer CTAs spend less on ramp-up and
+  // partials (measured ~2% on the batch-256 mixes).  With fewer units the
+  // tail of the last wave costs more, so stay at 1024 or below.
+  if (pairs * ((max_ctx + 2047) / 2048) >= 8LL * device_sm_count() &&
+      2048 % d->block_size == 0)
+    return 2048;
   int ps = 1024;
   while (ps > 2 * d->block_size && ps > 64 &&
          pairs * ((max_ctx + ps - 1) / ps) < target)
