@@ -127,11 +127,16 @@ const char* pa_last_error(void);
  *                 entries past a sequence's last block are ignored
  *   context_lens  [num_seqs] int32, tokens per sequence, the newest included
  *   workspace     pa_decode_workspace_bytes(desc) bytes of device memory the
- *                 caller owns, 16-byte aligned (may be NULL when that size is
- *                 0): partition partials and per-(sequence, KV head)
- *                 counters the call resets on its stream.  Its contents need
+ *                 caller owns, 16-byte aligned (always > 0): partition
+ *                 partials and per-(sequence, KV head) counters (more than
+ *                 one partition only) and the order in which sequences are
+ *                 served (longest first, so the grid ends on short work),
+ *                 all written by the call on its stream.  Its contents need
  *                 no initialisation and are scratch after the call; calls
  *                 that share a workspace must not overlap on the device.
+ * Launches: a one-CTA prep kernel (the longest-first order; counter reset),
+ * the decode, and with more than 16 partitions or PA_REDUCE_KERNEL the
+ * reduce kernel, chained by programmatic dependent launch.
  * Computation: fp32 scores, fp32 online softmax, fp32 accumulation; the
  * output is rounded once to dtype.
  * Errors: PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED / PA_ERR_WORKSPACE before

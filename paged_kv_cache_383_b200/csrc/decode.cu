@@ -72,6 +72,7 @@ struct DecodeArgs {
   float* ws_o;   // [num_seqs, num_q_heads, max_parts, head_dim]
   float* ws_ml;  // [num_seqs, num_q_heads, max_parts, 2] = (max, sum), log2 units
   int* counters; // [num_seqs, num_kv_heads] finished partitions (fused mode)
+  const int32_t* order;  // [num_seqs] sequence served by grid row z
   int fused;     // 1: the last partition CTA combines; 0: the reduce kernel
   int32_t* dev_err;
   float scale_log2;  // scale * log2(e): scores are kept in base-2 units
@@ -249,12 +250,19 @@ __global__ void __launch_bounds__(kThreads)
 
   const int part = blockIdx.x;
   const int kvh = blockIdx.y;
-  const int b = blockIdx.z;
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
   dev::pdl_trigger();  // the reduce may start its prologue early
+  // Grid rows are handed out longest sequence first (the order the prep
+  // kernel wrote, which this grid may only read after waiting for it), so
+  // the last CTAs to start are short ones and the tail of the grid is short.
+  int b = blockIdx.z;
+  if (a.order) {
+    dev::pdl_wait();
+    b = a.order[blockIdx.z];
+  }
   const int PS = a.partition_size;
   const int pages_per_part = PS / BS;
   const int page0 = part * pages_per_part;
@@ -717,17 +725,63 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 // ---------------------------------------------------------------------------
-// Zero the per-(sequence, KV head) partition counters before a decode that
-// combines in place.  Launched with programmatic stream serialization: it
-// lets the decode launch at once, waits for the previous kernel (which may
-// still read the counters), zeroes them, and the decode's own wait then
-// covers both.
-__global__ void zero_counters_kernel(int* counters, int n) {
+// Prep kernel (one CTA), run before every decode: orders the sequences
+// longest first (a counting sort on context_len >> shift, 1024 buckets,
+// descending) into `order`, and zeroes the per-(sequence, KV head) partition
+// counters when the decode combines in place.  Launched with programmatic
+// stream serialization: it sorts while the previous kernel drains (it reads
+// only host-written lengths), then waits for that kernel, which may still
+// read `order` and the counters, before writing them.  The decode's own wait
+// covers the prep kernel.  Within one bucket the order follows the atomics;
+// results do not depend on it (each sequence is computed on its own and
+// partials are combined in partition order).
+constexpr int kPrepThreads = 1024;
+constexpr int kPrepBuckets = 1024;
+
+__global__ void __launch_bounds__(kPrepThreads)
+    prep_kernel(const int32_t* __restrict__ context_lens, int num_seqs,
+                int shift, int32_t* __restrict__ order, int* counters,
+                int n_counters) {
+  __shared__ int hist[kPrepBuckets];
+  __shared__ int warp_sum[kPrepThreads / 32];
   dev::pdl_trigger();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  auto bucket = [&](int i) {
+    const int L = context_lens[i];
+    const int k = L <= 0 ? 0 : min(L >> shift, kPrepBuckets - 1);
+    return kPrepBuckets - 1 - k;  // longest first
+  };
+  hist[tid] = 0;
+  __syncthreads();
+  for (int i = tid; i < num_seqs; i += kPrepThreads)
+    atomicAdd(&hist[bucket(i)], 1);
+  __syncthreads();
+  // Exclusive scan of the 1024 bucket counts (one per thread).
+  const int c = hist[tid];
+  int x = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sum[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  hist[tid] = x - c + (warp > 0 ? warp_sum[warp - 1] : 0);
+  __syncthreads();
   dev::pdl_wait();
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += gridDim.x * blockDim.x)
-    counters[i] = 0;
+  for (int i = tid; i < num_seqs; i += kPrepThreads)
+    order[atomicAdd(&hist[bucket(i)], 1)] = i;
+  for (int i = tid; i < n_counters; i += kPrepThreads) counters[i] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -884,13 +938,15 @@ int resolve_partition(const pa_decode_desc* d, int max_ctx) {
   if (d->partition_size > 0) return d->partition_size;
   const int64_t pairs = static_cast<int64_t>(d->num_seqs) * d->num_kv_heads;
   const int64_t target = 3LL * device_sm_count();
-  // Plenty of work units even at 2048 tokens each (at least 8 per SM if every
-  // sequence were max_ctx long): fewer, longer CTAs spend less on ramp-up and
-  // partials (measured ~2% on the batch-256 mixes).  With fewer units the
-  // tail of the last wave costs more, so stay at 1024 or below.
-  if (pairs * ((max_ctx + 2047) / 2048) >= 8LL * device_sm_count() &&
-      2048 % d->block_size == 0)
-    return 2048;
+  // Long partitions (fewer CTAs, less ramp-up and fewer partials) as long as
+  // the grid keeps at least 6 units per SM were every sequence max_ctx long;
+  // the prep kernel's longest-first order keeps the tail short.  Measured:
+  // 4096 is best on the batch-256 and 8-sequence long-context mixes, 2048 on
+  // the batch-64 mix (8192 loses everywhere).
+  for (int big = 4096; big >= 2048; big /= 2)
+    if (pairs * ((max_ctx + big - 1) / big) >= 6LL * device_sm_count() &&
+        big % d->block_size == 0)
+      return big;
   int ps = 1024;
   while (ps > 2 * d->block_size && ps > 64 &&
          pairs * ((max_ctx + ps - 1) / ps) < target)
@@ -958,17 +1014,44 @@ pa_status check_desc(const pa_decode_desc* d) {
   return PA_OK;
 }
 
-size_t workspace_bytes(const pa_decode_desc* d) {
+// Workspace layout, in bytes from the start: partials o and (m, l) and the
+// partition counters (only with more than one partition), then the sequence
+// order; each piece 16-byte aligned.
+struct WsLayout {
+  size_t o = 0, ml = 0, counters = 0, order = 0, total = 0;
+};
+
+WsLayout ws_layout(const pa_decode_desc* d) {
+  auto up16 = [](size_t x) { return (x + 15) & ~size_t(15); };
   const int max_ctx = resolve_max_ctx(d);
   const int ps = resolve_partition(d, max_ctx);
   const int64_t parts = max_ctx > 0 ? (max_ctx + ps - 1) / ps : 1;
-  if (parts <= 1) return 0;
-  const size_t partials = static_cast<size_t>(d->num_seqs) * d->num_q_heads *
-                          parts * (d->head_dim + 2) * sizeof(float);
-  const size_t counters =
-      (static_cast<size_t>(d->num_seqs) * d->num_kv_heads * sizeof(int) + 15) &
-      ~size_t(15);
-  return partials + counters;
+  WsLayout w;
+  size_t at = 0;
+  if (parts > 1) {
+    const size_t rows = static_cast<size_t>(d->num_seqs) * d->num_q_heads *
+                        static_cast<size_t>(parts);
+    w.o = at;
+    at += up16(rows * d->head_dim * sizeof(float));
+    w.ml = at;
+    at += up16(rows * 2 * sizeof(float));
+    w.counters = at;
+    at += up16(static_cast<size_t>(d->num_seqs) * d->num_kv_heads *
+               sizeof(int));
+  }
+  w.order = at;
+  at += up16(static_cast<size_t>(d->num_seqs) * sizeof(int32_t));
+  w.total = at;
+  return w;
+}
+
+size_t workspace_bytes(const pa_decode_desc* d) { return ws_layout(d).total; }
+
+// Bucket shift for the prep kernel's sort: max_ctx >> shift < 1024.
+int order_shift(int max_ctx) {
+  int shift = 0;
+  while ((max_ctx >> shift) >= kPrepBuckets) ++shift;
+  return shift;
 }
 
 // Combine partitions inside the decode kernel (few partitions) or with the
@@ -996,27 +1079,31 @@ pa_status launch(const pa_decode_desc* d, DecodeArgs& a, const CUtensorMap& km,
                   cudaGetErrorString(e));
     if (dev >= 0 && dev < 64) configured[dev] = true;
   }
-  // Every kernel here (the counter reset, the decode, the reduce) is
+  // Every kernel here (the prep, the decode, the reduce) is
   // launched with programmatic stream serialization: each may start while
   // its predecessor drains and waits (griddepcontrol.wait) before touching
   // memory the predecessor writes.
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = kUsePdl;
-  if (a.max_parts > 1 && a.fused) {
-    const int n = d->num_seqs * d->num_kv_heads;
-    cudaLaunchConfig_t zcfg = {};
-    zcfg.gridDim = dim3((n + 1023) / 1024 < 64 ? (n + 1023) / 1024 : 64);
-    zcfg.blockDim = dim3(1024);
-    zcfg.stream = stream;
-    zcfg.attrs = attr;
-    zcfg.numAttrs = 1;
-    const cudaError_t ze =
-        cudaLaunchKernelEx(&zcfg, zero_counters_kernel, a.counters, n);
+  {
+    const int n = (a.max_parts > 1 && a.fused)
+                      ? d->num_seqs * d->num_kv_heads
+                      : 0;
+    cudaLaunchConfig_t pcfg = {};
+    pcfg.gridDim = dim3(1);
+    pcfg.blockDim = dim3(kPrepThreads);
+    pcfg.stream = stream;
+    pcfg.attrs = attr;
+    pcfg.numAttrs = 1;
+    const cudaError_t pe = cudaLaunchKernelEx(
+        &pcfg, prep_kernel, a.context_lens, d->num_seqs,
+        order_shift(a.max_context_len), const_cast<int32_t*>(a.order),
+        a.counters, n);
     count_launch();
-    if (ze != cudaSuccess)
-      return fail(PA_ERR_CUDA, "pa_decode: counter reset failed: %s",
-                  cudaGetErrorString(ze));
+    if (pe != cudaSuccess)
+      return fail(PA_ERR_CUDA, "pa_decode: prep launch failed: %s",
+                  cudaGetErrorString(pe));
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.max_parts, d->num_kv_heads, d->num_seqs);
@@ -1172,16 +1259,12 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache,
   a.q = q;
   a.block_tables = block_tables;
   a.context_lens = context_lens;
-  a.ws_o = static_cast<float*>(workspace);
-  a.ws_ml = need > 0 ? static_cast<float*>(workspace) +
-                           static_cast<size_t>(desc->num_seqs) *
-                               desc->num_q_heads * parts * desc->head_dim
-                     : nullptr;
-  a.counters = need > 0 ? reinterpret_cast<int*>(
-                               a.ws_ml + 2 * static_cast<size_t>(
-                                                 desc->num_seqs) *
-                                             desc->num_q_heads * parts)
-                         : nullptr;
+  const pagedkv::WsLayout wl = pagedkv::ws_layout(desc);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.ws_o = parts > 1 ? reinterpret_cast<float*>(ws + wl.o) : nullptr;
+  a.ws_ml = parts > 1 ? reinterpret_cast<float*>(ws + wl.ml) : nullptr;
+  a.counters = parts > 1 ? reinterpret_cast<int*>(ws + wl.counters) : nullptr;
+  a.order = reinterpret_cast<const int32_t*>(ws + wl.order);
   a.fused = pagedkv::use_fused(desc, parts) ? 1 : 0;
   a.dev_err = dev_err;
   a.scale_log2 = scale * pagedkv::kLog2e;
