@@ -791,10 +791,13 @@ def run_extras_only(args):
 
 
 def run_e2e(args, w, inp, dev, pkv, flow, world, rank, ps):
-    """Same step through the public API with host buffers: per step the
-    block manager appends one token to every sequence, the tables are
-    rebuilt, inputs go host->device from pinned memory, the output comes
-    back device->host."""
+    """Same step through the public API with host buffers.  Every step:
+    the block manager appends one token to every sequence and rebuilds the
+    tables (on the host), the step's inputs (q, the new tokens' K/V, slots,
+    tables, lengths) go host->device from pinned memory in one packed copy,
+    then cache write and decode, and the output comes back device->host;
+    one sync per step.  The host work of step n+1 runs while the GPU works
+    on step n (two pinned staging buffers); nothing else overlaps steps."""
     import torch
     bm = pkv.BlockManager(inp.num_blocks, w.block_size,
                           free_order=_free_order(inp))
@@ -803,77 +806,101 @@ def run_e2e(args, w, inp, dev, pkv, flow, world, rank, ps):
         bm.add_seq(int(b))
     bm.append_batch(ids, inp.lengths.astype(np.int32) - 1)
     steps = args.steps
-    max_blocks = int(wl_blocks(inp.lengths + steps + args.warmup + 1,
-                               w.block_size).max())
-    pin = dict(
-        q=inp.q.cpu().pin_memory(), k=inp.k_new.cpu().pin_memory(),
-        v=inp.v_new.cpu().pin_memory(),
-        out=torch.empty(inp.q.shape, dtype=inp.q.dtype).pin_memory())
-    dq = torch.empty_like(inp.q)
-    dk = torch.empty_like(inp.k_new)
-    dv = torch.empty_like(inp.v_new)
-    dout = torch.empty_like(inp.q)
-    ones = np.ones(w.num_seqs, dtype=np.int32)
-    stream = torch.cuda.current_stream(dev)
-    t_slots = torch.empty(w.num_seqs, dtype=torch.int64).pin_memory()
-    t_table = torch.empty(w.num_seqs, max_blocks,
-                          dtype=torch.int32).pin_memory()
-    t_lens = torch.empty(w.num_seqs, dtype=torch.int32).pin_memory()
-    h2d = d2h = 0
-    tot_bytes = 0
+    final_lens = inp.lengths + steps + args.warmup + 1
+    max_blocks = int(wl_blocks(final_lens, w.block_size).max())
+    B = w.num_seqs
+    # packed staging layout: (name, bytes, dtype, shape), 256-byte aligned
+    parts = [("q", inp.q), ("k", inp.k_new), ("v", inp.v_new)]
+    fields, off = {}, 0
+    for name, t in parts:
+        fields[name] = (off, t.nbytes, t.dtype, tuple(t.shape))
+        off = (off + t.nbytes + 255) & ~255
+    for name, nbytes, dt, shape in (
+            ("slots", B * 8, torch.int64, (B,)),
+            ("table", B * max_blocks * 4, torch.int32, (B, max_blocks)),
+            ("lens", B * 4, torch.int32, (B,))):
+        fields[name] = (off, nbytes, dt, shape)
+        off = (off + nbytes + 255) & ~255
+    total = off
 
-    def one(record):
-        nonlocal h2d, d2h, tot_bytes
-        stream.synchronize()          # pinned staging buffers are reused
-        slots, pairs = bm.append_batch(ids, ones, slots_out=t_slots.numpy())
-        table, lens = bm.block_table(ids, max_blocks,
-                                     table_out=t_table.numpy(),
-                                     lens_out=t_lens.numpy())
-        dq.copy_(pin["q"], non_blocking=True)
-        dk.copy_(pin["k"], non_blocking=True)
-        dv.copy_(pin["v"], non_blocking=True)
-        d_slots = t_slots.to(dev, non_blocking=True)
-        d_table = t_table.to(dev, non_blocking=True)
-        d_lens = t_lens.to(dev, non_blocking=True)
+    def views(buf):
+        return {k: buf[o:o + n].view(dt).view(shape)
+                for k, (o, n, dt, shape) in fields.items()}
+
+    stage = [torch.empty(total, dtype=torch.uint8).pin_memory()
+             for _ in range(2)]
+    hv = [views(x) for x in stage]
+    for v in hv:
+        for name, t in parts:
+            v[name].copy_(t.cpu())
+    dstage = torch.empty(total, dtype=torch.uint8, device=dev)
+    dv = views(dstage)
+    dout = torch.empty_like(inp.q)
+    hout = torch.empty(inp.q.shape, dtype=inp.q.dtype).pin_memory()
+    desc = pkv.make_desc(inp.q, inp.k_cache, dv["table"],
+                         partition_size=ps,
+                         max_context_len=int(final_lens.max()))
+    ws = torch.empty(max(pkv.pa_decode_workspace_bytes(desc), 16),
+                     dtype=torch.uint8, device=dev)
+    ones = np.ones(B, dtype=np.int32)
+    stream = torch.cuda.current_stream(dev)
+
+    def prepare(i):
+        """Host work of one step into staging buffer i."""
+        _, pairs = bm.append_batch(ids, ones, slots_out=hv[i]["slots"].numpy())
+        _, lens = bm.block_table(ids, max_blocks,
+                                 table_out=hv[i]["table"].numpy(),
+                                 lens_out=hv[i]["lens"].numpy())
+        return pairs, int(lens.sum())
+
+    def launch(i, pairs):
+        dstage.copy_(stage[i], non_blocking=True)
         nb = 0
         if len(pairs):
             d_pairs = torch.from_numpy(pairs).pin_memory().to(
                 dev, non_blocking=True)
             pkv.pa_copy_blocks(inp.k_cache, inp.v_cache, d_pairs)
-            nb += pairs.nbytes
-        pkv.pa_cache_write(inp.k_cache, inp.v_cache, dk, dv, d_slots)
-        pkv.pa_decode(dout, dq, inp.k_cache, inp.v_cache, d_table, d_lens,
-                      w.softmax_scale, partition_size=ps,
-                      max_context_len=int(lens.max()))
-        pin["out"].copy_(dout, non_blocking=True)
-        stream.synchronize()
-        if record:
-            h2d = (pin["q"].nbytes + pin["k"].nbytes + pin["v"].nbytes
-                   + slots.nbytes + table.nbytes + lens.nbytes + nb)
-            d2h = pin["out"].nbytes
-            tot_bytes += kv_bytes(lens, w)
+            nb = pairs.nbytes
+        pkv.pa_cache_write(inp.k_cache, inp.v_cache, dv["k"], dv["v"],
+                           dv["slots"])
+        pkv.pa_decode(dout, dv["q"], inp.k_cache, inp.v_cache, dv["table"],
+                      dv["lens"], w.softmax_scale, desc=desc, workspace=ws)
+        hout.copy_(dout, non_blocking=True)
+        return nb
 
-    for _ in range(args.warmup):
-        one(False)
+    tot_tokens, h2d = 0, 0
+    nxt = prepare(0)
+    for n in range(args.warmup):
+        launch(n % 2, nxt[0])
+        nxt = prepare((n + 1) % 2)
+        stream.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(steps):
-        one(True)
+    for n in range(args.warmup, args.warmup + steps):
+        pairs, tok = nxt
+        nb = launch(n % 2, pairs)
+        tot_tokens += tok
+        h2d = total + nb
+        if n + 1 < args.warmup + steps:
+            nxt = prepare((n + 1) % 2)
+        stream.synchronize()
     b.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(a.elapsed_time(b), world)
     bm.close()
+    tot_bytes = tot_tokens * w.num_kv_heads * w.head_dim * 2 * 2
     return {"value": round(world * tot_bytes / (ms * 1e-3) / 1e9, 2),
             "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h),
+            "d2h_bytes_per_step": int(hout.nbytes),
             "ms_per_step": round(ms / steps, 4),
-            "includes": "host block-manager append + table build, pinned "
-                        "H2D of q/new K,V/slots/tables/lengths, cache write, "
-                        "decode, D2H of the output, one sync per step"}
+            "includes": "host block-manager append + table build (for the "
+                        "next step, while the GPU runs this one), one packed "
+                        "pinned H2D of q/new K,V/slots/tables/lengths, cache "
+                        "write, decode, D2H of the output, one sync per step"}
 
 
 def wl_blocks(lengths, bs):
