@@ -63,6 +63,7 @@ constexpr int kMaxGroup = 8;                       // query heads per KV head
 constexpr int kMaxPartition = 8192;
 constexpr int kMaxParts = 16384;                   // partitions per sequence
 constexpr int kFusedMaxParts = 16;  // up to this many: combine in the decode
+constexpr int kWarpPartsMaxPartition = 1024;  // warp_parts up to this size
 
 struct DecodeArgs {
   void* out;
@@ -74,6 +75,8 @@ struct DecodeArgs {
   int* counters; // [num_seqs, num_kv_heads] finished partitions (fused mode)
   const int32_t* order;  // [num_seqs] sequence served by grid row z
   int fused;     // 1: the last partition CTA combines; 0: the reduce kernel
+  int warp_parts;  // 1: a CTA serves kConsumers consecutive partitions, one
+                   // per consumer warp (reduce kernel path, short partitions)
   int32_t* dev_err;
   float scale_log2;  // scale * log2(e): scores are kept in base-2 units
   int num_q_heads;
@@ -248,7 +251,10 @@ __global__ void __launch_bounds__(kThreads)
   // must start on a 1024-byte boundary of the shared window.
   uint8_t* smem = smem_dyn + ((1024u - (dev::smem_u32(smem_dyn) & 1023u)) & 1023u);
 
-  const int part = blockIdx.x;
+  // Partitions this CTA serves: one, or (warp_parts) kConsumers consecutive
+  // ones, consumer warp w taking partition part + w.
+  const int nsub = a.warp_parts ? kConsumers : 1;
+  const int part = blockIdx.x * nsub;
   const int kvh = blockIdx.y;
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -280,7 +286,7 @@ __global__ void __launch_bounds__(kThreads)
       a.block_tables + static_cast<int64_t>(b) * a.max_blocks_per_seq + page0;
   const int row_left = a.max_blocks_per_seq - page0;
   const int ctx = a.context_lens[b];
-  for (int i = tid; i < pages_per_part && i < row_left; i += kThreads)
+  for (int i = tid; i < nsub * pages_per_part && i < row_left; i += kThreads)
     bt_s[i] = bt_row[i];
   if (ctx < 0 || ctx > a.max_blocks_per_seq * BS || ctx > a.max_context_len) {
     if (part == 0 && kvh == 0 && tid == 0)
@@ -290,7 +296,8 @@ __global__ void __launch_bounds__(kThreads)
   const int n_parts = ctx > 0 ? (ctx + PS - 1) / PS : 1;
   if (part >= n_parts) return;
   const int tok0 = part * PS;
-  const int n_tok = min(ctx - tok0, PS);  // 0 only when ctx == 0
+  // Tokens (and staged pages) of this CTA's partitions; 0 only when ctx == 0.
+  const int n_tok = min(ctx - tok0, nsub * PS);
   const int n_pages = (n_tok + BS - 1) / BS;
   const int G = a.group;
 
@@ -314,13 +321,15 @@ __global__ void __launch_bounds__(kThreads)
   if (bad) {
     if (tid == 0) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
     if (n_parts > 1) {
-      if (tid < G) {  // mark the partition empty for the combine
-        const int64_t row =
-            (static_cast<int64_t>(b) * a.num_q_heads + kvh * G + tid) *
-                a.max_parts + part;
-        a.ws_ml[2 * row] = -INFINITY;
-        a.ws_ml[2 * row + 1] = 0.f;
-      }
+      // mark the CTA's partitions empty for the combine
+      for (int k = 0; k < nsub && part + k < n_parts; ++k)
+        if (tid < G) {
+          const int64_t row =
+              (static_cast<int64_t>(b) * a.num_q_heads + kvh * G + tid) *
+                  a.max_parts + part + k;
+          a.ws_ml[2 * row] = -INFINITY;
+          a.ws_ml[2 * row + 1] = 0.f;
+        }
       if (a.fused) {  // still counts as finished: the others may be fine
         __threadfence();
         __syncthreads();
@@ -342,7 +351,19 @@ __global__ void __launch_bounds__(kThreads)
     if (lane == 0 && n_pages > 0) {
       dev::prefetch_tmap(&kmap);
       dev::prefetch_tmap(&vmap);
-      for (int i = 0; i < n_pages; ++i) {
+      // warp_parts: pages are interleaved across the partitions (index i is
+      // page i / kConsumers of partition i % kConsumers), so consumer warp w
+      // still gets every page i = w (mod kConsumers) and owns its stages;
+      // pages past a shorter partition's end are skipped, which only ever
+      // stops the reuse of that warp's stages.
+      const int n_iter =
+          a.warp_parts ? kConsumers * min(n_pages, pages_per_part) : n_pages;
+      for (int i = 0; i < n_iter; ++i) {
+        int slot = i;
+        if (a.warp_parts) {
+          slot = (i % kConsumers) * pages_per_part + i / kConsumers;
+          if (slot >= n_pages) continue;
+        }
         const int s = i % S;
         if (i >= S && !dev::mbar_wait(empty0 + s * 8, ((i / S) - 1) & 1)) {
           dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
@@ -350,7 +371,7 @@ __global__ void __launch_bounds__(kThreads)
         }
         const uint32_t full = full0 + s * 8;
         dev::mbar_arrive_expect_tx(full, Geo::kStageBytes);
-        const int y = (bt_s[i] * a.num_kv_heads + kvh) * BS;
+        const int y = (bt_s[slot] * a.num_kv_heads + kvh) * BS;
         const uint32_t kdst = ring + s * Geo::kStageBytes;
 #pragma unroll
         for (int bx = 0; bx < Geo::kBoxes; ++bx) {
@@ -399,7 +420,12 @@ __global__ void __launch_bounds__(kThreads)
     const int mi = lane >> 3;
     const int j = lane & 7;
 
-    for (int i = cw; i < n_pages; i += kConsumers) {
+    // Tokens this warp's pages cover: the CTA's partition (the warps share
+    // it), or with warp_parts this warp's own partition part + cw.
+    const int w_tok = a.warp_parts ? max(0, min(n_tok - cw * PS, PS)) : n_tok;
+    const int w_iter =
+        a.warp_parts ? kConsumers * ((w_tok + BS - 1) / BS) : n_pages;
+    for (int i = cw; i < w_iter; i += kConsumers) {
       const int s = i % S;
       if (!dev::mbar_wait(full0 + s * 8, (i / S) & 1)) {
         dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
@@ -407,7 +433,8 @@ __global__ void __launch_bounds__(kThreads)
       }
       const uint32_t kb = ring + s * Geo::kStageBytes;
       const uint32_t vb = kb + Geo::kPageBytes;
-      const int nv = min(BS, n_tok - i * BS);
+      const int pg = a.warp_parts ? i / kConsumers : i;  // page of w_tok
+      const int nv = min(BS, w_tok - pg * BS);
       if (nv < BS) {
         // Slots past the context get P = 0, but 0 * NaN is NaN in the MMA:
         // clear the V rows the sequence never wrote (last page only).
@@ -502,6 +529,48 @@ __global__ void __launch_bounds__(kThreads)
       if (lane == 0) dev::mbar_arrive(empty0 + s * 8);
     }
 
+    if (a.warp_parts) {
+      // This warp's partition is complete: write its partial directly
+      // (no merge with the other warps, which hold other partitions).
+      const int mypart = part + cw;
+      if (mypart < n_parts) {
+        float lt[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float l = l_run[h];
+          l += __shfl_xor_sync(0xffffffffu, l, 4);
+          l += __shfl_xor_sync(0xffffffffu, l, 8);
+          l += __shfl_xor_sync(0xffffffffu, l, 16);
+          lt[h] = l;
+        }
+        const int64_t row0 =
+            static_cast<int64_t>(b) * a.num_q_heads + kvh * G;
+#pragma unroll
+        for (int dt = 0; dt < D / 16; ++dt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int g = 2 * t4 + (e & 1);
+            if (g < G) {
+              const int64_t row = (row0 + g) * a.max_parts + mypart;
+              const float l = lt[e & 1];
+              a.ws_o[row * D + dt * 16 + g4 + (e >> 1) * 8] =
+                  l > 0.f ? o[dt][e] / l : 0.f;
+            }
+          }
+        if (g4 == 0) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int g = 2 * t4 + h;
+            if (g < G) {
+              const int64_t row = (row0 + g) * a.max_parts + mypart;
+              a.ws_ml[2 * row] = m_run[h];
+              a.ws_ml[2 * row + 1] = lt[h];
+            }
+          }
+        }
+      }
+      return;
+    }
     // Hand this warp's state to the epilogue area (aliases the ring).
     dev::named_barrier(1, kConsumers * 32);
     float* ep = reinterpret_cast<float*>(smem) + cw * Geo::kEpiWarpFloats;
@@ -1065,8 +1134,8 @@ pa_status launch(const pa_decode_desc* d, DecodeArgs& a, const CUtensorMap& km,
                  const CUtensorMap& vm, cudaStream_t stream) {
   constexpr int S = stages_for(BS, D);
   auto kern = decode_kernel<T, BS, D, S, kMma>;
-  const size_t smem =
-      smem_bytes_for<BS, D, S, kMma>(a.partition_size / BS);
+  const size_t smem = smem_bytes_for<BS, D, S, kMma>(
+      (a.warp_parts ? kConsumers : 1) * a.partition_size / BS);
   int dev = 0;
   cudaGetDevice(&dev);
   static bool configured[64] = {false};
@@ -1106,7 +1175,9 @@ pa_status launch(const pa_decode_desc* d, DecodeArgs& a, const CUtensorMap& km,
                   cudaGetErrorString(pe));
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.max_parts, d->num_kv_heads, d->num_seqs);
+  cfg.gridDim = dim3(a.warp_parts ? (a.max_parts + kConsumers - 1) / kConsumers
+                                   : a.max_parts,
+                     d->num_kv_heads, d->num_seqs);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -1266,6 +1337,12 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache,
   a.counters = parts > 1 ? reinterpret_cast<int*>(ws + wl.counters) : nullptr;
   a.order = reinterpret_cast<const int32_t*>(ws + wl.order);
   a.fused = pagedkv::use_fused(desc, parts) ? 1 : 0;
+  // Short partitions combined by the reduce kernel: one partition per
+  // consumer warp, kConsumers per CTA (fewer, longer CTAs; no merge).
+  a.warp_parts = (desc->kernel != PA_KERNEL_SIMT && !a.fused && parts > 1 &&
+                  ps <= pagedkv::kWarpPartsMaxPartition)
+                     ? 1
+                     : 0;
   a.dev_err = dev_err;
   a.scale_log2 = scale * pagedkv::kLog2e;
   a.num_q_heads = desc->num_q_heads;
