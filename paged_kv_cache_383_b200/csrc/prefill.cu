@@ -17,23 +17,29 @@
 // per KV head a tile holds 128/G tokens and each K/V byte serves all G heads.
 //   * Warp 0, lane 0 loads the Q tile with one 3-D TMA box per half of
 //     head_dim, then streams 64-key K and V tiles page by page (2-D TMA boxes
-//     of block_size rows x 128 B, 128-byte swizzle, no multicast) into a
-//     3-stage ring.  Pages are placed so that a tile is the canonical
-//     128-byte-swizzled layout the tensor core reads.
+//     of block_size rows x 128 B, 128-byte swizzle, no multicast) into
+//     separate 2-stage K and V rings: a K stage is free again once S(j) has
+//     read it, a V stage once P(j).V has, and V tile j is loaded after K
+//     tile j+1 since it is needed a tile later.  Pages are placed so that a
+//     tile is the canonical 128-byte-swizzled layout the tensor core reads.
 //   * Warp 1 allocates 256 tensor-memory columns; its lane 0 issues
-//     S = Q K^T (M=128, N=64) and O += P V (M=128, N=128, V read MN-major)
-//     as tcgen05.mma with fp32 accumulators in tensor memory, and signals
-//     completion with tcgen05.commit.  S and P are double-buffered, so the
-//     tensor cores compute S(j+1) and P(j-1).V while the softmax warps work
-//     on tile j.
+//     S = Q K^T (M=128, N=64, both operands in shared memory) and
+//     O += P V (M=128, N=128; P read from tensor memory, V from shared
+//     memory, MN-major) as tcgen05.mma with fp32 accumulators, and signals
+//     completion with tcgen05.commit.  S is double-buffered and P is written
+//     over the S it came from, so the tensor cores compute S(j+1) and
+//     P(j-1).V while the softmax warps work on tile j; S(j+2) is issued once
+//     P(j).V has finished reading that buffer.
 //   * Warps 2..5 own one tensor-memory row each (thread = query row): they
 //     read S with tcgen05.ld, apply the causal mask (diagonal tiles only),
 //     keep the online softmax in registers (no shuffles: a row is one
-//     thread), compute the exponentials before waiting for the previous P.V,
-//     rescale O in tensor memory only when the running maximum grows by more
-//     than 2^8 (the final division uses the same reference, so the result is
-//     unchanged), and write P to shared memory as a 16-bit rounded part plus
-//     its residual so P . V keeps ~16 mantissa bits.
+//     thread), rescale O in tensor memory only when the running maximum
+//     grows by more than 2^8 (the final division uses the same reference,
+//     so the result is unchanged), and store P with tcgen05.st as a 16-bit
+//     rounded part plus its residual so P . V keeps ~16 mantissa bits.
+//   * Shared memory is ~99 KB (Q, the rings, barriers, the block-table slice)
+//     and tensor memory 256 columns, so two CTAs share an SM: one CTA's
+//     softmax runs while the other's tiles are on the tensor cores.
 //   * Every wait is bounded (1 s) and reports PA_ERR_DEVICE_TIMEOUT; tensor
 //     memory is always released.  A barrier that is waited on by parity is
 //     never allowed to run two phases ahead of its waiter: each double
@@ -49,6 +55,7 @@
 #include "device_utils.cuh"
 #include "pagedkv.h"
 #include "status.h"
+#include "tcgen05_ts.cuh"
 
 namespace pagedkv {
 namespace {
@@ -57,7 +64,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kRows = 128;      // query rows per tile (tensor memory lanes)
 constexpr int kKeys = 64;       // keys per K/V tile
 constexpr int kD = 128;         // head_dim
-constexpr int kStages = 3;      // K/V ring depth
+constexpr int kKStages = 2;     // K ring depth
+constexpr int kVStages = 2;     // V ring depth
 constexpr int kThreads = 192;   // producer, MMA, 4 softmax warps
 constexpr int kTmemCols = 256;  // S: cols [0, 64), O: cols [128, 256)
 constexpr float kRescaleLog2 = 8.f;
@@ -82,16 +90,14 @@ constexpr int kQBytes = kRows * kD * 2;                 // 32 KB, two halves
 constexpr int kHalfQ = kRows * 128;                     // 16 KB
 constexpr int kTileHalf = kKeys * 128;                  // 8 KB: 64 keys x 64 d
 constexpr int kKVTile = 2 * kTileHalf;                  // 16 KB per K or V
-constexpr int kStageBytes = 2 * kKVTile;                // K + V
-constexpr int kPBytes = kRows * kKeys * 2;              // 16 KB per P part
-constexpr int kPBuf = 2 * kPBytes;                      // rounded + residual
 constexpr int kOffQ = 0;
-constexpr int kOffRing = kOffQ + kQBytes;
-constexpr int kOffP = kOffRing + kStages * kStageBytes;  // 2 P buffers
-constexpr int kOffBars = kOffP + 2 * kPBuf;
-// barriers: q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2],
-// p_full[2], o_ready[2], done, then the tensor-memory base address word.
-constexpr int kNumBars = 1 + 2 * kStages + 4 * 2 + 1;
+constexpr int kOffK = kOffQ + kQBytes;
+constexpr int kOffV = kOffK + kKStages * kKVTile;
+constexpr int kOffBars = kOffV + kVStages * kKVTile;
+// barriers: q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
+// s_full[2], s_free[2], p_full[2], o_ready[2], done, then the tensor-memory
+// base address word.
+constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 4 * 2 + 1;
 constexpr int kOffTable = kOffBars + kNumBars * 8 + 16;
 
 size_t prefill_smem_bytes(int max_pages) {
@@ -99,7 +105,7 @@ size_t prefill_smem_bytes(int max_pages) {
 }
 
 template <typename T, int BS, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap,
                    const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap,
@@ -113,14 +119,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       smem_dyn + ((1024u - (dev::smem_u32(smem_dyn) & 1023u)) & 1023u);
   const uint32_t base = dev::smem_u32(smem);
   const uint32_t q_s = base + kOffQ;
-  const uint32_t ring = base + kOffRing;
-  const uint32_t p_s = base + kOffP;
+  const uint32_t kring = base + kOffK;
+  const uint32_t vring = base + kOffV;
   const uint32_t bars = base + kOffBars;
   const uint32_t q_full = bars;
-  const uint32_t kv_full0 = bars + 8;
-  const uint32_t kv_empty0 = kv_full0 + kStages * 8;
+  const uint32_t k_full0 = bars + 8;
+  const uint32_t k_empty0 = k_full0 + kKStages * 8;
+  const uint32_t v_full0 = k_empty0 + kKStages * 8;
+  const uint32_t v_empty0 = v_full0 + kVStages * 8;
   // Double-buffer barriers: tile t uses element t & 1, phase t >> 1.
-  const uint32_t s_full0 = kv_empty0 + kStages * 8;
+  const uint32_t s_full0 = v_empty0 + kVStages * 8;
   const uint32_t s_free0 = s_full0 + 16;
   const uint32_t p_full0 = s_free0 + 16;
   const uint32_t o_ready0 = p_full0 + 16;
@@ -163,9 +171,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 0) {
     dev::mbar_init(q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      dev::mbar_init(kv_full0 + 8 * s, 1);
-      dev::mbar_init(kv_empty0 + 8 * s, 1);
+    for (int s = 0; s < kKStages; ++s) {
+      dev::mbar_init(k_full0 + 8 * s, 1);
+      dev::mbar_init(k_empty0 + 8 * s, 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      dev::mbar_init(v_full0 + 8 * s, 1);
+      dev::mbar_init(v_empty0 + 8 * s, 1);
     }
     for (int i = 0; i < 2; ++i) {
       dev::mbar_init(s_full0 + 8 * i, 1);
@@ -189,8 +201,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   dev::tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  const uint32_t s_tmem = tbase;        // S buffers: columns [0, 64), [64, 128)
-  const uint32_t o_tmem = tbase + 128;  // O: columns [128, 256)
+  // S / P buffers: columns [0, 64) and [64, 128); O: columns [128, 256).
+  // P(j) (rounded part in the first 32 columns, residual in the next 32,
+  // two 16-bit values per column) overwrites S(j) once it has been read.
+  const uint32_t s_tmem = tbase;
+  const uint32_t o_tmem = tbase + 128;
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -201,17 +216,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_arrive_expect_tx(q_full, kQBytes);
       dev::tma_load_3d(q_s, &qmap, 0, kvh * G, q0 + tok0, q_full);
       dev::tma_load_3d(q_s + kHalfQ, &qmap, 64, kvh * G, q0 + tok0, q_full);
-      for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % kStages;
-        if (j >= kStages &&
-            !dev::mbar_wait(kv_empty0 + 8 * s, ((j / kStages) - 1) & 1)) {
-          dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
-          break;
-        }
-        const uint32_t full = kv_full0 + 8 * s;
-        dev::mbar_arrive_expect_tx(full, kStageBytes);
-        const uint32_t kt = ring + s * kStageBytes;
-        const uint32_t vt = kt + kKVTile;
+      // K tile j and V tile j-1 per step: a K stage is free once S(j) has
+      // read it, a V stage once P(j).V has, and V is needed a tile later.
+      auto load = [&](int j, bool is_v) -> bool {
+        const int ns = is_v ? kVStages : kKStages;
+        const int s = j % ns;
+        const uint32_t empty = (is_v ? v_empty0 : k_empty0) + 8 * s;
+        if (j >= ns && !dev::mbar_wait(empty, ((j / ns) - 1) & 1))
+          return false;
+        const uint32_t full = (is_v ? v_full0 : k_full0) + 8 * s;
+        dev::mbar_arrive_expect_tx(full, kKVTile);
+        const uint32_t dst = (is_v ? vring : kring) + s * kKVTile;
+        const CUtensorMap* map = is_v ? &vmap : &kmap;
 #pragma unroll
         for (int p = 0; p < kPagesPerTile; ++p) {
           const int page = j * kPagesPerTile + p;
@@ -219,10 +235,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int32_t phys = page < n_pages ? bt_s[page] : bt_s[0];
           const int y = (phys * a.num_kv_heads + kvh) * BS;
           const uint32_t off = p * BS * 128;
-          dev::tma_load_2d(kt + off, &kmap, 0, y, full);
-          dev::tma_load_2d(kt + kTileHalf + off, &kmap, 64, y, full);
-          dev::tma_load_2d(vt + off, &vmap, 0, y, full);
-          dev::tma_load_2d(vt + kTileHalf + off, &vmap, 64, y, full);
+          dev::tma_load_2d(dst + off, map, 0, y, full);
+          dev::tma_load_2d(dst + kTileHalf + off, map, 64, y, full);
+        }
+        return true;
+      };
+      for (int t = 0; t <= n_tiles; ++t) {
+        if ((t < n_tiles && !load(t, false)) || (t >= 1 && !load(t - 1, true))) {
+          dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
+          break;
         }
       }
     }
@@ -238,40 +259,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_pv = dev::umma_idesc_f16(kBf16, kRows, kD,
                                                         false, true);
       auto issue_pv = [&](int t) -> bool {
-        if (!dev::mbar_wait(p_full0 + 8 * (t & 1), (t >> 1) & 1)) return false;
+        if (!dev::mbar_wait(p_full0 + 8 * (t & 1), (t >> 1) & 1) ||
+            !dev::mbar_wait(v_full0 + 8 * (t % kVStages), (t / kVStages) & 1))
+          return false;
         dev::tc_fence_after();
-        const uint32_t vt = ring + (t % kStages) * kStageBytes + kKVTile;
-        const uint32_t pb = p_s + (t & 1) * kPBuf;
+        const uint32_t vt = vring + (t % kVStages) * kKVTile;
+        const uint32_t pt = s_tmem + (t & 1) * kKeys;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {  // P rounded part, residual
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk) {
-            const uint64_t ad =
-                dev::sw128_desc(pb + part * kPBytes + kk * 32, 16, 1024);
             // V as the MN-major B operand: 64-wide d halves kTileHalf apart,
             // 8-key groups 1024 bytes apart.
             const uint64_t bd =
                 dev::sw128_desc(vt + kk * 2048, kTileHalf, 1024);
-            dev::umma_f16(o_tmem, ad, bd, idesc_pv,
-                          (t > 0 || part > 0 || kk > 0) ? 1u : 0u);
+            dev::umma_f16_ts(o_tmem, pt + part * (kKeys / 2) + kk * 8, bd,
+                             idesc_pv, (t > 0 || part > 0 || kk > 0) ? 1u : 0u);
           }
         }
         dev::umma_commit(o_ready0 + 8 * (t & 1));
-        dev::umma_commit(kv_empty0 + 8 * (t % kStages));
+        dev::umma_commit(v_empty0 + 8 * (t % kVStages));
         return true;
       };
       ok = dev::mbar_wait(q_full, 0);
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % kStages;
-        // S buffer j & 1 is free once the softmax warps have read S(j-2).
-        if (!dev::mbar_wait(kv_full0 + 8 * s, (j / kStages) & 1) ||
+        const int s = j % kKStages;
+        // Buffer j & 1 is free once the softmax warps have read S(j-2) and
+        // P(j-2).V has read the P written over it.
+        if (!dev::mbar_wait(k_full0 + 8 * s, (j / kKStages) & 1) ||
             (j >= 2 &&
-             !dev::mbar_wait(s_free0 + 8 * (j & 1), ((j >> 1) - 1) & 1))) {
+             (!dev::mbar_wait(s_free0 + 8 * (j & 1), ((j >> 1) - 1) & 1) ||
+              !dev::mbar_wait(o_ready0 + 8 * (j & 1), ((j >> 1) - 1) & 1)))) {
           ok = false;
           break;
         }
         dev::tc_fence_after();
-        const uint32_t kt = ring + s * kStageBytes;
+        const uint32_t kt = kring + s * kKVTile;
         const uint32_t sd = s_tmem + (j & 1) * kKeys;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
@@ -283,6 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           dev::umma_f16(sd, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
         dev::umma_commit(s_full0 + 8 * (j & 1));
+        dev::umma_commit(k_empty0 + 8 * s);
         if (j >= 1 && !issue_pv(j - 1)) {
           ok = false;
           break;
@@ -342,14 +366,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (k0 + kKeys > L) {
       // Keys past the context get P = 0, but 0 * NaN is NaN in the MMA:
       // clear the V rows of slots the sequence never wrote (and of pages
-      // past it).  Warp q clears rows 16q .. 16q+15 of the last tile.
-      const uint32_t vt = ring + (j % kStages) * kStageBytes + kKVTile;
+      // past it).  Warp q clears rows 16q .. 16q+15 of the last tile, once
+      // it has landed (P(j).V, the stage's next reader, waits for p_full).
+      ok = __all_sync(0xffffffffu,
+                      dev::mbar_wait(v_full0 + 8 * (j % kVStages),
+                                     (j / kVStages) & 1));
+      if (!ok) break;
+      const uint32_t vt = vring + (j % kVStages) * kKVTile;
       for (int idx = lane; idx < 16 * 16; idx += 32) {
         const int krow = quarter * 16 + (idx >> 4), ch = idx & 15;
         if (k0 + krow >= L)
           dev::st_shared_zero16(vt + (ch >> 3) * kTileHalf + krow * 128 +
                                 (ch & 7) * 16);
       }
+      dev::fence_proxy_async_smem();  // visible to the tensor cores' P.V
     }
     // Causal mask: only tiles that reach past this row's position.
     const int lim = qpos - k0;
@@ -393,32 +423,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       dev::tmem_st_wait();
     }
-    // P buffer j & 1 was last read by P(j-2).V.
-    if (j >= 2) {
-      ok = wait_pv(j - 2);
-      if (!ok) break;
-    }
-    // Row r of the K-major 128-byte-swizzled A operand (16-byte chunk ch at
-    // ch ^ (r % 8)): rounded part, then the residual.
-    uint8_t* prow_hi = smem + kOffP + (j & 1) * kPBuf + r * 128;
-    uint8_t* prow_lo = prow_hi + kPBytes;
+    // P over S(j) in its tensor-memory buffer: rounded part, then residual.
+    {
+      uint32_t hw[kKeys / 2], lw[kKeys / 2];
 #pragma unroll
-    for (int ch = 0; ch < kKeys / 8; ++ch) {
-      uint32_t hw[4], lw[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float p0 = sv[8 * ch + 2 * e], p1 = sv[8 * ch + 2 * e + 1];
+      for (int e = 0; e < kKeys / 2; ++e) {
+        const float p0 = sv[2 * e], p1 = sv[2 * e + 1];
         hw[e] = M::pack(p0, p1);
         const float2 hf = M::unpack(hw[e]);
         lw[e] = M::pack(p0 - hf.x, p1 - hf.y);
       }
-      const int sw = (ch ^ (r & 7)) * 16;
-      *reinterpret_cast<uint4*>(prow_hi + sw) =
-          make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(prow_lo + sw) =
-          make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      const uint32_t pa = s_tmem + (j & 1) * kKeys + lane_off;
+      dev::tmem_st32u(pa, hw);
+      dev::tmem_st32u(pa + kKeys / 2, lw);
+      dev::tmem_st_wait();
     }
-    dev::fence_proxy_async_smem();
     dev::tc_fence_before();
     __syncwarp();
     if (lane == 0) dev::mbar_arrive(p_full0 + 8 * (j & 1));
