@@ -245,35 +245,54 @@ def run_native(args, rank, world, local):
         step()
     torch.cuda.synchronize()
 
-    # Timed region: exactly K steps, events only at its two ends (an event
-    # between the kernels would break their programmatic-launch overlap).
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
+    # K/V a step reads at least once; below twice the L2 size the data would
+    # stay cached between steps, so L2 is flushed (a 256 MB write) between
+    # timed steps and each step is timed on its own.
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    unique_bytes = spec.info.get("unique_kv_bytes_per_step", step_bytes)
+    flush = unique_bytes < 2 * l2_bytes
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) \
+        if flush else None
+
+    def timed(fn):
+        """Total ms of args.steps calls of fn on the stream."""
+        if not flush:
+            # events only at the two ends (an event between the kernels
+            # would break their programmatic-launch overlap)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1)
+        evs = [(torch.cuda.Event(enable_timing=True),
+                torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for e0, e1 in evs:
+            flush_buf.fill_(1)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return sum(e0.elapsed_time(e1) for e0, e1 in evs)
+
+    # Timed region: exactly K steps.
     launches0 = pkv.pa_launch_count()
     barrier(world)
     torch.cuda.synchronize()
-    t0.record(stream)
-    for _ in range(args.steps):
-        step()
-    t1.record(stream)
-    torch.cuda.synchronize()
+    ms_local = timed(step)
     barrier(world)
     launches = pkv.pa_launch_count() - launches0
-    ms_local = t0.elapsed_time(t1)
     ms_total = max_over_ranks(ms_local, world)
-    # The dominant kernel's launch duration: K back-to-back pa_decode calls on
-    # the same inputs, timed the same way on the same stream.
-    d0 = torch.cuda.Event(enable_timing=True)
-    d1 = torch.cuda.Event(enable_timing=True)
-    d0.record(stream)
-    for _ in range(args.steps):
-        pkv.pa_decode(out, inp.q, inp.k_cache, inp.v_cache, bt, cl,
-                      w.softmax_scale, desc=desc, workspace=ws, dev_err=err,
-                      stream=stream)
-    d1.record(stream)
-    torch.cuda.synchronize()
+    # The dominant kernel's launch duration: K pa_decode calls on the same
+    # inputs, timed the same way on the same stream.
+    dec_ms = max_over_ranks(timed(lambda: pkv.pa_decode(
+        out, inp.q, inp.k_cache, inp.v_cache, bt, cl, w.softmax_scale,
+        desc=desc, workspace=ws, dev_err=err, stream=stream)), world) \
+        / args.steps
     clk = clocks.stop()
-    dec_ms = max_over_ranks(d0.elapsed_time(d1), world) / args.steps
     if err.item() != 0:
         raise RuntimeError(f"device error flag {err.item()} during bench")
 
@@ -307,8 +326,11 @@ def run_native(args, rank, world, local):
             "kernel": args.kernel,
             "kv_bytes_per_step": step_bytes,
             **spec.info,
-            "l2": "inputs larger than L2 (no flush): "
-                  f"{step_bytes / 1e9:.2f} GB of K/V read per step",
+            "l2": (f"L2 flushed between timed steps (256 MB write outside "
+                   f"the per-step events): {unique_bytes / 1e6:.1f} MB of "
+                   f"K/V per step" if flush else
+                   f"inputs larger than L2 (no flush): {unique_bytes / 1e9:.2f}"
+                   f" GB of distinct K/V per step"),
             "parallelism": f"{world} independent replicas" if world > 1
                            else "1 GPU",
         },
@@ -323,8 +345,10 @@ def run_native(args, rank, world, local):
             "frac_of_spec_8000": round(achieved / SPEC_HBM_GBS, 4),
             "traffic": profiled_traffic(w.name),
             "decode_ms": round(dec_ms, 5),
-            "decode_ms_how": "K back-to-back pa_decode calls on the step's "
-                             "inputs, CUDA events on the launch stream",
+            "decode_ms_how": ("K pa_decode calls on the step's inputs, CUDA "
+                              "events on the launch stream" +
+                              (", L2 flushed before each" if flush else
+                               ", back to back")),
         },
         "gpu_launches": int(launches),
         "clocks": clk,
@@ -341,6 +365,9 @@ def run_native(args, rank, world, local):
         else:
             res["e2e"] = run_e2e(args, w, inp, dev, pkv, flow, world, rank,
                                  ps)
+    if flush and "e2e" in res:
+        res["e2e"]["l2"] = (f"the {unique_bytes / 1e6:.1f} MB of K/V stay in "
+                            f"L2 between end-to-end steps (not flushed there)")
     if want_cpu and w.lengths != "prefix":
         res["cpu_baseline"] = cpu_baseline(pool, inp, w, dev)
     if pool is not None:
@@ -537,12 +564,70 @@ def extras(args, w, inp, dev, pkv, bt, cl):
     out["torch_sum_read_gbs"] = round(4 * (1 << 30) / (a.elapsed_time(b) /
                                                         10 * 1e-3) / 1e9, 1)
     del x
+    out["identity_vs_shuffled"] = identity_vs_shuffled(pkv, w, inp, dev)
     from paged_kv_cache_383_b200 import workloads as wl
     out["prefill"] = [time_prefill(pkv, wl, n, c, dev)
                       for n, c in PREFILL_CASES]
     out["prefix_cache"] = prefix_cache_measure(pkv, dev)
     out["swap"] = swap_measure(pkv, dev)
     return out
+
+
+def identity_vs_shuffled(pkv, w, inp, dev):
+    """The same decode over the shuffled pool and over a copy laid out so
+    every sequence's blocks are consecutive (identity tables): the whole
+    batch, and batch 1 (its longest sequence; L2 flushed before each call,
+    the data being smaller than L2).  GB/s of K/V read."""
+    import torch
+    B = inp.block_tables.shape[0]
+    rows = [inp.block_tables[b][inp.block_tables[b] >= 0] for b in range(B)]
+    order = torch.from_numpy(np.concatenate(rows).astype(np.int64)).to(dev)
+    kc = inp.k_cache[order].contiguous()
+    vc = inp.v_cache[order].contiguous()
+    ident = np.full_like(inp.block_tables, -1)
+    base = 0
+    for b, r in enumerate(rows):
+        ident[b, :len(r)] = np.arange(base, base + len(r))
+        base += len(r)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def run(seqs, tables, k, v, flush):
+        q = inp.q[seqs].contiguous()
+        bt = torch.from_numpy(tables[seqs]).to(dev)
+        lens = inp.lengths[seqs]
+        cl = torch.from_numpy(lens.astype(np.int32)).to(dev)
+        o = torch.empty_like(q)
+        desc = pkv.make_desc(q, k, bt, max_context_len=int(lens.max()))
+        ws = torch.empty(pkv.pa_decode_workspace_bytes(desc),
+                         dtype=torch.uint8, device=dev)
+        f = lambda: pkv.pa_decode(o, q, k, v, bt, cl, w.softmax_scale,
+                                  desc=desc, workspace=ws)
+        for _ in range(3):
+            f()
+        n, total = 20, 0.0
+        for _ in range(n):
+            if flush:
+                flush_buf.fill_(1)
+            a = torch.cuda.Event(enable_timing=True)
+            b_ = torch.cuda.Event(enable_timing=True)
+            a.record()
+            f()
+            b_.record()
+            torch.cuda.synchronize()
+            total += a.elapsed_time(b_)
+        return round(kv_bytes(lens, w) / (total / n * 1e-3) / 1e9, 1)
+
+    allb = np.arange(B)
+    one = np.array([int(np.argmax(inp.lengths))])
+    res = {"batch_gbs_shuffled": run(allb, inp.block_tables, inp.k_cache,
+                                     inp.v_cache, False),
+           "batch_gbs_identity": run(allb, ident, kc, vc, False),
+           "batch1_tokens": int(inp.lengths[one[0]]),
+           "batch1_gbs_shuffled": run(one, inp.block_tables, inp.k_cache,
+                                      inp.v_cache, True),
+           "batch1_gbs_identity": run(one, ident, kc, vc, True)}
+    del kc, vc
+    return res
 
 
 def measured_bf16_peak():

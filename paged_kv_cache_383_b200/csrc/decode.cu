@@ -545,6 +545,22 @@ __global__ void __launch_bounds__(kThreads)
         }
         const int64_t row0 =
             static_cast<int64_t>(b) * a.num_q_heads + kvh * G;
+        if (n_parts == 1) {
+          // The reduce kernel skips single-partition rows: write the output.
+#pragma unroll
+          for (int dt = 0; dt < D / 16; ++dt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int g = 2 * t4 + (e & 1);
+              if (g < G) {
+                const float l = lt[e & 1];
+                static_cast<T*>(a.out)[(row0 + g) * D + dt * 16 + g4 +
+                                       (e >> 1) * 8] =
+                    from_float<T>(l > 0.f ? o[dt][e] / l : 0.f);
+              }
+            }
+          return;
+        }
 #pragma unroll
         for (int dt = 0; dt < D / 16; ++dt)
 #pragma unroll

@@ -216,3 +216,22 @@ def test_unwritten_slots_hold_nan(pkv, kernel, bs):
     for ps in (0, 64):
         out = _run(pkv, inp, kernel=kernel, partition_size=ps)
         check_decode(to_np(out), ref, inp.q.dtype, f"{kernel} ps={ps}")
+
+
+@pytest.mark.parametrize("ps", [16, 32, 64])
+def test_warp_partitions_ragged_groups(pkv, ps):
+    # Reduce-kernel path with short partitions: a CTA serves four
+    # partitions, one per consumer warp.  Lengths leave groups of 1-4
+    # partitions, partial last pages and partitions, an empty sequence and
+    # a one-token sequence.
+    lens = (0, 1, 16, 17, 48, 63, 64, 65, 100, 129, 200, 255)
+    w = wl.Workload("warp_parts", 41, len(lens), 32, 8, 128, 16, "bfloat16",
+                    "fixed", fixed_lengths=lens)
+    inp = wl.make_paged(w, device="cuda")
+    out = _run(pkv, inp, partition_size=ps, reduce="kernel")
+    assert torch.count_nonzero(out[0]) == 0
+    v0 = inp.v_cache[int(inp.block_tables[1, 0]), :, 0, :]
+    assert torch.equal(out[1], v0.repeat_interleave(4, dim=0))
+    _check_all(inp, out, f"warp partitions ps={ps}")
+    ref = _run(pkv, inp, partition_size=256, reduce="auto")
+    assert (out.float() - ref.float()).abs().max().item() <= 4e-3
