@@ -163,11 +163,17 @@ def measured_hbm_peak():
 
 
 def decode_source_hash() -> str:
+    """Hash of the decode kernel's code (decode.cu and device_utils.cuh with
+    comments and blank space removed, so a comment edit keeps a capture
+    current and any code change makes it stale)."""
     h = hashlib.sha256()
     for name in ("decode.cu", "device_utils.cuh"):
         with open(os.path.join(ROOT, "paged_kv_cache_383_b200", "csrc",
-                               name), "rb") as f:
-            h.update(f.read())
+                               name)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

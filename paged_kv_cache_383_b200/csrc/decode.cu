@@ -32,8 +32,17 @@
 //  * Compute variant SIMT: fp32 FMA dot products on the CUDA cores (kept to
 //    show what the tensor-core mapping buys).
 //  * A sequence that needs more than one partition writes (m, l, o/l) per
-//    partition to the workspace; a second kernel combines them.  A sequence
+//    partition to the workspace.  With at most 16 partitions the partition
+//    CTA that finishes last combines them (fence + ticket, nobody waits);
+//    otherwise, or on request, a separate reduce kernel does.  A sequence
 //    that fits one partition is written straight to `out`.
+//  * With the reduce kernel and partitions of <= 1024 tokens, a CTA serves
+//    four consecutive partitions, one per consumer warp (pages interleaved
+//    so each warp still owns its ring stages): no cross-warp merge.
+//  * A one-CTA prep kernel runs first: it orders the sequences longest
+//    first (grid row z serves order[z], so the grid ends on short work) and
+//    resets the partition counters.  Kernels are chained by programmatic
+//    dependent launch.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
