@@ -388,9 +388,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int k = 0; k < kKeys; ++k)
         if (k > lim) sv[k] = -INFINITY;
     }
-    float mx = sv[0];
+    // Eight independent partial maxima (and sums below): a 64-long serial
+    // chain of dependent instructions would stall the warp on each step.
+    float m8[8];
 #pragma unroll
-    for (int k = 1; k < kKeys; ++k) mx = fmaxf(mx, sv[k]);
+    for (int u = 0; u < 8; ++u) m8[u] = sv[u];
+#pragma unroll
+    for (int k = 8; k < kKeys; ++k) m8[k & 7] = fmaxf(m8[k & 7], sv[k]);
+    float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                     fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
     mx *= c;  // the scale is positive: max commutes with it
     float factor = 1.f;
     if (j == 0) {
@@ -401,10 +407,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       l *= factor;
     }
     // P = 2^(s * c - m_ref), before waiting for the tensor cores.
+    {
+      float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int k = 0; k < kKeys; ++k) {
-      sv[k] = dev::fast_exp2(fmaf(sv[k], c, -m_ref));
-      l += sv[k];
+      for (int k = 0; k < kKeys; ++k) {
+        sv[k] = dev::fast_exp2(fmaf(sv[k], c, -m_ref));
+        l8[k & 7] += sv[k];
+      }
+      l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) +
+           ((l8[4] + l8[5]) + (l8[6] + l8[7]));
     }
     if (__any_sync(0xffffffffu, factor != 1.f)) {
       // O must hold P(j-1).V before it is rescaled (P(j).V is not issued
