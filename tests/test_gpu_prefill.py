@@ -183,3 +183,27 @@ def test_speculative_verify_and_rollback(pkv):
     kp, vp, tables = _contiguous_pool(K, V, bs)
     check_decode(to_np(dec), oa.paged_decode(to_np(q), kp, vp, tables, lens,
                                              scale), q.dtype, "decode")
+
+
+def test_prompt_prefill_full_size_sampled(pkv):
+    """Whole prompts at the bench's full size (8 sequences, 1k-8k tokens,
+    every token new).  Row p of a prompt attends to positions 0..p, i.e. a
+    decode over the first p + 1 tokens, which the oracle computes for
+    sampled rows: first and last tokens, tile boundaries, random ones."""
+    w = wl.WORKLOADS["prompt_prefill_gqa8"]
+    lens = wl.make_paged(w, values=False).lengths
+    pin = wl.make_prefill(w, lens, device="cuda")
+    out = _run(pkv, pin)
+    inp = pin.paged
+    rng = np.random.default_rng(7)
+    kc, vc = to_np(inp.k_cache), to_np(inp.v_cache)
+    for b in (0, int(np.argmax(lens)), w.num_seqs - 1):
+        L = int(lens[b])
+        pos = sorted({0, 1, 15, 16, 63, 64, 127, 128, L - 2, L - 1,
+                      *rng.integers(0, L, size=6).tolist()})
+        rows = pin.query_start[b] + np.array(pos)
+        q = to_np(pin.q)[rows]
+        tables = np.repeat(inp.block_tables[b:b + 1], len(pos), axis=0)
+        ref = oa.paged_decode(q, kc, vc, tables, np.array(pos) + 1,
+                              w.softmax_scale)
+        check_decode(to_np(out)[rows], ref, pin.q.dtype, f"prompt seq {b}")
