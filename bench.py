@@ -229,17 +229,17 @@ def run_native(args, rank, world, local):
     step_bytes = kv_bytes(inp.lengths, w)
 
     def writes():
+        # on the current stream (the timing stream, or a graph's capture
+        # stream)
         if pairs is not None:
-            pkv.pa_copy_blocks(inp.k_cache, inp.v_cache, pairs, dev_err=err,
-                               stream=stream)
+            pkv.pa_copy_blocks(inp.k_cache, inp.v_cache, pairs, dev_err=err)
         pkv.pa_cache_write(inp.k_cache, inp.v_cache, spec.write_k,
-                           spec.write_v, slots, dev_err=err, stream=stream)
+                           spec.write_v, slots, dev_err=err)
 
     def step():
         writes()
         pkv.pa_decode(out, inp.q, inp.k_cache, inp.v_cache, bt, cl,
-                      w.softmax_scale, desc=desc, workspace=ws, dev_err=err,
-                      stream=stream)
+                      w.softmax_scale, desc=desc, workspace=ws, dev_err=err)
 
     clocks = ClockSampler(local)
     t_spin = time.time()
@@ -361,6 +361,27 @@ def run_native(args, rank, world, local):
     }
     if rank == 0 and world == 1 and not args.no_extras:
         res["extras"] = extras(args, w, inp, dev, pkv, bt, cl)
+        # The same step captured once in a CUDA graph and replayed: what
+        # the host's launch calls cost per step.
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        g_ms = timed(graph.replay) / args.steps
+        res["extras"]["cuda_graph"] = {
+            "step_ms_eager": round(ms_step, 5),
+            "step_ms_graph": round(g_ms, 5),
+            "note": "one captured step (cache write, prep, decode) replayed "
+                    "K times, timed as the main step"}
+        del graph
         probe = res["extras"].get("read_probe_gbs")
         if probe:
             res["roofline"]["read_probe_gbs"] = probe

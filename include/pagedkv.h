@@ -32,6 +32,11 @@
  *     pa_decode ([KV-cache chapter] "PagedAttention: borrowing virtual
  *     memory...": a private copy is made before the first write into a shared
  *     block).
+ *   - pa_cache_write, pa_copy_blocks, pa_decode and pa_prefill only enqueue
+ *     kernels (no allocation, no synchronisation), so a sequence of them
+ *     can be captured in a CUDA graph and replayed; the graph keeps the
+ *     pointers and shapes it was captured with.  Call each shape once
+ *     outside capture first (the first call configures its kernel).
  *   - pa_last_error() returns a thread-local text describing the last
  *     non-OK status produced on the calling thread.
  */
