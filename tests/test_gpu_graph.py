@@ -84,3 +84,49 @@ def test_captured_step_replays_like_eager(pkv, name, ps):
                           w.softmax_scale, seqs=seqs)
     check_decode(to_np(replayed)[seqs], ref[seqs], q.dtype, "graph replay")
     del graph
+
+
+def test_captured_copy_and_prefill_replay_like_eager(pkv):
+    lens = (100, 300, 37)
+    w = wl.Workload("graph_prefill", 77, len(lens), 32, 8, 128, 16,
+                    "bfloat16", "fixed", fixed_lengths=lens)
+    pin = wl.make_prefill(w, (30, 120, 37), device="cuda")
+    inp = pin.paged
+    dev = inp.k_cache.device
+    bt = torch.from_numpy(inp.block_tables).to(dev)
+    cl = torch.from_numpy(inp.lengths.astype(np.int32)).to(dev)
+    qs = torch.from_numpy(pin.query_start).to(dev)
+    free = np.setdiff1d(np.arange(inp.num_blocks), inp.block_tables)
+    pairs = torch.tensor([[int(inp.block_tables[0, 0]), int(free[0])]],
+                         dtype=torch.int32, device=dev)
+    q = pin.q.clone()
+    out = torch.empty_like(q)
+    kw = dict(max_q_len=120, max_context_len=300)
+
+    def step():
+        pkv.pa_copy_blocks(inp.k_cache, inp.v_cache, pairs)
+        pkv.pa_prefill(out, q, inp.k_cache, inp.v_cache, bt, cl, qs,
+                       w.softmax_scale, **kw)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    g = torch.Generator(device=dev)
+    for trial in range(2):
+        g.manual_seed(200 + trial)
+        q.copy_(torch.randn(q.shape, generator=g, device=dev).to(q.dtype))
+        graph.replay()
+        torch.cuda.synchronize()
+        replayed = out.clone()
+        step()
+        torch.cuda.synchronize()
+        assert torch.equal(replayed, out), trial
+    src, dst = int(pairs[0, 0]), int(pairs[0, 1])
+    assert torch.equal(inp.k_cache[dst], inp.k_cache[src])
+    del graph
