@@ -470,6 +470,18 @@ int pa_bm_is_swapped(void* bm, int64_t seq_id);
 pa_status pa_bm_seq_blocks(void* bm, int64_t seq_id, int32_t* blocks_out,
                            int max_blocks, int* n_out);
 
+/* Pool sizing: how many blocks of block_size tokens fit in `bytes` for a
+ * model of num_layers layers, each holding K and V of num_kv_heads heads of
+ * head_dim 2-byte elements per token (a block id then names the same slot
+ * range in every layer's cache).  Per token and layer that is
+ * 2 * num_kv_heads * head_dim * 2 bytes ([Taming the Tail] "The Math of the
+ * Cache" counts 2 x layers x hidden x bytes; with grouped-query attention
+ * the per-layer width is num_kv_heads * head_dim).  Pass the share of free
+ * device memory the cache may take (a serving engine's memory-utilisation
+ * setting).  -1 (INVALID_ARG) for a non-positive shape or another dtype. */
+int64_t pa_pool_blocks(uint64_t bytes, int num_layers, int num_kv_heads,
+                       int head_dim, int block_size, pa_dtype dtype);
+
 /* Kernel launches this library has issued in this process (all devices,
  * all threads): lets a caller count the GPU work a timed region contained. */
 int64_t pa_launch_count(void);
@@ -482,8 +494,11 @@ int64_t pa_launch_count(void);
 pa_status pa_read_probe(const void* buf, size_t bytes, uint32_t* sink,
                         void* stream);
 
-/* Pool and sequence queries (-1 for an unknown handle / sequence / block). */
+/* Pool and sequence queries (-1 for an unknown handle / sequence / block).
+ * pa_bm_num_used = blocks referenced by a table or by the prefix cache
+ * (num_blocks - pa_bm_num_free). */
 int pa_bm_num_free(void* bm);
+int pa_bm_num_used(void* bm);
 int pa_bm_refcount(void* bm, int block);
 int64_t pa_bm_seq_len(void* bm, int64_t seq_id);
 int pa_bm_num_seq_blocks(void* bm, int64_t seq_id);

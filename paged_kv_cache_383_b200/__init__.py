@@ -258,6 +258,21 @@ def pa_swap_blocks(dst_k, dst_v, src_k, src_v, pairs, *, dev_err=None,
     _lib.check(st, "pa_swap_blocks")
 
 
+def pa_pool_blocks(nbytes: int, num_layers: int, num_kv_heads: int,
+                   head_dim: int, block_size: int, dtype) -> int:
+    """Blocks of block_size tokens (K and V of every layer) that fit in
+    ``nbytes``; ``dtype`` is torch.float16 or torch.bfloat16."""
+    import torch
+    code = {torch.float16: PA_F16, torch.bfloat16: PA_BF16}.get(dtype)
+    if code is None:
+        raise TypeError(f"expected float16 or bfloat16, got {dtype}")
+    n = _lib.load().pa_pool_blocks(int(nbytes), num_layers, num_kv_heads,
+                                   head_dim, block_size, code)
+    if n < 0:
+        _lib.check(_lib.PA_ERR_INVALID_ARG, "pa_pool_blocks")
+    return n
+
+
 def pa_cache_write(k_cache, v_cache, k, v, slot_mapping, *, dev_err=None,
                    stream=None):
     """Copy each new token's K and V rows into cache slot slot_mapping[t]
@@ -421,6 +436,9 @@ class BlockManager:
 
     def num_free(self) -> int:
         return self._lib.pa_bm_num_free(self._h)
+
+    def num_used(self) -> int:
+        return self._lib.pa_bm_num_used(self._h)
 
     def refcount(self, block: int) -> int:
         return self._lib.pa_bm_refcount(self._h, block)

@@ -118,6 +118,9 @@ SIGNATURES = {
     "pa_bm_refcount": (_int, [_vp, _int]),
     "pa_bm_seq_len": (_i64, [_vp, _i64]),
     "pa_bm_num_seq_blocks": (_int, [_vp, _i64]),
+    "pa_bm_num_used": (_int, [_vp]),
+    "pa_pool_blocks": (_i64, [ctypes.c_uint64, _int, _int, _int, _int,
+                              _int]),
     "pa_bm_match_prefix": (_st, [_vp, _i64, _pi32, _i64, _pi64]),
     "pa_bm_cache_insert": (_st, [_vp, _i64, _pi32, _i64]),
     "pa_bm_cache_evict": (_st, [_vp, _int, ctypes.POINTER(_int)]),

@@ -492,6 +492,28 @@ int pa_bm_num_free(void* p) {
   return bm ? static_cast<int>(bm->free_stack.size()) : -1;
 }
 
+int pa_bm_num_used(void* p) {
+  BlockManager* bm = as_bm(p);
+  return bm ? bm->num_blocks - static_cast<int>(bm->free_stack.size()) : -1;
+}
+
+int64_t pa_pool_blocks(uint64_t bytes, int num_layers, int num_kv_heads,
+                       int head_dim, int block_size, pa_dtype dtype) {
+  pagedkv::clear_error();
+  if (num_layers <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+      block_size <= 0 || (dtype != PA_F16 && dtype != PA_BF16)) {
+    fail(PA_ERR_INVALID_ARG,
+         "pa_pool_blocks: num_layers=%d num_kv_heads=%d head_dim=%d "
+         "block_size=%d dtype=%d", num_layers, num_kv_heads, head_dim,
+         block_size, static_cast<int>(dtype));
+    return -1;
+  }
+  // K and V, every layer, every KV head, block_size tokens, 2-byte elements.
+  const uint64_t per_block = 2ull * num_layers * num_kv_heads * head_dim *
+                             block_size * 2ull;
+  return static_cast<int64_t>(bytes / per_block);
+}
+
 int pa_bm_refcount(void* p, int block) {
   BlockManager* bm = as_bm(p);
   if (!bm || block < 0 || block >= bm->num_blocks) return -1;

@@ -236,3 +236,40 @@ def test_append_batch_partial_failure(pkv):
         bm.append_batch([0, 1, 2], [16, 50, 1])
     assert ei.value.num_done == 1
     assert bm.seq_len(0) == 16 and bm.seq_len(1) == 0 and bm.seq_len(2) == 0
+
+
+def test_num_used_counts_tables_and_cache(pkv):
+    bm = pkv.BlockManager(32, 4)
+    assert bm.num_used() == 0
+    bm.add_seq(0)
+    bm.append(0, 9)                       # 3 blocks
+    bm.fork(0, 1)                         # shared: still 3
+    assert bm.num_used() == 3
+    bm.cache_insert(0, list(range(8)))    # 2 full blocks cached
+    bm.free_seq(0)
+    bm.free_seq(1)
+    assert bm.num_used() == 2             # the cache still holds them
+    assert bm.num_used() + bm.num_free() == 32
+
+
+def test_pool_blocks_from_bytes(pkv):
+    import torch
+    # Llama-3-70B shape: 80 layers, 8 KV heads of 128 dims, bf16.  Per token
+    # 2 (K, V) x 80 x 8 x 128 x 2 B = 327,680 B (the pages' 2 x layers x
+    # hidden x bytes with the grouped-query width 8 x 128); 8,192 tokens
+    # take 2.68 GB.
+    per_token = 2 * 80 * 8 * 128 * 2
+    assert per_token == 327_680
+    assert per_token * 8192 == 2_684_354_560
+    n = pkv.pa_pool_blocks(per_token * 16 * 1000, 80, 8, 128, 16,
+                           torch.bfloat16)
+    assert n == 1000
+    assert pkv.pa_pool_blocks(per_token * 16 * 1000 - 1, 80, 8, 128, 16,
+                              torch.float16) == 999
+    # one layer, the batch-256 mix's pool: 4,096 B per token, block 16
+    assert pkv.pa_pool_blocks(64 << 30, 1, 8, 128, 16, torch.bfloat16) == \
+        (64 << 30) // (4096 * 16)
+    with pytest.raises(pkv.PagedKVError):
+        pkv.pa_pool_blocks(1 << 30, 0, 8, 128, 16, torch.bfloat16)
+    with pytest.raises(TypeError):
+        pkv.pa_pool_blocks(1 << 30, 1, 8, 128, 16, torch.float32)
