@@ -212,10 +212,8 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,
  * Layouts: q, out [total_q, num_q_heads, 128] dtype; query_start [num_seqs+1]
  * int32 on the device, non-decreasing, query_start[0] = 0 and
  * query_start[num_seqs] <= total_q; the rest as for pa_decode.
- * Supported: head_dim 128, block_size 16 or 32, G = 1, 2, 4 or 8, and a
- * max_context_len whose block-table slice fits shared memory (about 33,000
- * blocks: 530k tokens at block 16); else PA_ERR_UNSUPPORTED.  Above about
- * 3,400 blocks (54k tokens at block 16) one CTA instead of two fits an SM.  Runs on the
+ * Supported: head_dim 128, block_size 16 or 32, G = 1, 2, 4 or 8 (else
+ * PA_ERR_UNSUPPORTED); any context length the table holds.  Runs on the
  * tcgen05 tensor cores with fp32 accumulation in tensor memory; output
  * rounded once to dtype.
  * Device-side: a context or query range outside the table, a sequence with

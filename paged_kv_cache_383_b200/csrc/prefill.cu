@@ -37,9 +37,10 @@
 //     grows by more than 2^8 (the final division uses the same reference,
 //     so the result is unchanged), and store P with tcgen05.st as a 16-bit
 //     rounded part plus its residual so P . V keeps ~16 mantissa bits.
-//   * Shared memory is ~99 KB (Q, the rings, barriers, the block-table slice)
-//     and tensor memory 256 columns, so two CTAs share an SM: one CTA's
-//     softmax runs while the other's tiles are on the tensor cores.
+//   * Shared memory is ~99 KB (Q, the rings, barriers; block ids are read
+//     from global memory a tile ahead) and tensor memory 256 columns, so two
+//     CTAs share an SM at any context length: one CTA's softmax runs while
+//     the other's tiles are on the tensor cores.
 //   * Every wait is bounded (1 s) and reports PA_ERR_DEVICE_TIMEOUT; tensor
 //     memory is always released.  A barrier that is waited on by parity is
 //     never allowed to run two phases ahead of its waiter: each double
@@ -98,11 +99,8 @@ constexpr int kOffBars = kOffV + kVStages * kKVTile;
 // s_full[2], s_free[2], p_full[2], o_ready[2], done, then the tensor-memory
 // base address word.
 constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 4 * 2 + 1;
-constexpr int kOffTable = kOffBars + kNumBars * 8 + 16;
-
-size_t prefill_smem_bytes(int max_pages) {
-  return 1024 + kOffTable + ((static_cast<size_t>(max_pages) * 4 + 15) & ~15);
-}
+// 1024 bytes of slack for aligning the base, then the layout above.
+constexpr size_t kSmemBytes = 1024 + kOffBars + kNumBars * 8 + 16;
 
 template <typename T, int BS, int G>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -135,7 +133,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t done = o_ready0 + 16;
   uint32_t* tmem_slot =
       reinterpret_cast<uint32_t*>(smem + kOffBars + kNumBars * 8);
-  int32_t* bt_s = reinterpret_cast<int32_t*>(smem + kOffTable);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -160,14 +157,15 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int n_tiles = (kv_end + kKeys - 1) / kKeys;
   const int n_pages = (kv_end + BS - 1) / BS;
 
-  // Block ids of the pages the tile reads; every one is checked.
+  // Block ids of the pages the tile reads; every one is checked here, and
+  // the producer reads them again (from L2) a tile ahead of its loads, so
+  // shared memory does not grow with the context.
   int bad = 0;
   const int32_t* row = a.block_tables +
                        static_cast<int64_t>(b) * a.max_blocks_per_seq;
   for (int i = tid; i < n_pages; i += kThreads) {
     const int32_t p = row[i];
     bad |= (p < 0 || p >= a.num_blocks);
-    bt_s[i] = p;
   }
   if (tid == 0) {
     dev::mbar_init(q_full, 1);
@@ -216,9 +214,22 @@ __global__ void __launch_bounds__(kThreads, 2)
       dev::mbar_arrive_expect_tx(q_full, kQBytes);
       dev::tma_load_3d(q_s, &qmap, 0, kvh * G, q0 + tok0, q_full);
       dev::tma_load_3d(q_s + kHalfQ, &qmap, 64, kvh * G, q0 + tok0, q_full);
+      // Block ids of a tile's pages; pages past the sequence are masked, so
+      // they read the first page instead.
+      const int32_t first = row[0];
+      auto fetch = [&](int j, int32_t (&ids)[kPagesPerTile]) {
+#pragma unroll
+        for (int p = 0; p < kPagesPerTile; ++p) {
+          const int page = j * kPagesPerTile + p;
+          ids[p] = page < n_pages ? __ldg(row + page) : first;
+        }
+      };
+      int32_t cur[kPagesPerTile], nxt[kPagesPerTile], prv[kPagesPerTile];
+      fetch(0, nxt);
       // K tile j and V tile j-1 per step: a K stage is free once S(j) has
       // read it, a V stage once P(j).V has, and V is needed a tile later.
-      auto load = [&](int j, bool is_v) -> bool {
+      auto load = [&](int j, bool is_v,
+                      const int32_t (&ids)[kPagesPerTile]) -> bool {
         const int ns = is_v ? kVStages : kKStages;
         const int s = j % ns;
         const uint32_t empty = (is_v ? v_empty0 : k_empty0) + 8 * s;
@@ -230,10 +241,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const CUtensorMap* map = is_v ? &vmap : &kmap;
 #pragma unroll
         for (int p = 0; p < kPagesPerTile; ++p) {
-          const int page = j * kPagesPerTile + p;
-          // Pages past the sequence are masked; read a valid one instead.
-          const int32_t phys = page < n_pages ? bt_s[page] : bt_s[0];
-          const int y = (phys * a.num_kv_heads + kvh) * BS;
+          const int y = (ids[p] * a.num_kv_heads + kvh) * BS;
           const uint32_t off = p * BS * 128;
           dev::tma_load_2d(dst + off, map, 0, y, full);
           dev::tma_load_2d(dst + kTileHalf + off, map, 64, y, full);
@@ -241,10 +249,18 @@ __global__ void __launch_bounds__(kThreads, 2)
         return true;
       };
       for (int t = 0; t <= n_tiles; ++t) {
-        if ((t < n_tiles && !load(t, false)) || (t >= 1 && !load(t - 1, true))) {
+        if (t < n_tiles) {
+#pragma unroll
+          for (int p = 0; p < kPagesPerTile; ++p) cur[p] = nxt[p];
+          if (t + 1 < n_tiles) fetch(t + 1, nxt);  // in flight meanwhile
+        }
+        if ((t < n_tiles && !load(t, false, cur)) ||
+            (t >= 1 && !load(t - 1, true, prv))) {
           dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
           break;
         }
+#pragma unroll
+        for (int p = 0; p < kPagesPerTile; ++p) prv[p] = cur[p];
       }
     }
     return;
@@ -544,9 +560,9 @@ bool encode_cache(CUtensorMap* m, const void* cache, uint64_t rows, int bs,
 template <typename T, int BS, int G>
 pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
                  const CUtensorMap& qm, const CUtensorMap& km,
-                 const CUtensorMap& vm, int max_pages, cudaStream_t st) {
+                 const CUtensorMap& vm, cudaStream_t st) {
   auto kern = prefill_kernel<T, BS, G>;
-  const size_t smem = prefill_smem_bytes(max_pages);
+  const size_t smem = kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
       static_cast<int>(smem));
@@ -567,12 +583,12 @@ pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
 template <typename T, int BS>
 pa_status dispatch_group(const pa_prefill_desc* d, const PrefillArgs& a,
                          const CUtensorMap& qm, const CUtensorMap& km,
-                         const CUtensorMap& vm, int max_pages, cudaStream_t st) {
+                         const CUtensorMap& vm, cudaStream_t st) {
   switch (d->num_q_heads / d->num_kv_heads) {
-    case 1: return launch<T, BS, 1>(d, a, qm, km, vm, max_pages, st);
-    case 2: return launch<T, BS, 2>(d, a, qm, km, vm, max_pages, st);
-    case 4: return launch<T, BS, 4>(d, a, qm, km, vm, max_pages, st);
-    default: return launch<T, BS, 8>(d, a, qm, km, vm, max_pages, st);
+    case 1: return launch<T, BS, 1>(d, a, qm, km, vm, st);
+    case 2: return launch<T, BS, 2>(d, a, qm, km, vm, st);
+    case 4: return launch<T, BS, 4>(d, a, qm, km, vm, st);
+    default: return launch<T, BS, 8>(d, a, qm, km, vm, st);
   }
 }
 
@@ -624,11 +640,6 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
   const int max_ctx = d->max_context_len > 0
                           ? d->max_context_len
                           : d->max_blocks_per_seq * d->block_size;
-  const int max_pages = (max_ctx + d->block_size - 1) / d->block_size;
-  if (pagedkv::prefill_smem_bytes(max_pages) > 227 * 1024)
-    return fail(PA_ERR_UNSUPPORTED,
-                "pa_prefill: context of %d tokens needs a block-table slice "
-                "beyond shared memory", max_ctx);
   const int tok = pagedkv::kRows / G;
   CUtensorMap qm, km, vm;
   const uint64_t rows = static_cast<uint64_t>(d->num_blocks) *
@@ -655,12 +666,10 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
   if (d->dtype == PA_BF16)
     return d->block_size == 16
                ? pagedkv::dispatch_group<__nv_bfloat16, 16>(d, a, qm, km, vm,
-                                                            max_pages, s)
+                                                            s)
                : pagedkv::dispatch_group<__nv_bfloat16, 32>(d, a, qm, km, vm,
-                                                            max_pages, s);
+                                                            s);
   return d->block_size == 16
-             ? pagedkv::dispatch_group<__half, 16>(d, a, qm, km, vm, max_pages,
-                                                   s)
-             : pagedkv::dispatch_group<__half, 32>(d, a, qm, km, vm, max_pages,
-                                                   s);
+             ? pagedkv::dispatch_group<__half, 16>(d, a, qm, km, vm, s)
+             : pagedkv::dispatch_group<__half, 32>(d, a, qm, km, vm, s);
 }

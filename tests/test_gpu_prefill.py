@@ -207,3 +207,32 @@ def test_prompt_prefill_full_size_sampled(pkv):
         ref = oa.paged_decode(q, kc, vc, tables, np.array(pos) + 1,
                               w.softmax_scale)
         check_decode(to_np(out)[rows], ref, pin.q.dtype, f"prompt seq {b}")
+
+
+def test_long_context_chunk_sampled(pkv):
+    """Chunks at the end of 90k- and 70k-token contexts (block 16): the
+    producer reads block ids from global memory, so shared memory does not
+    grow with the context.  Sampled rows against the oracle (row i of a
+    chunk of n is a decode over the first L - n + i + 1 tokens)."""
+    w = wl.Workload("long_prefill", 15, 2, 32, 8, 128, 16, "bfloat16",
+                    "fixed", fixed_lengths=(90_000, 70_001))
+    pin = wl.make_prefill(w, (256, 200), device="cuda")
+    out = _run(pkv, pin)
+    inp = pin.paged
+    bs = w.block_size
+    for b in (0, 1):
+        L, n = int(inp.lengths[b]), int(pin.q_lens[b])
+        local = np.array([0, 1, 63, 64, 127, n - 1])
+        rows = pin.query_start[b] + local
+        pos = L - n + local
+        # the sequence's own blocks, copied to the host as a sub-pool
+        need = int(pos.max()) // bs + 1
+        ids = torch.from_numpy(
+            inp.block_tables[b, :need].astype(np.int64)).cuda()
+        kc = to_np(inp.k_cache.index_select(0, ids))
+        vc = to_np(inp.v_cache.index_select(0, ids))
+        sub = np.repeat(np.arange(need, dtype=np.int32)[None, :], len(pos),
+                        axis=0)
+        ref = oa.paged_decode(to_np(pin.q)[rows], kc, vc, sub, pos + 1,
+                              w.softmax_scale)
+        check_decode(to_np(out)[rows], ref, pin.q.dtype, f"long seq {b}")
