@@ -209,10 +209,10 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,
  *     out[query_start[b] + i, h, :] = softmax(scale * K_b[0..p] q) V_b[0..p]
  * with query head h reading KV head h / G.  q_len = 1 is decode; q_len = L a
  * whole prompt.
- * Layouts: q, out [total_q, num_q_heads, 128] dtype; query_start [num_seqs+1]
+ * Layouts: q, out [total_q, num_q_heads, head_dim] dtype; query_start [num_seqs+1]
  * int32 on the device, non-decreasing, query_start[0] = 0 and
  * query_start[num_seqs] <= total_q; the rest as for pa_decode.
- * Supported: head_dim 128, block_size 16 or 32, G = 1, 2, 4 or 8 (else
+ * Supported: head_dim 64 or 128, block_size 16 or 32, G = 1, 2, 4 or 8 (else
  * PA_ERR_UNSUPPORTED); any context length the table holds.  Runs on the
  * tcgen05 tensor cores with fp32 accumulation in tensor memory; output
  * rounded once to dtype.

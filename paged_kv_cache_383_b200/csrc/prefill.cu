@@ -64,11 +64,10 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kRows = 128;      // query rows per tile (tensor memory lanes)
 constexpr int kKeys = 64;       // keys per K/V tile
-constexpr int kD = 128;         // head_dim
 constexpr int kKStages = 2;     // K ring depth
 constexpr int kVStages = 2;     // V ring depth
 constexpr int kThreads = 192;   // producer, MMA, 4 softmax warps
-constexpr int kTmemCols = 256;  // S: cols [0, 64), O: cols [128, 256)
+constexpr int kTmemCols = 256;  // S/P: cols [0, 128), O: cols [128, 128 + D)
 constexpr float kRescaleLog2 = 8.f;
 
 struct PrefillArgs {
@@ -86,28 +85,41 @@ struct PrefillArgs {
   int total_q;
 };
 
-// Shared memory (offsets from a 1024-byte aligned base).
-constexpr int kQBytes = kRows * kD * 2;                 // 32 KB, two halves
-constexpr int kHalfQ = kRows * 128;                     // 16 KB
-constexpr int kTileHalf = kKeys * 128;                  // 8 KB: 64 keys x 64 d
-constexpr int kKVTile = 2 * kTileHalf;                  // 16 KB per K or V
-constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
-constexpr int kOffV = kOffK + kKStages * kKVTile;
-constexpr int kOffBars = kOffV + kVStages * kKVTile;
 // barriers: q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
 // s_full[2], s_free[2], p_full[2], o_ready[2], done, then the tensor-memory
 // base address word.
 constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 4 * 2 + 1;
-// 1024 bytes of slack for aligning the base, then the layout above.
-constexpr size_t kSmemBytes = 1024 + kOffBars + kNumBars * 8 + 16;
+constexpr int kTileHalf = kKeys * 128;  // 8 KB: 64 keys x 64 dims (128 B)
 
-template <typename T, int BS, int G>
+// Shared memory for head_dim D (offsets from a 1024-byte aligned base): the
+// head dimension is held in 64-element halves of 128 bytes, each its own
+// 128-byte-swizzled region.
+template <int D>
+struct Layout {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kHalfQ = kRows * 128;             // 16 KB
+  static constexpr int kQBytes = kHalves * kHalfQ;
+  static constexpr int kKVTile = kHalves * kTileHalf;     // per K or V tile
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + kKStages * kKVTile;
+  static constexpr int kOffBars = kOffV + kVStages * kKVTile;
+  // 1024 bytes of slack for aligning the base, then the layout above.
+  static constexpr size_t kSmemBytes = 1024 + kOffBars + kNumBars * 8 + 16;
+};
+
+template <typename T, int BS, int G, int D>
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap,
                    const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap,
                    const PrefillArgs a) {
+  using Lay = Layout<D>;
+  constexpr int kHalves = Lay::kHalves;
+  constexpr int kHalfQ = Lay::kHalfQ;
+  constexpr int kQBytes = Lay::kQBytes;
+  constexpr int kKVTile = Lay::kKVTile;
+  constexpr int kOffBars = Lay::kOffBars;
   constexpr int kTok = kRows / G;         // new tokens per tile
   constexpr int kPagesPerTile = kKeys / BS;
   constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
@@ -116,9 +128,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint8_t* smem =
       smem_dyn + ((1024u - (dev::smem_u32(smem_dyn) & 1023u)) & 1023u);
   const uint32_t base = dev::smem_u32(smem);
-  const uint32_t q_s = base + kOffQ;
-  const uint32_t kring = base + kOffK;
-  const uint32_t vring = base + kOffV;
+  const uint32_t q_s = base + Lay::kOffQ;
+  const uint32_t kring = base + Lay::kOffK;
+  const uint32_t vring = base + Lay::kOffV;
   const uint32_t bars = base + kOffBars;
   const uint32_t q_full = bars;
   const uint32_t k_full0 = bars + 8;
@@ -212,8 +224,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       dev::prefetch_tmap(&kmap);
       dev::prefetch_tmap(&vmap);
       dev::mbar_arrive_expect_tx(q_full, kQBytes);
-      dev::tma_load_3d(q_s, &qmap, 0, kvh * G, q0 + tok0, q_full);
-      dev::tma_load_3d(q_s + kHalfQ, &qmap, 64, kvh * G, q0 + tok0, q_full);
+#pragma unroll
+      for (int h = 0; h < kHalves; ++h)
+        dev::tma_load_3d(q_s + h * kHalfQ, &qmap, 64 * h, kvh * G, q0 + tok0,
+                         q_full);
       // Block ids of a tile's pages; pages past the sequence are masked, so
       // they read the first page instead.
       const int32_t first = row[0];
@@ -243,8 +257,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int p = 0; p < kPagesPerTile; ++p) {
           const int y = (ids[p] * a.num_kv_heads + kvh) * BS;
           const uint32_t off = p * BS * 128;
-          dev::tma_load_2d(dst + off, map, 0, y, full);
-          dev::tma_load_2d(dst + kTileHalf + off, map, 64, y, full);
+#pragma unroll
+          for (int h = 0; h < kHalves; ++h)
+            dev::tma_load_2d(dst + h * kTileHalf + off, map, 64 * h, y, full);
         }
         return true;
       };
@@ -272,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = dev::umma_idesc_f16(kBf16, kRows, kKeys,
                                                         false, false);
-      constexpr uint32_t idesc_pv = dev::umma_idesc_f16(kBf16, kRows, kD,
+      constexpr uint32_t idesc_pv = dev::umma_idesc_f16(kBf16, kRows, D,
                                                         false, true);
       auto issue_pv = [&](int t) -> bool {
         if (!dev::mbar_wait(p_full0 + 8 * (t & 1), (t >> 1) & 1) ||
@@ -313,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t kt = kring + s * kKVTile;
         const uint32_t sd = s_tmem + (j & 1) * kKeys;
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
           const int h = kk >> 2, k4 = kk & 3;
           const uint64_t ad = dev::sw128_desc(q_s + h * kHalfQ + k4 * 32, 16,
                                               1024);
@@ -389,8 +404,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                                      (j / kVStages) & 1));
       if (!ok) break;
       const uint32_t vt = vring + (j % kVStages) * kKVTile;
-      for (int idx = lane; idx < 16 * 16; idx += 32) {
-        const int krow = quarter * 16 + (idx >> 4), ch = idx & 15;
+      for (int idx = lane; idx < 16 * 8 * kHalves; idx += 32) {
+        const int krow = quarter * 16 + idx / (8 * kHalves);
+        const int ch = idx % (8 * kHalves);
         if (k0 + krow >= L)
           dev::st_shared_zero16(vt + (ch >> 3) * kTileHalf + krow * 128 +
                                 (ch & 7) * 16);
@@ -440,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (!ok) break;
       dev::tc_fence_after();
 #pragma unroll
-      for (int col = 0; col < kD; col += 32) {
+      for (int col = 0; col < D; col += 32) {
         float ov[32];
         dev::tmem_ld32(o_tmem + lane_off + col, ov);
         dev::tmem_ld_wait();
@@ -476,9 +492,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float inv = l > 0.f ? 1.f / l : 0.f;
     T* dst = static_cast<T*>(a.out) +
              (static_cast<int64_t>(q0 + tok) * a.num_q_heads + kvh * G + g) *
-                 kD;
+                 D;
 #pragma unroll
-    for (int col = 0; col < kD; col += 32) {
+    for (int col = 0; col < D; col += 32) {
       float ov[32];
       dev::tmem_ld32(o_tmem + lane_off + col, ov);
       dev::tmem_ld_wait();
@@ -524,16 +540,16 @@ CUtensorMapDataType tma_type(pa_dtype t) {
                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
 }
 
-// q [total_q, Hq, 128] as a 3-D tensor; box = 64 dims x G heads x tokens.
-bool encode_q(CUtensorMap* m, const void* q, int total_q, int hq, int g,
-              int tok, pa_dtype dt) {
+// q [total_q, Hq, D] as a 3-D tensor; box = 64 dims x G heads x tokens.
+bool encode_q(CUtensorMap* m, const void* q, int total_q, int hq, int hd,
+              int g, int tok, pa_dtype dt) {
   auto enc = encoder();
   if (!enc) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD),
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(hd),
                         static_cast<cuuint64_t>(hq),
                         static_cast<cuuint64_t>(total_q)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * 2,
-                           static_cast<cuuint64_t>(hq) * kD * 2};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(hd) * 2,
+                           static_cast<cuuint64_t>(hq) * hd * 2};
   cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(g),
                        static_cast<cuuint32_t>(tok)};
   cuuint32_t es[3] = {1u, 1u, 1u};
@@ -543,12 +559,12 @@ bool encode_q(CUtensorMap* m, const void* q, int total_q, int hq, int g,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool encode_cache(CUtensorMap* m, const void* cache, uint64_t rows, int bs,
-                  pa_dtype dt) {
+bool encode_cache(CUtensorMap* m, const void* cache, uint64_t rows, int hd,
+                  int bs, pa_dtype dt) {
   auto enc = encoder();
   if (!enc) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), rows};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD) * 2};
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(hd), rows};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(hd) * 2};
   cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(bs)};
   cuuint32_t es[2] = {1u, 1u};
   return enc(m, tma_type(dt), 2, const_cast<void*>(cache), dims, strides, box,
@@ -557,12 +573,12 @@ bool encode_cache(CUtensorMap* m, const void* cache, uint64_t rows, int bs,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, int BS, int G>
+template <typename T, int BS, int G, int D>
 pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
                  const CUtensorMap& qm, const CUtensorMap& km,
                  const CUtensorMap& vm, cudaStream_t st) {
-  auto kern = prefill_kernel<T, BS, G>;
-  const size_t smem = kSmemBytes;
+  auto kern = prefill_kernel<T, BS, G, D>;
+  const size_t smem = Layout<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
       static_cast<int>(smem));
@@ -580,16 +596,28 @@ pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
   return PA_OK;
 }
 
-template <typename T, int BS>
+template <typename T, int BS, int D>
 pa_status dispatch_group(const pa_prefill_desc* d, const PrefillArgs& a,
                          const CUtensorMap& qm, const CUtensorMap& km,
                          const CUtensorMap& vm, cudaStream_t st) {
   switch (d->num_q_heads / d->num_kv_heads) {
-    case 1: return launch<T, BS, 1>(d, a, qm, km, vm, st);
-    case 2: return launch<T, BS, 2>(d, a, qm, km, vm, st);
-    case 4: return launch<T, BS, 4>(d, a, qm, km, vm, st);
-    default: return launch<T, BS, 8>(d, a, qm, km, vm, st);
+    case 1: return launch<T, BS, 1, D>(d, a, qm, km, vm, st);
+    case 2: return launch<T, BS, 2, D>(d, a, qm, km, vm, st);
+    case 4: return launch<T, BS, 4, D>(d, a, qm, km, vm, st);
+    default: return launch<T, BS, 8, D>(d, a, qm, km, vm, st);
   }
+}
+
+template <typename T>
+pa_status dispatch_shape(const pa_prefill_desc* d, const PrefillArgs& a,
+                         const CUtensorMap& qm, const CUtensorMap& km,
+                         const CUtensorMap& vm, cudaStream_t st) {
+  if (d->head_dim == 128)
+    return d->block_size == 16
+               ? dispatch_group<T, 16, 128>(d, a, qm, km, vm, st)
+               : dispatch_group<T, 32, 128>(d, a, qm, km, vm, st);
+  return d->block_size == 16 ? dispatch_group<T, 16, 64>(d, a, qm, km, vm, st)
+                             : dispatch_group<T, 32, 64>(d, a, qm, km, vm, st);
 }
 
 }  // namespace
@@ -618,10 +646,11 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
                 d->max_blocks_per_seq, d->total_q, d->max_q_len,
                 static_cast<int>(d->dtype));
   const int G = d->num_q_heads / d->num_kv_heads;
-  if (d->head_dim != 128 || (d->block_size != 16 && d->block_size != 32) ||
+  if ((d->head_dim != 64 && d->head_dim != 128) ||
+      (d->block_size != 16 && d->block_size != 32) ||
       (G != 1 && G != 2 && G != 4 && G != 8))
     return fail(PA_ERR_UNSUPPORTED,
-                "pa_prefill: needs head_dim 128 (got %d), block_size 16 or 32 "
+                "pa_prefill: needs head_dim 64 or 128 (got %d), block_size 16 or 32 "
                 "(got %d) and a query group of 1, 2, 4 or 8 (got %d)",
                 d->head_dim, d->block_size, G);
   if (d->num_seqs == 0 || d->total_q == 0 || d->max_q_len == 0) return PA_OK;
@@ -644,10 +673,12 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
   CUtensorMap qm, km, vm;
   const uint64_t rows = static_cast<uint64_t>(d->num_blocks) *
                         d->num_kv_heads * d->block_size;
-  if (!pagedkv::encode_q(&qm, q, d->total_q, d->num_q_heads, G, tok,
-                         d->dtype) ||
-      !pagedkv::encode_cache(&km, k_cache, rows, d->block_size, d->dtype) ||
-      !pagedkv::encode_cache(&vm, v_cache, rows, d->block_size, d->dtype))
+  if (!pagedkv::encode_q(&qm, q, d->total_q, d->num_q_heads, d->head_dim, G,
+                         tok, d->dtype) ||
+      !pagedkv::encode_cache(&km, k_cache, rows, d->head_dim, d->block_size,
+                             d->dtype) ||
+      !pagedkv::encode_cache(&vm, v_cache, rows, d->head_dim, d->block_size,
+                             d->dtype))
     return fail(PA_ERR_CUDA, "pa_prefill: cuTensorMapEncodeTiled failed");
   pagedkv::PrefillArgs a;
   a.out = out;
@@ -664,12 +695,6 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
   a.total_q = d->total_q;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d->dtype == PA_BF16)
-    return d->block_size == 16
-               ? pagedkv::dispatch_group<__nv_bfloat16, 16>(d, a, qm, km, vm,
-                                                            s)
-               : pagedkv::dispatch_group<__nv_bfloat16, 32>(d, a, qm, km, vm,
-                                                            s);
-  return d->block_size == 16
-             ? pagedkv::dispatch_group<__half, 16>(d, a, qm, km, vm, s)
-             : pagedkv::dispatch_group<__half, 32>(d, a, qm, km, vm, s);
+    return pagedkv::dispatch_shape<__nv_bfloat16>(d, a, qm, km, vm, s);
+  return pagedkv::dispatch_shape<__half>(d, a, qm, km, vm, s);
 }

@@ -43,15 +43,16 @@ def _check(pin, out, what, seqs=None):
 @pytest.mark.parametrize("dtype", ["bfloat16", "float16"])
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (32, 8), (64, 8)])
 @pytest.mark.parametrize("bs", [16, 32])
-def test_mixed_chunks(pkv, dtype, hq, hkv, bs):
+@pytest.mark.parametrize("head_dim", [64, 128])
+def test_mixed_chunks(pkv, dtype, hq, hkv, bs, head_dim):
     # whole prompts, chunks, single tokens and a few speculative tokens
     lens = (1, 17, 130, 300, 520, 64, 700, 33)
     qlens = (1, 17, 130, 57, 1, 4, 200, 33)
-    w = wl.Workload("prefill", 11, len(lens), hq, hkv, 128, bs, dtype,
+    w = wl.Workload("prefill", 11, len(lens), hq, hkv, head_dim, bs, dtype,
                     "fixed", fixed_lengths=lens)
     pin = wl.make_prefill(w, qlens, device="cuda")
     out = _run(pkv, pin)
-    _check(pin, out, f"{dtype}/{hq}:{hkv}/bs{bs}")
+    _check(pin, out, f"{dtype}/{hq}:{hkv}/bs{bs}/d{head_dim}")
 
 
 def test_single_token_matches_decode(pkv):
@@ -99,9 +100,10 @@ def test_bad_block_id_is_flagged(pkv):
 
 
 @pytest.mark.parametrize("bs", [16, 32])
-def test_unwritten_slots_hold_nan(pkv, bs):
+@pytest.mark.parametrize("head_dim", [64, 128])
+def test_unwritten_slots_hold_nan(pkv, bs, head_dim):
     lens = (1, 15, 17, 100, 333, 1000)
-    w = wl.Workload("prefill_nan", 14, len(lens), 32, 8, 128, bs,
+    w = wl.Workload("prefill_nan", 14, len(lens), 32, 8, head_dim, bs,
                     "bfloat16", "fixed", fixed_lengths=lens)
     pin = wl.make_prefill(w, (1, 15, 5, 100, 40, 300), device="cuda")
     _check(pin, _run(pkv, pin), "clean pool")
