@@ -32,9 +32,6 @@ __global__ void cache_write_kernel(uint4* __restrict__ k_cache,
                                    int num_kv_heads, int block_size,
                                    int64_t num_slots, int32_t* dev_err) {
   dev::pdl_trigger();  // a following decode may run its prologue now
-  // Launched early (programmatic serialization): the previous kernel may
-  // still read the cache, so wait for it before any store.
-  dev::pdl_wait();
   const int row_chunks = head_chunks * num_kv_heads;
   for (int64_t t0 = static_cast<int64_t>(blockIdx.x) * kTok; t0 < num_tokens;
        t0 += static_cast<int64_t>(gridDim.x) * kTok) {
@@ -82,7 +79,6 @@ __global__ void copy_blocks_kernel(uint4* __restrict__ k_cache,
                                    int64_t block_chunks, int num_blocks,
                                    int32_t* dev_err) {
   dev::pdl_trigger();
-  dev::pdl_wait();  // as above: the previous kernel may still read blocks
   const int pair = blockIdx.x;
   const int32_t src = pairs[2 * pair];
   const int32_t dst = pairs[2 * pair + 1];
@@ -95,16 +91,6 @@ __global__ void copy_blocks_kernel(uint4* __restrict__ k_cache,
   const uint4* s = cache + static_cast<int64_t>(src) * block_chunks;
   uint4* d = cache + static_cast<int64_t>(dst) * block_chunks;
   for (int64_t i = threadIdx.x; i < block_chunks; i += blockDim.x) d[i] = s[i];
-}
-
-// Programmatic stream serialization for a launch: the kernel may start
-// while the previous one in the stream drains, and waits for it
-// (griddepcontrol.wait) before touching memory that kernel may use.
-void pdl_attr(cudaLaunchAttribute (&attr)[1], cudaLaunchConfig_t* cfg) {
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg->attrs = attr;
-  cfg->numAttrs = 1;
 }
 
 int sm_count() {
@@ -167,20 +153,14 @@ pa_status pa_cache_write(void* k_cache, void* v_cache, const void* k,
   int64_t blocks = (num_tokens + pagedkv::kTok - 1) / pagedkv::kTok;
   const int64_t cap = static_cast<int64_t>(pagedkv::sm_count()) * 16;
   if (blocks > cap) blocks = cap;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
-  cfg.blockDim = dim3(threads);
-  cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  pagedkv::pdl_attr(attr, &cfg);
-  cudaError_t e = cudaLaunchKernelEx(
-      &cfg, pagedkv::cache_write_kernel, static_cast<uint4*>(k_cache),
-      static_cast<uint4*>(v_cache), static_cast<const uint4*>(k),
-      static_cast<const uint4*>(v), slot_mapping, num_tokens, head_chunks,
-      num_kv_heads, block_size,
+  pagedkv::cache_write_kernel<<<static_cast<unsigned>(blocks), threads, 0,
+                                static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), slot_mapping,
+      num_tokens, head_chunks, num_kv_heads, block_size,
       static_cast<int64_t>(num_blocks) * block_size, dev_err);
   pagedkv::count_launch();
-  if (e == cudaSuccess) e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return fail(PA_ERR_CUDA, "pa_cache_write: launch failed: %s",
                 cudaGetErrorString(e));
@@ -206,17 +186,12 @@ pa_status pa_copy_blocks(void* k_cache, void* v_cache, const int32_t* pairs,
                 "pa_copy_blocks: caches must be 16-byte aligned");
   const int64_t block_chunks =
       static_cast<int64_t>(num_kv_heads) * block_size * head_dim * 2 / 16;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(num_pairs, 2);
-  cfg.blockDim = dim3(256);
-  cfg.stream = static_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  pagedkv::pdl_attr(attr, &cfg);
-  cudaError_t e = cudaLaunchKernelEx(
-      &cfg, pagedkv::copy_blocks_kernel, static_cast<uint4*>(k_cache),
-      static_cast<uint4*>(v_cache), pairs, block_chunks, num_blocks, dev_err);
+  pagedkv::copy_blocks_kernel<<<dim3(num_pairs, 2), 256, 0,
+                                static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), pairs,
+      block_chunks, num_blocks, dev_err);
   pagedkv::count_launch();
-  if (e == cudaSuccess) e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess)
     return fail(PA_ERR_CUDA, "pa_copy_blocks: launch failed: %s",
                 cudaGetErrorString(e));
