@@ -163,11 +163,11 @@ def measured_hbm_peak():
 
 
 def decode_source_hash() -> str:
-    """Hash of the decode kernel's code (decode.cu and device_utils.cuh with
-    comments and blank space removed, so a comment edit keeps a capture
-    current and any code change makes it stale)."""
+    """Hash of the decode kernel's code (decode.cu, device_utils.cuh and
+    order.cuh with comments and blank space removed, so a comment edit
+    keeps a capture current and any code change makes it stale)."""
     h = hashlib.sha256()
-    for name in ("decode.cu", "device_utils.cuh"):
+    for name in ("decode.cu", "device_utils.cuh", "order.cuh"):
         with open(os.path.join(ROOT, "paged_kv_cache_383_b200", "csrc",
                                name)) as f:
             text = f.read()
@@ -597,6 +597,7 @@ def extras(args, w, inp, dev, pkv, bt, cl):
                       for n, c in PREFILL_CASES]
     out["prefix_cache"] = prefix_cache_measure(pkv, dev)
     out["swap"] = swap_measure(pkv, dev)
+    out["spec_verify"] = spec_verify_measure(pkv, dev)
     return out
 
 
@@ -697,7 +698,9 @@ def time_prefill(pkv, wl, name, chunk, dev, iters=10):
     qs = torch.from_numpy(pin.query_start).to(dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     kw = dict(max_q_len=int(pin.q_lens.max()),
-              max_context_len=int(inp.lengths.max()), dev_err=err)
+              max_context_len=int(inp.lengths.max()), dev_err=err,
+              workspace=torch.empty(4 * w.num_seqs + 16, dtype=torch.uint8,
+                                    device=dev))
     for _ in range(3):
         pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl, qs,
                        w.softmax_scale, **kw)
@@ -775,7 +778,9 @@ def prefix_cache_measure(pkv, dev, requests=128, prompt_len=2048,
         out = torch.empty_like(q)
         qsd = torch.from_numpy(qs).to(dev)
         kw = dict(max_q_len=int(q_lens.max()),
-                  max_context_len=int(lens.max()))
+                  max_context_len=int(lens.max()),
+                  workspace=torch.empty(4 * len(lens) + 16, dtype=torch.uint8,
+                                        device=dev))
         for _ in range(2):
             pkv.pa_prefill(out, q, kc, vc, bt, cl, qsd, d ** -0.5, **kw)
         a = torch.cuda.Event(enable_timing=True)
@@ -886,6 +891,45 @@ def swap_measure(pkv, dev, group_size=64, seed=383010):
     return res
 
 
+def spec_verify_measure(pkv, dev, drafts=4):
+    """Speculative verification on the batch-256 mix (Llama-3-70B heads,
+    log-normal lengths, block 16, bf16): every sequence checks ``drafts``
+    new tokens in one pa_prefill call.  Reported as GB/s of K/V read (it
+    reads every cached token once, like a decode) beside the decode of the
+    same batch."""
+    import torch
+    from paged_kv_cache_383_b200 import workloads as wl
+    w = wl.WORKLOADS["llama3_70b_gqa8"]
+    lens = wl.make_paged(w, values=False).lengths
+    pin = wl.make_prefill(w, np.full(w.num_seqs, drafts), device=dev)
+    inp = pin.paged
+    bt = torch.from_numpy(inp.block_tables).to(dev)
+    cl = torch.from_numpy(inp.lengths.astype(np.int32)).to(dev)
+    qs = torch.from_numpy(pin.query_start).to(dev)
+    out = torch.empty_like(pin.q)
+    kw = dict(max_q_len=drafts, max_context_len=int(lens.max()),
+              workspace=torch.empty(4 * w.num_seqs + 16, dtype=torch.uint8,
+                                    device=dev))
+    f = lambda: pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl,
+                               qs, w.softmax_scale, **kw)
+    for _ in range(3):
+        f()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(20):
+        f()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / 20
+    return {"seqs": w.num_seqs, "drafts": drafts,
+            "kv_bytes": kv_bytes(inp.lengths, w), "ms": round(ms, 4),
+            "kv_gbs": round(kv_bytes(inp.lengths, w) / (ms * 1e-3) / 1e9, 1),
+            "tflops": round(prefill_flops(inp.lengths, pin.q_lens,
+                                          w.num_q_heads, w.head_dim)
+                            / (ms * 1e-3) / 1e12, 1)}
+
+
 def run_extras_only(args):
     import torch
     import paged_kv_cache_383_b200 as pkv
@@ -899,6 +943,7 @@ def run_extras_only(args):
             "prefill": res,
             "prefix_cache": prefix_cache_measure(pkv, dev),
             "swap": swap_measure(pkv, dev),
+            "spec_verify": spec_verify_measure(pkv, dev),
             "gpu_launches": pkv.pa_launch_count()}
 
 

@@ -234,10 +234,21 @@ typedef struct {
   int max_context_len;  /* host bound on context_lens[] (0: table capacity) */
 } pa_prefill_desc;
 
+/* Bytes of device workspace pa_prefill needs for this shape (the sequence
+ * order: num_seqs int32, rounded up to 16). */
+size_t pa_prefill_workspace_bytes(const pa_prefill_desc* desc);
+
+/* workspace: pa_prefill_workspace_bytes(desc) bytes of caller-owned device
+ * memory, 16-byte aligned (PA_ERR_WORKSPACE otherwise); scratch after the
+ * call, and calls sharing it must not overlap on the device.  The call
+ * launches a one-CTA kernel that orders the sequences longest context
+ * first, then the prefill, whose grid rows serve them in that order (a
+ * long sequence never starts last), chained by programmatic launch. */
 pa_status pa_prefill(void* out, const void* q, const void* k_cache,
                      const void* v_cache, const int32_t* block_tables,
                      const int32_t* context_lens, const int32_t* query_start,
                      float scale, const pa_prefill_desc* desc,
+                     void* workspace, size_t workspace_bytes,
                      int32_t* dev_err, void* stream);
 
 /* ------------------------------------------------------------------------

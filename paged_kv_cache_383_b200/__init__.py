@@ -188,11 +188,14 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens,
 
 def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens,
                query_start, scale: float, *, max_q_len: int,
-               max_context_len: int = 0, dev_err=None, stream=None):
+               max_context_len: int = 0, workspace=None, dev_err=None,
+               stream=None):
     """Causal attention of each sequence's new tokens (rows
     query_start[b] .. query_start[b+1]-1 of ``q``) over its paged K/V, the
     new tokens being the last ones of the context.  ``max_q_len`` bounds
-    every sequence's new-token count (sizes the grid).  Returns ``out``."""
+    every sequence's new-token count (sizes the grid).  ``workspace`` (a
+    uint8 device tensor of ``pa_prefill_workspace_bytes(desc)`` bytes) is
+    allocated per call when not given.  Returns ``out``."""
     import torch
     lib = _lib.load()
     total_q, num_q_heads, head_dim = q.shape
@@ -208,6 +211,11 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens,
         max_blocks_per_seq=block_tables.shape[1], num_blocks=num_blocks,
         dtype=_dtype_code(q), total_q=total_q, max_q_len=max_q_len,
         max_context_len=max_context_len)
+    need = lib.pa_prefill_workspace_bytes(ctypes.byref(desc))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8,
+                                device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
     st = lib.pa_prefill(
         _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"),
         _dev(v_cache, "v_cache"),
@@ -215,6 +223,7 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens,
         _dev(context_lens, "context_lens", torch.int32),
         _dev(query_start, "query_start", torch.int32),
         ctypes.c_float(scale), ctypes.byref(desc),
+        _dev(workspace, "workspace"), ctypes.c_size_t(ws_bytes),
         _dev(dev_err, "dev_err", torch.int32), _stream(stream))
     _lib.check(st, "pa_prefill")
     return out

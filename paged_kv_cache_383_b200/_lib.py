@@ -94,7 +94,10 @@ SIGNATURES = {
     "pa_decode_noalloc": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
                                 ctypes.POINTER(pa_decode_desc), _vp, _vp]),
     "pa_prefill": (_st, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float,
-                         ctypes.POINTER(pa_prefill_desc), _vp, _vp]),
+                         ctypes.POINTER(pa_prefill_desc), _vp, ctypes.c_size_t,
+                         _vp, _vp]),
+    "pa_prefill_workspace_bytes": (ctypes.c_size_t,
+                                   [ctypes.POINTER(pa_prefill_desc)]),
     "pa_cache_write": (_st, [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int,
                              _int, _int, _vp, _vp]),
     "pa_copy_blocks": (_st, [_vp, _vp, _vp, _int, _int, _int, _int, _int, _int,

@@ -51,6 +51,7 @@
 #include <cstdint>
 
 #include "device_utils.cuh"
+#include "order.cuh"
 #include "pagedkv.h"
 #include "status.h"
 
@@ -829,53 +830,15 @@ __global__ void __launch_bounds__(kThreads)
 // covers the prep kernel.  Within one bucket the order follows the atomics;
 // results do not depend on it (each sequence is computed on its own and
 // partials are combined in partition order).
-constexpr int kPrepThreads = 1024;
-constexpr int kPrepBuckets = 1024;
-
-__global__ void __launch_bounds__(kPrepThreads)
+__global__ void __launch_bounds__(kOrderThreads)
     prep_kernel(const int32_t* __restrict__ context_lens, int num_seqs,
                 int shift, int32_t* __restrict__ order, int* counters,
                 int n_counters) {
-  __shared__ int hist[kPrepBuckets];
-  __shared__ int warp_sum[kPrepThreads / 32];
   dev::pdl_trigger();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  auto bucket = [&](int i) {
-    const int L = context_lens[i];
-    const int k = L <= 0 ? 0 : min(L >> shift, kPrepBuckets - 1);
-    return kPrepBuckets - 1 - k;  // longest first
-  };
-  hist[tid] = 0;
-  __syncthreads();
-  for (int i = tid; i < num_seqs; i += kPrepThreads)
-    atomicAdd(&hist[bucket(i)], 1);
-  __syncthreads();
-  // Exclusive scan of the 1024 bucket counts (one per thread).
-  const int c = hist[tid];
-  int x = c;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) warp_sum[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    int w = warp_sum[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    warp_sum[lane] = w;  // inclusive over warps
-  }
-  __syncthreads();
-  hist[tid] = x - c + (warp > 0 ? warp_sum[warp - 1] : 0);
-  __syncthreads();
-  dev::pdl_wait();
-  for (int i = tid; i < num_seqs; i += kPrepThreads)
-    order[atomicAdd(&hist[bucket(i)], 1)] = i;
-  for (int i = tid; i < n_counters; i += kPrepThreads) counters[i] = 0;
+  sort_longest_first(context_lens, num_seqs, shift, order,
+                     [] { dev::pdl_wait(); });
+  for (int i = threadIdx.x; i < n_counters; i += kOrderThreads)
+    counters[i] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -1141,12 +1104,6 @@ WsLayout ws_layout(const pa_decode_desc* d) {
 
 size_t workspace_bytes(const pa_decode_desc* d) { return ws_layout(d).total; }
 
-// Bucket shift for the prep kernel's sort: max_ctx >> shift < 1024.
-int order_shift(int max_ctx) {
-  int shift = 0;
-  while ((max_ctx >> shift) >= kPrepBuckets) ++shift;
-  return shift;
-}
 
 // Combine partitions inside the decode kernel (few partitions) or with the
 // separate reduce kernel.
@@ -1186,7 +1143,7 @@ pa_status launch(const pa_decode_desc* d, DecodeArgs& a, const CUtensorMap& km,
                       : 0;
     cudaLaunchConfig_t pcfg = {};
     pcfg.gridDim = dim3(1);
-    pcfg.blockDim = dim3(kPrepThreads);
+    pcfg.blockDim = dim3(kOrderThreads);
     pcfg.stream = stream;
     pcfg.attrs = attr;
     pcfg.numAttrs = 1;

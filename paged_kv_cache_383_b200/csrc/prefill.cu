@@ -54,6 +54,7 @@
 #include <cstdint>
 
 #include "device_utils.cuh"
+#include "order.cuh"
 #include "pagedkv.h"
 #include "status.h"
 #include "tcgen05_ts.cuh"
@@ -72,6 +73,7 @@ constexpr float kRescaleLog2 = 8.f;
 
 struct PrefillArgs {
   void* out;
+  const int32_t* order;  // [num_seqs] sequence served by grid row z
   const int32_t* block_tables;
   const int32_t* context_lens;
   const int32_t* query_start;
@@ -147,7 +149,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       reinterpret_cast<uint32_t*>(smem + kOffBars + kNumBars * 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int qt = blockIdx.x, kvh = blockIdx.y;
+  // Grid rows serve sequences longest first (the order kernel, which this
+  // grid follows by programmatic launch, wrote it): the grid's tail is short
+  // work even when a few long sequences dominate.
+  dev::pdl_wait();
+  const int b = a.order[blockIdx.z];
   const int L = a.context_lens[b];
   const int q0 = a.query_start[b];
   const int q_len = a.query_start[b + 1] - q0;
@@ -573,6 +580,21 @@ bool encode_cache(CUtensorMap* m, const void* cache, uint64_t rows, int hd,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// One CTA: the longest-first order of the sequences (by context length),
+// launched in stream order after whatever came before (which may still have
+// read the order), and letting the prefill launch early behind it.
+__global__ void __launch_bounds__(kOrderThreads)
+    prefill_order_kernel(const int32_t* __restrict__ context_lens,
+                         int num_seqs, int shift, int32_t* __restrict__ order) {
+  dev::pdl_trigger();
+  sort_longest_first(context_lens, num_seqs, shift, order, [] {});
+}
+
+size_t prefill_workspace_bytes(const pa_prefill_desc* d) {
+  return (static_cast<size_t>(d->num_seqs) * sizeof(int32_t) + 15) &
+         ~size_t(15);
+}
+
 template <typename T, int BS, int G, int D>
 pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
                  const CUtensorMap& qm, const CUtensorMap& km,
@@ -586,10 +608,20 @@ pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
     return fail(PA_ERR_CUDA, "pa_prefill: cudaFuncSetAttribute(%zu): %s",
                 smem, cudaGetErrorString(e));
   constexpr int kTok = kRows / G;
-  dim3 grid((d->max_q_len + kTok - 1) / kTok, d->num_kv_heads, d->num_seqs);
-  kern<<<grid, kThreads, smem, st>>>(qm, km, vm, a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim =
+      dim3((d->max_q_len + kTok - 1) / kTok, d->num_kv_heads, d->num_seqs);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, qm, km, vm, a);
   count_launch();
-  e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess)
     return fail(PA_ERR_CUDA, "pa_prefill: launch failed: %s",
                 cudaGetErrorString(e));
@@ -630,7 +662,8 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
                                 const int32_t* block_tables,
                                 const int32_t* context_lens,
                                 const int32_t* query_start, float scale,
-                                const pa_prefill_desc* d, int32_t* dev_err,
+                                const pa_prefill_desc* d, void* workspace,
+                                size_t workspace_bytes, int32_t* dev_err,
                                 void* stream) {
   pagedkv::clear_error();
   if (!d) return fail(PA_ERR_INVALID_ARG, "pa_prefill: desc is NULL");
@@ -650,8 +683,8 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
       (d->block_size != 16 && d->block_size != 32) ||
       (G != 1 && G != 2 && G != 4 && G != 8))
     return fail(PA_ERR_UNSUPPORTED,
-                "pa_prefill: needs head_dim 64 or 128 (got %d), block_size 16 or 32 "
-                "(got %d) and a query group of 1, 2, 4 or 8 (got %d)",
+                "pa_prefill: needs head_dim 64 or 128 (got %d), block_size "
+                "16 or 32 (got %d) and a query group of 1, 2, 4 or 8 (got %d)",
                 d->head_dim, d->block_size, G);
   if (d->num_seqs == 0 || d->total_q == 0 || d->max_q_len == 0) return PA_OK;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens ||
@@ -661,6 +694,11 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
       !pagedkv::aligned16(k_cache) || !pagedkv::aligned16(v_cache))
     return fail(PA_ERR_INVALID_ARG,
                 "pa_prefill: out, q and the caches must be 16-byte aligned");
+  const size_t need = pagedkv::prefill_workspace_bytes(d);
+  if (!workspace || workspace_bytes < need || !pagedkv::aligned16(workspace))
+    return fail(PA_ERR_WORKSPACE,
+                "pa_prefill: workspace of %zu bytes (16-byte aligned) needed, "
+                "got %zu at %p", need, workspace_bytes, workspace);
   if (d->num_blocks == 0 || d->num_seqs > 65535 || d->num_kv_heads > 65535)
     return fail(PA_ERR_INVALID_ARG, "pa_prefill: bad pool or batch size");
   if (static_cast<int64_t>(d->num_blocks) * d->num_kv_heads * d->block_size >
@@ -682,6 +720,7 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
     return fail(PA_ERR_CUDA, "pa_prefill: cuTensorMapEncodeTiled failed");
   pagedkv::PrefillArgs a;
   a.out = out;
+  a.order = static_cast<const int32_t*>(workspace);
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.query_start = query_start;
@@ -694,7 +733,21 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
   a.max_context_len = max_ctx;
   a.total_q = d->total_q;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  pagedkv::prefill_order_kernel<<<1, pagedkv::kOrderThreads, 0, s>>>(
+      context_lens, d->num_seqs, pagedkv::order_shift(max_ctx),
+      static_cast<int32_t*>(workspace));
+  pagedkv::count_launch();
+  const cudaError_t oe = cudaGetLastError();
+  if (oe != cudaSuccess)
+    return fail(PA_ERR_CUDA, "pa_prefill: order launch failed: %s",
+                cudaGetErrorString(oe));
   if (d->dtype == PA_BF16)
     return pagedkv::dispatch_shape<__nv_bfloat16>(d, a, qm, km, vm, s);
   return pagedkv::dispatch_shape<__half>(d, a, qm, km, vm, s);
+}
+
+extern "C" size_t pa_prefill_workspace_bytes(const pa_prefill_desc* d) {
+  pagedkv::clear_error();
+  if (!d || d->num_seqs < 0) return 0;
+  return pagedkv::prefill_workspace_bytes(d);
 }

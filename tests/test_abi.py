@@ -116,3 +116,25 @@ def test_zero_sized_calls_are_noops(pkv):
                               None) == 0
     assert lib.pa_cache_write(None, None, None, None, None, 3, 8, 128, 16, 4,
                               1, None, None) == _lib.PA_ERR_INVALID_ARG
+
+
+def test_prefill_needs_its_order_workspace(pkv):
+    from paged_kv_cache_383_b200 import _lib
+    lib = _lib.load()
+    d = _lib.pa_prefill_desc(num_seqs=5, num_q_heads=8, num_kv_heads=2,
+                             head_dim=128, block_size=16,
+                             max_blocks_per_seq=4, num_blocks=16, dtype=1,
+                             total_q=20, max_q_len=4, max_context_len=64)
+    # the sequence order: 5 int32, rounded up to 16 bytes
+    assert lib.pa_prefill_workspace_bytes(ctypes.byref(d)) == 32
+    fake = 0x1000
+    args = [fake] * 7 + [ctypes.c_float(1.0), ctypes.byref(d)]
+    for ws, nbytes in ((None, 32), (fake, 16), (fake + 4, 32)):
+        st = lib.pa_prefill(*args, ws, nbytes, None, None)
+        assert st == _lib.PA_ERR_WORKSPACE, (ws, nbytes)
+        assert b"workspace" in lib.pa_last_error()
+    d0 = _lib.pa_prefill_desc(num_seqs=0, num_q_heads=8, num_kv_heads=2,
+                              head_dim=128, block_size=16,
+                              max_blocks_per_seq=4, num_blocks=16, dtype=1)
+    assert lib.pa_prefill(*([None] * 7), ctypes.c_float(1.0),
+                          ctypes.byref(d0), None, 0, None, None) == 0

@@ -238,3 +238,22 @@ def test_long_context_chunk_sampled(pkv):
         ref = oa.paged_decode(to_np(pin.q)[rows], kc, vc, sub, pos + 1,
                               w.softmax_scale)
         check_decode(to_np(out)[rows], ref, pin.q.dtype, f"long seq {b}")
+
+
+def test_more_sequences_than_order_threads(pkv):
+    """1300 sequences (more than the one-CTA longest-first sort has threads),
+    uniform 1..200-token contexts, 0..5 new tokens each: the grid rows follow
+    the sort's order, so every sequence must still land in its own rows.
+    Sampled sequences against the oracle, and no row left unwritten."""
+    w = wl.Workload("many_seqs", 31, 1300, 16, 2, 64, 16, "bfloat16",
+                    "uniform", low=1, high=200)
+    lens = wl.make_paged(w, values=False).lengths
+    q_lens = np.minimum(lens, np.random.default_rng(3).integers(0, 6, 1300))
+    pin = wl.make_prefill(w, q_lens, device="cuda")
+    out = _run(pkv, pin)
+    assert not torch.isnan(out).any()
+    rng = np.random.default_rng(4)
+    seqs = sorted({0, 1, 1023, 1024, 1299, int(np.argmax(lens)),
+                   int(np.argmin(lens)), *rng.integers(0, 1300, 25).tolist()})
+    seqs = [b for b in seqs if q_lens[b] > 0]
+    _check(pin, out, "1300 sequences", seqs=seqs)
