@@ -953,8 +953,12 @@ def run_e2e(args, w, inp, dev, pkv, flow, world, rank, ps):
     tables (on the host), the step's inputs (q, the new tokens' K/V, slots,
     tables, lengths) go host->device from pinned memory in one packed copy,
     then cache write and decode, and the output comes back device->host;
-    one sync per step.  The host work of step n+1 runs while the GPU works
-    on step n (two pinned staging buffers); nothing else overlaps steps."""
+    the host waits for each step's output.  Steps are pipelined the way a
+    serving loop overlaps them: while the GPU decodes step n, the host
+    builds step n+1's inputs and copies them up on a copy stream, and
+    earlier steps' outputs come down on another; the host reads step n's
+    output while step n+2 is issued (three staging buffers on each side).
+    Every step's copies and kernels lie inside the timed region."""
     import torch
     bm = pkv.BlockManager(inp.num_blocks, w.block_size,
                           free_order=_free_order(inp))
@@ -984,66 +988,96 @@ def run_e2e(args, w, inp, dev, pkv, flow, world, rank, ps):
         return {k: buf[o:o + n].view(dt).view(shape)
                 for k, (o, n, dt, shape) in fields.items()}
 
+    depth = 3
     stage = [torch.empty(total, dtype=torch.uint8).pin_memory()
-             for _ in range(2)]
+             for _ in range(depth)]
     hv = [views(x) for x in stage]
     for v in hv:
         for name, t in parts:
             v[name].copy_(t.cpu())
-    dstage = torch.empty(total, dtype=torch.uint8, device=dev)
-    dv = views(dstage)
-    dout = torch.empty_like(inp.q)
-    hout = torch.empty(inp.q.shape, dtype=inp.q.dtype).pin_memory()
-    desc = pkv.make_desc(inp.q, inp.k_cache, dv["table"],
+    dstage = [torch.empty(total, dtype=torch.uint8, device=dev)
+              for _ in range(depth)]
+    dv = [views(x) for x in dstage]
+    dout = [torch.empty_like(inp.q) for _ in range(depth)]
+    hout = [torch.empty(inp.q.shape, dtype=inp.q.dtype).pin_memory()
+            for _ in range(depth)]
+    desc = pkv.make_desc(inp.q, inp.k_cache, dv[0]["table"],
                          partition_size=ps,
                          max_context_len=int(final_lens.max()))
     ws = torch.empty(max(pkv.pa_decode_workspace_bytes(desc), 16),
                      dtype=torch.uint8, device=dev)
     ones = np.ones(B, dtype=np.int32)
     stream = torch.cuda.current_stream(dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_up = [torch.cuda.Event() for _ in range(depth)]
+    ev_run = [torch.cuda.Event() for _ in range(depth)]
+    ev_down = [torch.cuda.Event() for _ in range(depth)]
 
     def prepare(i):
         """Host work of one step into staging buffer i."""
+        ev_up[i].synchronize()          # its previous upload has left
         _, pairs = bm.append_batch(ids, ones, slots_out=hv[i]["slots"].numpy())
         _, lens = bm.block_table(ids, max_blocks,
                                  table_out=hv[i]["table"].numpy(),
                                  lens_out=hv[i]["lens"].numpy())
         return pairs, int(lens.sum())
 
+    def upload(i):
+        up.wait_event(ev_run[i])        # kernels of `depth` steps ago
+        with torch.cuda.stream(up):
+            dstage[i].copy_(stage[i], non_blocking=True)
+        ev_up[i].record(up)
+
     def launch(i, pairs):
-        dstage.copy_(stage[i], non_blocking=True)
+        stream.wait_event(ev_up[i])
+        stream.wait_event(ev_down[i])   # dout[i] of `depth` steps ago
         nb = 0
         if len(pairs):
             d_pairs = torch.from_numpy(pairs).pin_memory().to(
                 dev, non_blocking=True)
             pkv.pa_copy_blocks(inp.k_cache, inp.v_cache, d_pairs)
             nb = pairs.nbytes
-        pkv.pa_cache_write(inp.k_cache, inp.v_cache, dv["k"], dv["v"],
-                           dv["slots"])
-        pkv.pa_decode(dout, dv["q"], inp.k_cache, inp.v_cache, dv["table"],
-                      dv["lens"], w.softmax_scale, desc=desc, workspace=ws)
-        hout.copy_(dout, non_blocking=True)
+        pkv.pa_cache_write(inp.k_cache, inp.v_cache, dv[i]["k"], dv[i]["v"],
+                           dv[i]["slots"])
+        pkv.pa_decode(dout[i], dv[i]["q"], inp.k_cache, inp.v_cache,
+                      dv[i]["table"], dv[i]["lens"], w.softmax_scale,
+                      desc=desc, workspace=ws)
+        ev_run[i].record(stream)
+        down.wait_event(ev_run[i])
+        with torch.cuda.stream(down):
+            hout[i].copy_(dout[i], non_blocking=True)
+        ev_down[i].record(down)
         return nb
 
-    tot_tokens, h2d = 0, 0
-    nxt = prepare(0)
-    for n in range(args.warmup):
-        launch(n % 2, nxt[0])
-        nxt = prepare((n + 1) % 2)
-        stream.synchronize()
+    def run(n0, count, start=None):
+        """Steps n0 .. n0+count-1; returns (tokens attended, pair bytes)."""
+        if count == 0:
+            return 0, 0
+        if start is not None:
+            up.wait_event(start)
+        tokens, nb = 0, 0
+        nxt = prepare(n0 % depth)
+        upload(n0 % depth)
+        for n in range(n0, n0 + count):
+            pairs, tok = nxt
+            nb = max(nb, launch(n % depth, pairs))
+            tokens += tok
+            if n + 1 < n0 + count:
+                nxt = prepare((n + 1) % depth)
+                upload((n + 1) % depth)
+            if n >= n0 + depth - 1:
+                ev_down[(n - depth + 1) % depth].synchronize()  # its output
+        stream.wait_event(ev_down[(n0 + count - 1) % depth])
+        return tokens, nb
+
+    run(0, args.warmup)
+    torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for n in range(args.warmup, args.warmup + steps):
-        pairs, tok = nxt
-        nb = launch(n % 2, pairs)
-        tot_tokens += tok
-        h2d = total + nb
-        if n + 1 < args.warmup + steps:
-            nxt = prepare((n + 1) % 2)
-        stream.synchronize()
+    tot_tokens, nb = run(args.warmup, steps, start=a)
     b.record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -1051,13 +1085,14 @@ def run_e2e(args, w, inp, dev, pkv, flow, world, rank, ps):
     bm.close()
     tot_bytes = tot_tokens * w.num_kv_heads * w.head_dim * 2 * 2
     return {"value": round(world * tot_bytes / (ms * 1e-3) / 1e9, 2),
-            "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(hout.nbytes),
+            "unit": "GB/s", "h2d_bytes_per_step": int(total + nb),
+            "d2h_bytes_per_step": int(hout[0].nbytes),
             "ms_per_step": round(ms / steps, 4),
-            "includes": "host block-manager append + table build (for the "
-                        "next step, while the GPU runs this one), one packed "
+            "includes": "host block-manager append + table build, one packed "
                         "pinned H2D of q/new K,V/slots/tables/lengths, cache "
-                        "write, decode, D2H of the output, one sync per step"}
+                        "write, decode, D2H of the output, host wait for each "
+                        "output; step n+1's host work and H2D and earlier "
+                        "steps' D2H overlap step n's kernels (3 buffers)"}
 
 
 def wl_blocks(lengths, bs):

@@ -213,7 +213,8 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,
  * int32 on the device, non-decreasing, query_start[0] = 0 and
  * query_start[num_seqs] <= total_q; the rest as for pa_decode.
  * Supported: head_dim 64 or 128, block_size 16 or 32, G = 1, 2, 4 or 8 (else
- * PA_ERR_UNSUPPORTED); any context length the table holds.  Runs on the
+ * PA_ERR_UNSUPPORTED); any context length the table holds; max_q_len up to
+ * 65535 tiles of 128 / G new tokens (PA_ERR_UNSUPPORTED above).  Runs on the
  * tcgen05 tensor cores with fp32 accumulation in tensor memory; output
  * rounded once to dtype.
  * Device-side: a context or query range outside the table, a sequence with
@@ -243,7 +244,9 @@ size_t pa_prefill_workspace_bytes(const pa_prefill_desc* desc);
  * call, and calls sharing it must not overlap on the device.  The call
  * launches a one-CTA kernel that orders the sequences longest context
  * first, then the prefill, whose grid rows serve them in that order (a
- * long sequence never starts last), chained by programmatic launch. */
+ * long sequence never starts last) and start each sequence's query tiles
+ * from its last (the one that sees the most keys), chained by programmatic
+ * launch. */
 pa_status pa_prefill(void* out, const void* q, const void* k_cache,
                      const void* v_cache, const int32_t* block_tables,
                      const int32_t* context_lens, const int32_t* query_start,

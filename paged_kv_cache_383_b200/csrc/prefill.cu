@@ -149,10 +149,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       reinterpret_cast<uint32_t*>(smem + kOffBars + kNumBars * 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = blockIdx.x, kvh = blockIdx.y;
-  // Grid rows serve sequences longest first (the order kernel, which this
-  // grid follows by programmatic launch, wrote it): the grid's tail is short
-  // work even when a few long sequences dominate.
+  // CTAs start in the order x (KV head), y, z.  y counts query tiles from
+  // the last one, which sees the most keys (the causal triangle), and z
+  // serves sequences longest first (the order kernel, which this grid
+  // follows by programmatic launch, wrote it): the grid's tail is short
+  // work even when a few long sequences or whole prompts dominate.
+  const int kvh = blockIdx.x;
+  const int qt = gridDim.y - 1 - blockIdx.y;
   dev::pdl_wait();
   const int b = a.order[blockIdx.z];
   const int L = a.context_lens[b];
@@ -165,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     return;
   }
   const int tok0 = qt * kTok;
-  if (qt == gridDim.x - 1 && q_len > tok0 + kTok) {
+  if (qt == static_cast<int>(gridDim.y) - 1 && q_len > tok0 + kTok) {
     // max_q_len was below this sequence's new-token count: the grid misses
     // rows, which are left unwritten.
     if (kvh == 0 && tid == 0) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
@@ -610,7 +613,7 @@ pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
   constexpr int kTok = kRows / G;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim =
-      dim3((d->max_q_len + kTok - 1) / kTok, d->num_kv_heads, d->num_seqs);
+      dim3(d->num_kv_heads, (d->max_q_len + kTok - 1) / kTok, d->num_seqs);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -701,6 +704,10 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
                 "got %zu at %p", need, workspace_bytes, workspace);
   if (d->num_blocks == 0 || d->num_seqs > 65535 || d->num_kv_heads > 65535)
     return fail(PA_ERR_INVALID_ARG, "pa_prefill: bad pool or batch size");
+  if ((d->max_q_len + pagedkv::kRows / G - 1) / (pagedkv::kRows / G) > 65535)
+    return fail(PA_ERR_UNSUPPORTED,
+                "pa_prefill: max_q_len %d needs more than 65535 query tiles",
+                d->max_q_len);
   if (static_cast<int64_t>(d->num_blocks) * d->num_kv_heads * d->block_size >
       0x7fffffffLL)
     return fail(PA_ERR_UNSUPPORTED, "pa_prefill: pool exceeds 2^31 rows");

@@ -138,3 +138,19 @@ def test_prefill_needs_its_order_workspace(pkv):
                               max_blocks_per_seq=4, num_blocks=16, dtype=1)
     assert lib.pa_prefill(*([None] * 7), ctypes.c_float(1.0),
                           ctypes.byref(d0), None, 0, None, None) == 0
+
+
+def test_prefill_refuses_more_query_tiles_than_the_grid_holds(pkv):
+    from paged_kv_cache_383_b200 import _lib
+    lib = _lib.load()
+    # G = 1: 128 new tokens per tile, 65535 tiles at most
+    d = _lib.pa_prefill_desc(num_seqs=1, num_q_heads=2, num_kv_heads=2,
+                             head_dim=128, block_size=16,
+                             max_blocks_per_seq=1 << 20, num_blocks=1 << 20,
+                             dtype=1, total_q=128 * 65535 + 1,
+                             max_q_len=128 * 65535 + 1)
+    fake = 0x1000
+    st = lib.pa_prefill(*([fake] * 7), ctypes.c_float(1.0), ctypes.byref(d),
+                        fake, 16, None, None)
+    assert st == _lib.PA_ERR_UNSUPPORTED
+    assert b"query tiles" in lib.pa_last_error()
