@@ -1082,6 +1082,16 @@ def run_e2e(args, w, inp, dev, pkv, flow, world, rank, ps):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(a.elapsed_time(b), world)
+    # The last step's output, as it reached the host, must equal a decode of
+    # the same inputs run on its own now (the kernel is deterministic).
+    last = (args.warmup + steps - 1) % depth
+    again = torch.empty_like(dout[last])
+    pkv.pa_decode(again, dv[last]["q"], inp.k_cache, inp.v_cache,
+                  dv[last]["table"], dv[last]["lens"], w.softmax_scale,
+                  desc=desc, workspace=ws)
+    if steps and not torch.equal(again.cpu(), hout[last]):
+        raise RuntimeError("end-to-end output differs from a plain decode "
+                           "of the same step")
     bm.close()
     tot_bytes = tot_tokens * w.num_kv_heads * w.head_dim * 2 * 2
     return {"value": round(world * tot_bytes / (ms * 1e-3) / 1e9, 2),

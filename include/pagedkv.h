@@ -509,6 +509,15 @@ int64_t pa_launch_count(void);
 pa_status pa_read_probe(const void* buf, size_t bytes, uint32_t* sink,
                         void* stream);
 
+/* Self-test of the kernels' bounded waits (no counterpart in the pages): one
+ * warp allocates 32 tensor-memory columns and waits on an mbarrier that
+ * nothing arrives at.  After the wait limit (1 s of device time) it sets
+ * *dev_err = PA_ERR_DEVICE_TIMEOUT (if still 0), frees the tensor memory and
+ * returns, which is what the decode and prefill kernels do when a copy
+ * never lands.  dev_err: a device int32, required (PA_ERR_INVALID_ARG
+ * otherwise).  Asynchronous on `stream`. */
+pa_status pa_wait_probe(int32_t* dev_err, void* stream);
+
 /* Pool and sequence queries (-1 for an unknown handle / sequence / block).
  * pa_bm_num_used = blocks referenced by a table or by the prefix cache
  * (num_blocks - pa_bm_num_free). */

@@ -30,7 +30,7 @@ __all__ = [
     "pa_copy_blocks",
     "pa_decode_workspace_bytes", "pa_decode_partition_size", "make_desc",
     "BlockManager", "PagedKVError", "NoFreeBlocksError", "library_path",
-    "pa_launch_count", "pa_read_probe",
+    "pa_launch_count", "pa_read_probe", "pa_wait_probe",
     "PA_KERNEL_AUTO", "PA_KERNEL_MMA", "PA_KERNEL_SIMT",
 ]
 
@@ -51,6 +51,19 @@ def pa_read_probe(buf, sink, stream=None):
         _dev(buf, "buf"), buf.numel() * buf.element_size(),
         _dev(sink, "sink", torch.int32), _stream(stream))
     _lib.check(st, "pa_read_probe")
+
+
+def pa_wait_probe(dev_err, stream=None):
+    """Make one bounded device wait run out (about 1 s of device time): the
+    kernel sets ``dev_err`` (an int32 CUDA tensor) to PA_ERR_DEVICE_TIMEOUT,
+    frees its tensor memory and returns, as the attention kernels do when a
+    copy never lands."""
+    import torch
+    if dev_err is None:
+        raise ValueError("pa_wait_probe needs a dev_err tensor")
+    st = _lib.load().pa_wait_probe(_dev(dev_err, "dev_err", torch.int32),
+                                   _stream(stream))
+    _lib.check(st, "pa_wait_probe")
 
 
 def pa_launch_count() -> int:

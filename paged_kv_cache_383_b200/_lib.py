@@ -117,6 +117,7 @@ SIGNATURES = {
     "pa_bm_block_table": (_st, [_vp, _pi64, _int, _int, _pi32, _pi32]),
     "pa_launch_count": (_i64, []),
     "pa_read_probe": (_st, [_vp, ctypes.c_size_t, _vp, _vp]),
+    "pa_wait_probe": (_st, [_vp, _vp]),
     "pa_bm_num_free": (_int, [_vp]),
     "pa_bm_refcount": (_int, [_vp, _int]),
     "pa_bm_seq_len": (_i64, [_vp, _i64]),

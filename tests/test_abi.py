@@ -154,3 +154,10 @@ def test_prefill_refuses_more_query_tiles_than_the_grid_holds(pkv):
                         fake, 16, None, None)
     assert st == _lib.PA_ERR_UNSUPPORTED
     assert b"query tiles" in lib.pa_last_error()
+
+
+def test_wait_probe_needs_an_error_word(pkv):
+    from paged_kv_cache_383_b200 import _lib
+    lib = _lib.load()
+    assert lib.pa_wait_probe(None, None) == _lib.PA_ERR_INVALID_ARG
+    assert b"error word" in lib.pa_last_error()
