@@ -59,6 +59,11 @@ def parse_args():
     p.add_argument("--extras-only", action="store_true",
                    help="time only the side measurements (prefill, prefix "
                         "cache, swap) and print them (tuning and profiling)")
+    p.add_argument("--extra", default="all",
+                   choices=["all", "prefill", "prefix_cache", "swap",
+                            "spec_verify"],
+                   help="with --extras-only: run just this side measurement "
+                        "(small profiling captures)")
     return p.parse_args()
 
 
@@ -936,15 +941,22 @@ def run_extras_only(args):
     from paged_kv_cache_383_b200 import workloads as wl
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    res = [time_prefill(pkv, wl, n, c, dev, iters=max(args.steps, 1))
-           for n, c in PREFILL_CASES]
-    return {"metric": "side measurements: prefill attention TFLOP/s "
-                      "(algorithmic), prefix cache, swap",
-            "prefill": res,
-            "prefix_cache": prefix_cache_measure(pkv, dev),
-            "swap": swap_measure(pkv, dev),
-            "spec_verify": spec_verify_measure(pkv, dev),
-            "gpu_launches": pkv.pa_launch_count()}
+    want = lambda name: args.extra in ("all", name)
+    res = {"metric": "side measurements: prefill attention TFLOP/s "
+                     "(algorithmic), prefix cache, swap, speculative "
+                     "verification"}
+    if want("prefill"):
+        res["prefill"] = [time_prefill(pkv, wl, n, c, dev,
+                                       iters=max(args.steps, 1))
+                          for n, c in PREFILL_CASES]
+    if want("prefix_cache"):
+        res["prefix_cache"] = prefix_cache_measure(pkv, dev)
+    if want("swap"):
+        res["swap"] = swap_measure(pkv, dev)
+    if want("spec_verify"):
+        res["spec_verify"] = spec_verify_measure(pkv, dev)
+    res["gpu_launches"] = pkv.pa_launch_count()
+    return res
 
 
 def run_e2e(args, w, inp, dev, pkv, flow, world, rank, ps):
