@@ -915,24 +915,34 @@ def spec_verify_measure(pkv, dev, drafts=4):
     kw = dict(max_q_len=drafts, max_context_len=int(lens.max()),
               workspace=torch.empty(4 * w.num_seqs + 16, dtype=torch.uint8,
                                     device=dev))
-    f = lambda: pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl,
-                               qs, w.softmax_scale, **kw)
-    for _ in range(3):
-        f()
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(20):
-        f()
-    b.record()
-    torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / 20
+
+    def time_kernel(kernel):
+        f = lambda: pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt,
+                                   cl, qs, w.softmax_scale, kernel=kernel,
+                                   **kw)
+        for _ in range(3):
+            f()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(20):
+            f()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / 20
+
+    ms = time_kernel("auto")
+    ms_keys = time_kernel("keys")
+    gbs = lambda t: round(kv_bytes(inp.lengths, w) / (t * 1e-3) / 1e9, 1)
     return {"seqs": w.num_seqs, "drafts": drafts,
             "kv_bytes": kv_bytes(inp.lengths, w), "ms": round(ms, 4),
-            "kv_gbs": round(kv_bytes(inp.lengths, w) / (ms * 1e-3) / 1e9, 1),
+            "kv_gbs": gbs(ms),
             "tflops": round(prefill_flops(inp.lengths, pin.q_lens,
                                           w.num_q_heads, w.head_dim)
-                            / (ms * 1e-3) / 1e12, 1)}
+                            / (ms * 1e-3) / 1e12, 1),
+            "kernel": "auto (the tile kernel)",
+            "ms_keys_kernel": round(ms_keys, 4),
+            "kv_gbs_keys_kernel": gbs(ms_keys)}
 
 
 def run_extras_only(args):

@@ -221,6 +221,26 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,
  * more new tokens than max_q_len, or a block id outside the pool sets
  * *dev_err = PA_ERR_DEVICE_OOB and the affected rows are unspecified.
  * ---------------------------------------------------------------------- */
+/* Which prefill kernel runs:
+ *   PA_PREFILL_AUTO  -- PA_PREFILL_TILE (the faster of the two on every
+ *                       shape measured so far).
+ *   PA_PREFILL_TILE  -- tiles of 128 query rows (new token, query head) on
+ *                       the MMA's M side, 64 keys on N; any q_len.
+ *   PA_PREFILL_KEYS  -- keys on M (128 per tile), the <= 32 query rows of
+ *                       one KV head on N: S^T = K Q^T, O^T += V^T P^T, so no
+ *                       MMA row is padding when few tokens are new
+ *                       (speculative verification).  Needs head_dim 128 and
+ *                       max_q_len * G <= 32 (PA_ERR_UNSUPPORTED otherwise);
+ *                       persistent, one CTA per SM.  Same results within
+ *                       the tolerance; slower than PA_PREFILL_TILE today
+ *                       (four softmax warps per SM and a cross-warp row
+ *                       maximum every 128 keys). */
+typedef enum {
+  PA_PREFILL_AUTO = 0,
+  PA_PREFILL_TILE = 1,
+  PA_PREFILL_KEYS = 2
+} pa_prefill_kernel;
+
 typedef struct {
   int num_seqs;
   int num_q_heads;
@@ -233,6 +253,7 @@ typedef struct {
   int total_q;          /* rows of q and out */
   int max_q_len;        /* host bound on any sequence's new-token count */
   int max_context_len;  /* host bound on context_lens[] (0: table capacity) */
+  int kernel;           /* pa_prefill_kernel (0: automatic) */
 } pa_prefill_desc;
 
 /* Bytes of device workspace pa_prefill needs for this shape (the sequence

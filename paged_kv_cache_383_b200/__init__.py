@@ -37,6 +37,8 @@ __all__ = [
 _KERNELS = {"auto": PA_KERNEL_AUTO, "mma": PA_KERNEL_MMA,
             "simt": PA_KERNEL_SIMT}
 _REDUCES = {"auto": _lib.PA_REDUCE_AUTO, "kernel": _lib.PA_REDUCE_KERNEL}
+_PREFILL_KERNELS = {"auto": _lib.PA_PREFILL_AUTO, "tile": _lib.PA_PREFILL_TILE,
+                    "keys": _lib.PA_PREFILL_KEYS}
 
 
 def library_path() -> str:
@@ -201,12 +203,14 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens,
 
 def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens,
                query_start, scale: float, *, max_q_len: int,
-               max_context_len: int = 0, workspace=None, dev_err=None,
-               stream=None):
+               max_context_len: int = 0, kernel: str = "auto",
+               workspace=None, dev_err=None, stream=None):
     """Causal attention of each sequence's new tokens (rows
     query_start[b] .. query_start[b+1]-1 of ``q``) over its paged K/V, the
     new tokens being the last ones of the context.  ``max_q_len`` bounds
-    every sequence's new-token count (sizes the grid).  ``workspace`` (a
+    every sequence's new-token count (sizes the grid).  ``kernel``: "auto",
+    "tile" (query rows on the MMA's M side) or "keys" (keys on M; head_dim
+    128 and max_q_len * G <= 32).  ``workspace`` (a
     uint8 device tensor of ``pa_prefill_workspace_bytes(desc)`` bytes) is
     allocated per call when not given.  Returns ``out``."""
     import torch
@@ -223,7 +227,7 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens,
         num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=block_size,
         max_blocks_per_seq=block_tables.shape[1], num_blocks=num_blocks,
         dtype=_dtype_code(q), total_q=total_q, max_q_len=max_q_len,
-        max_context_len=max_context_len)
+        max_context_len=max_context_len, kernel=_PREFILL_KERNELS[kernel])
     need = lib.pa_prefill_workspace_bytes(ctypes.byref(desc))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8,

@@ -69,8 +69,11 @@ class pa_prefill_desc(ctypes.Structure):
         ("total_q", ctypes.c_int),
         ("max_q_len", ctypes.c_int),
         ("max_context_len", ctypes.c_int),
+        ("kernel", ctypes.c_int),
     ]
 
+
+PA_PREFILL_AUTO, PA_PREFILL_TILE, PA_PREFILL_KEYS = 0, 1, 2
 
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int32

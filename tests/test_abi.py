@@ -161,3 +161,29 @@ def test_wait_probe_needs_an_error_word(pkv):
     lib = _lib.load()
     assert lib.pa_wait_probe(None, None) == _lib.PA_ERR_INVALID_ARG
     assert b"error word" in lib.pa_last_error()
+
+
+def test_prefill_kernel_choice_is_checked(pkv):
+    from paged_kv_cache_383_b200 import _lib
+    lib = _lib.load()
+    fake = 0x1000
+
+    def call(**kw):
+        base = dict(num_seqs=2, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                    block_size=16, max_blocks_per_seq=4, num_blocks=16,
+                    dtype=1, total_q=20, max_q_len=10, max_context_len=64)
+        base.update(kw)
+        d = _lib.pa_prefill_desc(**base)
+        return lib.pa_prefill(*([fake] * 7), ctypes.c_float(1.0),
+                              ctypes.byref(d), None, 0, None, None)
+
+    assert call(kernel=7) == _lib.PA_ERR_INVALID_ARG
+    # keys on M: G = 4, so at most 8 new tokens per sequence; head_dim 128
+    assert call(kernel=_lib.PA_PREFILL_KEYS) == _lib.PA_ERR_UNSUPPORTED
+    assert b"keys-on-M" in lib.pa_last_error()
+    assert call(kernel=_lib.PA_PREFILL_KEYS, max_q_len=8,
+                head_dim=64) == _lib.PA_ERR_UNSUPPORTED
+    # a valid choice gets as far as the workspace check
+    assert call(kernel=_lib.PA_PREFILL_KEYS,
+                max_q_len=8) == _lib.PA_ERR_WORKSPACE
+    assert call(kernel=_lib.PA_PREFILL_TILE) == _lib.PA_ERR_WORKSPACE

@@ -12,7 +12,7 @@ from helpers import check_decode, poison_unwritten, to_np
 pytestmark = pytest.mark.gpu
 
 
-def _run(pkv, pin, tables=None, err=None):
+def _run(pkv, pin, tables=None, err=None, kernel="auto"):
     inp = pin.paged
     w = inp.workload
     out = torch.full_like(pin.q, float("nan"))
@@ -22,7 +22,8 @@ def _run(pkv, pin, tables=None, err=None):
     qs = torch.from_numpy(pin.query_start).cuda()
     pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl, qs,
                    w.softmax_scale, max_q_len=int(max(pin.q_lens.max(), 1)),
-                   max_context_len=int(inp.lengths.max()), dev_err=err)
+                   max_context_len=int(inp.lengths.max()), dev_err=err,
+                   kernel=kernel)
     torch.cuda.synchronize()
     return out
 
@@ -257,3 +258,114 @@ def test_more_sequences_than_order_threads(pkv):
                    int(np.argmin(lens)), *rng.integers(0, 1300, 25).tolist()})
     seqs = [b for b in seqs if q_lens[b] > 0]
     _check(pin, out, "1300 sequences", seqs=seqs)
+
+
+# ---------------------------------------------------------------------------
+# The keys-on-M kernel (S^T = K Q^T, O^T += V^T P^T; q_len * G <= 32)
+
+
+@pytest.mark.parametrize("dtype", ["bfloat16", "float16"])
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (32, 8), (64, 8)])
+@pytest.mark.parametrize("bs", [16, 32])
+def test_keys_kernel_mixed(pkv, dtype, hq, hkv, bs):
+    """Contexts around the 128-key tile edges, 0 .. 32/G new tokens each;
+    both kernels against the oracle."""
+    qmax = 32 // (hq // hkv)
+    lens = (1, 17, 130, 300, 520, 64, 700, 33, 129, 128, 255, 256)
+    want = (1, qmax, 2, qmax, 1, 3, qmax, 0, qmax, 1, 2, qmax)
+    qlens = tuple(min(L, q) for L, q in zip(lens, want))
+    w = wl.Workload("prefill_keys", 21, len(lens), hq, hkv, 128, bs, dtype,
+                    "fixed", fixed_lengths=lens)
+    pin = wl.make_prefill(w, qlens, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for kernel in ("keys", "tile"):
+        out = _run(pkv, pin, err=err, kernel=kernel)
+        assert err.item() == 0
+        _check(pin, out, f"{kernel} {dtype}/{hq}:{hkv}/bs{bs}")
+
+
+def test_keys_kernel_many_units(pkv):
+    """1300 sequences x 2 KV heads = 2600 units over one persistent CTA per
+    SM (each CTA serves many units back to back), 0 .. 4 new tokens each."""
+    w = wl.Workload("many_keys", 33, 1300, 16, 2, 128, 16, "bfloat16",
+                    "uniform", low=1, high=400)
+    lens = wl.make_paged(w, values=False).lengths
+    q_lens = np.minimum(lens, np.random.default_rng(5).integers(0, 5, 1300))
+    pin = wl.make_prefill(w, q_lens, device="cuda")
+    out = _run(pkv, pin, kernel="keys")
+    assert not torch.isnan(out).any()
+    rng = np.random.default_rng(6)
+    seqs = sorted({0, 1, 147, 148, 1299, int(np.argmax(lens)),
+                   *rng.integers(0, 1300, 30).tolist()})
+    _check(pin, out, "keys, 1300 sequences",
+           seqs=[b for b in seqs if q_lens[b] > 0])
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+def test_keys_kernel_unwritten_slots_hold_nan(pkv, bs):
+    lens = (1, 15, 17, 100, 333, 1000, 128, 129)
+    w = wl.Workload("keys_nan", 22, len(lens), 32, 8, 128, bs, "bfloat16",
+                    "fixed", fixed_lengths=lens)
+    pin = wl.make_prefill(w, (1, 8, 5, 8, 3, 8, 8, 2), device="cuda")
+    _check(pin, _run(pkv, pin, kernel="keys"), "clean pool")
+    poison_unwritten(pin.paged)
+    _check(pin, _run(pkv, pin, kernel="keys"), "poisoned pool")
+
+
+def test_keys_kernel_bad_block_id_is_flagged(pkv):
+    w = wl.Workload("keysbad", 23, 3, 32, 8, 128, 16, "bfloat16", "fixed",
+                    fixed_lengths=(300, 300, 300))
+    pin = wl.make_prefill(w, (4, 4, 4), device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tables = pin.paged.block_tables.copy()
+    tables[1, 5] = pin.paged.num_blocks + 3
+    out = _run(pkv, pin, tables=tables, err=err, kernel="keys")
+    assert err.item() == 5
+    _check(pin, out, "other sequences intact", seqs=[0, 2])
+
+
+def test_speculative_verify_full_size_sampled(pkv):
+    """4 draft tokens for each of the 256 sequences of the batch-256 decode
+    mix (the bench's verification workload); sampled sequences against the
+    oracle, over each sequence's own blocks."""
+    w = wl.WORKLOADS["llama3_70b_gqa8"]
+    pin = wl.make_prefill(w, np.full(w.num_seqs, 4), device="cuda")
+    out = _run(pkv, pin)
+    inp = pin.paged
+    lens = inp.lengths
+    for b in (0, int(np.argmax(lens)), int(np.argmin(lens)), 100, 255):
+        L = int(lens[b])
+        need = (L + w.block_size - 1) // w.block_size
+        ids = torch.from_numpy(
+            inp.block_tables[b, :need].astype(np.int64)).cuda()
+        kc = to_np(inp.k_cache.index_select(0, ids))
+        vc = to_np(inp.v_cache.index_select(0, ids))
+        rows = np.arange(pin.query_start[b], pin.query_start[b + 1])
+        sub = np.arange(need, dtype=np.int32)[None, :]
+        ref = oa.paged_prefill(to_np(pin.q)[rows], kc, vc, sub,
+                               np.array([L]), np.array([0, len(rows)],
+                                                       dtype=np.int32),
+                               w.softmax_scale)
+        check_decode(to_np(out)[rows], ref, pin.q.dtype, f"verify seq {b}")
+
+
+def test_keys_kernel_long_context(pkv):
+    """4 new tokens at the end of 90k- and 70k-token contexts: few units, so
+    most CTAs idle and each busy one streams ~700 tiles."""
+    w = wl.Workload("long_keys", 16, 2, 64, 8, 128, 32, "float16", "fixed",
+                    fixed_lengths=(90_000, 70_001))
+    pin = wl.make_prefill(w, (4, 3), device="cuda")
+    out = _run(pkv, pin, kernel="keys")
+    inp = pin.paged
+    for b in (0, 1):
+        L, n = int(inp.lengths[b]), int(pin.q_lens[b])
+        need = (L + w.block_size - 1) // w.block_size
+        ids = torch.from_numpy(
+            inp.block_tables[b, :need].astype(np.int64)).cuda()
+        kc = to_np(inp.k_cache.index_select(0, ids))
+        vc = to_np(inp.v_cache.index_select(0, ids))
+        rows = pin.query_start[b] + np.arange(n)
+        sub = np.repeat(np.arange(need, dtype=np.int32)[None, :], n, axis=0)
+        ref = oa.paged_decode(to_np(pin.q)[rows], kc, vc, sub,
+                              L - n + np.arange(n) + 1, w.softmax_scale)
+        check_decode(to_np(out)[rows], ref, pin.q.dtype, f"long seq {b}")
