@@ -378,6 +378,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   // Padding rows (no query) see every key the tile loads; never stored.
   const int qpos = valid ? L - q_len + tok : kv_end - 1;
   const float c = a.scale_log2;
+  // A warp whose 32 rows are all padding (few new tokens: 4 drafts x 8 heads
+  // fill one warp's rows of 128) computes nothing: it keeps the barrier
+  // protocol and its share of the V clearing only.  Its rows of P hold stale
+  // values, which reach only its own (never stored) rows of O.
+  const bool idle = quarter * 32 >= n_q * G;
   float m_ref = -INFINITY, l = 0.f;
   bool ok = true;
   // Wait results are made warp-uniform: the tcgen05 loads and stores below
@@ -390,17 +395,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     ok = __all_sync(0xffffffffu,
                     dev::mbar_wait(s_full0 + 8 * (j & 1), (j >> 1) & 1));
     if (!ok) break;
-    dev::tc_fence_after();
     float sv[kKeys];
-    {
+    if (!idle) {
+      dev::tc_fence_after();
       const uint32_t sa = s_tmem + (j & 1) * kKeys + lane_off;
       float (&lo)[32] = *reinterpret_cast<float(*)[32]>(sv);
       float (&hi)[32] = *reinterpret_cast<float(*)[32]>(sv + 32);
       dev::tmem_ld32(sa, lo);
       dev::tmem_ld32(sa + 32, hi);
       dev::tmem_ld_wait();
+      dev::tc_fence_before();
     }
-    dev::tc_fence_before();
     __syncwarp();
     if (lane == 0) dev::mbar_arrive(s_free0 + 8 * (j & 1));
     const int k0 = j * kKeys;
@@ -422,6 +427,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                                 (ch & 7) * 16);
       }
       dev::fence_proxy_async_smem();  // visible to the tensor cores' P.V
+    }
+    if (idle) {
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(p_full0 + 8 * (j & 1));
+      continue;
     }
     // Causal mask: only tiles that reach past this row's position.
     const int lim = qpos - k0;
@@ -496,8 +506,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) dev::mbar_arrive(p_full0 + 8 * (j & 1));
   }
   // Epilogue: O / l -> out[token, query head].
-  if (ok) ok = wait_pv(n_tiles - 1);
-  if (ok) {
+  if (ok && !idle) ok = wait_pv(n_tiles - 1);
+  if (ok && !idle) {
     dev::tc_fence_after();
     const float inv = l > 0.f ? 1.f / l : 0.f;
     T* dst = static_cast<T*>(a.out) +
@@ -520,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
     }
-  } else {
+  } else if (!ok) {
     dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
   }
   dev::tc_fence_before();
