@@ -104,6 +104,9 @@ typedef struct {
   int max_context_len;
   pa_kernel kernel;
   pa_reduce reduce;
+  int out_fp32;  /* 0: out has q's dtype (rounded once).  1: out is float32,
+                    the value before that rounding (a check of the kernel's
+                    own error apart from the output rounding). */
 } pa_decode_desc;
 
 /* Library version string, and the text of a status code. */
@@ -126,6 +129,7 @@ const char* pa_last_error(void);
  *
  * Layouts (all dense, row-major):
  *   out, q        [num_seqs, num_q_heads, head_dim]          dtype
+ *                 (out float32 when desc->out_fp32 = 1)
  *   k_cache,
  *   v_cache       [num_blocks, num_kv_heads, block_size, head_dim]  dtype
  *   block_tables  [num_seqs, max_blocks_per_seq] int32 physical block ids;
@@ -209,7 +213,8 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,
  *     out[query_start[b] + i, h, :] = softmax(scale * K_b[0..p] q) V_b[0..p]
  * with query head h reading KV head h / G.  q_len = 1 is decode; q_len = L a
  * whole prompt.
- * Layouts: q, out [total_q, num_q_heads, head_dim] dtype; query_start [num_seqs+1]
+ * Layouts: q, out [total_q, num_q_heads, head_dim] dtype (out float32 with
+ * desc->out_fp32); query_start [num_seqs+1]
  * int32 on the device, non-decreasing, query_start[0] = 0 and
  * query_start[num_seqs] <= total_q; the rest as for pa_decode.
  * Supported: head_dim 64 or 128, block_size 16 or 32, G = 1, 2, 4 or 8 (else
@@ -254,6 +259,7 @@ typedef struct {
   int max_q_len;        /* host bound on any sequence's new-token count */
   int max_context_len;  /* host bound on context_lens[] (0: table capacity) */
   int kernel;           /* pa_prefill_kernel (0: automatic) */
+  int out_fp32;         /* as in pa_decode_desc: 1 = out is float32 */
 } pa_prefill_desc;
 
 /* Bytes of device workspace pa_prefill needs for this shape (the sequence

@@ -9,6 +9,7 @@ if the library is missing, every call raises.
 
 Layouts (see include/pagedkv.h for the full contract):
   q, out            [num_seqs, num_q_heads, head_dim]            fp16 / bf16
+                    (out may be float32: the value before the final rounding)
   k_cache, v_cache  [num_blocks, num_kv_heads, block_size, head_dim]
   block_tables      [num_seqs, max_blocks_per_seq] int32
   context_lens      [num_seqs] int32
@@ -123,6 +124,19 @@ def make_desc(q, k_cache, block_tables, *, partition_size: int = 0,
         reduce=_REDUCES[reduce])
 
 
+def _out_mode(desc, out, dt):
+    """``out`` in q's dtype, or float32: the value before the final rounding
+    (desc.out_fp32 follows the tensor)."""
+    import torch
+    if out.dtype == dt:
+        desc.out_fp32 = 0
+    elif out.dtype == torch.float32:
+        desc.out_fp32 = 1
+    else:
+        raise TypeError(f"out dtype {out.dtype} is neither q's dtype {dt} "
+                        "nor float32")
+
+
 def pa_decode_workspace_bytes(desc: pa_decode_desc) -> int:
     return int(_lib.load().pa_decode_workspace_bytes(ctypes.byref(desc)))
 
@@ -150,9 +164,10 @@ def pa_decode(out, q, k_cache, v_cache, block_tables, context_lens,
                          max_context_len=max_context_len, kernel=kernel,
                          reduce=reduce)
     dt = q.dtype
-    for name, t in (("out", out), ("k_cache", k_cache), ("v_cache", v_cache)):
+    for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
         if t.dtype != dt:
             raise TypeError(f"{name} dtype {t.dtype} != q dtype {dt}")
+    _out_mode(desc, out, dt)
     need = int(lib.pa_decode_workspace_bytes(ctypes.byref(desc)))
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -187,9 +202,10 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens,
                          partition_size=partition_size,
                          max_context_len=max_context_len, kernel=kernel,
                          reduce=reduce)
-    for name, t in (("out", out), ("k_cache", k_cache), ("v_cache", v_cache)):
+    for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
         if t.dtype != q.dtype:
             raise TypeError(f"{name} dtype {t.dtype} != q dtype {q.dtype}")
+    _out_mode(desc, out, q.dtype)
     st = lib.pa_decode_noalloc(
         _dev(out, "out"), _dev(q, "q"), _dev(k_cache, "k_cache"),
         _dev(v_cache, "v_cache"),
@@ -219,7 +235,7 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens,
     num_blocks, num_kv_heads, block_size, hd2 = k_cache.shape
     if hd2 != head_dim or out.shape != q.shape:
         raise ValueError("q, out and the caches disagree on shape")
-    for name, t in (("out", out), ("k_cache", k_cache), ("v_cache", v_cache)):
+    for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
         if t.dtype != q.dtype:
             raise TypeError(f"{name} dtype {t.dtype} != q dtype {q.dtype}")
     desc = _lib.pa_prefill_desc(
@@ -228,6 +244,7 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens,
         max_blocks_per_seq=block_tables.shape[1], num_blocks=num_blocks,
         dtype=_dtype_code(q), total_q=total_q, max_q_len=max_q_len,
         max_context_len=max_context_len, kernel=_PREFILL_KERNELS[kernel])
+    _out_mode(desc, out, q.dtype)
     need = lib.pa_prefill_workspace_bytes(ctypes.byref(desc))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8,

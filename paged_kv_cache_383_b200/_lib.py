@@ -53,6 +53,7 @@ class pa_decode_desc(ctypes.Structure):
         ("max_context_len", ctypes.c_int),
         ("kernel", ctypes.c_int),
         ("reduce", ctypes.c_int),
+        ("out_fp32", ctypes.c_int),
     ]
 
 
@@ -70,6 +71,7 @@ class pa_prefill_desc(ctypes.Structure):
         ("max_q_len", ctypes.c_int),
         ("max_context_len", ctypes.c_int),
         ("kernel", ctypes.c_int),
+        ("out_fp32", ctypes.c_int),
     ]
 
 

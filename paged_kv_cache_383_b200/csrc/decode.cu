@@ -97,6 +97,7 @@ struct DecodeArgs {
   int partition_size;
   int max_parts;
   int max_context_len;
+  int out_f32;   // 1: out is float32 (the value before the cast to T)
 };
 
 // Shared-memory geometry of one (block_size, head_dim, stages) instance.
@@ -182,6 +183,18 @@ __device__ __forceinline__ float warp_max_xor(float v, int lo_mask,
   return v;
 }
 
+// Final store of one output element: rounded once to the output dtype, or,
+// on request, the fp32 value itself (lets tests separate the kernel's error
+// from the output rounding).
+template <typename T>
+__device__ __forceinline__ void store_out(const DecodeArgs& a, int64_t idx,
+                                          float v) {
+  if (a.out_f32)
+    static_cast<float*>(a.out)[idx] = v;
+  else
+    static_cast<T*>(a.out)[idx] = from_float<T>(v);
+}
+
 // ---------------------------------------------------------------------------
 // Fused combine of one (sequence, KV head)'s partitions, run by threads
 // [t, ...) step nt of the partition CTA that finished last:
@@ -240,11 +253,11 @@ __device__ __forceinline__ void combine_partials(const DecodeArgs& a, int b,
         for (int e = 0; e < kDT; ++e) acc[e] += w * oj[u][e];
       }
     }
-    T* dst = static_cast<T*>(a.out) +
-             (static_cast<int64_t>(b) * a.num_q_heads + kvh * G + g) * D + d0;
+    const int64_t dst =
+        (static_cast<int64_t>(b) * a.num_q_heads + kvh * G + g) * D + d0;
 #pragma unroll
     for (int e = 0; e < kDT; ++e)
-      dst[e] = from_float<T>(W > 0.f ? acc[e] / W : 0.f);
+      store_out<T>(a, dst + e, W > 0.f ? acc[e] / W : 0.f);
   }
 }
 
@@ -564,9 +577,8 @@ __global__ void __launch_bounds__(kThreads)
               const int g = 2 * t4 + (e & 1);
               if (g < G) {
                 const float l = lt[e & 1];
-                static_cast<T*>(a.out)[(row0 + g) * D + dt * 16 + g4 +
-                                       (e >> 1) * 8] =
-                    from_float<T>(l > 0.f ? o[dt][e] / l : 0.f);
+                store_out<T>(a, (row0 + g) * D + dt * 16 + g4 + (e >> 1) * 8,
+                             l > 0.f ? o[dt][e] / l : 0.f);
               }
             }
           return;
@@ -791,8 +803,8 @@ __global__ void __launch_bounds__(kThreads)
     }
     const int qh = kvh * G + g;
     if (!split) {
-      static_cast<T*>(a.out)[(static_cast<int64_t>(b) * a.num_q_heads + qh) * D +
-                             d] = from_float<T>(val);
+      store_out<T>(a, (static_cast<int64_t>(b) * a.num_q_heads + qh) * D + d,
+                   val);
     } else {
       const int64_t row =
           (static_cast<int64_t>(b) * a.num_q_heads + qh) * a.max_parts + part;
@@ -929,8 +941,8 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
         tv += s_acc[w][d] * sc;
       }
     }
-    static_cast<T*>(a.out)[(static_cast<int64_t>(b) * a.num_q_heads + qh) *
-                               D + d] = from_float<T>(tw > 0.f ? tv / tw : 0.f);
+    store_out<T>(a, (static_cast<int64_t>(b) * a.num_q_heads + qh) * D + d,
+                 tw > 0.f ? tv / tw : 0.f);
   }
 }
 
@@ -1047,6 +1059,8 @@ pa_status check_desc(const pa_decode_desc* d) {
   if (d->reduce != PA_REDUCE_AUTO && d->reduce != PA_REDUCE_KERNEL)
     return fail(PA_ERR_INVALID_ARG, "pa_decode: reduce %d",
                 static_cast<int>(d->reduce));
+  if (d->out_fp32 != 0 && d->out_fp32 != 1)
+    return fail(PA_ERR_INVALID_ARG, "pa_decode: out_fp32 %d", d->out_fp32);
   if (d->kernel != PA_KERNEL_AUTO && d->kernel != PA_KERNEL_SIMT &&
       d->kernel != PA_KERNEL_MMA)
     return fail(PA_ERR_INVALID_ARG, "pa_decode: kernel %d",
@@ -1335,6 +1349,7 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache,
   a.partition_size = ps;
   a.max_parts = parts;
   a.max_context_len = max_ctx;
+  a.out_f32 = desc->out_fp32;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool mma = desc->kernel != PA_KERNEL_SIMT;

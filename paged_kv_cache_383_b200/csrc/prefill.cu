@@ -85,6 +85,7 @@ struct PrefillArgs {
   int num_blocks;
   int max_context_len;
   int total_q;
+  int out_f32;  // 1: out is float32 (the value before the cast to T)
 };
 
 // barriers: q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
@@ -510,15 +511,22 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (ok && !idle) {
     dev::tc_fence_after();
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    T* dst = static_cast<T*>(a.out) +
-             (static_cast<int64_t>(q0 + tok) * a.num_q_heads + kvh * G + g) *
-                 D;
+    const int64_t idx =
+        (static_cast<int64_t>(q0 + tok) * a.num_q_heads + kvh * G + g) * D;
+    T* dst = static_cast<T*>(a.out) + idx;
+    float* dst32 = static_cast<float*>(a.out) + idx;  // out_f32 only
 #pragma unroll
     for (int col = 0; col < D; col += 32) {
       float ov[32];
       dev::tmem_ld32(o_tmem + lane_off + col, ov);
       dev::tmem_ld_wait();
-      if (valid) {
+      if (valid && a.out_f32) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(dst32 + col + e) =
+              make_float4(ov[e] * inv, ov[e + 1] * inv, ov[e + 2] * inv,
+                          ov[e + 3] * inv);
+      } else if (valid) {
 #pragma unroll
         for (int e = 0; e < 32; e += 8) {
           uint4 w;
@@ -1084,22 +1092,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     dev::tc_fence_before();
     __syncwarp();
     if (lane == 0) dev::mbar_arrive(o_free0 + 8 * ob);
-    T* out = static_cast<T*>(a.out);
 #pragma unroll
     for (int r = 0; r < N; r += 2) {
       const uint32_t w = M::pack(ov[r] * inv[r], ov[r + 1] * inv[r + 1]);
-      if (r < R) {
-        const int64_t row = static_cast<int64_t>(v.q0 + r / G) * a.num_q_heads +
-                            v.kvh * G + r % G;
-        reinterpret_cast<uint16_t*>(out)[row * 128 + kl] =
-            static_cast<uint16_t>(w & 0xffffu);
-      }
-      if (r + 1 < R) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (r + h >= R) continue;
         const int64_t row =
-            static_cast<int64_t>(v.q0 + (r + 1) / G) * a.num_q_heads +
-            v.kvh * G + (r + 1) % G;
-        reinterpret_cast<uint16_t*>(out)[row * 128 + kl] =
-            static_cast<uint16_t>(w >> 16);
+            static_cast<int64_t>(v.q0 + (r + h) / G) * a.num_q_heads +
+            v.kvh * G + (r + h) % G;
+        if (a.out_f32)
+          static_cast<float*>(a.out)[row * 128 + kl] = ov[r + h] * inv[r + h];
+        else
+          static_cast<uint16_t*>(a.out)[row * 128 + kl] =
+              static_cast<uint16_t>(h ? w >> 16 : w & 0xffffu);
       }
     }
     g += v.n_tiles;
@@ -1319,6 +1325,8 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
   const int G = d->num_q_heads / d->num_kv_heads;
   if (d->kernel < PA_PREFILL_AUTO || d->kernel > PA_PREFILL_KEYS)
     return fail(PA_ERR_INVALID_ARG, "pa_prefill: kernel %d", d->kernel);
+  if (d->out_fp32 != 0 && d->out_fp32 != 1)
+    return fail(PA_ERR_INVALID_ARG, "pa_prefill: out_fp32 %d", d->out_fp32);
   const bool keys_fit =
       d->head_dim == 128 &&
       static_cast<int64_t>(d->max_q_len) * G <= pagedkv::kVerRows &&
@@ -1391,6 +1399,7 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
   a.num_blocks = d->num_blocks;
   a.max_context_len = max_ctx;
   a.total_q = d->total_q;
+  a.out_f32 = d->out_fp32;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   pagedkv::prefill_order_kernel<<<1, pagedkv::kOrderThreads, 0, s>>>(
       context_lens, d->num_seqs, pagedkv::order_shift(max_ctx),

@@ -107,3 +107,19 @@ def poison_unwritten(inp) -> None:
     free = torch.from_numpy(np.flatnonzero(~used)).to(inp.k_cache.device)
     inp.k_cache[free] = float("nan")
     inp.v_cache[free] = float("nan")
+
+
+def check_strict(out32, ref, what=""):
+    """The tolerance with no carve-out, for float32 outputs (the kernel's
+    value before the final rounding): every element within 2e-3 absolute,
+    every element with |ref| >= 0.2 within 1e-2 relative."""
+    out32 = np.asarray(out32, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert out32.shape == ref.shape
+    assert np.isfinite(out32).all(), f"{what}: non-finite output"
+    err = np.abs(out32 - ref)
+    big = np.abs(ref) >= REL_FLOOR
+    rel = np.where(big, err / np.maximum(np.abs(ref), 1e-30), 0.0)
+    assert err.max() <= ATOL, f"{what}: max abs err {err.max():.3e}"
+    assert rel.max() <= RTOL, f"{what}: max rel err {rel.max():.3e}"
+    return float(err.max()), float(rel.max())
