@@ -187,3 +187,22 @@ def test_prefill_kernel_choice_is_checked(pkv):
     assert call(kernel=_lib.PA_PREFILL_KEYS,
                 max_q_len=8) == _lib.PA_ERR_WORKSPACE
     assert call(kernel=_lib.PA_PREFILL_TILE) == _lib.PA_ERR_WORKSPACE
+
+
+def test_out_fp32_flag_is_checked(pkv):
+    from paged_kv_cache_383_b200 import _lib
+    lib = _lib.load()
+    fake = 0x1000
+    d = _desc(out_fp32=2)
+    assert lib.pa_decode(fake, fake, fake, fake, fake, fake,
+                         ctypes.c_float(1.0), ctypes.byref(d), None, 0, None,
+                         None) == _lib.PA_ERR_INVALID_ARG
+    assert b"out_fp32" in lib.pa_last_error()
+    p = _lib.pa_prefill_desc(num_seqs=2, num_q_heads=8, num_kv_heads=2,
+                             head_dim=128, block_size=16,
+                             max_blocks_per_seq=4, num_blocks=16, dtype=1,
+                             total_q=8, max_q_len=4, max_context_len=64,
+                             out_fp32=3)
+    assert lib.pa_prefill(*([fake] * 7), ctypes.c_float(1.0),
+                          ctypes.byref(p), None, 0, None,
+                          None) == _lib.PA_ERR_INVALID_ARG
