@@ -71,6 +71,58 @@ constexpr int kThreads = 192;   // producer, MMA, 4 softmax warps
 constexpr int kTmemCols = 256;  // S/P: cols [0, 128), O: cols [128, 128 + D)
 constexpr float kRescaleLog2 = 8.f;
 
+// Tensor-memory access shapes with four threads per lane, used when at most
+// 32 query rows are real.  16x256b: thread t gets lanes t/4 and t/4 + 8 of
+// the 16 addressed, columns 2 (t % 4) and 2 (t % 4) + 1 of every 8 (the
+// layout of an m16n8 accumulator).  16x128b: the same lanes, column t % 4 of
+// every 4.
+__device__ __forceinline__ void tmem_ld16x256_x8(uint32_t taddr,
+                                                 float (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, "
+      "%7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, "
+      "%21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]),
+        "=f"(v[5]), "=f"(v[6]), "=f"(v[7]), "=f"(v[8]), "=f"(v[9]),
+        "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]),
+        "=f"(v[15]), "=f"(v[16]), "=f"(v[17]), "=f"(v[18]), "=f"(v[19]),
+        "=f"(v[20]), "=f"(v[21]), "=f"(v[22]), "=f"(v[23]), "=f"(v[24]),
+        "=f"(v[25]), "=f"(v[26]), "=f"(v[27]), "=f"(v[28]), "=f"(v[29]),
+        "=f"(v[30]), "=f"(v[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld16x256_x4(uint32_t taddr,
+                                                 float (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0, %1, %2, %3, %4, %5, %6, "
+      "%7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]),
+        "=f"(v[5]), "=f"(v[6]), "=f"(v[7]), "=f"(v[8]), "=f"(v[9]),
+        "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]),
+        "=f"(v[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16x256_x4(uint32_t taddr,
+                                                 const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%16], {%0, %1, %2, %3, %4, "
+      "%5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15};" ::"f"(v[0]),
+      "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+      "f"(v[7]), "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]),
+      "f"(v[13]), "f"(v[14]), "f"(v[15]), "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16x128_x8(uint32_t taddr,
+                                                 const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x8.b32 [%16], {%0, %1, %2, %3, %4, "
+      "%5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15};" ::"r"(v[0]),
+      "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+      "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]),
+      "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(taddr)
+      : "memory");
+}
+
 struct PrefillArgs {
   void* out;
   const int32_t* order;  // [num_seqs] sequence served by grid row z
@@ -111,7 +163,7 @@ struct Layout {
   static constexpr size_t kSmemBytes = 1024 + kOffBars + kNumBars * 8 + 16;
 };
 
-template <typename T, int BS, int G, int D>
+template <typename T, int BS, int G, int D, bool SQ>
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap,
                    const __grid_constant__ CUtensorMap kmap,
@@ -169,9 +221,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     return;
   }
   const int tok0 = qt * kTok;
-  if (qt == static_cast<int>(gridDim.y) - 1 && q_len > tok0 + kTok) {
-    // max_q_len was below this sequence's new-token count: the grid misses
-    // rows, which are left unwritten.
+  if ((qt == static_cast<int>(gridDim.y) - 1 && q_len > tok0 + kTok) ||
+      (SQ && q_len * G > 32)) {
+    // max_q_len was below this sequence's new-token count: the grid (or the
+    // few-row layout) misses rows, which are left unwritten.
     if (kvh == 0 && tid == 0) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
   }
   if (tok0 >= q_len) return;
@@ -234,11 +287,24 @@ __global__ void __launch_bounds__(kThreads, 2)
       dev::prefetch_tmap(&qmap);
       dev::prefetch_tmap(&kmap);
       dev::prefetch_tmap(&vmap);
-      dev::mbar_arrive_expect_tx(q_full, kQBytes);
+      if constexpr (SQ) {
+        // Few query rows: 8/G tokens of G heads (eight rows) into the first
+        // eight rows of each 32-row quarter; the rest of the tile is padding.
+        constexpr int kQTok = 8 / G;
+        dev::mbar_arrive_expect_tx(q_full, 4 * kHalves * 8 * 128);
 #pragma unroll
-      for (int h = 0; h < kHalves; ++h)
-        dev::tma_load_3d(q_s + h * kHalfQ, &qmap, 64 * h, kvh * G, q0 + tok0,
-                         q_full);
+        for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+          for (int h = 0; h < kHalves; ++h)
+            dev::tma_load_3d(q_s + h * kHalfQ + qq * 32 * 128, &qmap, 64 * h,
+                             kvh * G, q0 + tok0 + qq * kQTok, q_full);
+      } else {
+        dev::mbar_arrive_expect_tx(q_full, kQBytes);
+#pragma unroll
+        for (int h = 0; h < kHalves; ++h)
+          dev::tma_load_3d(q_s + h * kHalfQ, &qmap, 64 * h, kvh * G,
+                           q0 + tok0, q_full);
+      }
       // Block ids of a tile's pages; pages past the sequence are masked, so
       // they read the first page instead.
       const int32_t first = row[0];
@@ -365,6 +431,178 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncwarp();
     dev::tc_fence_after();
     dev::tmem_dealloc(tbase, kTmemCols);
+    return;
+  }
+
+  if constexpr (SQ) {
+    // ------------- softmax warps, few query rows (<= 32 real) -------------
+    // Query row r = i * G + h (token i, head h) sits in lane
+    // 32 * (r / 8) + r % 8: each warp owns eight rows, and four threads
+    // share a row, each taking 16 of a tile's 64 keys (the 16x256b shape).
+    // Lanes 8 .. 31 of every quarter are padding: never read back.
+    const int quarter = warp & 3;
+    const int c4 = lane & 3;                  // this thread's key pairs
+    const int rr = quarter * 8 + (lane >> 2);  // query row
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const int t_loc = rr / G;
+    const int hq = rr - t_loc * G;
+    const bool valid = t_loc < n_q;
+    const int qpos = valid ? L - q_len + tok0 + t_loc : kv_end - 1;
+    const bool idle = quarter * 8 >= n_q * G;  // no real row in this warp
+    const float c = a.scale_log2;
+    float m_ref = -INFINITY, l = 0.f;  // l: this thread's keys only
+    bool ok = true;
+    auto wait_pv = [&](int t) {
+      return __all_sync(0xffffffffu, dev::mbar_wait(o_ready0 + 8 * (t & 1),
+                                                    (t >> 1) & 1));
+    };
+    for (int j = 0; j < n_tiles && ok; ++j) {
+      ok = __all_sync(0xffffffffu,
+                      dev::mbar_wait(s_full0 + 8 * (j & 1), (j >> 1) & 1));
+      if (!ok) break;
+      float sa[32];
+      if (!idle) {
+        dev::tc_fence_after();
+        tmem_ld16x256_x8(s_tmem + (j & 1) * kKeys + lane_off, sa);
+        dev::tmem_ld_wait();
+        dev::tc_fence_before();
+      }
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(s_free0 + 8 * (j & 1));
+      const int k0 = j * kKeys;
+      if (k0 + kKeys > L) {
+        // As below: clear the V rows past the context in the last tile.
+        ok = __all_sync(0xffffffffu,
+                        dev::mbar_wait(v_full0 + 8 * (j % kVStages),
+                                       (j / kVStages) & 1));
+        if (!ok) break;
+        const uint32_t vt = vring + (j % kVStages) * kKVTile;
+        for (int idx = lane; idx < 16 * 8 * kHalves; idx += 32) {
+          const int krow = quarter * 16 + idx / (8 * kHalves);
+          const int ch = idx % (8 * kHalves);
+          if (k0 + krow >= L)
+            dev::st_shared_zero16(vt + (ch >> 3) * kTileHalf + krow * 128 +
+                                  (ch & 7) * 16);
+        }
+        dev::fence_proxy_async_smem();
+      }
+      if (idle) {
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(p_full0 + 8 * (j & 1));
+        continue;
+      }
+      // sa[4k], sa[4k + 1]: this row, keys 8k + 2 c4 and 8k + 2 c4 + 1.
+      float sv[16];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        sv[2 * k] = sa[4 * k];
+        sv[2 * k + 1] = sa[4 * k + 1];
+      }
+      const int lim = qpos - k0;
+      if (lim < kKeys - 1) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+#pragma unroll
+          for (int e = 0; e < 2; ++e)
+            if (8 * k + 2 * c4 + e > lim) sv[2 * k + e] = -INFINITY;
+      }
+      float m4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) m4[u] = fmaxf(sv[u], sv[u + 4]);
+#pragma unroll
+      for (int k = 8; k < 16; ++k) m4[k & 3] = fmaxf(m4[k & 3], sv[k]);
+      float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      mx *= c;
+      float factor = 1.f;
+      if (j == 0) {
+        m_ref = mx;
+      } else if (mx > m_ref + kRescaleLog2) {
+        factor = dev::fast_exp2(m_ref - mx);
+        m_ref = mx;
+        l *= factor;
+      }
+      {
+        float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          sv[k] = dev::fast_exp2(fmaf(sv[k], c, -m_ref));
+          l4[k & 3] += sv[k];
+        }
+        l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+      }
+      if (__any_sync(0xffffffffu, factor != 1.f)) {
+        ok = wait_pv(j - 1);
+        if (!ok) break;
+        dev::tc_fence_after();
+#pragma unroll
+        for (int col = 0; col < D; col += 32) {
+          float ov[16];
+          tmem_ld16x256_x4(o_tmem + lane_off + col, ov);
+          dev::tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) ov[e] *= factor;
+          tmem_st16x256_x4(o_tmem + lane_off + col, ov);
+        }
+        dev::tmem_st_wait();
+      }
+      // P over S(j): column 4k + c4 of each half holds keys 8k + 2 c4 and
+      // 8k + 2 c4 + 1; the padding lane (t/4 + 8) gets zeros.
+      {
+        uint32_t hw[16], lw[16];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t w = M::pack(sv[2 * k], sv[2 * k + 1]);
+          const float2 hf = M::unpack(w);
+          hw[2 * k] = w;
+          hw[2 * k + 1] = 0u;
+          lw[2 * k] = M::pack(sv[2 * k] - hf.x, sv[2 * k + 1] - hf.y);
+          lw[2 * k + 1] = 0u;
+        }
+        const uint32_t pa = s_tmem + (j & 1) * kKeys + lane_off;
+        tmem_st16x128_x8(pa, hw);
+        tmem_st16x128_x8(pa + kKeys / 2, lw);
+        dev::tmem_st_wait();
+      }
+      dev::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(p_full0 + 8 * (j & 1));
+    }
+    // Epilogue: the row sum over the four threads, O / l -> out.
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    if (ok && !idle) ok = wait_pv(n_tiles - 1);
+    if (ok && !idle) {
+      dev::tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const int64_t idx =
+          (static_cast<int64_t>(q0 + tok0 + t_loc) * a.num_q_heads + kvh * G +
+           hq) * D + 2 * c4;
+#pragma unroll
+      for (int col = 0; col < D; col += 32) {
+        float ov[16];
+        tmem_ld16x256_x4(o_tmem + lane_off + col, ov);
+        dev::tmem_ld_wait();
+        if (valid) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int64_t e = idx + col + 8 * k;  // dims e, e + 1
+            if (a.out_f32)
+              *reinterpret_cast<float2*>(static_cast<float*>(a.out) + e) =
+                  make_float2(ov[4 * k] * inv, ov[4 * k + 1] * inv);
+            else
+              *reinterpret_cast<uint32_t*>(static_cast<T*>(a.out) + e) =
+                  M::pack(ov[4 * k] * inv, ov[4 * k + 1] * inv);
+          }
+        }
+      }
+    } else if (!ok) {
+      dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
+    }
+    dev::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) dev::mbar_arrive(done);
     return;
   }
 
@@ -1187,11 +1425,11 @@ size_t prefill_workspace_bytes(const pa_prefill_desc* d) {
          ~size_t(15);
 }
 
-template <typename T, int BS, int G, int D>
+template <typename T, int BS, int G, int D, bool SQ>
 pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
                  const CUtensorMap& qm, const CUtensorMap& km,
                  const CUtensorMap& vm, cudaStream_t st) {
-  auto kern = prefill_kernel<T, BS, G, D>;
+  auto kern = prefill_kernel<T, BS, G, D, SQ>;
   const size_t smem = Layout<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1220,28 +1458,29 @@ pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
   return PA_OK;
 }
 
-template <typename T, int BS, int D>
+template <typename T, int BS, int D, bool SQ>
 pa_status dispatch_group(const pa_prefill_desc* d, const PrefillArgs& a,
                          const CUtensorMap& qm, const CUtensorMap& km,
                          const CUtensorMap& vm, cudaStream_t st) {
   switch (d->num_q_heads / d->num_kv_heads) {
-    case 1: return launch<T, BS, 1, D>(d, a, qm, km, vm, st);
-    case 2: return launch<T, BS, 2, D>(d, a, qm, km, vm, st);
-    case 4: return launch<T, BS, 4, D>(d, a, qm, km, vm, st);
-    default: return launch<T, BS, 8, D>(d, a, qm, km, vm, st);
+    case 1: return launch<T, BS, 1, D, SQ>(d, a, qm, km, vm, st);
+    case 2: return launch<T, BS, 2, D, SQ>(d, a, qm, km, vm, st);
+    case 4: return launch<T, BS, 4, D, SQ>(d, a, qm, km, vm, st);
+    default: return launch<T, BS, 8, D, SQ>(d, a, qm, km, vm, st);
   }
 }
 
-template <typename T>
+template <typename T, bool SQ>
 pa_status dispatch_shape(const pa_prefill_desc* d, const PrefillArgs& a,
                          const CUtensorMap& qm, const CUtensorMap& km,
                          const CUtensorMap& vm, cudaStream_t st) {
   if (d->head_dim == 128)
     return d->block_size == 16
-               ? dispatch_group<T, 16, 128>(d, a, qm, km, vm, st)
-               : dispatch_group<T, 32, 128>(d, a, qm, km, vm, st);
-  return d->block_size == 16 ? dispatch_group<T, 16, 64>(d, a, qm, km, vm, st)
-                             : dispatch_group<T, 32, 64>(d, a, qm, km, vm, st);
+               ? dispatch_group<T, 16, 128, SQ>(d, a, qm, km, vm, st)
+               : dispatch_group<T, 32, 128, SQ>(d, a, qm, km, vm, st);
+  return d->block_size == 16
+             ? dispatch_group<T, 16, 64, SQ>(d, a, qm, km, vm, st)
+             : dispatch_group<T, 32, 64, SQ>(d, a, qm, km, vm, st);
 }
 
 template <typename T, int BS, int G>
@@ -1374,7 +1613,12 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
   const int max_ctx = d->max_context_len > 0
                           ? d->max_context_len
                           : d->max_blocks_per_seq * d->block_size;
-  const int tok = use_keys ? pagedkv::kVerRows / G : pagedkv::kRows / G;
+  // At most 32 query rows per KV head (a few new tokens): the tile kernel
+  // spreads them over the four softmax warps, eight rows each.
+  const bool small_q = !use_keys && static_cast<int64_t>(d->max_q_len) * G <= 32;
+  const int tok = use_keys  ? pagedkv::kVerRows / G
+                  : small_q ? 8 / G
+                            : pagedkv::kRows / G;
   CUtensorMap qm, km, vm;
   const uint64_t rows = static_cast<uint64_t>(d->num_blocks) *
                         d->num_kv_heads * d->block_size;
@@ -1413,9 +1657,13 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
     return d->dtype == PA_BF16
                ? pagedkv::dispatch_verify<__nv_bfloat16>(d, a, qm, km, vm, s)
                : pagedkv::dispatch_verify<__half>(d, a, qm, km, vm, s);
-  if (d->dtype == PA_BF16)
-    return pagedkv::dispatch_shape<__nv_bfloat16>(d, a, qm, km, vm, s);
-  return pagedkv::dispatch_shape<__half>(d, a, qm, km, vm, s);
+  if (small_q)
+    return d->dtype == PA_BF16
+               ? pagedkv::dispatch_shape<__nv_bfloat16, true>(d, a, qm, km, vm, s)
+               : pagedkv::dispatch_shape<__half, true>(d, a, qm, km, vm, s);
+  return d->dtype == PA_BF16
+             ? pagedkv::dispatch_shape<__nv_bfloat16, false>(d, a, qm, km, vm, s)
+             : pagedkv::dispatch_shape<__half, false>(d, a, qm, km, vm, s);
 }
 
 extern "C" size_t pa_prefill_workspace_bytes(const pa_prefill_desc* d) {
