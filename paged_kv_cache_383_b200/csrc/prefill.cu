@@ -37,6 +37,11 @@
 //     grows by more than 2^8 (the final division uses the same reference,
 //     so the result is unchanged), and store P with tcgen05.st as a 16-bit
 //     rounded part plus its residual so P . V keeps ~16 mantissa bits.
+//   * With at most 32 query rows per KV head (a few new tokens), a
+//     compile-time variant spreads the rows over all four softmax warps,
+//     eight per lane quarter, and reads S / writes P / reads O with the
+//     16-lane tensor-memory shapes: four threads per row, 16 keys each.  A
+//     warp whose rows are all padding computes nothing.
 //   * Shared memory is ~99 KB (Q, the rings, barriers; block ids are read
 //     from global memory a tile ahead) and tensor memory 256 columns, so two
 //     CTAs share an SM at any context length: one CTA's softmax runs while
