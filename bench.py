@@ -603,6 +603,7 @@ def extras(args, w, inp, dev, pkv, bt, cl):
     out["prefix_cache"] = prefix_cache_measure(pkv, dev)
     out["swap"] = swap_measure(pkv, dev)
     out["spec_verify"] = spec_verify_measure(pkv, dev)
+    out["spec_verify_8"] = spec_verify_measure(pkv, dev, drafts=8)
     return out
 
 
@@ -932,8 +933,10 @@ def spec_verify_measure(pkv, dev, drafts=4):
         return a.elapsed_time(b) / 20
 
     ms = time_kernel("auto")
-    ms_keys = time_kernel("keys")
-    gbs = lambda t: round(kv_bytes(inp.lengths, w) / (t * 1e-3) / 1e9, 1)
+    keys_fit = drafts * (w.num_q_heads // w.num_kv_heads) <= 32
+    ms_keys = time_kernel("keys") if keys_fit else None
+    gbs = lambda t: round(kv_bytes(inp.lengths, w) / (t * 1e-3) / 1e9, 1) \
+        if t else None
     return {"seqs": w.num_seqs, "drafts": drafts,
             "kv_bytes": kv_bytes(inp.lengths, w), "ms": round(ms, 4),
             "kv_gbs": gbs(ms),
@@ -941,7 +944,7 @@ def spec_verify_measure(pkv, dev, drafts=4):
                                           w.num_q_heads, w.head_dim)
                             / (ms * 1e-3) / 1e12, 1),
             "kernel": "auto (the tile kernel)",
-            "ms_keys_kernel": round(ms_keys, 4),
+            "ms_keys_kernel": round(ms_keys, 4) if ms_keys else None,
             "kv_gbs_keys_kernel": gbs(ms_keys)}
 
 
@@ -965,6 +968,7 @@ def run_extras_only(args):
         res["swap"] = swap_measure(pkv, dev)
     if want("spec_verify"):
         res["spec_verify"] = spec_verify_measure(pkv, dev)
+        res["spec_verify_8"] = spec_verify_measure(pkv, dev, drafts=8)
     res["gpu_launches"] = pkv.pa_launch_count()
     return res
 

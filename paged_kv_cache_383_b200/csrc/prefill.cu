@@ -37,9 +37,9 @@
 //     grows by more than 2^8 (the final division uses the same reference,
 //     so the result is unchanged), and store P with tcgen05.st as a 16-bit
 //     rounded part plus its residual so P . V keeps ~16 mantissa bits.
-//   * With at most 32 query rows per KV head (a few new tokens), a
+//   * With at most 64 query rows per KV head (a few new tokens), a
 //     compile-time variant spreads the rows over all four softmax warps,
-//     eight per lane quarter, and reads S / writes P / reads O with the
+//     8 or 16 per lane quarter, and reads S / writes P / reads O with the
 //     16-lane tensor-memory shapes: four threads per row, 16 keys each.  A
 //     warp whose rows are all padding computes nothing.
 //   * Shared memory is ~99 KB (Q, the rings, barriers; block ids are read
@@ -168,7 +168,7 @@ struct Layout {
   static constexpr size_t kSmemBytes = 1024 + kOffBars + kNumBars * 8 + 16;
 };
 
-template <typename T, int BS, int G, int D, bool SQ>
+template <typename T, int BS, int G, int D, int RQ>
 __global__ void __launch_bounds__(kThreads, 2)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap,
                    const __grid_constant__ CUtensorMap kmap,
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   const int tok0 = qt * kTok;
   if ((qt == static_cast<int>(gridDim.y) - 1 && q_len > tok0 + kTok) ||
-      (SQ && q_len * G > 32)) {
+      (RQ > 0 && q_len * G > 4 * RQ)) {
     // max_q_len was below this sequence's new-token count: the grid (or the
     // few-row layout) misses rows, which are left unwritten.
     if (kvh == 0 && tid == 0) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
@@ -292,11 +292,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       dev::prefetch_tmap(&qmap);
       dev::prefetch_tmap(&kmap);
       dev::prefetch_tmap(&vmap);
-      if constexpr (SQ) {
-        // Few query rows: 8/G tokens of G heads (eight rows) into the first
-        // eight rows of each 32-row quarter; the rest of the tile is padding.
-        constexpr int kQTok = 8 / G;
-        dev::mbar_arrive_expect_tx(q_full, 4 * kHalves * 8 * 128);
+      if constexpr (RQ > 0) {
+        // Few query rows: RQ/G tokens of G heads (RQ rows) into the first RQ
+        // rows of each 32-row quarter; the rest of the tile is padding.
+        constexpr int kQTok = RQ / G;
+        dev::mbar_arrive_expect_tx(q_full, 4 * kHalves * RQ * 128);
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq)
 #pragma unroll
@@ -439,23 +439,36 @@ __global__ void __launch_bounds__(kThreads, 2)
     return;
   }
 
-  if constexpr (SQ) {
-    // ------------- softmax warps, few query rows (<= 32 real) -------------
+  if constexpr (RQ > 0) {
+    // ------ softmax warps, few query rows (<= 4 * RQ real, RQ per quarter) --
     // Query row r = i * G + h (token i, head h) sits in lane
-    // 32 * (r / 8) + r % 8: each warp owns eight rows, and four threads
-    // share a row, each taking 16 of a tile's 64 keys (the 16x256b shape).
-    // Lanes 8 .. 31 of every quarter are padding: never read back.
+    // 32 * (r / RQ) + r % RQ: each warp owns RQ rows, and four threads share
+    // a row, each taking 16 of a tile's 64 keys (the 16x256b shape gives a
+    // thread lanes t/4 and t/4 + 8: one row when RQ = 8, the other lane
+    // being padding, two rows when RQ = 16).  Lanes RQ .. 31 of every
+    // quarter are padding: never read back.
+    constexpr int kR = RQ / 8;  // rows per thread
     const int quarter = warp & 3;
-    const int c4 = lane & 3;                  // this thread's key pairs
-    const int rr = quarter * 8 + (lane >> 2);  // query row
+    const int c4 = lane & 3;  // this thread's key pairs
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const int t_loc = rr / G;
-    const int hq = rr - t_loc * G;
-    const bool valid = t_loc < n_q;
-    const int qpos = valid ? L - q_len + tok0 + t_loc : kv_end - 1;
-    const bool idle = quarter * 8 >= n_q * G;  // no real row in this warp
+    int t_loc[kR], hq[kR], qpos[kR];
+    bool valid[kR];
+#pragma unroll
+    for (int x = 0; x < kR; ++x) {
+      const int rr = quarter * RQ + (lane >> 2) + 8 * x;  // query row
+      t_loc[x] = rr / G;
+      hq[x] = rr - t_loc[x] * G;
+      valid[x] = t_loc[x] < n_q;
+      qpos[x] = valid[x] ? L - q_len + tok0 + t_loc[x] : kv_end - 1;
+    }
+    const bool idle = quarter * RQ >= n_q * G;  // no real row in this warp
     const float c = a.scale_log2;
-    float m_ref = -INFINITY, l = 0.f;  // l: this thread's keys only
+    float m_ref[kR], l[kR];  // l: this thread's keys only
+#pragma unroll
+    for (int x = 0; x < kR; ++x) {
+      m_ref[x] = -INFINITY;
+      l[x] = 0.f;
+    }
     bool ok = true;
     auto wait_pv = [&](int t) {
       return __all_sync(0xffffffffu, dev::mbar_wait(o_ready0 + 8 * (t & 1),
@@ -496,48 +509,52 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (lane == 0) dev::mbar_arrive(p_full0 + 8 * (j & 1));
         continue;
       }
-      // sa[4k], sa[4k + 1]: this row, keys 8k + 2 c4 and 8k + 2 c4 + 1.
-      float sv[16];
+      // sa[4k + 2x + e]: row x, key 8k + 2 c4 + e.
+      float sv[kR][16];
+      float factor[kR];
+      bool grow = false;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        sv[2 * k] = sa[4 * k];
-        sv[2 * k + 1] = sa[4 * k + 1];
-      }
-      const int lim = qpos - k0;
-      if (lim < kKeys - 1) {
+      for (int x = 0; x < kR; ++x) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
+        for (int k = 0; k < 8; ++k) {
+          sv[x][2 * k] = sa[4 * k + 2 * x];
+          sv[x][2 * k + 1] = sa[4 * k + 2 * x + 1];
+        }
+        const int lim = qpos[x] - k0;
+        if (lim < kKeys - 1) {
 #pragma unroll
-          for (int e = 0; e < 2; ++e)
-            if (8 * k + 2 * c4 + e > lim) sv[2 * k + e] = -INFINITY;
-      }
-      float m4[4];
+          for (int k = 0; k < 8; ++k)
 #pragma unroll
-      for (int u = 0; u < 4; ++u) m4[u] = fmaxf(sv[u], sv[u + 4]);
+            for (int e = 0; e < 2; ++e)
+              if (8 * k + 2 * c4 + e > lim) sv[x][2 * k + e] = -INFINITY;
+        }
+        float m4[4];
 #pragma unroll
-      for (int k = 8; k < 16; ++k) m4[k & 3] = fmaxf(m4[k & 3], sv[k]);
-      float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      mx *= c;
-      float factor = 1.f;
-      if (j == 0) {
-        m_ref = mx;
-      } else if (mx > m_ref + kRescaleLog2) {
-        factor = dev::fast_exp2(m_ref - mx);
-        m_ref = mx;
-        l *= factor;
-      }
-      {
+        for (int u = 0; u < 4; ++u) m4[u] = fmaxf(sv[x][u], sv[x][u + 4]);
+#pragma unroll
+        for (int k = 8; k < 16; ++k) m4[k & 3] = fmaxf(m4[k & 3], sv[x][k]);
+        float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        mx *= c;
+        factor[x] = 1.f;
+        if (j == 0) {
+          m_ref[x] = mx;
+        } else if (mx > m_ref[x] + kRescaleLog2) {
+          factor[x] = dev::fast_exp2(m_ref[x] - mx);
+          m_ref[x] = mx;
+          l[x] *= factor[x];
+          grow = true;
+        }
         float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          sv[k] = dev::fast_exp2(fmaf(sv[k], c, -m_ref));
-          l4[k & 3] += sv[k];
+          sv[x][k] = dev::fast_exp2(fmaf(sv[x][k], c, -m_ref[x]));
+          l4[k & 3] += sv[x][k];
         }
-        l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        l[x] += (l4[0] + l4[1]) + (l4[2] + l4[3]);
       }
-      if (__any_sync(0xffffffffu, factor != 1.f)) {
+      if (__any_sync(0xffffffffu, grow)) {
         ok = wait_pv(j - 1);
         if (!ok) break;
         dev::tc_fence_after();
@@ -547,24 +564,35 @@ __global__ void __launch_bounds__(kThreads, 2)
           tmem_ld16x256_x4(o_tmem + lane_off + col, ov);
           dev::tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) ov[e] *= factor;
+          for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int x = 0; x < kR; ++x) {
+              ov[4 * k + 2 * x] *= factor[x];
+              ov[4 * k + 2 * x + 1] *= factor[x];
+            }
           tmem_st16x256_x4(o_tmem + lane_off + col, ov);
         }
         dev::tmem_st_wait();
       }
       // P over S(j): column 4k + c4 of each half holds keys 8k + 2 c4 and
-      // 8k + 2 c4 + 1; the padding lane (t/4 + 8) gets zeros.
+      // 8k + 2 c4 + 1 of row x in lane t/4 + 8x; a padding lane gets zeros.
       {
         uint32_t hw[16], lw[16];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t w = M::pack(sv[2 * k], sv[2 * k + 1]);
-          const float2 hf = M::unpack(w);
-          hw[2 * k] = w;
-          hw[2 * k + 1] = 0u;
-          lw[2 * k] = M::pack(sv[2 * k] - hf.x, sv[2 * k + 1] - hf.y);
-          lw[2 * k + 1] = 0u;
-        }
+        for (int k = 0; k < 8; ++k)
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            if (x < kR) {
+              const uint32_t w = M::pack(sv[x][2 * k], sv[x][2 * k + 1]);
+              const float2 hf = M::unpack(w);
+              hw[2 * k + x] = w;
+              lw[2 * k + x] =
+                  M::pack(sv[x][2 * k] - hf.x, sv[x][2 * k + 1] - hf.y);
+            } else {
+              hw[2 * k + x] = 0u;
+              lw[2 * k + x] = 0u;
+            }
+          }
         const uint32_t pa = s_tmem + (j & 1) * kKeys + lane_off;
         tmem_st16x128_x8(pa, hw);
         tmem_st16x128_x8(pa + kKeys / 2, lw);
@@ -574,31 +602,39 @@ __global__ void __launch_bounds__(kThreads, 2)
       __syncwarp();
       if (lane == 0) dev::mbar_arrive(p_full0 + 8 * (j & 1));
     }
-    // Epilogue: the row sum over the four threads, O / l -> out.
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    // Epilogue: the row sums over the four threads, O / l -> out.
+    float inv[kR];
+#pragma unroll
+    for (int x = 0; x < kR; ++x) {
+      l[x] += __shfl_xor_sync(0xffffffffu, l[x], 1);
+      l[x] += __shfl_xor_sync(0xffffffffu, l[x], 2);
+      inv[x] = l[x] > 0.f ? 1.f / l[x] : 0.f;
+    }
     if (ok && !idle) ok = wait_pv(n_tiles - 1);
     if (ok && !idle) {
       dev::tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const int64_t idx =
-          (static_cast<int64_t>(q0 + tok0 + t_loc) * a.num_q_heads + kvh * G +
-           hq) * D + 2 * c4;
 #pragma unroll
       for (int col = 0; col < D; col += 32) {
         float ov[16];
         tmem_ld16x256_x4(o_tmem + lane_off + col, ov);
         dev::tmem_ld_wait();
-        if (valid) {
+#pragma unroll
+        for (int x = 0; x < kR; ++x) {
+          if (!valid[x]) continue;
+          const int64_t idx =
+              (static_cast<int64_t>(q0 + tok0 + t_loc[x]) * a.num_q_heads +
+               kvh * G + hq[x]) * D + 2 * c4 + col;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const int64_t e = idx + col + 8 * k;  // dims e, e + 1
+            const int64_t e = idx + 8 * k;  // dims e, e + 1
+            const float v0 = ov[4 * k + 2 * x] * inv[x];
+            const float v1 = ov[4 * k + 2 * x + 1] * inv[x];
             if (a.out_f32)
               *reinterpret_cast<float2*>(static_cast<float*>(a.out) + e) =
-                  make_float2(ov[4 * k] * inv, ov[4 * k + 1] * inv);
+                  make_float2(v0, v1);
             else
               *reinterpret_cast<uint32_t*>(static_cast<T*>(a.out) + e) =
-                  M::pack(ov[4 * k] * inv, ov[4 * k + 1] * inv);
+                  M::pack(v0, v1);
           }
         }
       }
@@ -1430,11 +1466,11 @@ size_t prefill_workspace_bytes(const pa_prefill_desc* d) {
          ~size_t(15);
 }
 
-template <typename T, int BS, int G, int D, bool SQ>
+template <typename T, int BS, int G, int D, int RQ>
 pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
                  const CUtensorMap& qm, const CUtensorMap& km,
                  const CUtensorMap& vm, cudaStream_t st) {
-  auto kern = prefill_kernel<T, BS, G, D, SQ>;
+  auto kern = prefill_kernel<T, BS, G, D, RQ>;
   const size_t smem = Layout<D>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1463,29 +1499,29 @@ pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
   return PA_OK;
 }
 
-template <typename T, int BS, int D, bool SQ>
+template <typename T, int BS, int D, int RQ>
 pa_status dispatch_group(const pa_prefill_desc* d, const PrefillArgs& a,
                          const CUtensorMap& qm, const CUtensorMap& km,
                          const CUtensorMap& vm, cudaStream_t st) {
   switch (d->num_q_heads / d->num_kv_heads) {
-    case 1: return launch<T, BS, 1, D, SQ>(d, a, qm, km, vm, st);
-    case 2: return launch<T, BS, 2, D, SQ>(d, a, qm, km, vm, st);
-    case 4: return launch<T, BS, 4, D, SQ>(d, a, qm, km, vm, st);
-    default: return launch<T, BS, 8, D, SQ>(d, a, qm, km, vm, st);
+    case 1: return launch<T, BS, 1, D, RQ>(d, a, qm, km, vm, st);
+    case 2: return launch<T, BS, 2, D, RQ>(d, a, qm, km, vm, st);
+    case 4: return launch<T, BS, 4, D, RQ>(d, a, qm, km, vm, st);
+    default: return launch<T, BS, 8, D, RQ>(d, a, qm, km, vm, st);
   }
 }
 
-template <typename T, bool SQ>
+template <typename T, int RQ>
 pa_status dispatch_shape(const pa_prefill_desc* d, const PrefillArgs& a,
                          const CUtensorMap& qm, const CUtensorMap& km,
                          const CUtensorMap& vm, cudaStream_t st) {
   if (d->head_dim == 128)
     return d->block_size == 16
-               ? dispatch_group<T, 16, 128, SQ>(d, a, qm, km, vm, st)
-               : dispatch_group<T, 32, 128, SQ>(d, a, qm, km, vm, st);
+               ? dispatch_group<T, 16, 128, RQ>(d, a, qm, km, vm, st)
+               : dispatch_group<T, 32, 128, RQ>(d, a, qm, km, vm, st);
   return d->block_size == 16
-             ? dispatch_group<T, 16, 64, SQ>(d, a, qm, km, vm, st)
-             : dispatch_group<T, 32, 64, SQ>(d, a, qm, km, vm, st);
+             ? dispatch_group<T, 16, 64, RQ>(d, a, qm, km, vm, st)
+             : dispatch_group<T, 32, 64, RQ>(d, a, qm, km, vm, st);
 }
 
 template <typename T, int BS, int G>
@@ -1618,12 +1654,14 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
   const int max_ctx = d->max_context_len > 0
                           ? d->max_context_len
                           : d->max_blocks_per_seq * d->block_size;
-  // At most 32 query rows per KV head (a few new tokens): the tile kernel
-  // spreads them over the four softmax warps, eight rows each.
-  const bool small_q = !use_keys && static_cast<int64_t>(d->max_q_len) * G <= 32;
-  const int tok = use_keys  ? pagedkv::kVerRows / G
-                  : small_q ? 8 / G
-                            : pagedkv::kRows / G;
+  // At most 64 query rows per KV head (a few new tokens): the tile kernel
+  // spreads them over the four softmax warps, 8 (up to 32 rows) or 16 (up
+  // to 64) per warp.
+  const int64_t q_rows = static_cast<int64_t>(d->max_q_len) * G;
+  const int rq = use_keys ? 0 : q_rows <= 32 ? 8 : q_rows <= 64 ? 16 : 0;
+  const int tok = use_keys ? pagedkv::kVerRows / G
+                  : rq > 0 ? rq / G
+                           : pagedkv::kRows / G;
   CUtensorMap qm, km, vm;
   const uint64_t rows = static_cast<uint64_t>(d->num_blocks) *
                         d->num_kv_heads * d->block_size;
@@ -1662,13 +1700,17 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
     return d->dtype == PA_BF16
                ? pagedkv::dispatch_verify<__nv_bfloat16>(d, a, qm, km, vm, s)
                : pagedkv::dispatch_verify<__half>(d, a, qm, km, vm, s);
-  if (small_q)
+  if (rq == 8)
     return d->dtype == PA_BF16
-               ? pagedkv::dispatch_shape<__nv_bfloat16, true>(d, a, qm, km, vm, s)
-               : pagedkv::dispatch_shape<__half, true>(d, a, qm, km, vm, s);
+               ? pagedkv::dispatch_shape<__nv_bfloat16, 8>(d, a, qm, km, vm, s)
+               : pagedkv::dispatch_shape<__half, 8>(d, a, qm, km, vm, s);
+  if (rq == 16)
+    return d->dtype == PA_BF16
+               ? pagedkv::dispatch_shape<__nv_bfloat16, 16>(d, a, qm, km, vm, s)
+               : pagedkv::dispatch_shape<__half, 16>(d, a, qm, km, vm, s);
   return d->dtype == PA_BF16
-             ? pagedkv::dispatch_shape<__nv_bfloat16, false>(d, a, qm, km, vm, s)
-             : pagedkv::dispatch_shape<__half, false>(d, a, qm, km, vm, s);
+             ? pagedkv::dispatch_shape<__nv_bfloat16, 0>(d, a, qm, km, vm, s)
+             : pagedkv::dispatch_shape<__half, 0>(d, a, qm, km, vm, s);
 }
 
 extern "C" size_t pa_prefill_workspace_bytes(const pa_prefill_desc* d) {

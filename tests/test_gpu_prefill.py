@@ -369,3 +369,25 @@ def test_keys_kernel_long_context(pkv):
         ref = oa.paged_decode(to_np(pin.q)[rows], kc, vc, sub,
                               L - n + np.arange(n) + 1, w.softmax_scale)
         check_decode(to_np(out)[rows], ref, pin.q.dtype, f"long seq {b}")
+
+
+@pytest.mark.parametrize("dtype", ["bfloat16", "float16"])
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (32, 8), (64, 8)])
+@pytest.mark.parametrize("bs", [16, 32])
+def test_few_rows_33_to_64(pkv, dtype, hq, hkv, bs):
+    """33 .. 64 query rows per KV head (the tile kernel's 16-rows-per-warp
+    layout: two rows per thread), contexts around the tile edges."""
+    G = hq // hkv
+    qmax = 64 // G
+    lens = (1, 17, 130, 300, 520, 64, 700, 33, 129, 128, 255, 256)
+    want = (1, qmax, qmax - 1, 32 // G + 1, 2, qmax, qmax, 0, qmax, 1, 5,
+            qmax)
+    qlens = tuple(min(L, q) for L, q in zip(lens, want))
+    assert 32 < max(qlens) * G <= 64
+    w = wl.Workload("prefill_rows64", 24, len(lens), hq, hkv, 128, bs, dtype,
+                    "fixed", fixed_lengths=lens)
+    pin = wl.make_prefill(w, qlens, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = _run(pkv, pin, err=err)
+    assert err.item() == 0
+    _check(pin, out, f"rows<=64 {dtype}/{hq}:{hkv}/bs{bs}")

@@ -67,10 +67,14 @@ def test_decode_paths_round_once(pkv, dtype, d, kernel, ps, reduce):
 
 
 @pytest.mark.parametrize("dtype", ["bfloat16", "float16"])
-@pytest.mark.parametrize("kernel", ["tile", "keys"])
-def test_prefill_paths_round_once(pkv, dtype, kernel):
+@pytest.mark.parametrize("kernel,maxq", [("tile", 4), ("tile", 16),
+                                         ("tile", 40), ("keys", 4)])
+def test_prefill_paths_round_once(pkv, dtype, kernel, maxq):
+    """G = 4: up to 16 / 64 / 160 query rows per KV head reach the tile
+    kernel's 8-rows-per-warp, 16-rows-per-warp and plain layouts."""
     lens = (1, 3, 6, 40, 700, 130, 2, 257)
-    qlens = (1, 3, 4, 4, 4, 2, 2, 4)
+    qlens = tuple(min(L, q) for L, q in
+                  zip(lens, (1, 3, maxq, maxq, maxq, 2, 2, maxq)))
     w = wl.Workload("rounding_pf", 42, len(lens), 32, 8, 128, 16, dtype,
                     "fixed", fixed_lengths=lens, scale=1.0)
     pin = wl.make_prefill(w, qlens, device="cuda")
@@ -78,7 +82,7 @@ def test_prefill_paths_round_once(pkv, dtype, kernel):
     bt = torch.from_numpy(inp.block_tables).cuda()
     cl = torch.from_numpy(inp.lengths.astype(np.int32)).cuda()
     qs = torch.from_numpy(pin.query_start).cuda()
-    kw = dict(max_q_len=4, max_context_len=int(inp.lengths.max()),
+    kw = dict(max_q_len=max(qlens), max_context_len=int(inp.lengths.max()),
               kernel=kernel)
     out = torch.empty_like(pin.q)
     out32 = torch.empty(pin.q.shape, dtype=torch.float32, device="cuda")
