@@ -181,9 +181,13 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache,
  *   - A shape whose pa_decode_workspace_bytes() exceeds
  *     PA_NOALLOC_SCRATCH_BYTES is rejected with PA_ERR_WORKSPACE and a
  *     message naming both sizes (use a larger partition_size or pa_decode).
- *   - The first call on a device looks up the area's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *   - The first call in a CUDA context looks up the area's device address
+ *     (cudaGetSymbolAddress, with that context current) and keeps it, keyed
+ *     on the context's unique id; make that first call before any stream
+ *     capture.  A device reset (cudaDeviceReset) or a context the caller
+ *     creates through the driver API gives a new id, so the address is
+ *     looked up again there rather than reused.  The lookup is guarded by a
+ *     mutex, so first calls from several host threads are safe.
  *   - Every call uses the same area, which keeps the previous call's data;
  *     what must start at zero (the per-sequence partition counters) is reset
  *     on the call's stream.  Calls that overlap on the GPU (other streams,

@@ -49,6 +49,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "device_utils.cuh"
 #include "order.cuh"
@@ -59,7 +60,7 @@
 // this library's module on every GPU that loads it, for callers that cannot
 // allocate device memory.  In host code this name is only a stand-in, not a
 // device address: scratch_address() below asks the runtime for the address,
-// once per device.
+// once per CUDA context.
 static __device__ __align__(256) unsigned char
     g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
 
@@ -1212,29 +1213,71 @@ pa_status dispatch_shape(const pa_decode_desc* d, DecodeArgs& a,
                             : launch<T, 32, 64, kMma>(d, a, km, vm, st);
 }
 
+// The built-in scratch's device address belongs to a CUDA context, not to a
+// device ordinal: after cudaDeviceReset, or under a context the caller made
+// current through the driver API, the module is loaded again and the array
+// may sit elsewhere.  So the cache is keyed on the current context's unique
+// id (cuCtxGetId, never reused within a process), filled under a mutex.
+using PFN_ctxGetCurrent = CUresult (*)(CUcontext*);
+using PFN_ctxGetId = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename F>
+F driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion(name, &p, 12000, cudaEnableDefault,
+                                       &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<F>(p);
+  return nullptr;
+}
+
+// Unique id of the calling thread's current context; false if there is none.
+bool current_context_id(unsigned long long* id) {
+  static const PFN_ctxGetCurrent get_current =
+      driver_fn<PFN_ctxGetCurrent>("cuCtxGetCurrent");
+  static const PFN_ctxGetId get_id = driver_fn<PFN_ctxGetId>("cuCtxGetId");
+  CUcontext ctx = nullptr;
+  return get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx &&
+         get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 void* scratch_address(pa_status* st) {
-  constexpr int kMaxDevices = 64;
-  static void* addr[kMaxDevices] = {nullptr};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    *st = fail(PA_ERR_CUDA, "pa_decode_noalloc: no usable current device (%s)",
-               cudaGetErrorString(e));
+  struct Entry {
+    unsigned long long ctx_id;
+    void* addr;
+  };
+  constexpr int kMaxEntries = 64;
+  static std::mutex mu;
+  static Entry cache[kMaxEntries];
+  static int used = 0;
+  unsigned long long id = 0;
+  if (current_context_id(&id)) {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+      if (cache[i].ctx_id == id) {
+        *st = PA_OK;
+        return cache[i].addr;
+      }
+  }
+  // First call in this context (or no context yet: the runtime creates the
+  // device's primary context here).
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, ::g_noalloc_scratch);
+  if (e != cudaSuccess || !p) {
+    *st = fail(PA_ERR_CUDA,
+               "pa_decode_noalloc: cudaGetSymbolAddress of the built-in "
+               "scratch failed: %s", cudaGetErrorString(e));
     return nullptr;
   }
-  if (!addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, ::g_noalloc_scratch);
-    if (e != cudaSuccess || !p) {
-      *st = fail(PA_ERR_CUDA,
-                 "pa_decode_noalloc: cudaGetSymbolAddress of the built-in "
-                 "scratch failed: %s", cudaGetErrorString(e));
-      return nullptr;
-    }
-    addr[dev] = p;
+  if (current_context_id(&id)) {
+    std::lock_guard<std::mutex> lock(mu);
+    bool known = false;
+    for (int i = 0; i < used; ++i) known |= cache[i].ctx_id == id;
+    if (!known && used < kMaxEntries) cache[used++] = Entry{id, p};
   }
   *st = PA_OK;
-  return addr[dev];
+  return p;
 }
 
 }  // namespace
