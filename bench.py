@@ -201,6 +201,38 @@ def kv_bytes(lengths, w) -> int:
     return int(np.sum(lengths)) * w.num_kv_heads * w.head_dim * 2 * 2
 
 
+def make_timer(stream, steps, flush_buf):
+    """timed(fn) -> total ms of ``steps`` calls of fn on ``stream``, CUDA
+    events on that stream.  With ``flush_buf`` (data below twice the L2
+    size) a write of that buffer flushes L2 before each call, outside the
+    per-call events; otherwise the calls run back to back between two
+    events (an event between the kernels would break their
+    programmatic-launch overlap)."""
+    import torch
+
+    def timed(fn):
+        if flush_buf is None:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(steps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1)
+        evs = [(torch.cuda.Event(enable_timing=True),
+                torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for e0, e1 in evs:
+            flush_buf.fill_(1)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return sum(e0.elapsed_time(e1) for e0, e1 in evs)
+    return timed
+
+
 def run_native(args, rank, world, local):
     import torch
     import paged_kv_cache_383_b200 as pkv
@@ -265,29 +297,7 @@ def run_native(args, rank, world, local):
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) \
         if flush else None
 
-    def timed(fn):
-        """Total ms of args.steps calls of fn on the stream."""
-        if not flush:
-            # events only at the two ends (an event between the kernels
-            # would break their programmatic-launch overlap)
-            e0 = torch.cuda.Event(enable_timing=True)
-            e1 = torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(args.steps):
-                fn()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            return e0.elapsed_time(e1)
-        evs = [(torch.cuda.Event(enable_timing=True),
-                torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        for e0, e1 in evs:
-            flush_buf.fill_(1)
-            e0.record(stream)
-            fn()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        return sum(e0.elapsed_time(e1) for e0, e1 in evs)
+    timed = make_timer(stream, args.steps, flush_buf)
 
     # Timed region: exactly K steps.
     launches0 = pkv.pa_launch_count()
@@ -391,6 +401,8 @@ def run_native(args, rank, world, local):
         if probe:
             res["roofline"]["read_probe_gbs"] = probe
             res["roofline"]["frac_of_read_probe"] = round(achieved / probe, 4)
+        res["extras"]["configs"] = config_block(args, pkv, flow, wl, dev,
+                                                probe)
     if not args.no_e2e:
         if w.lengths == "prefix":
             res["e2e"] = run_e2e_fixed(args, w, spec, dev, pkv, world, ps)
@@ -404,6 +416,106 @@ def run_native(args, rank, world, local):
         res["cpu_baseline"] = cpu_baseline(pool, inp, w, dev)
     if pool is not None:
         pool.close()
+    return res
+
+
+# The serving mixes besides the headline one (batch 256, block 16): each is
+# timed like the headline line, into extras["configs"].
+CONFIG_WORKLOADS = ("tiny_mha_d64", "llama3_8b_gqa4", "llama3_70b_gqa8_bs32",
+                    "shared_prefix_cow", "long_context_split")
+
+
+def config_block(args, pkv, flow, wl, dev, probe_gbs):
+    """Per configuration: the step (copy-on-write copies and cache write
+    where the mix has them, then the decode) and the decode alone, each over
+    K calls timed with CUDA events on the launch stream exactly like the
+    headline line (L2 flushed between calls when the distinct K/V is below
+    twice the L2 size), with the clocks sampled during the timed calls.
+    GB/s are algorithmic K/V bytes (logical bytes for the shared-prefix mix:
+    its prefix is read once per sequence and stays in L2)."""
+    import torch
+    peak, peak_kind = measured_hbm_peak()
+    stream = torch.cuda.current_stream(dev)
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    steps = max(args.steps, 10)
+    res = {}
+    for name in CONFIG_WORKLOADS:
+        w = wl.WORKLOADS[name]
+        spec = setup_prefix(w, dev, pkv, flow, wl) if w.lengths == "prefix" \
+            else setup_paged(w, dev, wl)
+        inp = spec.inp
+        out = torch.empty_like(inp.q)
+        desc = pkv.make_desc(inp.q, inp.k_cache, spec.bt,
+                             partition_size=w.partition_size,
+                             max_context_len=int(inp.lengths.max()))
+        ws = torch.empty(max(pkv.pa_decode_workspace_bytes(desc), 16),
+                         dtype=torch.uint8, device=dev)
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+        def decode():
+            pkv.pa_decode(out, inp.q, inp.k_cache, inp.v_cache, spec.bt,
+                          spec.cl, w.softmax_scale, desc=desc, workspace=ws,
+                          dev_err=err)
+
+        def step():
+            if spec.pairs is not None:
+                pkv.pa_copy_blocks(inp.k_cache, inp.v_cache, spec.pairs,
+                                   dev_err=err)
+            pkv.pa_cache_write(inp.k_cache, inp.v_cache, spec.write_k,
+                               spec.write_v, spec.slots, dev_err=err)
+            decode()
+
+        for _ in range(5):
+            step()
+        torch.cuda.synchronize()
+        step_bytes = kv_bytes(inp.lengths, w)
+        unique = spec.info.get("unique_kv_bytes_per_step", step_bytes)
+        flush = unique < 2 * l2_bytes
+        flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev) \
+            if flush else None
+        timed = make_timer(stream, steps, flush_buf)
+        # the timed calls last milliseconds: the clocks are sampled over an
+        # untimed 0.5 s run of the same step just before them, and the
+        # timed calls themselves
+        clocks = ClockSampler(dev.index or 0)
+        t0 = time.time()
+        while time.time() - t0 < 0.5:
+            step()
+            torch.cuda.synchronize()
+        ms_step = timed(step) / steps
+        ms_dec = timed(decode) / steps
+        clk = clocks.stop()
+        if err.item() != 0:
+            raise RuntimeError(f"{name}: device error flag {err.item()}")
+        dec_gbs = step_bytes / (ms_dec * 1e-3) / 1e9
+        entry = {
+            "step": spec.info["step"],
+            "seqs": w.num_seqs, "heads_q_kv": [w.num_q_heads,
+                                               w.num_kv_heads],
+            "head_dim": w.head_dim, "block_size": w.block_size,
+            "dtype": w.dtype, "tokens": int(inp.lengths.sum()),
+            "kv_bytes": step_bytes,
+            "partition_size": pkv.pa_decode_partition_size(desc),
+            "partition_spec": w.partition_size or "auto",
+            "ms_step": round(ms_step, 5), "ms_decode": round(ms_dec, 5),
+            "step_gbs": round(step_bytes / (ms_step * 1e-3) / 1e9, 1),
+            "decode_gbs": round(dec_gbs, 1),
+            "seq_layers_per_s": round(w.num_seqs / (ms_dec * 1e-3), 1),
+            "frac_of_copy_peak": round(dec_gbs / peak, 4),
+            "copy_peak": f"{peak} GB/s ({peak_kind})",
+            "frac_of_read_probe": round(dec_gbs / probe_gbs, 4)
+            if probe_gbs else None,
+            "frac_of_spec_8000": round(dec_gbs / SPEC_HBM_GBS, 4),
+            "l2": "flushed between calls" if flush else "inputs larger than "
+                                                        "L2, back to back",
+            "calls": steps, "clocks": clk,
+            "clocks_how": "nvidia-smi every 100 ms over a 0.5 s untimed run "
+                          "of the step and the timed calls"}
+        if w.lengths == "prefix":
+            entry["note"] = spec.info["note"]
+        res[name] = entry
+        del spec, inp, out, ws, flush_buf
+        torch.cuda.empty_cache()
     return res
 
 
@@ -607,11 +719,14 @@ def extras(args, w, inp, dev, pkv, bt, cl):
     return out
 
 
-def identity_vs_shuffled(pkv, w, inp, dev):
+def identity_vs_shuffled(pkv, w, inp, dev, repeats=12, calls=10):
     """The same decode over the shuffled pool and over a copy laid out so
     every sequence's blocks are consecutive (identity tables): the whole
     batch, and batch 1 (its longest sequence; L2 flushed before each call,
-    the data being smaller than L2).  GB/s of K/V read."""
+    the data being smaller than L2).  The two arms alternate, ``repeats``
+    times, each time ``calls`` calls; each arm reports the median and the
+    min..max of its repeats (GB/s of K/V read), so a difference of about a
+    percent can be told from run-to-run noise."""
     import torch
     B = inp.block_tables.shape[0]
     rows = [inp.block_tables[b][inp.block_tables[b] >= 0] for b in range(B)]
@@ -625,7 +740,7 @@ def identity_vs_shuffled(pkv, w, inp, dev):
         base += len(r)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
-    def run(seqs, tables, k, v, flush):
+    def prepare(seqs, tables, k, v):
         q = inp.q[seqs].contiguous()
         bt = torch.from_numpy(tables[seqs]).to(dev)
         lens = inp.lengths[seqs]
@@ -638,8 +753,11 @@ def identity_vs_shuffled(pkv, w, inp, dev):
                                   desc=desc, workspace=ws)
         for _ in range(3):
             f()
-        n, total = 20, 0.0
-        for _ in range(n):
+        return f, kv_bytes(lens, w)
+
+    def once(f, nbytes, flush):
+        total = 0.0
+        for _ in range(calls):
             if flush:
                 flush_buf.fill_(1)
             a = torch.cuda.Event(enable_timing=True)
@@ -649,17 +767,32 @@ def identity_vs_shuffled(pkv, w, inp, dev):
             b_.record()
             torch.cuda.synchronize()
             total += a.elapsed_time(b_)
-        return round(kv_bytes(lens, w) / (total / n * 1e-3) / 1e9, 1)
+        return nbytes / (total / calls * 1e-3) / 1e9
+
+    def compare(seqs, flush):
+        arms = {"shuffled": prepare(seqs, inp.block_tables, inp.k_cache,
+                                    inp.v_cache),
+                "identity": prepare(seqs, ident, kc, vc)}
+        got = {k: [] for k in arms}
+        for r in range(repeats):
+            for k in (("shuffled", "identity") if r % 2 == 0
+                      else ("identity", "shuffled")):
+                got[k].append(once(*arms[k], flush))
+        out = {}
+        for k, v in got.items():
+            out[f"{k}_gbs_median"] = round(float(np.median(v)), 1)
+            out[f"{k}_gbs_range"] = [round(min(v), 1), round(max(v), 1)]
+        lo_i, hi_i = out["identity_gbs_range"]
+        lo_s, hi_s = out["shuffled_gbs_range"]
+        out["ranges_overlap"] = bool(lo_i <= hi_s and lo_s <= hi_i)
+        return out
 
     allb = np.arange(B)
     one = np.array([int(np.argmax(inp.lengths))])
-    res = {"batch_gbs_shuffled": run(allb, inp.block_tables, inp.k_cache,
-                                     inp.v_cache, False),
-           "batch_gbs_identity": run(allb, ident, kc, vc, False),
+    res = {"repeats": repeats, "calls_per_repeat": calls,
+           "batch": compare(allb, False),
            "batch1_tokens": int(inp.lengths[one[0]]),
-           "batch1_gbs_shuffled": run(one, inp.block_tables, inp.k_cache,
-                                      inp.v_cache, True),
-           "batch1_gbs_identity": run(one, ident, kc, vc, True)}
+           "batch1": compare(one, True)}
     del kc, vc
     return res
 
@@ -691,7 +824,9 @@ PREFILL_CASES = (
 
 def time_prefill(pkv, wl, name, chunk, dev, iters=10):
     """pa_prefill on a prefill workload: CUDA events around ``iters``
-    back-to-back launches on the launch stream (inputs > L2)."""
+    back-to-back launches on the launch stream (inputs > L2), for each
+    precision of P in P . V (the default "auto" adds P's residual only in
+    the tiles that need it; "split" in every tile; "single" never)."""
     import torch
     w = wl.WORKLOADS[name]
     rng_lens = wl.make_paged(w, values=False).lengths
@@ -707,31 +842,42 @@ def time_prefill(pkv, wl, name, chunk, dev, iters=10):
               max_context_len=int(inp.lengths.max()), dev_err=err,
               workspace=torch.empty(4 * w.num_seqs + 16, dtype=torch.uint8,
                                     device=dev))
-    for _ in range(3):
-        pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl, qs,
-                       w.softmax_scale, **kw)
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(iters):
-        pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl, qs,
-                       w.softmax_scale, **kw)
-    b.record()
-    torch.cuda.synchronize()
-    if err.item():
-        raise RuntimeError(f"pa_prefill device error {err.item()}")
-    ms = a.elapsed_time(b) / iters
+    def run(pv):
+        for _ in range(3):
+            pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl, qs,
+                           w.softmax_scale, pv=pv, **kw)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(iters):
+            pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl, qs,
+                           w.softmax_scale, pv=pv, **kw)
+        b.record()
+        torch.cuda.synchronize()
+        if err.item():
+            raise RuntimeError(f"pa_prefill device error {err.item()}")
+        return a.elapsed_time(b) / iters
+
     flops = prefill_flops(inp.lengths, pin.q_lens, w.num_q_heads, w.head_dim)
     peak, kind = measured_bf16_peak()
-    tf = flops / (ms * 1e-3) / 1e12
+    ms = {pv: run(pv) for pv in ("auto", "split", "single")}
+    tf = {pv: flops / (t * 1e-3) / 1e12 for pv, t in ms.items()}
     return {"workload": name, "seqs": w.num_seqs,
             "new_tokens": int(pin.q_lens.sum()),
-            "context_tokens": int(inp.lengths.sum()), "ms": round(ms, 4),
-            "tflops": round(tf, 1), "peak_tflops": peak,
+            "context_tokens": int(inp.lengths.sum()),
+            "ms": round(ms["auto"], 4), "tflops": round(tf["auto"], 1),
+            "peak_tflops": peak,
             "peak_kind": f"{kind} bf16 dense (cuBLAS GEMM)",
-            "frac": round(tf / peak, 4),
-            "note": "P.V runs twice (rounded P and its residual): the tensor "
-                    "cores do 1.5x the algorithmic FLOPs"}
+            "frac": round(tf["auto"] / peak, 4),
+            "pv": "auto (P's residual . V only in tiles where a key may end "
+                  "with weight > 1/16)",
+            "tflops_pv_split": round(tf["split"], 1),
+            "frac_pv_split": round(tf["split"] / peak, 4),
+            "tflops_pv_single": round(tf["single"], 1),
+            "frac_pv_single": round(tf["single"] / peak, 4),
+            "note": "algorithmic FLOPs (4 D per query head, new token and "
+                    "key attended); with pv=split the tensor cores do 1.5x "
+                    "that (P.V twice)"}
 
 
 def prefix_cache_measure(pkv, dev, requests=128, prompt_len=2048,
@@ -917,10 +1063,10 @@ def spec_verify_measure(pkv, dev, drafts=4):
               workspace=torch.empty(4 * w.num_seqs + 16, dtype=torch.uint8,
                                     device=dev))
 
-    def time_kernel(kernel):
+    def time_kernel(kernel, pv="auto"):
         f = lambda: pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt,
                                    cl, qs, w.softmax_scale, kernel=kernel,
-                                   **kw)
+                                   pv=pv, **kw)
         for _ in range(3):
             f()
         a = torch.cuda.Event(enable_timing=True)
@@ -933,8 +1079,8 @@ def spec_verify_measure(pkv, dev, drafts=4):
         return a.elapsed_time(b) / 20
 
     ms = time_kernel("auto")
-    keys_fit = drafts * (w.num_q_heads // w.num_kv_heads) <= 32
-    ms_keys = time_kernel("keys") if keys_fit else None
+    ms_split = time_kernel("auto", "split")
+    ms_single = time_kernel("auto", "single")
     gbs = lambda t: round(kv_bytes(inp.lengths, w) / (t * 1e-3) / 1e9, 1) \
         if t else None
     return {"seqs": w.num_seqs, "drafts": drafts,
@@ -943,9 +1089,10 @@ def spec_verify_measure(pkv, dev, drafts=4):
             "tflops": round(prefill_flops(inp.lengths, pin.q_lens,
                                           w.num_q_heads, w.head_dim)
                             / (ms * 1e-3) / 1e12, 1),
-            "kernel": "auto (the tile kernel)",
-            "ms_keys_kernel": round(ms_keys, 4) if ms_keys else None,
-            "kv_gbs_keys_kernel": gbs(ms_keys)}
+            "kernel": "the tile kernel",
+            "pv": "auto",
+            "kv_gbs_pv_split": gbs(ms_split),
+            "kv_gbs_pv_single": gbs(ms_single)}
 
 
 def run_extras_only(args):

@@ -230,25 +230,40 @@ pa_status pa_decode_noalloc(void* out, const void* q, const void* k_cache,
  * more new tokens than max_q_len, or a block id outside the pool sets
  * *dev_err = PA_ERR_DEVICE_OOB and the affected rows are unspecified.
  * ---------------------------------------------------------------------- */
-/* Which prefill kernel runs:
- *   PA_PREFILL_AUTO  -- PA_PREFILL_TILE (the faster of the two on every
- *                       shape measured so far).
- *   PA_PREFILL_TILE  -- tiles of 128 query rows (new token, query head) on
- *                       the MMA's M side, 64 keys on N; any q_len.
- *   PA_PREFILL_KEYS  -- keys on M (128 per tile), the <= 32 query rows of
- *                       one KV head on N: S^T = K Q^T, O^T += V^T P^T, so no
- *                       MMA row is padding when few tokens are new
- *                       (speculative verification).  Needs head_dim 128 and
- *                       max_q_len * G <= 32 (PA_ERR_UNSUPPORTED otherwise);
- *                       persistent, one CTA per SM.  Same results within
- *                       the tolerance; slower than PA_PREFILL_TILE today
- *                       (four softmax warps per SM and a cross-warp row
- *                       maximum every 128 keys). */
+/* Which prefill kernel runs (PA_PREFILL_AUTO and PA_PREFILL_TILE are the
+ * same): tiles of 128 query rows (new token, query head) on the MMA's M side,
+ * 64 keys on N; with at most 64 query rows per KV head (a few new tokens) the
+ * rows are spread over all four softmax warps.  Any other value is
+ * PA_ERR_INVALID_ARG. */
 typedef enum {
   PA_PREFILL_AUTO = 0,
-  PA_PREFILL_TILE = 1,
-  PA_PREFILL_KEYS = 2
+  PA_PREFILL_TILE = 1
 } pa_prefill_kernel;
+
+/* Precision of P in the tile kernel's P . V (the tensor cores take 16-bit
+ * operands, so the softmax weights P are rounded to dtype).  One rounding
+ * moves each weight by up to 2^-8 of itself in bf16 (2^-11 in fp16); on a
+ * row whose weight sits on a few keys that moves the output by up to
+ * 2^-8 |v|, more than the 2e-3 tolerance.  Adding residual . V, with the
+ * residual = P - round(P) rounded again, keeps about 16 bits of P at the cost
+ * of a second P . V MMA.
+ *   PA_PV_AUTO    -- the residual only in tiles where some row has a key
+ *                    with p > l / 16, l being the row's running sum of
+ *                    weights including that tile (such a key may end with a
+ *                    weight above 1/16); in every other tile each key ends
+ *                    with a weight below 1/16 and the single rounding's
+ *                    errors, of either sign, average out.  Within the
+ *                    tolerance on every workload tested; on long rows
+ *                    only the first few tiles need the residual.
+ *   PA_PV_SPLIT   -- the residual in every tile.
+ *   PA_PV_SINGLE  -- never: one rounding of P (as FlashAttention does);
+ *                    fastest, but short or peaky rows may exceed 2e-3.
+ */
+typedef enum {
+  PA_PV_AUTO = 0,
+  PA_PV_SPLIT = 1,
+  PA_PV_SINGLE = 2
+} pa_prefill_pv;
 
 typedef struct {
   int num_seqs;
@@ -264,6 +279,7 @@ typedef struct {
   int max_context_len;  /* host bound on context_lens[] (0: table capacity) */
   int kernel;           /* pa_prefill_kernel (0: automatic) */
   int out_fp32;         /* as in pa_decode_desc: 1 = out is float32 */
+  int pv;               /* pa_prefill_pv (0: per tile, as needed) */
 } pa_prefill_desc;
 
 /* Bytes of device workspace pa_prefill needs for this shape (the sequence

@@ -38,8 +38,9 @@ __all__ = [
 _KERNELS = {"auto": PA_KERNEL_AUTO, "mma": PA_KERNEL_MMA,
             "simt": PA_KERNEL_SIMT}
 _REDUCES = {"auto": _lib.PA_REDUCE_AUTO, "kernel": _lib.PA_REDUCE_KERNEL}
-_PREFILL_KERNELS = {"auto": _lib.PA_PREFILL_AUTO, "tile": _lib.PA_PREFILL_TILE,
-                    "keys": _lib.PA_PREFILL_KEYS}
+_PREFILL_KERNELS = {"auto": _lib.PA_PREFILL_AUTO, "tile": _lib.PA_PREFILL_TILE}
+_PREFILL_PV = {"auto": _lib.PA_PV_AUTO, "split": _lib.PA_PV_SPLIT,
+               "single": _lib.PA_PV_SINGLE}
 
 
 def library_path() -> str:
@@ -220,13 +221,14 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens,
 def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens,
                query_start, scale: float, *, max_q_len: int,
                max_context_len: int = 0, kernel: str = "auto",
-               workspace=None, dev_err=None, stream=None):
+               pv: str = "auto", workspace=None, dev_err=None, stream=None):
     """Causal attention of each sequence's new tokens (rows
     query_start[b] .. query_start[b+1]-1 of ``q``) over its paged K/V, the
     new tokens being the last ones of the context.  ``max_q_len`` bounds
-    every sequence's new-token count (sizes the grid).  ``kernel``: "auto",
-    "tile" (query rows on the MMA's M side) or "keys" (keys on M; head_dim
-    128 and max_q_len * G <= 32).  ``workspace`` (a
+    every sequence's new-token count (sizes the grid).  ``kernel``: "auto"
+    or "tile" (the same kernel).  ``pv``: precision of P in P . V --
+    "auto" (P's residual added in the tiles that need it), "split" (in every
+    tile) or "single" (one rounding of P).  ``workspace`` (a
     uint8 device tensor of ``pa_prefill_workspace_bytes(desc)`` bytes) is
     allocated per call when not given.  Returns ``out``."""
     import torch
@@ -243,7 +245,8 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens,
         num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=block_size,
         max_blocks_per_seq=block_tables.shape[1], num_blocks=num_blocks,
         dtype=_dtype_code(q), total_q=total_q, max_q_len=max_q_len,
-        max_context_len=max_context_len, kernel=_PREFILL_KERNELS[kernel])
+        max_context_len=max_context_len, kernel=_PREFILL_KERNELS[kernel],
+        pv=_PREFILL_PV[pv])
     _out_mode(desc, out, q.dtype)
     need = lib.pa_prefill_workspace_bytes(ctypes.byref(desc))
     if workspace is None:

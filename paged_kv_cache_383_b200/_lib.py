@@ -72,10 +72,13 @@ class pa_prefill_desc(ctypes.Structure):
         ("max_context_len", ctypes.c_int),
         ("kernel", ctypes.c_int),
         ("out_fp32", ctypes.c_int),
+        ("pv", ctypes.c_int),
     ]
 
 
-PA_PREFILL_AUTO, PA_PREFILL_TILE, PA_PREFILL_KEYS = 0, 1, 2
+PA_PREFILL_AUTO, PA_PREFILL_TILE = 0, 1
+# pa_prefill_pv
+PA_PV_AUTO, PA_PV_SPLIT, PA_PV_SINGLE = 0, 1, 2
 
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int32

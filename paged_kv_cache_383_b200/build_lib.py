@@ -1,9 +1,13 @@
 """Build libpagedkv.so in place with nvcc for sm_100a.
 
-Usage: python -m paged_kv_cache_383_b200.build_lib [--verbose]
+Each source compiles to its own object (in parallel) under ``_build/``; the
+objects are then linked into one shared library.
+
+Usage: python -m paged_kv_cache_383_b200.build_lib [--verbose] [--ptxas]
 """
 from __future__ import annotations
 
+import concurrent.futures as cf
 import os
 import shutil
 import subprocess
@@ -14,10 +18,13 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libpagedkv.so")
+OBJ_DIR = os.path.join(HERE, "_build")
 
 SOURCES = ["status.cpp", "block_manager.cpp", "cache_ops.cu", "decode.cu",
            "prefill.cu", "probe.cu", "swap.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3,-Wall",
+         "--split-compile=0"]
 
 
 def nvcc() -> str:
@@ -26,6 +33,24 @@ def nvcc() -> str:
         if cand and os.path.exists(cand):
             return cand
     raise RuntimeError("nvcc not found")
+
+
+def _compile(src: str, ptxas_verbose: bool, verbose: bool) -> str:
+    obj = os.path.join(OBJ_DIR, os.path.basename(src) + ".o")
+    cmd = [nvcc(), *ARCH, *FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src,
+           "-o", obj + ".tmp"]
+    if ptxas_verbose:
+        cmd.insert(1, "-Xptxas=-v")
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError(f"nvcc failed on {src}:\n" + res.stdout +
+                           res.stderr)
+    if verbose or ptxas_verbose:
+        sys.stdout.write(res.stdout + res.stderr)
+    os.replace(obj + ".tmp", obj)
+    return obj
 
 
 def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
@@ -37,18 +62,17 @@ def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
     if (os.path.exists(LIB) and os.path.getmtime(LIB) >= newest
             and not ptxas_verbose):
         return LIB
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17",
-           "-Xcompiler", "-fPIC,-O3,-Wall", "-shared",
-           "-I", INCLUDE, "-I", CSRC, "-o", LIB + ".tmp", *srcs]
-    if ptxas_verbose:
-        cmd.insert(1, "-Xptxas=-v")
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    workers = max(1, min(len(srcs), os.cpu_count() or 1))
+    with cf.ThreadPoolExecutor(workers) as pool:
+        objs = list(pool.map(lambda s: _compile(s, ptxas_verbose, verbose),
+                             srcs))
+    cmd = [nvcc(), *ARCH, "-shared", "-o", LIB + ".tmp", *objs]
     if verbose:
         print(" ".join(cmd), flush=True)
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
-    if verbose or ptxas_verbose:
-        sys.stdout.write(res.stdout + res.stderr)
+        raise RuntimeError("nvcc link failed:\n" + res.stdout + res.stderr)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

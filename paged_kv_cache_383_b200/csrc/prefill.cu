@@ -35,8 +35,10 @@
 //     keep the online softmax in registers (no shuffles: a row is one
 //     thread), rescale O in tensor memory only when the running maximum
 //     grows by more than 2^8 (the final division uses the same reference,
-//     so the result is unchanged), and store P with tcgen05.st as a 16-bit
-//     rounded part plus its residual so P . V keeps ~16 mantissa bits.
+//     so the result is unchanged), and store P with tcgen05.st as 16-bit
+//     values.  In the tiles where some row may end with a key of weight
+//     above 1/16 they also store P's residual (P minus its rounding), and a
+//     second MMA adds residual . V, so those weights keep ~16 bits.
 //   * With at most 64 query rows per KV head (a few new tokens), a
 //     compile-time variant spreads the rows over all four softmax warps,
 //     8 or 16 per lane quarter, and reads S / writes P / reads O with the
@@ -75,6 +77,15 @@ constexpr int kVStages = 2;     // V ring depth
 constexpr int kThreads = 192;   // producer, MMA, 4 softmax warps
 constexpr int kTmemCols = 256;  // S/P: cols [0, 128), O: cols [128, 128 + D)
 constexpr float kRescaleLog2 = 8.f;
+// P . V runs on 16-bit P.  A single rounding of P moves each weight by up to
+// 2^-8 of itself (bf16), which on a row whose weight sits on a few keys can
+// move the output by more than the 2e-3 tolerance.  So P is also split into a
+// rounded part and its residual, and a second MMA adds residual . V, for every
+// tile in which some row has a key with p > l / kSplitInv, where l is the
+// row's running sum including this tile: such a key's final weight may exceed
+// 1/kSplitInv.  Keys of the other tiles each end with a weight below
+// 1/kSplitInv, and their rounding errors, of either sign, average out.
+constexpr float kSplitInv = 16.f;
 
 // Tensor-memory access shapes with four threads per lane, used when at most
 // 32 query rows are real.  16x256b: thread t gets lanes t/4 and t/4 + 8 of
@@ -143,6 +154,7 @@ struct PrefillArgs {
   int max_context_len;
   int total_q;
   int out_f32;  // 1: out is float32 (the value before the cast to T)
+  int pv_split;  // pa_prefill_pv: 0 per tile as needed, 1 always, 2 never
 };
 
 // barriers: q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
@@ -164,8 +176,9 @@ struct Layout {
   static constexpr int kOffK = kOffQ + kQBytes;
   static constexpr int kOffV = kOffK + kKStages * kKVTile;
   static constexpr int kOffBars = kOffV + kVStages * kKVTile;
-  // 1024 bytes of slack for aligning the base, then the layout above.
-  static constexpr size_t kSmemBytes = 1024 + kOffBars + kNumBars * 8 + 16;
+  // 1024 bytes of slack for aligning the base, then the layout above; after
+  // the barriers, the tensor-memory address word and two residual votes.
+  static constexpr size_t kSmemBytes = 1024 + kOffBars + kNumBars * 8 + 32;
 };
 
 template <typename T, int BS, int G, int D, int RQ>
@@ -205,6 +218,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t done = o_ready0 + 16;
   uint32_t* tmem_slot =
       reinterpret_cast<uint32_t*>(smem + kOffBars + kNumBars * 8);
+  // Residual votes of P buffer i: a softmax warp whose rows need P's
+  // residual in tile t stores t + 1 into word t & 1 before it arrives on
+  // p_full, and the MMA issuer reads the word after that barrier; a stale
+  // word holds t - 1 or less, so the words never need clearing.
+  volatile uint32_t* pv_vote = tmem_slot + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // CTAs start in the order x (KV head), y, z.  y counts query tiles from
@@ -266,6 +284,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     dev::mbar_init(done, 4);
     dev::fence_mbar_init();
+    pv_vote[0] = 0u;
+    pv_vote[1] = 0u;
   }
   bad = __syncthreads_or(bad);
   if (bad) {
@@ -378,8 +398,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         dev::tc_fence_after();
         const uint32_t vt = vring + (t % kVStages) * kKVTile;
         const uint32_t pt = s_tmem + (t & 1) * kKeys;
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {  // P rounded part, residual
+        const int parts =
+            a.pv_split == 1 ||
+                    (a.pv_split == 0 &&
+                     pv_vote[t & 1] == static_cast<uint32_t>(t) + 1u)
+                ? 2
+                : 1;
+        for (int part = 0; part < parts; ++part) {  // P rounded, residual
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk) {
             // V as the MN-major B operand: 64-wide d halves kTileHalf apart,
@@ -512,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       // sa[4k + 2x + e]: row x, key 8k + 2 c4 + e.
       float sv[kR][16];
       float factor[kR];
-      bool grow = false;
+      bool grow = false, want = false;
 #pragma unroll
       for (int x = 0; x < kR; ++x) {
 #pragma unroll
@@ -553,7 +578,15 @@ __global__ void __launch_bounds__(kThreads, 2)
           l4[k & 3] += sv[x][k];
         }
         l[x] += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+        // Residual vote, as in the one-row-per-thread layout: the row's sum
+        // so far is spread over its four threads.
+        if (a.pv_split == 0) {
+          float lr = l[x] + __shfl_xor_sync(0xffffffffu, l[x], 1);
+          lr += __shfl_xor_sync(0xffffffffu, lr, 2);
+          want |= valid[x] && dev::fast_exp2(mx - m_ref[x]) * kSplitInv > lr;
+        }
       }
+      const bool split = __any_sync(0xffffffffu, want || a.pv_split == 1);
       if (__any_sync(0xffffffffu, grow)) {
         ok = wait_pv(j - 1);
         if (!ok) break;
@@ -584,10 +617,14 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int x = 0; x < 2; ++x) {
             if (x < kR) {
               const uint32_t w = M::pack(sv[x][2 * k], sv[x][2 * k + 1]);
-              const float2 hf = M::unpack(w);
               hw[2 * k + x] = w;
-              lw[2 * k + x] =
-                  M::pack(sv[x][2 * k] - hf.x, sv[x][2 * k + 1] - hf.y);
+              if (split) {
+                const float2 hf = M::unpack(w);
+                lw[2 * k + x] =
+                    M::pack(sv[x][2 * k] - hf.x, sv[x][2 * k + 1] - hf.y);
+              } else {
+                lw[2 * k + x] = 0u;
+              }
             } else {
               hw[2 * k + x] = 0u;
               lw[2 * k + x] = 0u;
@@ -595,12 +632,15 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         const uint32_t pa = s_tmem + (j & 1) * kKeys + lane_off;
         tmem_st16x128_x8(pa, hw);
-        tmem_st16x128_x8(pa + kKeys / 2, lw);
+        if (a.pv_split != 2) tmem_st16x128_x8(pa + kKeys / 2, lw);
         dev::tmem_st_wait();
       }
       dev::tc_fence_before();
       __syncwarp();
-      if (lane == 0) dev::mbar_arrive(p_full0 + 8 * (j & 1));
+      if (lane == 0) {
+        if (split) pv_vote[j & 1] = static_cast<uint32_t>(j) + 1u;
+        dev::mbar_arrive(p_full0 + 8 * (j & 1));
+      }
     }
     // Epilogue: the row sums over the four threads, O / l -> out.
     float inv[kR];
@@ -749,6 +789,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) +
            ((l8[4] + l8[5]) + (l8[6] + l8[7]));
     }
+    // Does a key of this tile need P's residual?  Its p is at most
+    // 2^(mx - m_ref); it needs it if that can exceed l / kSplitInv.
+    const bool split = __any_sync(
+        0xffffffffu,
+        a.pv_split == 1 ||
+            (a.pv_split == 0 && valid &&
+             dev::fast_exp2(mx - m_ref) * kSplitInv > l));
     if (__any_sync(0xffffffffu, factor != 1.f)) {
       // O must hold P(j-1).V before it is rescaled (P(j).V is not issued
       // until this warp arrives on p_full below).
@@ -766,24 +813,36 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       dev::tmem_st_wait();
     }
-    // P over S(j) in its tensor-memory buffer: rounded part, then residual.
+    // P over S(j) in its tensor-memory buffer: rounded part, then residual
+    // (zeros when this warp's rows need none: another warp's rows may).
     {
       uint32_t hw[kKeys / 2], lw[kKeys / 2];
+      if (split) {
 #pragma unroll
-      for (int e = 0; e < kKeys / 2; ++e) {
-        const float p0 = sv[2 * e], p1 = sv[2 * e + 1];
-        hw[e] = M::pack(p0, p1);
-        const float2 hf = M::unpack(hw[e]);
-        lw[e] = M::pack(p0 - hf.x, p1 - hf.y);
+        for (int e = 0; e < kKeys / 2; ++e) {
+          const float p0 = sv[2 * e], p1 = sv[2 * e + 1];
+          hw[e] = M::pack(p0, p1);
+          const float2 hf = M::unpack(hw[e]);
+          lw[e] = M::pack(p0 - hf.x, p1 - hf.y);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < kKeys / 2; ++e) {
+          hw[e] = M::pack(sv[2 * e], sv[2 * e + 1]);
+          lw[e] = 0u;
+        }
       }
       const uint32_t pa = s_tmem + (j & 1) * kKeys + lane_off;
       dev::tmem_st32u(pa, hw);
-      dev::tmem_st32u(pa + kKeys / 2, lw);
+      if (a.pv_split != 2) dev::tmem_st32u(pa + kKeys / 2, lw);
       dev::tmem_st_wait();
     }
     dev::tc_fence_before();
     __syncwarp();
-    if (lane == 0) dev::mbar_arrive(p_full0 + 8 * (j & 1));
+    if (lane == 0) {
+      if (split) pv_vote[j & 1] = static_cast<uint32_t>(j) + 1u;
+      dev::mbar_arrive(p_full0 + 8 * (j & 1));
+    }
   }
   // Epilogue: O / l -> out[token, query head].
   if (ok && !idle) ok = wait_pv(n_tiles - 1);
@@ -820,577 +879,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else if (!ok) {
     dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
   }
-  dev::tc_fence_before();
-  __syncwarp();
-  if (lane == 0) dev::mbar_arrive(done);
-}
-
-// ---------------------------------------------------------------------------
-// Few new tokens per sequence (speculative verification, decode-like chunks):
-// the keys go on the MMA's M side.
-//
-// With q_len * G <= 32 query rows per KV head, the tile above would compute
-// 128 rows to use at most 32.  Here the roles of queries and keys swap:
-//     S^T = K Q^T      (M = 128 keys, N = 32 query rows, K = head_dim)
-//     O^T += V^T P^T   (M = head_dim, N = 32 query rows, K = 128 keys)
-// so every row the tensor cores compute is a real key or a real output
-// dimension.  Tensor memory holds S^T (one key per lane) and O^T (one output
-// dimension per lane); P^T goes through shared memory, as the K-major B
-// operand.  The softmax runs over lanes, so the per-row maximum of a tile is
-// combined across the four softmax warps through shared memory, behind an
-// mbarrier (bounded waits only).  Each thread keeps partial row sums for its
-// own keys; they are rescaled with the row maximum like O and summed across
-// threads once, in the epilogue.
-//
-// The CTA is persistent: it serves (KV head, sequence) units u = blockIdx.x,
-// blockIdx.x + gridDim.x, ... in the longest-first order, one CTA per SM
-// (about 227 KB of shared memory: 3 K and 3 V stages of 128 keys).  The
-// producer streams straight from one unit into the next; Q and O are double
-// buffered per unit, so the epilogue of one unit overlaps the next unit's
-// first tiles.
-//
-// Measured (4 drafts x 256 sequences, Llama-3-70B heads): 2.96 TB/s of K/V
-// against 4.78 for the tile kernel, which therefore stays the automatic
-// choice.  With one CTA per SM only four softmax warps are in flight, each
-// issuing about 1,500 instructions per 128-key tile (row maxima across
-// lanes, 64 sixteen-bit P^T stores) at a quarter of an instruction per
-// cycle; the tensor pipe is 8 % busy.  Two softmax warpgroups taking
-// alternate tiles, or a P^T layout that takes 16-byte stores, are the next
-// steps for this kernel.
-constexpr int kVerKeys = 128;                  // keys per tile (MMA M)
-constexpr int kVerRows = 32;                   // query rows (MMA N)
-constexpr int kVerKStages = 3;
-constexpr int kVerVStages = 3;
-constexpr int kVerHalf = kVerKeys * 128;       // 16 KB: 128 keys x 64 dims
-constexpr int kVerTile = 2 * kVerHalf;         // one K or V tile, D = 128
-constexpr int kVerQBuf = 2 * kVerRows * 128;   // 8 KB: Q rows, two halves
-constexpr int kVerPPart = 2 * kVerRows * 128;  // 8 KB: P^T, two key halves
-constexpr int kVerTmemCols = 4 * kVerRows;     // S^T x2, O^T x2
-// barriers: q_full[2], q_empty[2], k_full[3], k_empty[3], v_full[3],
-// v_empty[3], s_full[2], s_free[2], p_full, pv_done, o_free[2], red_full[2],
-// red_l_full, done
-constexpr int kVerNumBars = 2 + 2 + 2 * kVerKStages + 2 * kVerVStages + 2 + 2 +
-                            1 + 1 + 2 + 2 + 1 + 1;
-struct VerLayout {
-  static constexpr int kOffK = 0;
-  static constexpr int kOffV = kOffK + kVerKStages * kVerTile;
-  static constexpr int kOffQ = kOffV + kVerVStages * kVerTile;
-  static constexpr int kOffP = kOffQ + 2 * kVerQBuf;
-  static constexpr int kOffRedM = kOffP + 2 * kVerPPart;  // [2][4][rows]
-  static constexpr int kOffRedL = kOffRedM + 2 * 4 * kVerRows * 4;
-  static constexpr int kOffBars = kOffRedL + 4 * kVerRows * 4;
-  static constexpr size_t kSmemBytes = 1024 + kOffBars + kVerNumBars * 8 + 16;
-};
-static_assert(VerLayout::kSmemBytes <= 232448, "verify kernel shared memory");
-
-// A (KV head, sequence) unit, resolved identically by every role.
-struct VerUnit {
-  int b, kvh, L, q_len, q0, n_tiles, n_pages;
-};
-
-template <int BS, int G>
-__device__ __forceinline__ VerUnit ver_unit(const PrefillArgs& a, int u,
-                                            bool report) {
-  VerUnit v;
-  v.kvh = u % a.num_kv_heads;
-  v.b = a.order[u / a.num_kv_heads];
-  v.L = a.context_lens[v.b];
-  v.q0 = a.query_start[v.b];
-  v.q_len = a.query_start[v.b + 1] - v.q0;
-  v.n_tiles = 0;
-  v.n_pages = 0;
-  if (v.L < 0 || v.L > a.max_blocks_per_seq * BS || v.L > a.max_context_len ||
-      v.q_len < 0 || v.q_len > v.L || v.q0 < 0 || v.q0 + v.q_len > a.total_q ||
-      v.q_len * G > kVerRows) {
-    if (report && v.kvh == 0) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
-    return v;
-  }
-  if (v.q_len == 0) return v;
-  v.n_tiles = (v.L + kVerKeys - 1) / kVerKeys;
-  v.n_pages = (v.L + BS - 1) / BS;
-  return v;
-}
-
-// 16-bit element (row r, key k) of a K-major, 128-byte-swizzled operand with
-// kVerRows rows and 128 keys held as two 64-key halves.
-__device__ __forceinline__ uint32_t ver_p_addr(uint32_t base, int r, int k) {
-  const int kk = k & 63;
-  return base + (k >> 6) * (kVerRows * 128) + r * 128 +
-         ((((kk >> 3) ^ (r & 7))) << 4) + (kk & 7) * 2;
-}
-
-// A float as a signed integer with the same order (for finite values and
-// +-inf): non-negative floats keep their bits, negative ones flip the
-// magnitude bits.  The map is its own inverse.
-__device__ __forceinline__ int float_to_ordered(float x) {
-  const int b = __float_as_int(x);
-  return b ^ ((b >> 31) & 0x7fffffff);
-}
-__device__ __forceinline__ float ordered_to_float(int k) {
-  return __int_as_float(k ^ ((k >> 31) & 0x7fffffff));
-}
-
-__device__ __forceinline__ void st_shared_u16(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(
-                   static_cast<unsigned short>(v & 0xffffu))
-               : "memory");
-}
-
-template <typename T, int BS, int G>
-__global__ void __launch_bounds__(kThreads, 1)
-    verify_kernel(const __grid_constant__ CUtensorMap qmap,
-                  const __grid_constant__ CUtensorMap kmap,
-                  const __grid_constant__ CUtensorMap vmap,
-                  const PrefillArgs a, int num_units) {
-  constexpr int N = kVerRows;
-  constexpr int kPages = kVerKeys / BS;  // pages per tile
-  constexpr bool kBf16 = std::is_same<T, __nv_bfloat16>::value;
-  using M = dev::Mma<T>;
-  using Lay = VerLayout;
-  extern __shared__ uint8_t smem_dyn[];
-  uint8_t* smem =
-      smem_dyn + ((1024u - (dev::smem_u32(smem_dyn) & 1023u)) & 1023u);
-  const uint32_t base = dev::smem_u32(smem);
-  const uint32_t kring = base + Lay::kOffK;
-  const uint32_t vring = base + Lay::kOffV;
-  const uint32_t qbuf = base + Lay::kOffQ;
-  const uint32_t pbuf = base + Lay::kOffP;
-  float* red_m = reinterpret_cast<float*>(smem + Lay::kOffRedM);
-  float* red_l = reinterpret_cast<float*>(smem + Lay::kOffRedL);
-  const uint32_t bars = base + Lay::kOffBars;
-  const uint32_t q_full0 = bars;
-  const uint32_t q_empty0 = q_full0 + 16;
-  const uint32_t k_full0 = q_empty0 + 16;
-  const uint32_t k_empty0 = k_full0 + 8 * kVerKStages;
-  const uint32_t v_full0 = k_empty0 + 8 * kVerKStages;
-  const uint32_t v_empty0 = v_full0 + 8 * kVerVStages;
-  const uint32_t s_full0 = v_empty0 + 8 * kVerVStages;
-  const uint32_t s_free0 = s_full0 + 16;
-  const uint32_t p_full = s_free0 + 16;
-  const uint32_t pv_done = p_full + 8;
-  const uint32_t o_free0 = pv_done + 8;
-  const uint32_t red_full0 = o_free0 + 16;
-  const uint32_t red_l_full = red_full0 + 16;
-  const uint32_t done = red_l_full + 8;
-  uint32_t* tmem_slot =
-      reinterpret_cast<uint32_t*>(smem + Lay::kOffBars + kVerNumBars * 8);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-  if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
-      dev::mbar_init(q_full0 + 8 * i, 1);
-      dev::mbar_init(q_empty0 + 8 * i, 1);
-      dev::mbar_init(s_full0 + 8 * i, 1);
-      dev::mbar_init(s_free0 + 8 * i, 4);
-      dev::mbar_init(o_free0 + 8 * i, 4);
-      dev::mbar_init(red_full0 + 8 * i, 4);
-    }
-    for (int s = 0; s < kVerKStages; ++s) {
-      dev::mbar_init(k_full0 + 8 * s, 1);
-      dev::mbar_init(k_empty0 + 8 * s, 1);
-    }
-    for (int s = 0; s < kVerVStages; ++s) {
-      dev::mbar_init(v_full0 + 8 * s, 1);
-      dev::mbar_init(v_empty0 + 8 * s, 1);
-    }
-    dev::mbar_init(p_full, 4);
-    dev::mbar_init(pv_done, 1);
-    dev::mbar_init(red_l_full, 4);
-    dev::mbar_init(done, 4);
-    dev::fence_mbar_init();
-  }
-  if (warp == 1) {
-    dev::tmem_alloc(dev::smem_u32(tmem_slot), kVerTmemCols);
-    dev::tmem_relinquish();
-  }
-  dev::tc_fence_before();
-  __syncthreads();
-  dev::tc_fence_after();
-  const uint32_t tbase = *tmem_slot;
-  // Tensor memory: S^T buffers at columns [0, N) and [N, 2N), O^T buffers
-  // at [2N, 3N) and [3N, 4N).
-  const uint32_t s_tmem = tbase;
-  const uint32_t o_tmem = tbase + 2 * N;
-  // The order kernel (and whatever ran before it) must be done before the
-  // order, the lengths, the caches or the outputs are touched.
-  dev::pdl_wait();
-
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      dev::prefetch_tmap(&qmap);
-      dev::prefetch_tmap(&kmap);
-      dev::prefetch_tmap(&vmap);
-      int g = 0, ui = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-        const VerUnit v = ver_unit<BS, G>(a, u, true);
-        if (v.n_tiles == 0) continue;
-        const int32_t* row =
-            a.block_tables + static_cast<int64_t>(v.b) * a.max_blocks_per_seq;
-        auto page_id = [&](int page) -> int32_t {
-          const int32_t p = __ldg(row + (page < v.n_pages ? page : 0));
-          if (p < 0 || p >= a.num_blocks) {
-            dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
-            return 0;
-          }
-          return p;
-        };
-        const int qb = ui & 1;
-        if (ui >= 2 && !dev::mbar_wait(q_empty0 + 8 * qb, ((ui >> 1) - 1) & 1)) {
-          ok = false;
-          break;
-        }
-        dev::mbar_arrive_expect_tx(q_full0 + 8 * qb, kVerQBuf);
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-          dev::tma_load_3d(qbuf + qb * kVerQBuf + h * (N * 128), &qmap, 64 * h,
-                           v.kvh * G, v.q0, q_full0 + 8 * qb);
-        auto load = [&](int gt, int t, bool is_v,
-                        const int32_t (&ids)[kPages]) -> bool {
-          const int ns = is_v ? kVerVStages : kVerKStages;
-          const int s = gt % ns;
-          const uint32_t empty = (is_v ? v_empty0 : k_empty0) + 8 * s;
-          if (gt >= ns && !dev::mbar_wait(empty, ((gt / ns) - 1) & 1))
-            return false;
-          const uint32_t full = (is_v ? v_full0 : k_full0) + 8 * s;
-          dev::mbar_arrive_expect_tx(full, kVerTile);
-          const uint32_t dst = (is_v ? vring : kring) + s * kVerTile;
-          const CUtensorMap* map = is_v ? &vmap : &kmap;
-#pragma unroll
-          for (int p = 0; p < kPages; ++p) {
-            const int y = (ids[p] * a.num_kv_heads + v.kvh) * BS;
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-              dev::tma_load_2d(dst + h * kVerHalf + p * BS * 128, map, 64 * h,
-                               y, full);
-          }
-          (void)t;
-          return true;
-        };
-        // Block ids are read a tile ahead, so their latency overlaps the
-        // loads of the tile before.
-        int32_t cur[kPages], nxt[kPages], prv[kPages];
-#pragma unroll
-        for (int p = 0; p < kPages; ++p) nxt[p] = page_id(p);
-        for (int t = 0; t <= v.n_tiles; ++t) {
-          if (t < v.n_tiles) {
-#pragma unroll
-            for (int p = 0; p < kPages; ++p) cur[p] = nxt[p];
-            if (t + 1 < v.n_tiles) {
-#pragma unroll
-              for (int p = 0; p < kPages; ++p)
-                nxt[p] = page_id((t + 1) * kPages + p);
-            }
-          }
-          // K tile t, then V tile t-1 (needed a tile later).
-          if ((t < v.n_tiles && !load(g + t, t, false, cur)) ||
-              (t >= 1 && !load(g + t - 1, t - 1, true, prv))) {
-            ok = false;
-            break;
-          }
-#pragma unroll
-          for (int p = 0; p < kPages; ++p) prv[p] = cur[p];
-        }
-        g += v.n_tiles;
-        ++ui;
-      }
-      if (!ok) dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
-    }
-    return;
-  }
-
-  if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    bool ok = true;
-    if (lane == 0) {
-      constexpr uint32_t idesc_s =
-          dev::umma_idesc_f16(kBf16, kVerKeys, N, false, false);
-      constexpr uint32_t idesc_o =
-          dev::umma_idesc_f16(kBf16, 128, N, true, false);
-      int g = 0, ui = 0;
-      // O^T(ob) += V^T(gt) P^T(gt); the first tile of a unit overwrites O^T.
-      auto issue_pv = [&](int gt, bool first, int ob, int uidx) -> bool {
-        if (!dev::mbar_wait(p_full, gt & 1) ||
-            !dev::mbar_wait(v_full0 + 8 * (gt % kVerVStages),
-                            (gt / kVerVStages) & 1))
-          return false;
-        if (first && uidx >= 2 &&
-            !dev::mbar_wait(o_free0 + 8 * ob, ((uidx >> 1) - 1) & 1))
-          return false;
-        dev::tc_fence_after();
-        const uint32_t vt = vring + (gt % kVerVStages) * kVerTile;
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {  // P rounded part, residual
-#pragma unroll
-          for (int kk = 0; kk < kVerKeys / 16; ++kk) {
-            // V^T: the MN-major A operand (head_dim halves kVerHalf apart,
-            // 8-key groups 1024 bytes apart); P^T: K-major B, keys in two
-            // 64-key halves.
-            const uint64_t ad = dev::sw128_desc(vt + kk * 2048, kVerHalf, 1024);
-            const uint64_t bd = dev::sw128_desc(
-                pbuf + part * kVerPPart + (kk >> 2) * (N * 128) + (kk & 3) * 32,
-                16, 1024);
-            dev::umma_f16(o_tmem + ob * N, ad, bd, idesc_o,
-                          (first && part == 0 && kk == 0) ? 0u : 1u);
-          }
-        }
-        dev::umma_commit(pv_done);
-        dev::umma_commit(v_empty0 + 8 * (gt % kVerVStages));
-        return true;
-      };
-      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-        const VerUnit v = ver_unit<BS, G>(a, u, false);
-        if (v.n_tiles == 0) continue;
-        const int qb = ui & 1, ob = ui & 1;
-        if (!dev::mbar_wait(q_full0 + 8 * qb, (ui >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-        const uint32_t qs = qbuf + qb * kVerQBuf;
-        for (int t = 0; t < v.n_tiles; ++t) {
-          const int gt = g + t, s = gt % kVerKStages;
-          // S^T buffer gt & 1 is free once the softmax warps read S^T(gt-2).
-          if (!dev::mbar_wait(k_full0 + 8 * s, (gt / kVerKStages) & 1) ||
-              (gt >= 2 &&
-               !dev::mbar_wait(s_free0 + 8 * (gt & 1), ((gt >> 1) - 1) & 1))) {
-            ok = false;
-            break;
-          }
-          dev::tc_fence_after();
-          const uint32_t kt = kring + s * kVerTile;
-#pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk) {
-            const int h = kk >> 2, k4 = kk & 3;
-            const uint64_t ad =
-                dev::sw128_desc(kt + h * kVerHalf + k4 * 32, 16, 1024);
-            const uint64_t bd =
-                dev::sw128_desc(qs + h * (N * 128) + k4 * 32, 16, 1024);
-            dev::umma_f16(s_tmem + (gt & 1) * N, ad, bd, idesc_s,
-                          kk > 0 ? 1u : 0u);
-          }
-          dev::umma_commit(s_full0 + 8 * (gt & 1));
-          dev::umma_commit(k_empty0 + 8 * s);
-          if (t == v.n_tiles - 1) dev::umma_commit(q_empty0 + 8 * qb);
-          if (t >= 1 && !issue_pv(gt - 1, t == 1, ob, ui)) {
-            ok = false;
-            break;
-          }
-        }
-        if (ok) ok = issue_pv(g + v.n_tiles - 1, v.n_tiles == 1, ob, ui);
-        g += v.n_tiles;
-        ++ui;
-      }
-      if (!ok) dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
-      // Release tensor memory only after the softmax warps are done with it.
-      if (!dev::mbar_wait(done, 0))
-        dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
-    }
-    __syncwarp();
-    dev::tc_fence_after();
-    dev::tmem_dealloc(tbase, kVerTmemCols);
-    return;
-  }
-
-  // ---------------- softmax warps (thread = key, then output dimension) -----
-  const int quarter = warp & 3;  // tensor-memory lane quarter of this warp
-  const int kl = quarter * 32 + lane;  // key of a tile / dimension of O^T
-  const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-  const float c = a.scale_log2;
-  bool ok = true;
-  // Every wait below is made warp-uniform: the tcgen05 loads and stores are
-  // warp-collective.
-  auto wait_all = [&](uint32_t bar, uint32_t parity) {
-    return __all_sync(0xffffffffu, dev::mbar_wait(bar, parity));
-  };
-  int g = 0, ui = 0;
-  for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-    const VerUnit v = ver_unit<BS, G>(a, u, false);
-    if (v.n_tiles == 0) continue;
-    const int ob = ui & 1;
-    const int R = v.q_len * G;  // real query rows (<= N)
-    float m_ref[N], lp[N];
-#pragma unroll
-    for (int r = 0; r < N; ++r) {
-      m_ref[r] = -INFINITY;
-      lp[r] = 0.f;
-    }
-    for (int t = 0; t < v.n_tiles; ++t) {
-      const int gt = g + t;
-      if (!(ok = wait_all(s_full0 + 8 * (gt & 1), (gt >> 1) & 1))) break;
-      dev::tc_fence_after();
-      float sv[N];
-      dev::tmem_ld32(s_tmem + (gt & 1) * N + lane_off, sv);
-      dev::tmem_ld_wait();
-      dev::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive(s_free0 + 8 * (gt & 1));
-      // Causal mask: key kp is seen by new token i (row r = i * G + h) when
-      // kp <= L - q_len + i; rows past the real ones see the whole context.
-      // Keys past the context (unwritten slots may hold NaN) never pass.
-      const int kp = t * kVerKeys + kl;
-      const int lim = kp - (v.L - v.q_len);  // token index needed
-#pragma unroll
-      for (int r = 0; r < N; ++r) {
-        const bool vis = r < R ? (r / G) >= lim : kp < v.L;
-        if (!vis) sv[r] = -INFINITY;
-      }
-      // Tile maximum of each row: over this warp's 32 keys with one integer
-      // max-reduction per row (floats mapped to order-preserving integers),
-      // then over the four warps through shared memory.
-      float wm[N];
-#pragma unroll
-      for (int r = 0; r < N; ++r)
-        wm[r] = ordered_to_float(
-            __reduce_max_sync(0xffffffffu, float_to_ordered(sv[r])));
-      float* rm = red_m + (gt & 1) * (4 * N);
-      if (lane == 0) {
-#pragma unroll
-        for (int r = 0; r < N; r += 4)
-          *reinterpret_cast<float4*>(rm + quarter * N + r) =
-              make_float4(wm[r], wm[r + 1], wm[r + 2], wm[r + 3]);
-      }
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive(red_full0 + 8 * (gt & 1));
-      if (!(ok = wait_all(red_full0 + 8 * (gt & 1), (gt >> 1) & 1))) break;
-      float factor[N];
-      bool rescale = false;
-#pragma unroll
-      for (int r = 0; r < N; r += 4) {
-        float4 x[4];
-#pragma unroll
-        for (int w = 0; w < 4; ++w)
-          x[w] = *reinterpret_cast<const float4*>(rm + w * N + r);
-        const float mx[4] = {
-            fmaxf(fmaxf(x[0].x, x[1].x), fmaxf(x[2].x, x[3].x)) * c,
-            fmaxf(fmaxf(x[0].y, x[1].y), fmaxf(x[2].y, x[3].y)) * c,
-            fmaxf(fmaxf(x[0].z, x[1].z), fmaxf(x[2].z, x[3].z)) * c,
-            fmaxf(fmaxf(x[0].w, x[1].w), fmaxf(x[2].w, x[3].w)) * c};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          factor[r + e] = 1.f;
-          if (t == 0) {
-            m_ref[r + e] = mx[e];  // O^T is overwritten by this unit's P.V
-          } else if (mx[e] > m_ref[r + e] + kRescaleLog2) {
-            factor[r + e] = dev::fast_exp2(m_ref[r + e] - mx[e]);
-            m_ref[r + e] = mx[e];
-            lp[r + e] *= factor[r + e];
-            rescale = true;
-          }
-        }
-      }
-      // P = 2^(s * c - m_ref) (0 for masked keys); partial row sums.
-#pragma unroll
-      for (int r = 0; r < N; ++r) {
-        sv[r] = dev::fast_exp2(fmaf(sv[r], c, -m_ref[r]));
-        lp[r] += sv[r];
-      }
-      // P^T's buffer is free, and O^T holds P(gt-1).V, once that MMA is done.
-      if (gt >= 1 && !(ok = wait_all(pv_done, (gt - 1) & 1))) break;
-      if (rescale) {  // the same for every thread: the maxima are shared
-        dev::tc_fence_after();
-        float ov[N];
-        dev::tmem_ld32(o_tmem + ob * N + lane_off, ov);
-        dev::tmem_ld_wait();
-#pragma unroll
-        for (int r = 0; r < N; ++r) ov[r] *= factor[r];
-        dev::tmem_st32(o_tmem + ob * N + lane_off, ov);
-        dev::tmem_st_wait();
-      }
-      if ((t + 1) * kVerKeys > v.L) {
-        // Last tile: V rows of keys past the context get P = 0, but 0 * NaN
-        // is NaN in the MMA, so they are cleared once the tile has landed
-        // (P.V, the stage's next reader, waits for p_full).
-        if (!(ok = wait_all(v_full0 + 8 * (gt % kVerVStages),
-                            (gt / kVerVStages) & 1)))
-          break;
-        if (kp >= v.L) {
-          const uint32_t vt = vring + (gt % kVerVStages) * kVerTile;
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-              dev::st_shared_zero16(vt + h * kVerHalf + kl * 128 + ch * 16);
-        }
-      }
-      // P^T for this thread's key: a rounded 16-bit part and its residual.
-#pragma unroll
-      for (int r = 0; r < N; r += 2) {
-        const uint32_t hw = M::pack(sv[r], sv[r + 1]);
-        const float2 hf = M::unpack(hw);
-        const uint32_t lw = M::pack(sv[r] - hf.x, sv[r + 1] - hf.y);
-        st_shared_u16(ver_p_addr(pbuf, r, kl), hw);
-        st_shared_u16(ver_p_addr(pbuf, r + 1, kl), hw >> 16);
-        st_shared_u16(ver_p_addr(pbuf + kVerPPart, r, kl), lw);
-        st_shared_u16(ver_p_addr(pbuf + kVerPPart, r + 1, kl), lw >> 16);
-      }
-      dev::fence_proxy_async_smem();  // visible to the tensor cores
-      dev::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive(p_full);
-    }
-    if (!ok) break;
-    const int glast = g + v.n_tiles - 1;
-    // Row sums: this thread's keys, then the warp, then the four warps.
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-      for (int r = 0; r < N; ++r)
-        lp[r] += __shfl_xor_sync(0xffffffffu, lp[r], o);
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int r = 0; r < N; r += 4)
-        *reinterpret_cast<float4*>(red_l + quarter * N + r) =
-            make_float4(lp[r], lp[r + 1], lp[r + 2], lp[r + 3]);
-    }
-    __syncwarp();
-    if (lane == 0) dev::mbar_arrive(red_l_full);
-    if (!(ok = wait_all(red_l_full, ui & 1))) break;
-    float inv[N];
-#pragma unroll
-    for (int r = 0; r < N; r += 4) {
-      float4 x[4];
-#pragma unroll
-      for (int w = 0; w < 4; ++w)
-        x[w] = *reinterpret_cast<const float4*>(red_l + w * N + r);
-      const float l4[4] = {(x[0].x + x[1].x) + (x[2].x + x[3].x),
-                           (x[0].y + x[1].y) + (x[2].y + x[3].y),
-                           (x[0].z + x[1].z) + (x[2].z + x[3].z),
-                           (x[0].w + x[1].w) + (x[2].w + x[3].w)};
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        inv[r + e] = l4[e] > 0.f ? 1.f / l4[e] : 0.f;
-    }
-    // Epilogue: O^T / l -> out[token, query head, dimension kl].
-    if (!(ok = wait_all(pv_done, glast & 1))) break;
-    dev::tc_fence_after();
-    float ov[N];
-    dev::tmem_ld32(o_tmem + ob * N + lane_off, ov);
-    dev::tmem_ld_wait();
-    dev::tc_fence_before();
-    __syncwarp();
-    if (lane == 0) dev::mbar_arrive(o_free0 + 8 * ob);
-#pragma unroll
-    for (int r = 0; r < N; r += 2) {
-      const uint32_t w = M::pack(ov[r] * inv[r], ov[r + 1] * inv[r + 1]);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (r + h >= R) continue;
-        const int64_t row =
-            static_cast<int64_t>(v.q0 + (r + h) / G) * a.num_q_heads +
-            v.kvh * G + (r + h) % G;
-        if (a.out_f32)
-          static_cast<float*>(a.out)[row * 128 + kl] = ov[r + h] * inv[r + h];
-        else
-          static_cast<uint16_t*>(a.out)[row * 128 + kl] =
-              static_cast<uint16_t>(h ? w >> 16 : w & 0xffffu);
-      }
-    }
-    g += v.n_tiles;
-    ++ui;
-  }
-  if (!ok) dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
   dev::tc_fence_before();
   __syncwarp();
   if (lane == 0) dev::mbar_arrive(done);
@@ -1524,58 +1012,6 @@ pa_status dispatch_shape(const pa_prefill_desc* d, const PrefillArgs& a,
              : dispatch_group<T, 32, 64, RQ>(d, a, qm, km, vm, st);
 }
 
-template <typename T, int BS, int G>
-pa_status launch_verify(const pa_prefill_desc* d, const PrefillArgs& a,
-                        const CUtensorMap& qm, const CUtensorMap& km,
-                        const CUtensorMap& vm, cudaStream_t st) {
-  auto kern = verify_kernel<T, BS, G>;
-  const size_t smem = VerLayout::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(
-      kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-      static_cast<int>(smem));
-  if (e != cudaSuccess)
-    return fail(PA_ERR_CUDA, "pa_prefill: cudaFuncSetAttribute(%zu): %s",
-                smem, cudaGetErrorString(e));
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int units = d->num_seqs * d->num_kv_heads;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(units < sms ? units : sms);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, qm, km, vm, a, units);
-  count_launch();
-  if (e == cudaSuccess) e = cudaGetLastError();
-  if (e != cudaSuccess)
-    return fail(PA_ERR_CUDA, "pa_prefill: launch failed: %s",
-                cudaGetErrorString(e));
-  return PA_OK;
-}
-
-template <typename T>
-pa_status dispatch_verify(const pa_prefill_desc* d, const PrefillArgs& a,
-                          const CUtensorMap& qm, const CUtensorMap& km,
-                          const CUtensorMap& vm, cudaStream_t st) {
-  const bool bs16 = d->block_size == 16;
-  switch (d->num_q_heads / d->num_kv_heads) {
-    case 1: return bs16 ? launch_verify<T, 16, 1>(d, a, qm, km, vm, st)
-                        : launch_verify<T, 32, 1>(d, a, qm, km, vm, st);
-    case 2: return bs16 ? launch_verify<T, 16, 2>(d, a, qm, km, vm, st)
-                        : launch_verify<T, 32, 2>(d, a, qm, km, vm, st);
-    case 4: return bs16 ? launch_verify<T, 16, 4>(d, a, qm, km, vm, st)
-                        : launch_verify<T, 32, 4>(d, a, qm, km, vm, st);
-    default: return bs16 ? launch_verify<T, 16, 8>(d, a, qm, km, vm, st)
-                         : launch_verify<T, 32, 8>(d, a, qm, km, vm, st);
-  }
-}
-
 }  // namespace
 }  // namespace pagedkv
 
@@ -1603,25 +1039,12 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
                 d->max_blocks_per_seq, d->total_q, d->max_q_len,
                 static_cast<int>(d->dtype));
   const int G = d->num_q_heads / d->num_kv_heads;
-  if (d->kernel < PA_PREFILL_AUTO || d->kernel > PA_PREFILL_KEYS)
+  if (d->kernel != PA_PREFILL_AUTO && d->kernel != PA_PREFILL_TILE)
     return fail(PA_ERR_INVALID_ARG, "pa_prefill: kernel %d", d->kernel);
   if (d->out_fp32 != 0 && d->out_fp32 != 1)
     return fail(PA_ERR_INVALID_ARG, "pa_prefill: out_fp32 %d", d->out_fp32);
-  const bool keys_fit =
-      d->head_dim == 128 &&
-      static_cast<int64_t>(d->max_q_len) * G <= pagedkv::kVerRows &&
-      static_cast<int64_t>(d->num_seqs) * d->num_kv_heads <= 0x7fffffffLL;
-  if (d->kernel == PA_PREFILL_KEYS && !keys_fit)
-    return fail(PA_ERR_UNSUPPORTED,
-                "pa_prefill: the keys-on-M kernel needs head_dim 128, "
-                "max_q_len * G <= %d and fewer than 2^31 (sequence, KV "
-                "head) units (got head_dim %d, max_q_len %d, G %d)",
-                pagedkv::kVerRows, d->head_dim, d->max_q_len, G);
-  // Automatic choice: the tile kernel.  The keys-on-M kernel computes no
-  // padding rows but runs one CTA per SM with a cross-warp row maximum per
-  // tile; measured on 4 drafts x 256 sequences it reads 2.96 TB/s of K/V
-  // against 4.78 for the tile kernel, so it runs only on request.
-  const bool use_keys = d->kernel == PA_PREFILL_KEYS;
+  if (d->pv < PA_PV_AUTO || d->pv > PA_PV_SINGLE)
+    return fail(PA_ERR_INVALID_ARG, "pa_prefill: pv %d", d->pv);
   if ((d->head_dim != 64 && d->head_dim != 128) ||
       (d->block_size != 16 && d->block_size != 32) ||
       (G != 1 && G != 2 && G != 4 && G != 8))
@@ -1658,10 +1081,8 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
   // spreads them over the four softmax warps, 8 (up to 32 rows) or 16 (up
   // to 64) per warp.
   const int64_t q_rows = static_cast<int64_t>(d->max_q_len) * G;
-  const int rq = use_keys ? 0 : q_rows <= 32 ? 8 : q_rows <= 64 ? 16 : 0;
-  const int tok = use_keys ? pagedkv::kVerRows / G
-                  : rq > 0 ? rq / G
-                           : pagedkv::kRows / G;
+  const int rq = q_rows <= 32 ? 8 : q_rows <= 64 ? 16 : 0;
+  const int tok = rq > 0 ? rq / G : pagedkv::kRows / G;
   CUtensorMap qm, km, vm;
   const uint64_t rows = static_cast<uint64_t>(d->num_blocks) *
                         d->num_kv_heads * d->block_size;
@@ -1687,6 +1108,7 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
   a.max_context_len = max_ctx;
   a.total_q = d->total_q;
   a.out_f32 = d->out_fp32;
+  a.pv_split = d->pv;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   pagedkv::prefill_order_kernel<<<1, pagedkv::kOrderThreads, 0, s>>>(
       context_lens, d->num_seqs, pagedkv::order_shift(max_ctx),
@@ -1696,10 +1118,6 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
   if (oe != cudaSuccess)
     return fail(PA_ERR_CUDA, "pa_prefill: order launch failed: %s",
                 cudaGetErrorString(oe));
-  if (use_keys)
-    return d->dtype == PA_BF16
-               ? pagedkv::dispatch_verify<__nv_bfloat16>(d, a, qm, km, vm, s)
-               : pagedkv::dispatch_verify<__half>(d, a, qm, km, vm, s);
   if (rq == 8)
     return d->dtype == PA_BF16
                ? pagedkv::dispatch_shape<__nv_bfloat16, 8>(d, a, qm, km, vm, s)

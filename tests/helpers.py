@@ -123,3 +123,35 @@ def check_strict(out32, ref, what=""):
     assert err.max() <= ATOL, f"{what}: max abs err {err.max():.3e}"
     assert rel.max() <= RTOL, f"{what}: max rel err {rel.max():.3e}"
     return float(err.max()), float(rel.max())
+
+
+def prefill_both(pkv, out, *args, **kw):
+    """pa_prefill into ``out`` (the input dtype) and, on the same inputs,
+    into a float32 tensor (the kernel's value before the output rounding);
+    returns the float32 tensor."""
+    import torch
+    out32 = torch.full(out.shape, float("nan"), dtype=torch.float32,
+                       device=out.device)
+    pkv.pa_prefill(out32, *args, **kw)
+    pkv.pa_prefill(out, *args, **kw)
+    return out32
+
+
+def check_prefill(out, out32, ref, what="", rows=None):
+    """The tolerance for a prefill output, with the output-rounding floor
+    handled as its reading prescribes: the float32 value (before the output
+    rounding) must meet the tolerance with no carve-out -- every element
+    within 2e-3, every element with |ref| >= 0.2 within 1e-2 relative -- and
+    the dtype output must be exactly its round-to-nearest-even.  So the only
+    error past 2e-3 in the dtype output is that rounding itself: up to half
+    an ulp, 2^-9 |ref| in bf16, which at |ref| >= 0.5 leaves a rounded output
+    as little as 5e-5 of room under a flat 2e-3.  ``rows`` selects the rows
+    compared (all if None)."""
+    import torch
+    assert out32.dtype == torch.float32
+    if rows is not None:
+        idx = torch.as_tensor(np.asarray(rows), device=out.device)
+        out, out32 = out.index_select(0, idx), out32.index_select(0, idx)
+    assert torch.equal(out, out32.to(out.dtype)), (
+        f"{what}: dtype output is not the rounding of the float32 value")
+    return check_strict(to_np(out32), ref, what)

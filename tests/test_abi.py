@@ -177,16 +177,18 @@ def test_prefill_kernel_choice_is_checked(pkv):
         return lib.pa_prefill(*([fake] * 7), ctypes.c_float(1.0),
                               ctypes.byref(d), None, 0, None, None)
 
-    assert call(kernel=7) == _lib.PA_ERR_INVALID_ARG
-    # keys on M: G = 4, so at most 8 new tokens per sequence; head_dim 128
-    assert call(kernel=_lib.PA_PREFILL_KEYS) == _lib.PA_ERR_UNSUPPORTED
-    assert b"keys-on-M" in lib.pa_last_error()
-    assert call(kernel=_lib.PA_PREFILL_KEYS, max_q_len=8,
-                head_dim=64) == _lib.PA_ERR_UNSUPPORTED
+    for kernel in (7, 2, -1):
+        assert call(kernel=kernel) == _lib.PA_ERR_INVALID_ARG
+        assert b"kernel" in lib.pa_last_error()
     # a valid choice gets as far as the workspace check
-    assert call(kernel=_lib.PA_PREFILL_KEYS,
-                max_q_len=8) == _lib.PA_ERR_WORKSPACE
+    assert call(kernel=_lib.PA_PREFILL_AUTO) == _lib.PA_ERR_WORKSPACE
     assert call(kernel=_lib.PA_PREFILL_TILE) == _lib.PA_ERR_WORKSPACE
+    # precision of P in P . V: auto, split or single; nothing else
+    for pv in (-1, 3):
+        assert call(pv=pv) == _lib.PA_ERR_INVALID_ARG
+        assert b"pv" in lib.pa_last_error()
+    for pv in (_lib.PA_PV_AUTO, _lib.PA_PV_SPLIT, _lib.PA_PV_SINGLE):
+        assert call(pv=pv) == _lib.PA_ERR_WORKSPACE
 
 
 def test_out_fp32_flag_is_checked(pkv):

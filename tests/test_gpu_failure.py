@@ -13,7 +13,7 @@ from oracle import attention as oa
 from paged_kv_cache_383_b200 import _lib
 from paged_kv_cache_383_b200 import workloads as wl
 
-from helpers import check_decode, to_np
+from helpers import check_decode, check_prefill, prefill_both, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -38,9 +38,9 @@ def test_wait_runs_out_and_the_context_survives(pkv):
     qs = torch.from_numpy(pin.query_start).cuda()
     err.zero_()
     out = torch.empty_like(pin.q)
-    pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl, qs,
-                   w.softmax_scale, max_q_len=int(pin.q_lens.max()),
-                   max_context_len=int(inp.lengths.max()), dev_err=err)
+    out32 = prefill_both(pkv, out, pin.q, inp.k_cache, inp.v_cache, bt, cl,
+                         qs, w.softmax_scale, max_q_len=int(pin.q_lens.max()),
+                         max_context_len=int(inp.lengths.max()), dev_err=err)
     dq = torch.randn(4, w.num_q_heads, w.head_dim,
                      device="cuda").to(pin.q.dtype)
     dout = torch.empty_like(dq)
@@ -52,7 +52,7 @@ def test_wait_runs_out_and_the_context_survives(pkv):
     kc, vc = to_np(inp.k_cache), to_np(inp.v_cache)
     ref = oa.paged_prefill(to_np(pin.q), kc, vc, inp.block_tables,
                            inp.lengths, pin.query_start, w.softmax_scale)
-    check_decode(to_np(out), ref, pin.q.dtype, "prefill after the timeout")
+    check_prefill(out, out32, ref, "prefill after the timeout")
     ref = oa.paged_decode(to_np(dq), kc, vc, inp.block_tables, inp.lengths,
                           w.softmax_scale)
     check_decode(to_np(dout), ref, dq.dtype, "decode after the timeout")

@@ -7,12 +7,15 @@ import torch
 from oracle import attention as oa
 from paged_kv_cache_383_b200 import workloads as wl
 
-from helpers import check_decode, poison_unwritten, to_np
+from helpers import (check_decode, check_prefill, poison_unwritten,
+                     prefill_both, to_np)
 
 pytestmark = pytest.mark.gpu
 
 
 def _run(pkv, pin, tables=None, err=None, kernel="auto"):
+    """pa_prefill into a dtype output and a float32 one (the value before
+    the output rounding); returns (out, out32)."""
     inp = pin.paged
     w = inp.workload
     out = torch.full_like(pin.q, float("nan"))
@@ -20,15 +23,16 @@ def _run(pkv, pin, tables=None, err=None, kernel="auto"):
                           else tables).cuda()
     cl = torch.from_numpy(inp.lengths.astype(np.int32)).cuda()
     qs = torch.from_numpy(pin.query_start).cuda()
-    pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl, qs,
-                   w.softmax_scale, max_q_len=int(max(pin.q_lens.max(), 1)),
-                   max_context_len=int(inp.lengths.max()), dev_err=err,
-                   kernel=kernel)
+    out32 = prefill_both(pkv, out, pin.q, inp.k_cache, inp.v_cache, bt, cl,
+                         qs, w.softmax_scale,
+                         max_q_len=int(max(pin.q_lens.max(), 1)),
+                         max_context_len=int(inp.lengths.max()), dev_err=err,
+                         kernel=kernel)
     torch.cuda.synchronize()
-    return out
+    return out, out32
 
 
-def _check(pin, out, what, seqs=None):
+def _check(pin, outs, what, seqs=None):
     inp = pin.paged
     ref = oa.paged_prefill(to_np(pin.q), to_np(inp.k_cache),
                            to_np(inp.v_cache), inp.block_tables, inp.lengths,
@@ -38,7 +42,7 @@ def _check(pin, out, what, seqs=None):
                                      pin.query_start[b + 1])
                            for b in (seqs if seqs is not None
                                      else range(len(pin.q_lens)))])
-    return check_decode(to_np(out)[rows], ref[rows], pin.q.dtype, what)
+    return check_prefill(*outs, ref[rows], what, rows=rows)
 
 
 @pytest.mark.parametrize("dtype", ["bfloat16", "float16"])
@@ -68,7 +72,7 @@ def test_single_token_matches_decode(pkv):
                   w.softmax_scale, max_context_len=int(inp.lengths.max()))
     torch.cuda.synchronize()
     _check(pin, out, "prefill q_len=1")
-    assert (out.float() - dec.float()).abs().max().item() <= 4e-3
+    assert (out[0].float() - dec.float()).abs().max().item() <= 4e-3
 
 
 def test_sequences_without_new_tokens(pkv):
@@ -77,7 +81,7 @@ def test_sequences_without_new_tokens(pkv):
     pin = wl.make_prefill(w, (0, 50, 0), device="cuda")
     out = _run(pkv, pin)
     _check(pin, out, "middle sequence only")
-    assert out.shape[0] == 50
+    assert out[0].shape[0] == 50
 
 
 def test_chunked_prefill_full_size_sampled(pkv):
@@ -85,7 +89,7 @@ def test_chunked_prefill_full_size_sampled(pkv):
     pin = wl.make_prefill(w, np.full(w.num_seqs, 512), device="cuda")
     out = _run(pkv, pin)
     _check(pin, out, "chunked prefill", seqs=[0, 7, 15])
-    assert torch.isfinite(out.float()).all()
+    assert torch.isfinite(out[0].float()).all()
 
 
 def test_bad_block_id_is_flagged(pkv):
@@ -163,13 +167,14 @@ def test_speculative_verify_and_rollback(pkv):
         bt, cl, lens = flow.tables_on_device(bm, ids, 16, "cuda")
         assert list(lens) == [len(k) for k in K]
         out = torch.empty_like(q)
-        pkv.pa_prefill(out, q, kc, vc, bt, cl, torch.from_numpy(qs).cuda(),
-                       scale, max_q_len=max(n_new),
-                       max_context_len=int(lens.max()))
+        out32 = prefill_both(pkv, out, q, kc, vc, bt, cl,
+                             torch.from_numpy(qs).cuda(), scale,
+                             max_q_len=max(n_new),
+                             max_context_len=int(lens.max()))
         kp, vp, tables = _contiguous_pool(K, V, bs)
         ref = oa.paged_prefill(to_np(q), kp, vp, tables, lens, qs, scale)
         torch.cuda.synchronize()
-        check_decode(to_np(out), ref, q.dtype, f"step {n_new}")
+        check_prefill(out, out32, ref, f"step {n_new}")
         return q, bt, cl, lens, out
 
     step(prompts)                      # whole prompts
@@ -209,7 +214,7 @@ def test_prompt_prefill_full_size_sampled(pkv):
         tables = np.repeat(inp.block_tables[b:b + 1], len(pos), axis=0)
         ref = oa.paged_decode(q, kc, vc, tables, np.array(pos) + 1,
                               w.softmax_scale)
-        check_decode(to_np(out)[rows], ref, pin.q.dtype, f"prompt seq {b}")
+        check_prefill(*out, ref, f"prompt seq {b}", rows=rows)
 
 
 def test_long_context_chunk_sampled(pkv):
@@ -238,7 +243,7 @@ def test_long_context_chunk_sampled(pkv):
                         axis=0)
         ref = oa.paged_decode(to_np(pin.q)[rows], kc, vc, sub, pos + 1,
                               w.softmax_scale)
-        check_decode(to_np(out)[rows], ref, pin.q.dtype, f"long seq {b}")
+        check_prefill(*out, ref, f"long seq {b}", rows=rows)
 
 
 def test_more_sequences_than_order_threads(pkv):
@@ -252,7 +257,7 @@ def test_more_sequences_than_order_threads(pkv):
     q_lens = np.minimum(lens, np.random.default_rng(3).integers(0, 6, 1300))
     pin = wl.make_prefill(w, q_lens, device="cuda")
     out = _run(pkv, pin)
-    assert not torch.isnan(out).any()
+    assert not torch.isnan(out[0]).any()
     rng = np.random.default_rng(4)
     seqs = sorted({0, 1, 1023, 1024, 1299, int(np.argmax(lens)),
                    int(np.argmin(lens)), *rng.integers(0, 1300, 25).tolist()})
@@ -260,68 +265,52 @@ def test_more_sequences_than_order_threads(pkv):
     _check(pin, out, "1300 sequences", seqs=seqs)
 
 
-# ---------------------------------------------------------------------------
-# The keys-on-M kernel (S^T = K Q^T, O^T += V^T P^T; q_len * G <= 32)
-
-
 @pytest.mark.parametrize("dtype", ["bfloat16", "float16"])
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (32, 8), (64, 8)])
 @pytest.mark.parametrize("bs", [16, 32])
-def test_keys_kernel_mixed(pkv, dtype, hq, hkv, bs):
-    """Contexts around the 128-key tile edges, 0 .. 32/G new tokens each;
-    both kernels against the oracle."""
+def test_few_rows_up_to_32(pkv, dtype, hq, hkv, bs):
+    """At most 32 query rows per KV head (0 .. 32/G new tokens: the tile
+    kernel's 8-rows-per-warp layout), contexts around the 64-key tile and
+    128-key edges."""
     qmax = 32 // (hq // hkv)
     lens = (1, 17, 130, 300, 520, 64, 700, 33, 129, 128, 255, 256)
     want = (1, qmax, 2, qmax, 1, 3, qmax, 0, qmax, 1, 2, qmax)
     qlens = tuple(min(L, q) for L, q in zip(lens, want))
-    w = wl.Workload("prefill_keys", 21, len(lens), hq, hkv, 128, bs, dtype,
+    w = wl.Workload("prefill_rows32", 21, len(lens), hq, hkv, 128, bs, dtype,
                     "fixed", fixed_lengths=lens)
     pin = wl.make_prefill(w, qlens, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    for kernel in ("keys", "tile"):
-        out = _run(pkv, pin, err=err, kernel=kernel)
-        assert err.item() == 0
-        _check(pin, out, f"{kernel} {dtype}/{hq}:{hkv}/bs{bs}")
+    out = _run(pkv, pin, err=err)
+    assert err.item() == 0
+    _check(pin, out, f"rows<=32 {dtype}/{hq}:{hkv}/bs{bs}")
 
 
-def test_keys_kernel_many_units(pkv):
-    """1300 sequences x 2 KV heads = 2600 units over one persistent CTA per
-    SM (each CTA serves many units back to back), 0 .. 4 new tokens each."""
-    w = wl.Workload("many_keys", 33, 1300, 16, 2, 128, 16, "bfloat16",
+@pytest.mark.parametrize("bs", [16, 32])
+def test_few_rows_unwritten_slots_hold_nan(pkv, bs):
+    lens = (1, 15, 17, 100, 333, 1000, 128, 129)
+    w = wl.Workload("rows32_nan", 22, len(lens), 32, 8, 128, bs, "bfloat16",
+                    "fixed", fixed_lengths=lens)
+    pin = wl.make_prefill(w, (1, 8, 5, 8, 3, 8, 8, 2), device="cuda")
+    _check(pin, _run(pkv, pin), "clean pool")
+    poison_unwritten(pin.paged)
+    _check(pin, _run(pkv, pin), "poisoned pool")
+
+
+def test_few_rows_many_sequences(pkv):
+    """1300 sequences x 2 KV heads, 0 .. 4 new tokens each (G = 8: up to 32
+    rows per KV head)."""
+    w = wl.Workload("many_rows32", 33, 1300, 16, 2, 128, 16, "bfloat16",
                     "uniform", low=1, high=400)
     lens = wl.make_paged(w, values=False).lengths
     q_lens = np.minimum(lens, np.random.default_rng(5).integers(0, 5, 1300))
     pin = wl.make_prefill(w, q_lens, device="cuda")
-    out = _run(pkv, pin, kernel="keys")
-    assert not torch.isnan(out).any()
+    out = _run(pkv, pin)
+    assert not torch.isnan(out[0]).any()
     rng = np.random.default_rng(6)
     seqs = sorted({0, 1, 147, 148, 1299, int(np.argmax(lens)),
                    *rng.integers(0, 1300, 30).tolist()})
-    _check(pin, out, "keys, 1300 sequences",
+    _check(pin, out, "rows<=32, 1300 sequences",
            seqs=[b for b in seqs if q_lens[b] > 0])
-
-
-@pytest.mark.parametrize("bs", [16, 32])
-def test_keys_kernel_unwritten_slots_hold_nan(pkv, bs):
-    lens = (1, 15, 17, 100, 333, 1000, 128, 129)
-    w = wl.Workload("keys_nan", 22, len(lens), 32, 8, 128, bs, "bfloat16",
-                    "fixed", fixed_lengths=lens)
-    pin = wl.make_prefill(w, (1, 8, 5, 8, 3, 8, 8, 2), device="cuda")
-    _check(pin, _run(pkv, pin, kernel="keys"), "clean pool")
-    poison_unwritten(pin.paged)
-    _check(pin, _run(pkv, pin, kernel="keys"), "poisoned pool")
-
-
-def test_keys_kernel_bad_block_id_is_flagged(pkv):
-    w = wl.Workload("keysbad", 23, 3, 32, 8, 128, 16, "bfloat16", "fixed",
-                    fixed_lengths=(300, 300, 300))
-    pin = wl.make_prefill(w, (4, 4, 4), device="cuda")
-    err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    tables = pin.paged.block_tables.copy()
-    tables[1, 5] = pin.paged.num_blocks + 3
-    out = _run(pkv, pin, tables=tables, err=err, kernel="keys")
-    assert err.item() == 5
-    _check(pin, out, "other sequences intact", seqs=[0, 2])
 
 
 def test_speculative_verify_full_size_sampled(pkv):
@@ -346,29 +335,7 @@ def test_speculative_verify_full_size_sampled(pkv):
                                np.array([L]), np.array([0, len(rows)],
                                                        dtype=np.int32),
                                w.softmax_scale)
-        check_decode(to_np(out)[rows], ref, pin.q.dtype, f"verify seq {b}")
-
-
-def test_keys_kernel_long_context(pkv):
-    """4 new tokens at the end of 90k- and 70k-token contexts: few units, so
-    most CTAs idle and each busy one streams ~700 tiles."""
-    w = wl.Workload("long_keys", 16, 2, 64, 8, 128, 32, "float16", "fixed",
-                    fixed_lengths=(90_000, 70_001))
-    pin = wl.make_prefill(w, (4, 3), device="cuda")
-    out = _run(pkv, pin, kernel="keys")
-    inp = pin.paged
-    for b in (0, 1):
-        L, n = int(inp.lengths[b]), int(pin.q_lens[b])
-        need = (L + w.block_size - 1) // w.block_size
-        ids = torch.from_numpy(
-            inp.block_tables[b, :need].astype(np.int64)).cuda()
-        kc = to_np(inp.k_cache.index_select(0, ids))
-        vc = to_np(inp.v_cache.index_select(0, ids))
-        rows = pin.query_start[b] + np.arange(n)
-        sub = np.repeat(np.arange(need, dtype=np.int32)[None, :], n, axis=0)
-        ref = oa.paged_decode(to_np(pin.q)[rows], kc, vc, sub,
-                              L - n + np.arange(n) + 1, w.softmax_scale)
-        check_decode(to_np(out)[rows], ref, pin.q.dtype, f"long seq {b}")
+        check_prefill(*out, ref, f"verify seq {b}", rows=rows)
 
 
 @pytest.mark.parametrize("dtype", ["bfloat16", "float16"])

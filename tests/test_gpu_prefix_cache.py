@@ -9,7 +9,7 @@ import torch
 from oracle import attention as oa
 from paged_kv_cache_383_b200 import flow
 
-from helpers import check_decode, to_np
+from helpers import check_prefill, prefill_both, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -61,8 +61,8 @@ def test_shared_prompt_prefills_only_the_suffix(pkv, bs):
         bt, cl, lens = flow.tables_on_device(bm, [r], 32, "cuda")
         qs = torch.tensor([0, n_new], dtype=torch.int32, device="cuda")
         out = torch.empty_like(q)
-        pkv.pa_prefill(out, q, kc, vc, bt, cl, qs, scale, max_q_len=n_new,
-                       max_context_len=int(lens[0]))
+        out32 = prefill_both(pkv, out, q, kc, vc, bt, cl, qs, scale,
+                             max_q_len=n_new, max_context_len=int(lens[0]))
         bm.cache_insert(r, toks)
         Kr = np.concatenate([to_np(pk), to_np(qk)])
         Vr = np.concatenate([to_np(pv), to_np(qv)])
@@ -70,7 +70,7 @@ def test_shared_prompt_prefills_only_the_suffix(pkv, bs):
         ref = oa.paged_prefill(to_np(q), kp, vp, tables, lens,
                                np.array([0, n_new]), scale)
         torch.cuda.synchronize()
-        check_decode(to_np(out), ref, q.dtype, f"request {r}")
+        check_prefill(out, out32, ref, f"request {r}")
         K.append(Kr)
         V.append(Vr)
     shared = bs * (prompt_len // bs)

@@ -18,7 +18,7 @@ import torch
 from oracle import attention as oa
 from paged_kv_cache_383_b200 import flow
 
-from helpers import check_decode, to_np
+from helpers import check_decode, check_prefill, prefill_both, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -86,24 +86,27 @@ class Flow:
         bt, cl, lens = flow.tables_on_device(self.bm, seqs, 64, "cuda")
         qs = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
         q = self.rnd(int(qs[-1]), HQ, D)
-        out = torch.empty_like(q)
+        out, out32 = torch.empty_like(q), None
         if max(q_lens) == 1:
             self.pkv.pa_decode(out, q, self.kc, self.vc, bt, cl, SCALE,
                                max_context_len=int(lens.max()),
                                dev_err=self.err)
         else:
-            self.pkv.pa_prefill(out, q, self.kc, self.vc, bt, cl,
-                                torch.from_numpy(qs).cuda(), SCALE,
-                                max_q_len=max(q_lens),
-                                max_context_len=int(lens.max()),
-                                dev_err=self.err)
+            out32 = prefill_both(self.pkv, out, q, self.kc, self.vc, bt, cl,
+                                 torch.from_numpy(qs).cuda(), SCALE,
+                                 max_q_len=max(q_lens),
+                                 max_context_len=int(lens.max()),
+                                 dev_err=self.err)
         kp, vp, tables = _pool([self.K[s] for s in seqs],
                                [self.V[s] for s in seqs], BS)
         assert list(lens) == [len(self.K[s]) for s in seqs]
         ref = oa.paged_prefill(to_np(q), kp, vp, tables, lens, qs, SCALE)
         torch.cuda.synchronize()
         assert self.err.item() == 0, what
-        check_decode(to_np(out), ref, q.dtype, what)
+        if out32 is None:
+            check_decode(to_np(out), ref, q.dtype, what)
+        else:
+            check_prefill(out, out32, ref, what)
 
     def swap(self, seqs, out):
         if out:
