@@ -235,3 +235,4 @@ def test_warp_partitions_ragged_groups(pkv, ps):
     _check_all(inp, out, f"warp partitions ps={ps}")
     ref = _run(pkv, inp, partition_size=256, reduce="auto")
     assert (out.float() - ref.float()).abs().max().item() <= 4e-3
+
