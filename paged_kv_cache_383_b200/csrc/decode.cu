@@ -857,12 +857,14 @@ __global__ void __launch_bounds__(kOrderThreads)
 // ---------------------------------------------------------------------------
 // Partition reduce: out = sum_j w_j o_j / sum_j w_j, w_j = l_j 2^(m_j - M),
 // M = max_j m_j (all in base-2 units).
-// One CTA per (query head, sequence); warp w folds partitions w, w+8, ...
-// with a running max, six to eight partitions in flight per warp, and the
-// eight warp states are merged through shared memory.  Used when a sequence
-// has many partitions (the fused combine handles few), so the work per CTA
-// is long enough to pay for the launch.
-constexpr int kReduceWarps = 8;
+// One CTA per (query head, sequence); warp w folds partitions w, w+16, ...
+// with a running max, eight partitions in flight per warp (one 16- or 8-byte
+// load per lane each), and the sixteen warp states are merged through shared
+// memory.  The partials were just written by the decode and are read once,
+// so the time is the latency of a few rounds of loads: 128 partitions in
+// flight per CTA keep that to one or two rounds for the longest sequences.
+// Used when a sequence has many partitions (the fused combine handles few).
+constexpr int kReduceWarps = 16;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kReduceWarps * 32)
@@ -892,7 +894,8 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-  constexpr int kBatch = kPer == 4 ? 6 : 8;  // partitions in flight
+  constexpr int kBatch = 8;  // partitions in flight per warp
+  static_assert(kPer == 4 || kPer == 2, "head_dim 128 or 64");
   for (int j0 = warp; j0 < n_parts; j0 += kBatch * kReduceWarps) {
     float2 mlj[kBatch];
     float oj[kBatch][kPer];
@@ -900,10 +903,24 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
     for (int u = 0; u < kBatch; ++u) {
       const int j = j0 + u * kReduceWarps;
       mlj[u] = j < n_parts ? __ldcg(ml + j) : make_float2(-INFINITY, 0.f);
-#pragma unroll
-      for (int e = 0; e < kPer; ++e)
-        oj[u][e] =
-            j < n_parts ? __ldcg(o + static_cast<int64_t>(j) * D + e) : 0.f;
+      // this lane's kPer consecutive dims: one 16- (or 8-) byte load; a
+      // partial row is D floats, 16-byte aligned
+      const float* src = o + static_cast<int64_t>(j) * D;
+      if constexpr (kPer == 4) {
+        const float4 v = j < n_parts
+                             ? __ldcg(reinterpret_cast<const float4*>(src))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        oj[u][0] = v.x;
+        oj[u][1] = v.y;
+        oj[u][2] = v.z;
+        oj[u][3] = v.w;
+      } else {
+        const float2 v = j < n_parts
+                             ? __ldcg(reinterpret_cast<const float2*>(src))
+                             : make_float2(0.f, 0.f);
+        oj[u][0] = v.x;
+        oj[u][1] = v.y;
+      }
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
