@@ -22,14 +22,16 @@
 //     read it, a V stage once P(j).V has, and V tile j is loaded after K
 //     tile j+1 since it is needed a tile later.  Pages are placed so that a
 //     tile is the canonical 128-byte-swizzled layout the tensor core reads.
-//   * Warp 1 allocates 256 tensor-memory columns; its lane 0 issues
-//     S = Q K^T (M=128, N=64, both operands in shared memory) and
-//     O += P V (M=128, N=128; P read from tensor memory, V from shared
+//   * Warp 1 allocates 256 tensor-memory columns (S 64, P 64, O 128); its
+//     lane 0 issues S = Q K^T (M=128, N=64, both operands in shared memory)
+//     and O += P V (M=128, N=128; P read from tensor memory, V from shared
 //     memory, MN-major) as tcgen05.mma with fp32 accumulators, and signals
-//     completion with tcgen05.commit.  S is double-buffered and P is written
-//     over the S it came from, so the tensor cores compute S(j+1) and
-//     P(j-1).V while the softmax warps work on tile j; S(j+2) is issued once
-//     P(j).V has finished reading that buffer.
+//     completion with tcgen05.commit.  S and P have buffers of their own:
+//     S(j+1) is issued as soon as the softmax warps hold S(j) in registers,
+//     so it is ready when they finish tile j, and the softmax stores P(j+1)
+//     once P(j).V has read the P buffer.  (With P written over the S it came
+//     from, S(j+2) had to wait for P(j).V, and that round trip set half of
+//     every tile's period.)
 //   * Warps 2..5 own one tensor-memory row each (thread = query row): they
 //     read S with tcgen05.ld, apply the causal mask (diagonal tiles only),
 //     keep the online softmax in registers (no shuffles: a row is one
@@ -158,9 +160,9 @@ struct PrefillArgs {
 };
 
 // barriers: q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
-// s_full[2], s_free[2], p_full[2], o_ready[2], done, then the tensor-memory
-// base address word.
-constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 4 * 2 + 1;
+// s_full, s_free, p_full, o_ready, done, then the tensor-memory base address
+// word and the residual vote.
+constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 4 + 1;
 constexpr int kTileHalf = kKeys * 128;  // 8 KB: 64 keys x 64 dims (128 B)
 
 // Shared memory for head_dim D (offsets from a 1024-byte aligned base): the
@@ -210,18 +212,21 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t k_empty0 = k_full0 + kKStages * 8;
   const uint32_t v_full0 = k_empty0 + kKStages * 8;
   const uint32_t v_empty0 = v_full0 + kVStages * 8;
-  // Double-buffer barriers: tile t uses element t & 1, phase t >> 1.
-  const uint32_t s_full0 = v_empty0 + kVStages * 8;
-  const uint32_t s_free0 = s_full0 + 16;
-  const uint32_t p_full0 = s_free0 + 16;
-  const uint32_t o_ready0 = p_full0 + 16;
-  const uint32_t done = o_ready0 + 16;
+  // S, P and P.V barriers, one each: tile t completes phase t (waited on
+  // with parity t & 1).  s_full: S(t) is in tensor memory; s_free: the
+  // softmax warps have S(t) in registers; p_full: P(t) is in tensor memory;
+  // o_ready: P(t).V has completed (O is current, the P buffer is free).
+  const uint32_t s_full = v_empty0 + kVStages * 8;
+  const uint32_t s_free = s_full + 8;
+  const uint32_t p_full = s_free + 8;
+  const uint32_t o_ready = p_full + 8;
+  const uint32_t done = o_ready + 8;
   uint32_t* tmem_slot =
       reinterpret_cast<uint32_t*>(smem + kOffBars + kNumBars * 8);
-  // Residual votes of P buffer i: a softmax warp whose rows need P's
-  // residual in tile t stores t + 1 into word t & 1 before it arrives on
-  // p_full, and the MMA issuer reads the word after that barrier; a stale
-  // word holds t - 1 or less, so the words never need clearing.
+  // Residual vote: a softmax warp whose rows need P's residual in tile t
+  // stores t + 1 into the word before it arrives on p_full, and the MMA
+  // issuer reads it after that barrier; a stale word holds t or less, so it
+  // never needs clearing.
   volatile uint32_t* pv_vote = tmem_slot + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -276,16 +281,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       dev::mbar_init(v_full0 + 8 * s, 1);
       dev::mbar_init(v_empty0 + 8 * s, 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      dev::mbar_init(s_full0 + 8 * i, 1);
-      dev::mbar_init(s_free0 + 8 * i, 4);
-      dev::mbar_init(p_full0 + 8 * i, 4);
-      dev::mbar_init(o_ready0 + 8 * i, 1);
-    }
+    dev::mbar_init(s_full, 1);
+    dev::mbar_init(s_free, 4);
+    dev::mbar_init(p_full, 4);
+    dev::mbar_init(o_ready, 1);
     dev::mbar_init(done, 4);
     dev::fence_mbar_init();
     pv_vote[0] = 0u;
-    pv_vote[1] = 0u;
   }
   bad = __syncthreads_or(bad);
   if (bad) {
@@ -300,10 +302,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   dev::tc_fence_after();
   const uint32_t tbase = *tmem_slot;
-  // S / P buffers: columns [0, 64) and [64, 128); O: columns [128, 256).
-  // P(j) (rounded part in the first 32 columns, residual in the next 32,
-  // two 16-bit values per column) overwrites S(j) once it has been read.
+  // S: columns [0, 64); P: columns [64, 128) (rounded part in the first 32,
+  // residual in the next 32, two 16-bit values per column); O: columns
+  // [128, 256).  S and P have buffers of their own, so S(j+1) can be
+  // computed as soon as the softmax warps hold S(j) in registers, without
+  // waiting for P(j).V (which only P's buffer holds up).
   const uint32_t s_tmem = tbase;
+  const uint32_t p_tmem = tbase + kKeys;
   const uint32_t o_tmem = tbase + 128;
 
   if (warp == 0) {
@@ -392,16 +397,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       constexpr uint32_t idesc_pv = dev::umma_idesc_f16(kBf16, kRows, D,
                                                         false, true);
       auto issue_pv = [&](int t) -> bool {
-        if (!dev::mbar_wait(p_full0 + 8 * (t & 1), (t >> 1) & 1) ||
+        if (!dev::mbar_wait(p_full, t & 1) ||
             !dev::mbar_wait(v_full0 + 8 * (t % kVStages), (t / kVStages) & 1))
           return false;
         dev::tc_fence_after();
         const uint32_t vt = vring + (t % kVStages) * kKVTile;
-        const uint32_t pt = s_tmem + (t & 1) * kKeys;
         const int parts =
             a.pv_split == 1 ||
                     (a.pv_split == 0 &&
-                     pv_vote[t & 1] == static_cast<uint32_t>(t) + 1u)
+                     pv_vote[0] == static_cast<uint32_t>(t) + 1u)
                 ? 2
                 : 1;
         for (int part = 0; part < parts; ++part) {  // P rounded, residual
@@ -411,29 +415,24 @@ __global__ void __launch_bounds__(kThreads, 2)
             // 8-key groups 1024 bytes apart.
             const uint64_t bd =
                 dev::sw128_desc(vt + kk * 2048, kTileHalf, 1024);
-            dev::umma_f16_ts(o_tmem, pt + part * (kKeys / 2) + kk * 8, bd,
-                             idesc_pv, (t > 0 || part > 0 || kk > 0) ? 1u : 0u);
+            dev::umma_f16_ts(o_tmem, p_tmem + part * (kKeys / 2) + kk * 8,
+                             bd, idesc_pv,
+                             (t > 0 || part > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        dev::umma_commit(o_ready0 + 8 * (t & 1));
+        dev::umma_commit(o_ready);
         dev::umma_commit(v_empty0 + 8 * (t % kVStages));
         return true;
       };
-      ok = dev::mbar_wait(q_full, 0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int s = j % kKStages;
-        // Buffer j & 1 is free once the softmax warps have read S(j-2) and
-        // P(j-2).V has read the P written over it.
-        if (!dev::mbar_wait(k_full0 + 8 * s, (j / kKStages) & 1) ||
-            (j >= 2 &&
-             (!dev::mbar_wait(s_free0 + 8 * (j & 1), ((j >> 1) - 1) & 1) ||
-              !dev::mbar_wait(o_ready0 + 8 * (j & 1), ((j >> 1) - 1) & 1)))) {
-          ok = false;
-          break;
-        }
+      // S(t) = Q K(t)^T, once K(t) has landed and the softmax warps hold
+      // S(t-1) in registers.
+      auto issue_s = [&](int t) -> bool {
+        const int s = t % kKStages;
+        if (!dev::mbar_wait(k_full0 + 8 * s, (t / kKStages) & 1) ||
+            (t >= 1 && !dev::mbar_wait(s_free, (t - 1) & 1)))
+          return false;
         dev::tc_fence_after();
         const uint32_t kt = kring + s * kKVTile;
-        const uint32_t sd = s_tmem + (j & 1) * kKeys;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int h = kk >> 2, k4 = kk & 3;
@@ -441,18 +440,21 @@ __global__ void __launch_bounds__(kThreads, 2)
                                               1024);
           const uint64_t bd = dev::sw128_desc(kt + h * kTileHalf + k4 * 32,
                                               16, 1024);
-          dev::umma_f16(sd, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          dev::umma_f16(s_tmem, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
-        dev::umma_commit(s_full0 + 8 * (j & 1));
+        dev::umma_commit(s_full);
         dev::umma_commit(k_empty0 + 8 * s);
-        if (j >= 1 && !issue_pv(j - 1)) {
-          ok = false;
-          break;
-        }
+        return true;
+      };
+      // S(j+1) is issued while the softmax works on tile j, before P(j).V,
+      // which waits for the softmax.
+      ok = dev::mbar_wait(q_full, 0) && issue_s(0);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        if (j + 1 < n_tiles) ok = issue_s(j + 1);
+        if (ok) ok = issue_pv(j);
       }
       const int last = n_tiles - 1;
-      if (ok) ok = issue_pv(last);
-      if (ok) ok = dev::mbar_wait(o_ready0 + 8 * (last & 1), (last >> 1) & 1);
+      if (ok) ok = dev::mbar_wait(o_ready, last & 1);
       if (!ok) dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
       // Release tensor memory only after the softmax warps are done with it.
       if (!dev::mbar_wait(done, 0)) dev::set_error(a.dev_err,
@@ -496,22 +498,20 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     bool ok = true;
     auto wait_pv = [&](int t) {
-      return __all_sync(0xffffffffu, dev::mbar_wait(o_ready0 + 8 * (t & 1),
-                                                    (t >> 1) & 1));
+      return __all_sync(0xffffffffu, dev::mbar_wait(o_ready, t & 1));
     };
     for (int j = 0; j < n_tiles && ok; ++j) {
-      ok = __all_sync(0xffffffffu,
-                      dev::mbar_wait(s_full0 + 8 * (j & 1), (j >> 1) & 1));
+      ok = __all_sync(0xffffffffu, dev::mbar_wait(s_full, j & 1));
       if (!ok) break;
       float sa[32];
       if (!idle) {
         dev::tc_fence_after();
-        tmem_ld16x256_x8(s_tmem + (j & 1) * kKeys + lane_off, sa);
+        tmem_ld16x256_x8(s_tmem + lane_off, sa);
         dev::tmem_ld_wait();
         dev::tc_fence_before();
       }
       __syncwarp();
-      if (lane == 0) dev::mbar_arrive(s_free0 + 8 * (j & 1));
+      if (lane == 0) dev::mbar_arrive(s_free);
       const int k0 = j * kKeys;
       if (k0 + kKeys > L) {
         // As below: clear the V rows past the context in the last tile.
@@ -530,8 +530,15 @@ __global__ void __launch_bounds__(kThreads, 2)
         dev::fence_proxy_async_smem();
       }
       if (idle) {
+        // Like the other warps, arrive for tile j only once P(j-1).V is done:
+        // a warp that ran a tile ahead would have its arrival counted toward
+        // tile j-1 on the single p_full barrier.
+        if (j >= 1 && !wait_pv(j - 1)) {
+          ok = false;
+          break;
+        }
         __syncwarp();
-        if (lane == 0) dev::mbar_arrive(p_full0 + 8 * (j & 1));
+        if (lane == 0) dev::mbar_arrive(p_full);
         continue;
       }
       // sa[4k + 2x + e]: row x, key 8k + 2 c4 + e.
@@ -630,7 +637,13 @@ __global__ void __launch_bounds__(kThreads, 2)
               lw[2 * k + x] = 0u;
             }
           }
-        const uint32_t pa = s_tmem + (j & 1) * kKeys + lane_off;
+        // P(j-1).V must have read the P buffer before it is overwritten.
+        if (j >= 1 && !wait_pv(j - 1)) {
+          ok = false;
+          break;
+        }
+        dev::tc_fence_after();
+        const uint32_t pa = p_tmem + lane_off;
         tmem_st16x128_x8(pa, hw);
         if (a.pv_split != 2) tmem_st16x128_x8(pa + kKeys / 2, lw);
         dev::tmem_st_wait();
@@ -638,8 +651,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       dev::tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if (split) pv_vote[j & 1] = static_cast<uint32_t>(j) + 1u;
-        dev::mbar_arrive(p_full0 + 8 * (j & 1));
+        if (split) pv_vote[0] = static_cast<uint32_t>(j) + 1u;
+        dev::mbar_arrive(p_full);
       }
     }
     // Epilogue: the row sums over the four threads, O / l -> out.
@@ -700,25 +713,24 @@ __global__ void __launch_bounds__(kThreads, 2)
   const float c = a.scale_log2;
   // A warp whose 32 rows are all padding (few new tokens: 4 drafts x 8 heads
   // fill one warp's rows of 128) computes nothing: it keeps the barrier
-  // protocol and its share of the V clearing only.  Its rows of P hold stale
-  // values, which reach only its own (never stored) rows of O.
+  // protocol (including the wait for P(j-1).V before it arrives for tile j)
+  // and its share of the V clearing only.  Its rows of P hold stale values,
+  // which reach only its own (never stored) rows of O.
   const bool idle = quarter * 32 >= n_q * G;
   float m_ref = -INFINITY, l = 0.f;
   bool ok = true;
   // Wait results are made warp-uniform: the tcgen05 loads and stores below
   // are warp-collective.
   auto wait_pv = [&](int t) {  // P(t).V has completed
-    return __all_sync(0xffffffffu, dev::mbar_wait(o_ready0 + 8 * (t & 1),
-                                                  (t >> 1) & 1));
+    return __all_sync(0xffffffffu, dev::mbar_wait(o_ready, t & 1));
   };
   for (int j = 0; j < n_tiles && ok; ++j) {
-    ok = __all_sync(0xffffffffu,
-                    dev::mbar_wait(s_full0 + 8 * (j & 1), (j >> 1) & 1));
+    ok = __all_sync(0xffffffffu, dev::mbar_wait(s_full, j & 1));
     if (!ok) break;
     float sv[kKeys];
     if (!idle) {
       dev::tc_fence_after();
-      const uint32_t sa = s_tmem + (j & 1) * kKeys + lane_off;
+      const uint32_t sa = s_tmem + lane_off;
       float (&lo)[32] = *reinterpret_cast<float(*)[32]>(sv);
       float (&hi)[32] = *reinterpret_cast<float(*)[32]>(sv + 32);
       dev::tmem_ld32(sa, lo);
@@ -727,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       dev::tc_fence_before();
     }
     __syncwarp();
-    if (lane == 0) dev::mbar_arrive(s_free0 + 8 * (j & 1));
+    if (lane == 0) dev::mbar_arrive(s_free);
     const int k0 = j * kKeys;
     if (k0 + kKeys > L) {
       // Keys past the context get P = 0, but 0 * NaN is NaN in the MMA:
@@ -749,8 +761,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       dev::fence_proxy_async_smem();  // visible to the tensor cores' P.V
     }
     if (idle) {
+      // Like the other warps, arrive for tile j only once P(j-1).V is done:
+      // a warp that ran a tile ahead would have its arrival counted toward
+      // tile j-1 on the single p_full barrier.
+      if (j >= 1 && !wait_pv(j - 1)) {
+        ok = false;
+        break;
+      }
       __syncwarp();
-      if (lane == 0) dev::mbar_arrive(p_full0 + 8 * (j & 1));
+      if (lane == 0) dev::mbar_arrive(p_full);
       continue;
     }
     // Causal mask: only tiles that reach past this row's position.
@@ -832,7 +851,13 @@ __global__ void __launch_bounds__(kThreads, 2)
           lw[e] = 0u;
         }
       }
-      const uint32_t pa = s_tmem + (j & 1) * kKeys + lane_off;
+      // P(j-1).V must have read the P buffer before it is overwritten.
+      if (j >= 1 && !wait_pv(j - 1)) {
+        ok = false;
+        break;
+      }
+      dev::tc_fence_after();
+      const uint32_t pa = p_tmem + lane_off;
       dev::tmem_st32u(pa, hw);
       if (a.pv_split != 2) dev::tmem_st32u(pa + kKeys / 2, lw);
       dev::tmem_st_wait();
@@ -840,8 +865,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     dev::tc_fence_before();
     __syncwarp();
     if (lane == 0) {
-      if (split) pv_vote[j & 1] = static_cast<uint32_t>(j) + 1u;
-      dev::mbar_arrive(p_full0 + 8 * (j & 1));
+      if (split) pv_vote[0] = static_cast<uint32_t>(j) + 1u;
+      dev::mbar_arrive(p_full);
     }
   }
   // Epilogue: O / l -> out[token, query head].
