@@ -23,8 +23,10 @@ OBJ_DIR = os.path.join(HERE, "_build")
 SOURCES = ["status.cpp", "block_manager.cpp", "cache_ops.cu", "decode.cu",
            "prefill.cu", "probe.cu", "swap.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3,-Wall",
-         "--split-compile=0"]
+# No --split-compile: splitting a translation unit's device code into
+# partitions compiled in parallel made the generated code differ from build to
+# build, and the prefill kernel's speed with it (up to 8 %).
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3,-Wall"]
 
 
 def nvcc() -> str:

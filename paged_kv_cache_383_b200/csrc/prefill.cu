@@ -719,6 +719,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   const bool idle = quarter * 32 >= n_q * G;
   float m_ref = -INFINITY, l = 0.f;
   bool ok = true;
+  // The residual columns of this warp's rows hold something other than
+  // zeros (tensor memory starts undefined).
+  bool res_dirty = true;
   // Wait results are made warp-uniform: the tcgen05 loads and stores below
   // are warp-collective.
   auto wait_pv = [&](int t) {  // P(t).V has completed
@@ -779,15 +782,18 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int k = 0; k < kKeys; ++k)
         if (k > lim) sv[k] = -INFINITY;
     }
-    // Eight independent partial maxima (and sums below): a 64-long serial
-    // chain of dependent instructions would stall the warp on each step.
+    // Eight independent partial maxima of eight keys each (and eight partial
+    // sums below), three inputs per max instruction: a 64-long serial chain
+    // of dependent instructions would stall the warp on each step.
     float m8[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) m8[u] = sv[u];
-#pragma unroll
-    for (int k = 8; k < kKeys; ++k) m8[k & 7] = fmaxf(m8[k & 7], sv[k]);
-    float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                     fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+    for (int u = 0; u < 8; ++u)
+      m8[u] = dev::fmax3(dev::fmax3(sv[u], sv[u + 8], sv[u + 16]),
+                         dev::fmax3(sv[u + 24], sv[u + 32], sv[u + 40]),
+                         fmaxf(sv[u + 48], sv[u + 56]));
+    float mx = dev::fmax3(dev::fmax3(m8[0], m8[1], m8[2]),
+                          dev::fmax3(m8[3], m8[4], m8[5]),
+                          fmaxf(m8[6], m8[7]));
     mx *= c;  // the scale is positive: max commutes with it
     float factor = 1.f;
     if (j == 0) {
@@ -797,16 +803,25 @@ __global__ void __launch_bounds__(kThreads, 2)
       m_ref = mx;
       l *= factor;
     }
-    // P = 2^(s * c - m_ref), before waiting for the tensor cores.
+    // P = 2^(s * c - m_ref), before waiting for the tensor cores; the
+    // exponents and the sums take two keys per instruction.
     {
-      float l8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const float2 c2 = make_float2(c, c);
+      const float2 nm2 = make_float2(-m_ref, -m_ref);
+      float2 l4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int k = 0; k < kKeys; ++k) {
-        sv[k] = dev::fast_exp2(fmaf(sv[k], c, -m_ref));
-        l8[k & 7] += sv[k];
+      for (int e = 0; e < kKeys / 2; ++e) {
+        const float2 x =
+            dev::ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), c2, nm2);
+        sv[2 * e] = dev::fast_exp2(x.x);
+        sv[2 * e + 1] = dev::fast_exp2(x.y);
+        l4[e & 3] =
+            dev::fadd2(l4[e & 3], make_float2(sv[2 * e], sv[2 * e + 1]));
       }
-      l += ((l8[0] + l8[1]) + (l8[2] + l8[3])) +
-           ((l8[4] + l8[5]) + (l8[6] + l8[7]));
+      const float2 la = dev::fadd2(l4[0], l4[1]);
+      const float2 lb = dev::fadd2(l4[2], l4[3]);
+      l += (la.x + la.y) + (lb.x + lb.y);
     }
     // Does a key of this tile need P's residual?  Its p is at most
     // 2^(mx - m_ref); it needs it if that can exceed l / kSplitInv.
@@ -832,17 +847,21 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       dev::tmem_st_wait();
     }
-    // P over S(j) in its tensor-memory buffer: rounded part, then residual
-    // (zeros when this warp's rows need none: another warp's rows may).
+    // P(j) into its tensor-memory buffer: rounded part, then the residual.
+    // When this warp's rows need none, its residual columns must read as
+    // zeros (another warp's rows may make the MMA add them): they are
+    // cleared once after a tile that wrote a residual, not every tile.
     {
       uint32_t hw[kKeys / 2], lw[kKeys / 2];
+      const bool store_lw = a.pv_split != 2 && (split || res_dirty);
       if (split) {
+        const float2 m1 = make_float2(-1.f, -1.f);
 #pragma unroll
         for (int e = 0; e < kKeys / 2; ++e) {
-          const float p0 = sv[2 * e], p1 = sv[2 * e + 1];
-          hw[e] = M::pack(p0, p1);
-          const float2 hf = M::unpack(hw[e]);
-          lw[e] = M::pack(p0 - hf.x, p1 - hf.y);
+          const float2 pe = make_float2(sv[2 * e], sv[2 * e + 1]);
+          hw[e] = M::pack(pe.x, pe.y);
+          const float2 r = dev::ffma2(M::unpack(hw[e]), m1, pe);  // P - hi
+          lw[e] = M::pack(r.x, r.y);
         }
       } else {
 #pragma unroll
@@ -851,6 +870,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           lw[e] = 0u;
         }
       }
+      res_dirty = split;
       // P(j-1).V must have read the P buffer before it is overwritten.
       if (j >= 1 && !wait_pv(j - 1)) {
         ok = false;
@@ -859,7 +879,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       dev::tc_fence_after();
       const uint32_t pa = p_tmem + lane_off;
       dev::tmem_st32u(pa, hw);
-      if (a.pv_split != 2) dev::tmem_st32u(pa + kKeys / 2, lw);
+      if (store_lw) dev::tmem_st32u(pa + kKeys / 2, lw);
       dev::tmem_st_wait();
     }
     dev::tc_fence_before();
