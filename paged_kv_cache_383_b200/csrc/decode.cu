@@ -857,14 +857,16 @@ __global__ void __launch_bounds__(kOrderThreads)
 // ---------------------------------------------------------------------------
 // Partition reduce: out = sum_j w_j o_j / sum_j w_j, w_j = l_j 2^(m_j - M),
 // M = max_j m_j (all in base-2 units).
-// One CTA per (query head, sequence); warp w folds partitions w, w+16, ...
-// with a running max, eight partitions in flight per warp (one 16- or 8-byte
-// load per lane each), and the sixteen warp states are merged through shared
-// memory.  The partials were just written by the decode and are read once,
-// so the time is the latency of a few rounds of loads: 128 partitions in
-// flight per CTA keep that to one or two rounds for the longest sequences.
-// Used when a sequence has many partitions (the fused combine handles few).
-constexpr int kReduceWarps = 16;
+// One CTA per (query head, sequence); warp w folds partitions w, w+8, ...
+// with a running max, sixteen partitions in flight per warp (eight at
+// head_dim 64; one 16- or 8-byte load per lane each), and the eight warp
+// states are merged through shared memory.  The partials were just written
+// by the decode and are read once, so the time is the latency of a few
+// rounds of loads: 128 partitions in flight per CTA keep that to one or two
+// rounds for the longest sequences, and 256 threads let two CTAs share an SM
+// (the grid, one CTA per query head and sequence, is a few waves).  Used
+// when a sequence has many partitions (the fused combine handles few).
+constexpr int kReduceWarps = 8;
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kReduceWarps * 32)
@@ -894,7 +896,8 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
   float acc[kPer];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-  constexpr int kBatch = 8;  // partitions in flight per warp
+  // partitions in flight per warp (head_dim 64: 8, which needs no spill)
+  constexpr int kBatch = kPer == 4 ? 16 : 8;
   static_assert(kPer == 4 || kPer == 2, "head_dim 128 or 64");
   for (int j0 = warp; j0 < n_parts; j0 += kBatch * kReduceWarps) {
     float2 mlj[kBatch];
