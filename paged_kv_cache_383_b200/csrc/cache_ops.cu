@@ -90,7 +90,25 @@ __global__ void copy_blocks_kernel(uint4* __restrict__ k_cache,
   uint4* cache = blockIdx.y == 0 ? k_cache : v_cache;
   const uint4* s = cache + static_cast<int64_t>(src) * block_chunks;
   uint4* d = cache + static_cast<int64_t>(dst) * block_chunks;
-  for (int64_t i = threadIdx.x; i < block_chunks; i += blockDim.x) d[i] = s[i];
+  // Eight 16-byte loads in flight per thread before their stores: the
+  // source and destination share one array, so the compiler may not hoist a
+  // load above an earlier store, and a load-store loop would pay one memory
+  // round trip per chunk (a 32 KB block is then a single round of loads).
+  constexpr int kInFlight = 8;
+  const int64_t stride = blockDim.x;
+  for (int64_t i0 = threadIdx.x; i0 < block_chunks; i0 += stride * kInFlight) {
+    uint4 v[kInFlight];
+#pragma unroll
+    for (int u = 0; u < kInFlight; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < block_chunks) v[u] = s[i];
+    }
+#pragma unroll
+    for (int u = 0; u < kInFlight; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < block_chunks) d[i] = v[u];
+    }
+  }
 }
 
 int sm_count() {
