@@ -319,14 +319,17 @@ __global__ void __launch_bounds__(kThreads, 2)
       dev::prefetch_tmap(&vmap);
       if constexpr (RQ > 0) {
         // Few query rows: RQ/G tokens of G heads (RQ rows) into the first RQ
-        // rows of each 32-row quarter; the rest of the tile is padding.
+        // of each 16-row quarter of the 64-row A operand (the rest is
+        // padding).  With M = 64 the tensor cores put row 16q + i of S and O
+        // in tensor-memory lane 32q + i, and read P's row 16q + i from that
+        // lane: the same lanes the softmax warps use.
         constexpr int kQTok = RQ / G;
         dev::mbar_arrive_expect_tx(q_full, 4 * kHalves * RQ * 128);
 #pragma unroll
         for (int qq = 0; qq < 4; ++qq)
 #pragma unroll
           for (int h = 0; h < kHalves; ++h)
-            dev::tma_load_3d(q_s + h * kHalfQ + qq * 32 * 128, &qmap, 64 * h,
+            dev::tma_load_3d(q_s + h * kHalfQ + qq * 16 * 128, &qmap, 64 * h,
                              kvh * G, q0 + tok0 + qq * kQTok, q_full);
       } else {
         dev::mbar_arrive_expect_tx(q_full, kQBytes);
@@ -392,9 +395,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ---------------- MMA issuer ----------------
     bool ok = true;
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = dev::umma_idesc_f16(kBf16, kRows, kKeys,
+      // M = 128 query rows per MMA, or 64 in the few-row layouts (at most 16
+      // real rows per lane quarter): half the tensor work per tile.
+      constexpr int kMmaM = RQ > 0 ? 64 : kRows;
+      constexpr uint32_t idesc_qk = dev::umma_idesc_f16(kBf16, kMmaM, kKeys,
                                                         false, false);
-      constexpr uint32_t idesc_pv = dev::umma_idesc_f16(kBf16, kRows, D,
+      constexpr uint32_t idesc_pv = dev::umma_idesc_f16(kBf16, kMmaM, D,
                                                         false, true);
       auto issue_pv = [&](int t) -> bool {
         if (!dev::mbar_wait(p_full, t & 1) ||
