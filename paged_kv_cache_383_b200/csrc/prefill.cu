@@ -45,7 +45,9 @@
 //     compile-time variant spreads the rows over all four softmax warps,
 //     8 or 16 per lane quarter, and reads S / writes P / reads O with the
 //     16-lane tensor-memory shapes: four threads per row, 16 keys each.  A
-//     warp whose rows are all padding computes nothing.
+//     warp whose rows are all padding computes nothing.  Its MMAs use
+//     M = 64 (half the tensor work), whose accumulator rows 16q + i sit in
+//     lanes 32q + i, and the 16 KB of Q this frees holds a third V stage.
 //   * Shared memory is ~99 KB (Q, the rings, barriers; block ids are read
 //     from global memory a tile ahead) and tensor memory 256 columns, so two
 //     CTAs share an SM at any context length: one CTA's softmax runs while
@@ -74,8 +76,17 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kRows = 128;      // query rows per tile (tensor memory lanes)
 constexpr int kKeys = 64;       // keys per K/V tile
-constexpr int kKStages = 2;     // K ring depth
-constexpr int kVStages = 2;     // V ring depth
+// Ring depths and Q rows per layout.  Tiles of 128 query rows: two K and
+// two V stages.  The few-row layouts (M = 64 MMAs, a 64-row Q operand)
+// stream K/V at HBM speed; the 16 KB their Q operand does not need holds a
+// third V stage (a V stage is held longest: until P.V, after the softmax).
+template <int RQ> __host__ __device__ constexpr int k_stages() { return 2; }
+template <int RQ> __host__ __device__ constexpr int v_stages() {
+  return RQ > 0 ? 3 : 2;
+}
+template <int RQ> __host__ __device__ constexpr int q_rows() {
+  return RQ > 0 ? 64 : 128;
+}
 constexpr int kThreads = 192;   // producer, MMA, 4 softmax warps
 constexpr int kTmemCols = 256;  // S/P: cols [0, 128), O: cols [128, 128 + D)
 constexpr float kRescaleLog2 = 8.f;
@@ -162,26 +173,31 @@ struct PrefillArgs {
 // barriers: q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
 // s_full, s_free, p_full, o_ready, done, then the tensor-memory base address
 // word and the residual vote.
-constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 4 + 1;
+template <int KS, int VS> __host__ __device__ constexpr int num_bars() {
+  return 1 + 2 * KS + 2 * VS + 4 + 1;
+}
 constexpr int kTileHalf = kKeys * 128;  // 8 KB: 64 keys x 64 dims (128 B)
 
 // Shared memory for head_dim D (offsets from a 1024-byte aligned base): the
 // head dimension is held in 64-element halves of 128 bytes, each its own
 // 128-byte-swizzled region.
-template <int D>
+template <int D, int QR, int KS, int VS>
 struct Layout {
   static constexpr int kHalves = D / 64;
-  static constexpr int kHalfQ = kRows * 128;             // 16 KB
+  static constexpr int kHalfQ = QR * 128;                 // 16 or 8 KB
   static constexpr int kQBytes = kHalves * kHalfQ;
   static constexpr int kKVTile = kHalves * kTileHalf;     // per K or V tile
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kKStages * kKVTile;
-  static constexpr int kOffBars = kOffV + kVStages * kKVTile;
+  static constexpr int kOffV = kOffK + KS * kKVTile;
+  static constexpr int kOffBars = kOffV + VS * kKVTile;
   // 1024 bytes of slack for aligning the base, then the layout above; after
   // the barriers, the tensor-memory address word and two residual votes.
-  static constexpr size_t kSmemBytes = 1024 + kOffBars + kNumBars * 8 + 32;
+  static constexpr size_t kSmemBytes =
+      1024 + kOffBars + num_bars<KS, VS>() * 8 + 32;
 };
+template <int D, int RQ>
+using LayoutFor = Layout<D, q_rows<RQ>(), k_stages<RQ>(), v_stages<RQ>()>;
 
 template <typename T, int BS, int G, int D, int RQ>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -189,7 +205,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                    const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap,
                    const PrefillArgs a) {
-  using Lay = Layout<D>;
+  using Lay = LayoutFor<D, RQ>;
+  constexpr int kKStages = k_stages<RQ>();
+  constexpr int kVStages = v_stages<RQ>();
+  constexpr int kNumBars = num_bars<kKStages, kVStages>();
   constexpr int kHalves = Lay::kHalves;
   constexpr int kHalfQ = Lay::kHalfQ;
   constexpr int kQBytes = Lay::kQBytes;
@@ -1010,7 +1029,7 @@ pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
                  const CUtensorMap& qm, const CUtensorMap& km,
                  const CUtensorMap& vm, cudaStream_t st) {
   auto kern = prefill_kernel<T, BS, G, D, RQ>;
-  const size_t smem = Layout<D>::kSmemBytes;
+  const size_t smem = LayoutFor<D, RQ>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
       static_cast<int>(smem));
