@@ -268,7 +268,8 @@ def test_more_sequences_than_order_threads(pkv):
 @pytest.mark.parametrize("dtype", ["bfloat16", "float16"])
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (32, 8), (64, 8)])
 @pytest.mark.parametrize("bs", [16, 32])
-def test_few_rows_up_to_32(pkv, dtype, hq, hkv, bs):
+@pytest.mark.parametrize("head_dim", [64, 128])
+def test_few_rows_up_to_32(pkv, dtype, hq, hkv, bs, head_dim):
     """At most 32 query rows per KV head (0 .. 32/G new tokens: the tile
     kernel's 8-rows-per-warp layout), contexts around the 64-key tile and
     128-key edges."""
@@ -276,13 +277,13 @@ def test_few_rows_up_to_32(pkv, dtype, hq, hkv, bs):
     lens = (1, 17, 130, 300, 520, 64, 700, 33, 129, 128, 255, 256)
     want = (1, qmax, 2, qmax, 1, 3, qmax, 0, qmax, 1, 2, qmax)
     qlens = tuple(min(L, q) for L, q in zip(lens, want))
-    w = wl.Workload("prefill_rows32", 21, len(lens), hq, hkv, 128, bs, dtype,
-                    "fixed", fixed_lengths=lens)
+    w = wl.Workload("prefill_rows32", 21, len(lens), hq, hkv, head_dim, bs,
+                    dtype, "fixed", fixed_lengths=lens)
     pin = wl.make_prefill(w, qlens, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = _run(pkv, pin, err=err)
     assert err.item() == 0
-    _check(pin, out, f"rows<=32 {dtype}/{hq}:{hkv}/bs{bs}")
+    _check(pin, out, f"rows<=32 {dtype}/{hq}:{hkv}/bs{bs}/d{head_dim}")
 
 
 @pytest.mark.parametrize("bs", [16, 32])
@@ -341,7 +342,8 @@ def test_speculative_verify_full_size_sampled(pkv):
 @pytest.mark.parametrize("dtype", ["bfloat16", "float16"])
 @pytest.mark.parametrize("hq,hkv", [(8, 8), (16, 8), (32, 8), (64, 8)])
 @pytest.mark.parametrize("bs", [16, 32])
-def test_few_rows_33_to_64(pkv, dtype, hq, hkv, bs):
+@pytest.mark.parametrize("head_dim", [64, 128])
+def test_few_rows_33_to_64(pkv, dtype, hq, hkv, bs, head_dim):
     """33 .. 64 query rows per KV head (the tile kernel's 16-rows-per-warp
     layout: two rows per thread), contexts around the tile edges."""
     G = hq // hkv
@@ -351,10 +353,10 @@ def test_few_rows_33_to_64(pkv, dtype, hq, hkv, bs):
             qmax)
     qlens = tuple(min(L, q) for L, q in zip(lens, want))
     assert 32 < max(qlens) * G <= 64
-    w = wl.Workload("prefill_rows64", 24, len(lens), hq, hkv, 128, bs, dtype,
-                    "fixed", fixed_lengths=lens)
+    w = wl.Workload("prefill_rows64", 24, len(lens), hq, hkv, head_dim, bs,
+                    dtype, "fixed", fixed_lengths=lens)
     pin = wl.make_prefill(w, qlens, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     out = _run(pkv, pin, err=err)
     assert err.item() == 0
-    _check(pin, out, f"rows<=64 {dtype}/{hq}:{hkv}/bs{bs}")
+    _check(pin, out, f"rows<=64 {dtype}/{hq}:{hkv}/bs{bs}/d{head_dim}")

@@ -67,15 +67,16 @@ def test_decode_paths_round_once(pkv, dtype, d, kernel, ps, reduce):
 
 
 @pytest.mark.parametrize("dtype", ["bfloat16", "float16"])
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("kernel,maxq", [("tile", 4), ("tile", 16),
                                          ("tile", 40)])
-def test_prefill_paths_round_once(pkv, dtype, kernel, maxq):
+def test_prefill_paths_round_once(pkv, dtype, d, kernel, maxq):
     """G = 4: up to 16 / 64 / 160 query rows per KV head reach the tile
     kernel's 8-rows-per-warp, 16-rows-per-warp and plain layouts."""
     lens = (1, 3, 6, 40, 700, 130, 2, 257)
     qlens = tuple(min(L, q) for L, q in
                   zip(lens, (1, 3, maxq, maxq, maxq, 2, 2, maxq)))
-    w = wl.Workload("rounding_pf", 42, len(lens), 32, 8, 128, 16, dtype,
+    w = wl.Workload("rounding_pf", 42, len(lens), 32, 8, d, 16, dtype,
                     "fixed", fixed_lengths=lens, scale=1.0)
     pin = wl.make_prefill(w, qlens, device="cuda")
     inp = pin.paged
@@ -94,5 +95,5 @@ def test_prefill_paths_round_once(pkv, dtype, kernel, maxq):
     ref = oa.paged_prefill(to_np(pin.q), to_np(inp.k_cache),
                            to_np(inp.v_cache), inp.block_tables, inp.lengths,
                            pin.query_start, w.softmax_scale)
-    check_prefill(out, out32, ref, f"{kernel}/{dtype}")
+    check_prefill(out, out32, ref, f"{kernel}/{dtype}/d{d}")
     assert np.abs(ref).max() > 1.0
