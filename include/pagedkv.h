@@ -137,10 +137,11 @@ const char* pa_last_error(void);
  *   context_lens  [num_seqs] int32, tokens per sequence, the newest included
  *   workspace     pa_decode_workspace_bytes(desc) bytes of device memory the
  *                 caller owns, 16-byte aligned (always > 0): partition
- *                 partials and per-(sequence, KV head) counters (more than
- *                 one partition only) and the order in which sequences are
- *                 served (longest first, so the grid ends on short work),
- *                 all written by the call on its stream.  Its contents need
+ *                 partials, per-(sequence, KV head) counters and the order
+ *                 in which partitions are served (more than one partition
+ *                 only), and the order in which sequences are served
+ *                 (longest first, so the grid ends on short work), all
+ *                 written by the call on its stream.  Its contents need
  *                 no initialisation and are scratch after the call; calls
  *                 that share a workspace must not overlap on the device.
  * Launches: a one-CTA prep kernel (the longest-first order; counter reset),

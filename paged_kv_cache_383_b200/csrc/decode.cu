@@ -85,6 +85,10 @@ struct DecodeArgs {
   float* ws_ml;  // [num_seqs, num_q_heads, max_parts, 2] = (max, sum), log2 units
   int* counters; // [num_seqs, num_kv_heads] finished partitions (fused mode)
   const int32_t* order;  // [num_seqs] sequence served by grid row z
+  // [num_seqs * max_parts] partition units longest first (entry u: sequence
+  // u / max_parts, partition u % max_parts); non-null when the grid is
+  // (KV head, unit) rather than (partition, KV head, sequence)
+  const int32_t* units;
   int fused;     // 1: the last partition CTA combines; 0: the reduce kernel
   int warp_parts;  // 1: a CTA serves kConsumers consecutive partitions, one
                    // per consumer warp (reduce kernel path, short partitions)
@@ -278,20 +282,31 @@ __global__ void __launch_bounds__(kThreads)
   // Partitions this CTA serves: one, or (warp_parts) kConsumers consecutive
   // ones, consumer warp w taking partition part + w.
   const int nsub = a.warp_parts ? kConsumers : 1;
-  const int part = blockIdx.x * nsub;
-  const int kvh = blockIdx.y;
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
   dev::pdl_trigger();  // the reduce may start its prologue early
-  // Grid rows are handed out longest sequence first (the order the prep
-  // kernel wrote, which this grid may only read after waiting for it), so
-  // the last CTAs to start are short ones and the tail of the grid is short.
-  int b = blockIdx.z;
-  if (a.order) {
+  // Grid rows are handed out longest first (the order the prep kernel wrote,
+  // which this grid may only read after waiting for it), so the last CTAs
+  // to start are short ones and the tail of the grid is short: partition
+  // units by their token count (all KV heads of a unit side by side), or
+  // sequences by length (their partitions side by side).
+  int part, kvh, b;
+  if (a.units) {
+    kvh = blockIdx.x;
     dev::pdl_wait();
-    b = a.order[blockIdx.z];
+    const int u = a.units[blockIdx.y];
+    b = u / a.max_parts;
+    part = u - b * a.max_parts;
+  } else {
+    part = blockIdx.x * nsub;
+    kvh = blockIdx.y;
+    b = blockIdx.z;
+    if (a.order) {
+      dev::pdl_wait();
+      b = a.order[blockIdx.z];
+    }
   }
   const int PS = a.partition_size;
   const int pages_per_part = PS / BS;
@@ -835,23 +850,40 @@ __global__ void __launch_bounds__(kThreads)
 // ---------------------------------------------------------------------------
 // Prep kernel (one CTA), run before every decode: orders the sequences
 // longest first (a counting sort on context_len >> shift, 1024 buckets,
-// descending) into `order`, and zeroes the per-(sequence, KV head) partition
-// counters when the decode combines in place.  Launched with programmatic
-// stream serialization: it sorts while the previous kernel drains (it reads
-// only host-written lengths), then waits for that kernel, which may still
-// read `order` and the counters, before writing them.  The decode's own wait
-// covers the prep kernel.  Within one bucket the order follows the atomics;
-// results do not depend on it (each sequence is computed on its own and
-// partials are combined in partition order).
+// descending) into `order`, zeroes the per-(sequence, KV head) partition
+// counters when the decode combines in place, and with a unit grid orders
+// the (sequence, partition) units by token count into `units`.  Launched
+// with programmatic stream serialization: it sorts while the previous kernel
+// drains (it reads only host-written lengths), then waits for that kernel,
+// which may still read `order`, the counters and `units`, before writing
+// them.  The decode's own wait covers the prep kernel.  Within one bucket the
+// order follows the atomics; results do not depend on it (each unit is
+// computed on its own and partials are combined in partition order).
 __global__ void __launch_bounds__(kOrderThreads)
     prep_kernel(const int32_t* __restrict__ context_lens, int num_seqs,
                 int shift, int32_t* __restrict__ order, int* counters,
-                int n_counters) {
+                int n_counters, int32_t* __restrict__ units, int max_parts,
+                int partition_size, int unit_shift) {
   dev::pdl_trigger();
   sort_longest_first(context_lens, num_seqs, shift, order,
                      [] { dev::pdl_wait(); });
   for (int i = threadIdx.x; i < n_counters; i += kOrderThreads)
     counters[i] = 0;
+  if (units) {
+    // Partition units by token count, largest first: unit u is partition
+    // u % max_parts of sequence u / max_parts (empty past the sequence).
+    // The previous kernel has been waited for above.
+    counting_sort_desc(
+        num_seqs * max_parts,
+        [&](int u) {
+          const int b = u / max_parts;
+          const int p = u - b * max_parts;
+          const int left = context_lens[b] - p * partition_size;
+          const int n = left <= 0 ? 0 : min(left, partition_size);
+          return n >> unit_shift;
+        },
+        units, [] {});
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -1110,7 +1142,7 @@ pa_status check_desc(const pa_decode_desc* d) {
 // partition counters (only with more than one partition), then the sequence
 // order; each piece 16-byte aligned.
 struct WsLayout {
-  size_t o = 0, ml = 0, counters = 0, order = 0, total = 0;
+  size_t o = 0, ml = 0, counters = 0, units = 0, order = 0, total = 0;
 };
 
 WsLayout ws_layout(const pa_decode_desc* d) {
@@ -1130,6 +1162,9 @@ WsLayout ws_layout(const pa_decode_desc* d) {
     w.counters = at;
     at += up16(static_cast<size_t>(d->num_seqs) * d->num_kv_heads *
                sizeof(int));
+    w.units = at;
+    at += up16(static_cast<size_t>(d->num_seqs) * static_cast<size_t>(parts) *
+               sizeof(int32_t));
   }
   w.order = at;
   at += up16(static_cast<size_t>(d->num_seqs) * sizeof(int32_t));
@@ -1185,15 +1220,18 @@ pa_status launch(const pa_decode_desc* d, DecodeArgs& a, const CUtensorMap& km,
     const cudaError_t pe = cudaLaunchKernelEx(
         &pcfg, prep_kernel, a.context_lens, d->num_seqs,
         order_shift(a.max_context_len), const_cast<int32_t*>(a.order),
-        a.counters, n);
+        a.counters, n, const_cast<int32_t*>(a.units), a.max_parts,
+        a.partition_size, order_shift(a.partition_size));
     count_launch();
     if (pe != cudaSuccess)
       return fail(PA_ERR_CUDA, "pa_decode: prep launch failed: %s",
                   cudaGetErrorString(pe));
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.warp_parts ? (a.max_parts + kConsumers - 1) / kConsumers
-                                   : a.max_parts,
+  cfg.gridDim =
+      a.units ? dim3(d->num_kv_heads, d->num_seqs * a.max_parts, 1)
+              : dim3(a.warp_parts ? (a.max_parts + kConsumers - 1) / kConsumers
+                                  : a.max_parts,
                      d->num_kv_heads, d->num_seqs);
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
@@ -1413,6 +1451,20 @@ pa_status pa_decode(void* out, const void* q, const void* k_cache,
   a.max_parts = parts;
   a.max_context_len = max_ctx;
   a.out_f32 = desc->out_fp32;
+  // Long partitions, one per CTA, in a grid of a few waves: the grid runs
+  // (KV head, unit) with the units longest first, so the last CTAs hold the
+  // shortest partitions.  Ordered by sequence instead, the second wave can
+  // start full-length partitions of mid-length sequences and end on a long
+  // tail (batch 64 at 2048-token partitions: 6.12 -> 6.24 TB/s).  With many
+  // waves the sequence order already ends on short work, and with short
+  // partitions the extra sort in the prep kernel costs more than the tail
+  // (gridDim.y caps the unit count).
+  const int64_t n_units = static_cast<int64_t>(desc->num_seqs) * parts;
+  a.units = (parts > 1 && !a.warp_parts && ps >= 1024 && n_units <= 65535 &&
+             // at most four waves of three CTAs per SM
+             n_units * desc->num_kv_heads <= 12LL * pagedkv::device_sm_count())
+                ? reinterpret_cast<const int32_t*>(ws + wl.units)
+                : nullptr;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool mma = desc->kernel != PA_KERNEL_SIMT;

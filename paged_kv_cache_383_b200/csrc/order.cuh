@@ -1,9 +1,9 @@
-// Longest-first order of sequences by context length, for grids whose row z
-// serves sequence order[z]: the last CTAs to start then hold short work, so
-// the grid's tail is short.  A counting sort on context_len >> shift over
-// 1024 buckets, descending, run by one CTA of kOrderThreads threads.  Within
-// a bucket the order follows the atomics; callers' results do not depend on
-// it (each sequence is computed on its own).
+// Longest-first orders for grids whose rows serve the entries of a sorted
+// list (sequences by context length, or partitions by their token count): the
+// last CTAs to start then hold short work, so the grid's tail is short.  A
+// counting sort over 1024 buckets, descending, run by one CTA of
+// kOrderThreads threads.  Within a bucket the order follows the atomics;
+// callers' results do not depend on it (each unit is computed on its own).
 #pragma once
 
 #include <cstdint>
@@ -21,25 +21,23 @@ inline int order_shift(int max_ctx) {
   return shift;
 }
 
-// Called by all kOrderThreads threads of the CTA.  Counts and scans, then
-// calls before_write() (e.g. a wait for the previous kernel that may still
-// read `order`), then writes order[0 .. num_seqs).
-template <typename BeforeWrite>
-__device__ __forceinline__ void sort_longest_first(
-    const int32_t* __restrict__ context_lens, int num_seqs, int shift,
-    int32_t* __restrict__ order, BeforeWrite before_write) {
+// Called by all kOrderThreads threads of the CTA.  A counting sort of items
+// 0 .. n-1 by key_of(i) (a non-negative int, clipped to 1023), largest key
+// first: counts and scans, then calls before_write() (e.g. a wait for the
+// previous kernel that may still read `out`), then writes out[0 .. n).
+template <typename KeyOf, typename BeforeWrite>
+__device__ __forceinline__ void counting_sort_desc(int n, KeyOf key_of,
+                                                   int32_t* __restrict__ out,
+                                                   BeforeWrite before_write) {
   __shared__ int hist[kOrderBuckets];
   __shared__ int warp_sum[kOrderThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   auto bucket = [&](int i) {
-    const int L = context_lens[i];
-    const int k = L <= 0 ? 0 : min(L >> shift, kOrderBuckets - 1);
-    return kOrderBuckets - 1 - k;  // longest first
+    return kOrderBuckets - 1 - min(key_of(i), kOrderBuckets - 1);
   };
   hist[tid] = 0;
   __syncthreads();
-  for (int i = tid; i < num_seqs; i += kOrderThreads)
-    atomicAdd(&hist[bucket(i)], 1);
+  for (int i = tid; i < n; i += kOrderThreads) atomicAdd(&hist[bucket(i)], 1);
   __syncthreads();
   // Exclusive scan of the 1024 bucket counts (one per thread).
   const int c = hist[tid];
@@ -64,8 +62,22 @@ __device__ __forceinline__ void sort_longest_first(
   hist[tid] = x - c + (warp > 0 ? warp_sum[warp - 1] : 0);
   __syncthreads();
   before_write();
-  for (int i = tid; i < num_seqs; i += kOrderThreads)
-    order[atomicAdd(&hist[bucket(i)], 1)] = i;
+  for (int i = tid; i < n; i += kOrderThreads)
+    out[atomicAdd(&hist[bucket(i)], 1)] = i;
+}
+
+// The sequences by context_len >> shift over 1024 buckets, longest first.
+template <typename BeforeWrite>
+__device__ __forceinline__ void sort_longest_first(
+    const int32_t* __restrict__ context_lens, int num_seqs, int shift,
+    int32_t* __restrict__ order, BeforeWrite before_write) {
+  counting_sort_desc(
+      num_seqs,
+      [&](int i) {
+        const int L = context_lens[i];
+        return L <= 0 ? 0 : (L >> shift);
+      },
+      order, before_write);
 }
 
 }  // namespace

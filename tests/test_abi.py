@@ -89,9 +89,10 @@ def test_decode_needs_workspace_for_split(pkv):
     d = _desc(partition_size=16, max_blocks_per_seq=8)
     need = lib.pa_decode_workspace_bytes(ctypes.byref(d))
     # o: 2 seqs x 8 q heads x 8 partitions x 128 floats; (m, l): x 2 floats;
-    # 2 seqs x 2 kv heads int32 counters; 2 int32 of sequence order; each
-    # piece rounded up to 16 bytes
-    assert need == 2 * 8 * 8 * 128 * 4 + 2 * 8 * 8 * 2 * 4 + 16 + 16
+    # 2 seqs x 2 kv heads int32 counters; 2 seqs x 8 partitions int32 of
+    # unit order; 2 int32 of sequence order; each piece rounded up to 16
+    # bytes
+    assert need == 2 * 8 * 8 * 128 * 4 + 2 * 8 * 8 * 2 * 4 + 16 + 64 + 16
     fake = 0x1000
     st = lib.pa_decode(fake, fake, fake, fake, fake, fake,
                        ctypes.c_float(1.0), ctypes.byref(d), None, 0, None,

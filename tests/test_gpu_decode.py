@@ -110,6 +110,25 @@ def test_fused_and_kernel_reduce_agree(pkv):
     assert (fused.float() - kern.float()).abs().max().item() <= 2e-3
 
 
+UNIT_GRID = {
+    "gqa4_bf16_bs16": wl.Workload("unit_gqa4", 77, 20, 32, 8, 128, 16,
+                                  "bfloat16", "uniform", low=1, high=6000),
+    "mha_d64_f16_bs32": wl.Workload("unit_mha", 78, 20, 8, 8, 64, 32,
+                                    "float16", "uniform", low=1, high=6000),
+}
+
+
+@pytest.mark.parametrize("kernel", ["mma", "simt"])
+@pytest.mark.parametrize("name", list(UNIT_GRID))
+def test_unit_ordered_grid(pkv, name, kernel):
+    """1024-token partitions in a grid of under four waves: the decode runs
+    one CTA per (KV head, partition unit), units longest first; ragged
+    lengths from one token to six partitions, empty units included."""
+    inp = wl.make_paged(UNIT_GRID[name], device="cuda")
+    out = _run(pkv, inp, kernel=kernel, partition_size=1024)
+    _check_all(inp, out, f"unit grid {name}/{kernel}")
+
+
 def test_identity_vs_shuffled_tables(pkv):
     w = wl.WORKLOADS["llama3_8b_gqa4"].scaled(num_seqs=5, low=100, high=900)
     inp = wl.make_paged(w, device="cuda")
