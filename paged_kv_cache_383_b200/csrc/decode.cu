@@ -850,9 +850,9 @@ __global__ void __launch_bounds__(kThreads)
 // ---------------------------------------------------------------------------
 // Prep kernel (one CTA), run before every decode: orders the sequences
 // longest first (a counting sort on context_len >> shift, 1024 buckets,
-// descending) into `order`, zeroes the per-(sequence, KV head) partition
-// counters when the decode combines in place, and with a unit grid orders
-// the (sequence, partition) units by token count into `units`.  Launched
+// descending) into `order` (with a unit grid: the (sequence, partition)
+// units by token count into `units` instead), and zeroes the per-(sequence,
+// KV head) partition counters when the decode combines in place.  Launched
 // with programmatic stream serialization: it sorts while the previous kernel
 // drains (it reads only host-written lengths), then waits for that kernel,
 // which may still read `order`, the counters and `units`, before writing
@@ -865,14 +865,10 @@ __global__ void __launch_bounds__(kOrderThreads)
                 int n_counters, int32_t* __restrict__ units, int max_parts,
                 int partition_size, int unit_shift) {
   dev::pdl_trigger();
-  sort_longest_first(context_lens, num_seqs, shift, order,
-                     [] { dev::pdl_wait(); });
-  for (int i = threadIdx.x; i < n_counters; i += kOrderThreads)
-    counters[i] = 0;
   if (units) {
     // Partition units by token count, largest first: unit u is partition
     // u % max_parts of sequence u / max_parts (empty past the sequence).
-    // The previous kernel has been waited for above.
+    // The unit grid does not read `order`.
     counting_sort_desc(
         num_seqs * max_parts,
         [&](int u) {
@@ -882,8 +878,13 @@ __global__ void __launch_bounds__(kOrderThreads)
           const int n = left <= 0 ? 0 : min(left, partition_size);
           return n >> unit_shift;
         },
-        units, [] {});
+        units, [] { dev::pdl_wait(); });
+  } else {
+    sort_longest_first(context_lens, num_seqs, shift, order,
+                       [] { dev::pdl_wait(); });
   }
+  for (int i = threadIdx.x; i < n_counters; i += kOrderThreads)
+    counters[i] = 0;
 }
 
 // ---------------------------------------------------------------------------
