@@ -88,7 +88,7 @@ template <int RQ> __host__ __device__ constexpr int q_rows() {
   return RQ > 0 ? 64 : 128;
 }
 constexpr int kThreads = 192;   // producer, MMA, 4 softmax warps
-constexpr int kTmemCols = 256;  // S/P: cols [0, 128), O: cols [128, 128 + D)
+constexpr int kTmemCols = 256;  // S [0, 64), P [64, 128), O [128, 128 + D)
 constexpr float kRescaleLog2 = 8.f;
 // P . V runs on 16-bit P.  A single rounding of P moves each weight by up to
 // 2^-8 of itself (bf16), which on a row whose weight sits on a few keys can
@@ -639,8 +639,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         dev::tmem_st_wait();
       }
-      // P over S(j): column 4k + c4 of each half holds keys 8k + 2 c4 and
-      // 8k + 2 c4 + 1 of row x in lane t/4 + 8x; a padding lane gets zeros.
+      // P(j) into its buffer: column 4k + c4 of each half holds keys
+      // 8k + 2 c4 and 8k + 2 c4 + 1 of row x in lane t/4 + 8x; a padding
+      // lane gets zeros.
       {
         uint32_t hw[16], lw[16];
 #pragma unroll
