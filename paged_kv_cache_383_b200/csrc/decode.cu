@@ -49,6 +49,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <atomic>
 #include <mutex>
 
 #include "device_utils.cuh"
@@ -1003,10 +1004,19 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
 // ---------------------------------------------------------------------------
 // Host side.
 
+// SM count of the current device, looked up once per device ordinal (the
+// launch path asks on every call).
 int device_sm_count() {
-  int dev = 0, count = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int count = 148;
+  cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cached[dev].store(count, std::memory_order_relaxed);
   return count;
 }
 
