@@ -829,33 +829,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       m_ref = mx;
       l *= factor;
     }
-    // P = 2^(s * c - m_ref), before waiting for the tensor cores; the
-    // exponents and the sums take two keys per instruction.
-    {
-      const float2 c2 = make_float2(c, c);
-      const float2 nm2 = make_float2(-m_ref, -m_ref);
-      float2 l4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                      make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-      for (int e = 0; e < kKeys / 2; ++e) {
-        const float2 x =
-            dev::ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), c2, nm2);
-        sv[2 * e] = dev::fast_exp2(x.x);
-        sv[2 * e + 1] = dev::fast_exp2(x.y);
-        l4[e & 3] =
-            dev::fadd2(l4[e & 3], make_float2(sv[2 * e], sv[2 * e + 1]));
-      }
-      const float2 la = dev::fadd2(l4[0], l4[1]);
-      const float2 lb = dev::fadd2(l4[2], l4[3]);
-      l += (la.x + la.y) + (lb.x + lb.y);
-    }
-    // Does a key of this tile need P's residual?  Its p is at most
-    // 2^(mx - m_ref); it needs it if that can exceed l / kSplitInv.
-    const bool split = __any_sync(
-        0xffffffffu,
-        a.pv_split == 1 ||
-            (a.pv_split == 0 && valid &&
-             dev::fast_exp2(mx - m_ref) * kSplitInv > l));
     if (__any_sync(0xffffffffu, factor != 1.f)) {
       // O must hold P(j-1).V before it is rescaled (P(j).V is not issued
       // until this warp arrives on p_full below).
@@ -873,41 +846,72 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       dev::tmem_st_wait();
     }
-    // P(j) into its tensor-memory buffer: rounded part, then the residual.
-    // When this warp's rows need none, its residual columns must read as
-    // zeros (another warp's rows may make the MMA add them): they are
-    // cleared once after a tile that wrote a residual, not every tile.
+    // P = 2^(s * c - m_ref) in two halves of 32 keys, two keys per
+    // instruction for the exponents and the sums.  Each half's rounded part
+    // goes to tensor memory as soon as it is packed (once P(j-1).V has read
+    // the buffer), so the store of the first half overlaps the exponentials
+    // of the second.
+    uint32_t hw[kKeys / 2];
     {
-      uint32_t hw[kKeys / 2], lw[kKeys / 2];
-      const bool store_lw = a.pv_split != 2 && (split || res_dirty);
+      const float2 c2 = make_float2(c, c);
+      const float2 nm2 = make_float2(-m_ref, -m_ref);
+      float2 l4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int e = 16 * h; e < 16 * h + 16; ++e) {
+          const float2 x =
+              dev::ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), c2, nm2);
+          sv[2 * e] = dev::fast_exp2(x.x);
+          sv[2 * e + 1] = dev::fast_exp2(x.y);
+          l4[e & 3] =
+              dev::fadd2(l4[e & 3], make_float2(sv[2 * e], sv[2 * e + 1]));
+          hw[e] = M::pack(sv[2 * e], sv[2 * e + 1]);
+        }
+        if (h == 0) {
+          // P(j-1).V must have read the P buffer before it is overwritten.
+          if (j >= 1 && !wait_pv(j - 1)) ok = false;
+          if (!ok) break;
+          dev::tc_fence_after();
+        }
+        dev::tmem_st16u(p_tmem + lane_off + 16 * h,
+                        *reinterpret_cast<const uint32_t(*)[16]>(hw + 16 * h));
+      }
+      if (!ok) break;
+      const float2 la = dev::fadd2(l4[0], l4[1]);
+      const float2 lb = dev::fadd2(l4[2], l4[3]);
+      l += (la.x + la.y) + (lb.x + lb.y);
+    }
+    // Does a key of this tile need P's residual?  Its p is at most
+    // 2^(mx - m_ref); it needs it if that can exceed l / kSplitInv.
+    const bool split = __any_sync(
+        0xffffffffu,
+        a.pv_split == 1 ||
+            (a.pv_split == 0 && valid &&
+             dev::fast_exp2(mx - m_ref) * kSplitInv > l));
+    // The residual P - hi.  When this warp's rows need none, its residual
+    // columns must read as zeros (another warp's rows may make the MMA add
+    // them): they are cleared once after a tile that wrote a residual, not
+    // every tile.
+    if (a.pv_split != 2 && (split || res_dirty)) {
+      uint32_t lw[kKeys / 2];
       if (split) {
         const float2 m1 = make_float2(-1.f, -1.f);
 #pragma unroll
         for (int e = 0; e < kKeys / 2; ++e) {
-          const float2 pe = make_float2(sv[2 * e], sv[2 * e + 1]);
-          hw[e] = M::pack(pe.x, pe.y);
-          const float2 r = dev::ffma2(M::unpack(hw[e]), m1, pe);  // P - hi
+          const float2 r = dev::ffma2(M::unpack(hw[e]), m1,
+                                      make_float2(sv[2 * e], sv[2 * e + 1]));
           lw[e] = M::pack(r.x, r.y);
         }
       } else {
 #pragma unroll
-        for (int e = 0; e < kKeys / 2; ++e) {
-          hw[e] = M::pack(sv[2 * e], sv[2 * e + 1]);
-          lw[e] = 0u;
-        }
+        for (int e = 0; e < kKeys / 2; ++e) lw[e] = 0u;
       }
-      res_dirty = split;
-      // P(j-1).V must have read the P buffer before it is overwritten.
-      if (j >= 1 && !wait_pv(j - 1)) {
-        ok = false;
-        break;
-      }
-      dev::tc_fence_after();
-      const uint32_t pa = p_tmem + lane_off;
-      dev::tmem_st32u(pa, hw);
-      if (store_lw) dev::tmem_st32u(pa + kKeys / 2, lw);
-      dev::tmem_st_wait();
+      dev::tmem_st32u(p_tmem + lane_off + kKeys / 2, lw);
     }
+    res_dirty = split;
+    dev::tmem_st_wait();
     dev::tc_fence_before();
     __syncwarp();
     if (lane == 0) {

@@ -1,5 +1,5 @@
 // tcgen05 helpers used only by the prefill kernel: the MMA whose A operand
-// sits in tensor memory, and a 32-column store of 32-bit words.
+// sits in tensor memory, and 32- and 16-column stores of 32-bit words.
 #pragma once
 
 #include <cstdint>
@@ -35,6 +35,18 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr,
       "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
       "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]),
       "r"(v[31]), "r"(taddr)
+      : "memory");
+}
+
+// 32 lanes x 16 columns of 32-bit words from registers (this thread's lane).
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr,
+                                           const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%16], {%0, %1, %2, %3, %4, "
+      "%5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15};" ::"r"(v[0]),
+      "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+      "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]),
+      "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(taddr)
       : "memory");
 }
 
