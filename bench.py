@@ -840,8 +840,9 @@ def time_prefill(pkv, wl, name, chunk, dev, iters=10):
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     kw = dict(max_q_len=int(pin.q_lens.max()),
               max_context_len=int(inp.lengths.max()), dev_err=err,
-              workspace=torch.empty(4 * w.num_seqs + 16, dtype=torch.uint8,
-                                    device=dev))
+              workspace=torch.empty(
+                  pkv.pa_prefill_workspace_bytes(pin.q, inp.k_cache, bt),
+                  dtype=torch.uint8, device=dev))
     def run(pv):
         for _ in range(3):
             pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt, cl, qs,
@@ -931,8 +932,9 @@ def prefix_cache_measure(pkv, dev, requests=128, prompt_len=2048,
         qsd = torch.from_numpy(qs).to(dev)
         kw = dict(max_q_len=int(q_lens.max()),
                   max_context_len=int(lens.max()),
-                  workspace=torch.empty(4 * len(lens) + 16, dtype=torch.uint8,
-                                        device=dev))
+                  workspace=torch.empty(
+                      pkv.pa_prefill_workspace_bytes(q, kc, bt),
+                      dtype=torch.uint8, device=dev))
         for _ in range(2):
             pkv.pa_prefill(out, q, kc, vc, bt, cl, qsd, d ** -0.5, **kw)
         a = torch.cuda.Event(enable_timing=True)
@@ -1060,8 +1062,9 @@ def spec_verify_measure(pkv, dev, drafts=4):
     qs = torch.from_numpy(pin.query_start).to(dev)
     out = torch.empty_like(pin.q)
     kw = dict(max_q_len=drafts, max_context_len=int(lens.max()),
-              workspace=torch.empty(4 * w.num_seqs + 16, dtype=torch.uint8,
-                                    device=dev))
+              workspace=torch.empty(
+                  pkv.pa_prefill_workspace_bytes(pin.q, inp.k_cache, bt),
+                  dtype=torch.uint8, device=dev))
 
     def time_kernel(kernel, pv="auto"):
         f = lambda: pkv.pa_prefill(out, pin.q, inp.k_cache, inp.v_cache, bt,

@@ -146,7 +146,10 @@ const char* pa_last_error(void);
  *                 that share a workspace must not overlap on the device.
  * Launches: a one-CTA prep kernel (the longest-first order; counter reset),
  * the decode, and with more than 16 partitions or PA_REDUCE_KERNEL the
- * reduce kernel, chained by programmatic dependent launch.
+ * reduce kernel, chained by programmatic dependent launch.  The prep kernel
+ * reads context_lens before it waits for the kernel launched just before
+ * the call, so that kernel, if it lets its dependents start early, must
+ * not be the one that writes context_lens.
  * Computation: fp32 scores, fp32 online softmax, fp32 accumulation; the
  * output is rounded once to dtype.
  * Errors: PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED / PA_ERR_WORKSPACE before
@@ -283,18 +286,27 @@ typedef struct {
   int pv;               /* pa_prefill_pv (0: per tile, as needed) */
 } pa_prefill_desc;
 
-/* Bytes of device workspace pa_prefill needs for this shape (the sequence
- * order: num_seqs int32, rounded up to 16). */
+/* Bytes of device workspace pa_prefill needs for this shape: the sequence
+ * order (num_seqs int32) and the map of query tiles (8 bytes per tile, room
+ * for min(total_q / T + num_seqs, num_seqs * ceil(max_q_len / T)) tiles of
+ * T = 128 / G new tokens, G = num_q_heads / num_kv_heads), each rounded up
+ * to 16. */
 size_t pa_prefill_workspace_bytes(const pa_prefill_desc* desc);
 
 /* workspace: pa_prefill_workspace_bytes(desc) bytes of caller-owned device
  * memory, 16-byte aligned (PA_ERR_WORKSPACE otherwise); scratch after the
  * call, and calls sharing it must not overlap on the device.  The call
  * launches a one-CTA kernel that orders the sequences longest context
- * first, then the prefill, whose grid rows serve them in that order (a
- * long sequence never starts last) and start each sequence's query tiles
- * from its last (the one that sees the most keys), chained by programmatic
- * launch. */
+ * first and lists their query tiles (128 / G new tokens each) in that
+ * order, each sequence's last tile (the one that sees the most keys)
+ * first; then the prefill, one CTA per listed tile and KV head, chained by
+ * programmatic launch.  So a long sequence never starts last, and no CTA is
+ * spent on tiles past a shorter sequence's new tokens.  PA_ERR_UNSUPPORTED
+ * when that grid would exceed 2^31 - 1 CTAs.  The first kernel is itself
+ * launched programmatically: it reads context_lens and query_start before
+ * it waits for the kernel launched just before the call, so that kernel,
+ * if it lets its dependents start early, must not be the one that writes
+ * them. */
 pa_status pa_prefill(void* out, const void* q, const void* k_cache,
                      const void* v_cache, const int32_t* block_tables,
                      const int32_t* context_lens, const int32_t* query_start,

@@ -27,7 +27,8 @@ from ._lib import (PA_BF16, PA_F16, PA_KERNEL_AUTO, PA_KERNEL_MMA,
                    pa_decode_desc)
 
 __all__ = [
-    "pa_decode", "pa_decode_noalloc", "pa_prefill", "pa_cache_write",
+    "pa_decode", "pa_decode_noalloc", "pa_prefill", "pa_prefill_workspace_bytes",
+    "pa_cache_write",
     "pa_copy_blocks",
     "pa_decode_workspace_bytes", "pa_decode_partition_size", "make_desc",
     "BlockManager", "PagedKVError", "NoFreeBlocksError", "library_path",
@@ -218,6 +219,32 @@ def pa_decode_noalloc(out, q, k_cache, v_cache, block_tables, context_lens,
     return out
 
 
+def _prefill_desc(q, k_cache, block_tables, max_q_len, max_context_len,
+                  kernel="auto", pv="auto"):
+    total_q, num_q_heads, head_dim = q.shape
+    num_blocks, num_kv_heads, block_size, hd2 = k_cache.shape
+    if hd2 != head_dim:
+        raise ValueError("q and the caches disagree on head_dim")
+    return _lib.pa_prefill_desc(
+        num_seqs=block_tables.shape[0], num_q_heads=num_q_heads,
+        num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=block_size,
+        max_blocks_per_seq=block_tables.shape[1], num_blocks=num_blocks,
+        dtype=_dtype_code(q), total_q=total_q, max_q_len=max_q_len,
+        max_context_len=max_context_len, kernel=_PREFILL_KERNELS[kernel],
+        pv=_PREFILL_PV[pv])
+
+
+def pa_prefill_workspace_bytes(q, k_cache, block_tables, *,
+                               max_q_len: int | None = None) -> int:
+    """Bytes of device workspace ``pa_prefill`` needs for these tensors and
+    ``max_q_len`` (default: every row of ``q``): the sequence order and the
+    tile map (``pa_prefill_workspace_bytes`` of the C ABI)."""
+    if max_q_len is None:
+        max_q_len = q.shape[0]
+    desc = _prefill_desc(q, k_cache, block_tables, max_q_len, 0)
+    return int(_lib.load().pa_prefill_workspace_bytes(ctypes.byref(desc)))
+
+
 def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens,
                query_start, scale: float, *, max_q_len: int,
                max_context_len: int = 0, kernel: str = "auto",
@@ -225,28 +252,22 @@ def pa_prefill(out, q, k_cache, v_cache, block_tables, context_lens,
     """Causal attention of each sequence's new tokens (rows
     query_start[b] .. query_start[b+1]-1 of ``q``) over its paged K/V, the
     new tokens being the last ones of the context.  ``max_q_len`` bounds
-    every sequence's new-token count (sizes the grid).  ``kernel``: "auto"
-    or "tile" (the same kernel).  ``pv``: precision of P in P . V --
-    "auto" (P's residual added in the tiles that need it), "split" (in every
-    tile) or "single" (one rounding of P).  ``workspace`` (a
-    uint8 device tensor of ``pa_prefill_workspace_bytes(desc)`` bytes) is
-    allocated per call when not given.  Returns ``out``."""
+    every sequence's new-token count (it picks the layout; a sequence above
+    it is flagged and left unwritten).  ``kernel``: "auto" or "tile" (the
+    same kernel).  ``pv``: precision of P in P . V -- "auto" (P's residual
+    added in the tiles that need it), "split" (in every tile) or "single"
+    (one rounding of P).  ``workspace`` (a uint8 device tensor of
+    ``pa_prefill_workspace_bytes`` bytes) is allocated per call when not
+    given.  Returns ``out``."""
     import torch
     lib = _lib.load()
-    total_q, num_q_heads, head_dim = q.shape
-    num_blocks, num_kv_heads, block_size, hd2 = k_cache.shape
-    if hd2 != head_dim or out.shape != q.shape:
-        raise ValueError("q, out and the caches disagree on shape")
+    if out.shape != q.shape:
+        raise ValueError("q and out disagree on shape")
     for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
         if t.dtype != q.dtype:
             raise TypeError(f"{name} dtype {t.dtype} != q dtype {q.dtype}")
-    desc = _lib.pa_prefill_desc(
-        num_seqs=block_tables.shape[0], num_q_heads=num_q_heads,
-        num_kv_heads=num_kv_heads, head_dim=head_dim, block_size=block_size,
-        max_blocks_per_seq=block_tables.shape[1], num_blocks=num_blocks,
-        dtype=_dtype_code(q), total_q=total_q, max_q_len=max_q_len,
-        max_context_len=max_context_len, kernel=_PREFILL_KERNELS[kernel],
-        pv=_PREFILL_PV[pv])
+    desc = _prefill_desc(q, k_cache, block_tables, max_q_len, max_context_len,
+                         kernel, pv)
     _out_mode(desc, out, q.dtype)
     need = lib.pa_prefill_workspace_bytes(ctypes.byref(desc))
     if workspace is None:

@@ -24,11 +24,12 @@ inline int order_shift(int max_ctx) {
 // Called by all kOrderThreads threads of the CTA.  A counting sort of items
 // 0 .. n-1 by key_of(i) (a non-negative int, clipped to 1023), largest key
 // first: counts and scans, then calls before_write() (e.g. a wait for the
-// previous kernel that may still read `out`), then writes out[0 .. n).
-template <typename KeyOf, typename BeforeWrite>
-__device__ __forceinline__ void counting_sort_desc(int n, KeyOf key_of,
-                                                   int32_t* __restrict__ out,
-                                                   BeforeWrite before_write) {
+// previous kernel that may still read the output), then place(pos, i) for
+// every item, pos being its rank; thread t places items t, t + kOrderThreads,
+// ...
+template <typename KeyOf, typename Place, typename BeforeWrite>
+__device__ __forceinline__ void counting_sort_desc_place(
+    int n, KeyOf key_of, Place place, BeforeWrite before_write) {
   __shared__ int hist[kOrderBuckets];
   __shared__ int warp_sum[kOrderThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -63,7 +64,16 @@ __device__ __forceinline__ void counting_sort_desc(int n, KeyOf key_of,
   __syncthreads();
   before_write();
   for (int i = tid; i < n; i += kOrderThreads)
-    out[atomicAdd(&hist[bucket(i)], 1)] = i;
+    place(atomicAdd(&hist[bucket(i)], 1), i);
+}
+
+// The same, writing out[rank] = i.
+template <typename KeyOf, typename BeforeWrite>
+__device__ __forceinline__ void counting_sort_desc(int n, KeyOf key_of,
+                                                   int32_t* __restrict__ out,
+                                                   BeforeWrite before_write) {
+  counting_sort_desc_place(
+      n, key_of, [&](int pos, int i) { out[pos] = i; }, before_write);
 }
 
 // The sequences by context_len >> shift over 1024 buckets, longest first.

@@ -61,6 +61,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 
@@ -154,7 +155,7 @@ __device__ __forceinline__ void tmem_st16x128_x8(uint32_t taddr,
 
 struct PrefillArgs {
   void* out;
-  const int32_t* order;  // [num_seqs] sequence served by grid row z
+  const int2* tiles;  // tile map: (sequence, query tile) per grid row
   const int32_t* block_tables;
   const int32_t* context_lens;
   const int32_t* query_start;
@@ -249,15 +250,21 @@ __global__ void __launch_bounds__(kThreads, 2)
   volatile uint32_t* pv_vote = tmem_slot + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // CTAs start in the order x (KV head), y, z.  y counts query tiles from
-  // the last one, which sees the most keys (the causal triangle), and z
-  // serves sequences longest first (the order kernel, which this grid
-  // follows by programmatic launch, wrote it): the grid's tail is short
-  // work even when a few long sequences or whole prompts dominate.
-  const int kvh = blockIdx.x;
-  const int qt = gridDim.y - 1 - blockIdx.y;
+  // One CTA per (tile-map entry, KV head), the KV head varying fastest.  The
+  // map (written by the plan kernel, which this grid follows by programmatic
+  // launch) lists the sequences longest context first and each sequence's
+  // query tiles from its last one, which sees the most keys (the causal
+  // triangle): the grid's tail is short work even when a few long sequences
+  // or whole prompts dominate, and no CTA is spent on a tile past a shorter
+  // sequence's new tokens.  Entries past the last tile are (-1, 0).
+  const int kvh = static_cast<int>(blockIdx.x % a.num_kv_heads);
+  const int entry = static_cast<int>(blockIdx.x / a.num_kv_heads);
+  dev::pdl_trigger();  // the next call's plan kernel may start its reads
   dev::pdl_wait();
-  const int b = a.order[blockIdx.z];
+  const int2 tile = a.tiles[entry];
+  if (tile.x < 0) return;
+  const int b = tile.x;
+  const int qt = tile.y;
   const int L = a.context_lens[b];
   const int q0 = a.query_start[b];
   const int q_len = a.query_start[b + 1] - q0;
@@ -268,10 +275,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     return;
   }
   const int tok0 = qt * kTok;
-  if ((qt == static_cast<int>(gridDim.y) - 1 && q_len > tok0 + kTok) ||
-      (RQ > 0 && q_len * G > 4 * RQ)) {
-    // max_q_len was below this sequence's new-token count: the grid (or the
-    // few-row layout) misses rows, which are left unwritten.
+  if (RQ > 0 && q_len * G > 4 * RQ) {
+    // max_q_len was below this sequence's new-token count: the few-row
+    // layout misses rows, which are left unwritten.
     if (kvh == 0 && tid == 0) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
   }
   if (tok0 >= q_len) return;
@@ -1015,18 +1021,154 @@ bool encode_cache(CUtensorMap* m, const void* cache, uint64_t rows, int hd,
 }
 
 // One CTA: the longest-first order of the sequences (by context length),
-// launched in stream order after whatever came before (which may still have
-// read the order), and letting the prefill launch early behind it.
+// then the prefill's tile map in that order.  Sequence b's new tokens fill
+// ceil(q_len / tok) query tiles of tok tokens; the map lists them, the last
+// (the one that sees the most keys) first, as (b, tile) pairs, and (-1, 0)
+// after the last one up to its capacity `cap`.  A sequence whose rows fall
+// outside q, or that has more new tokens than its context or than
+// max_q_len, gets no tiles and sets PA_ERR_DEVICE_OOB; so does a map that
+// would overflow (rows of several sequences overlapping), which is cut at
+// `cap`.  Launched by programmatic stream serialization: it reads the
+// lengths and rows and sorts while the kernel before it drains, then waits
+// for that kernel (which may still read the workspace: the previous
+// prefill) before writing; the prefill launches early behind it.
 __global__ void __launch_bounds__(kOrderThreads)
-    prefill_order_kernel(const int32_t* __restrict__ context_lens,
-                         int num_seqs, int shift, int32_t* __restrict__ order) {
+    prefill_plan_kernel(const int32_t* __restrict__ context_lens,
+                        const int32_t* __restrict__ query_start, int num_seqs,
+                        int total_q, int max_q_len, int shift, int tok,
+                        int cap, int32_t* __restrict__ order,
+                        int2* __restrict__ tiles, int32_t* dev_err) {
   dev::pdl_trigger();
-  sort_longest_first(context_lens, num_seqs, shift, order, [] {});
+  __shared__ int s_b[kOrderThreads], s_n[kOrderThreads];
+  __shared__ int s_start[kOrderThreads];
+  __shared__ int s_warp[kOrderThreads / 32];
+  __shared__ int s_carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  bool bad = false;
+  auto tiles_of = [&](int b) {  // 0 (and flagged) for invalid rows
+    const int q0 = query_start[b], q1 = query_start[b + 1];
+    if (q0 < 0 || q1 < q0 || q1 > total_q || q1 - q0 > context_lens[b] ||
+        q1 - q0 > max_q_len) {
+      bad = true;
+      return 0;
+    }
+    return (q1 - q0 + tok - 1) / tok;
+  };
+  // Up to kOrderThreads sequences, one per thread: a sequence's tile count
+  // is loaded with its length and the sort places both at its rank in
+  // shared memory (the order itself is not stored); the ranks are scanned
+  // there too, so after the wait for the previous kernel only the map's
+  // stores are left.  More sequences go through `order` in global memory.
+  const bool one_pass = num_seqs <= kOrderThreads;
+  const int my_n = one_pass && tid < num_seqs ? tiles_of(tid) : 0;
+  auto key = [&](int i) {
+    const int L = context_lens[i];
+    return L <= 0 ? 0 : (L >> shift);
+  };
+  if (one_pass) {
+    counting_sort_desc_place(
+        num_seqs, key,
+        [&](int pos, int i) {  // i == tid
+          s_b[pos] = i;
+          s_n[pos] = my_n;
+        },
+        [] {});
+  } else {
+    counting_sort_desc_place(
+        num_seqs, key, [&](int pos, int i) { order[pos] = i; },
+        [] { dev::pdl_wait(); });
+  }
+  if (tid == 0) s_carry = 0;
+  __syncthreads();  // the placed ranks (and the order, for more sequences)
+  for (int base = 0; base < num_seqs; base += kOrderThreads) {
+    const int z = base + tid;
+    int b = -1, n = 0;
+    if (z < num_seqs) {
+      if (one_pass) {
+        b = s_b[z];
+        n = s_n[z];
+      } else {
+        b = order[z];
+        n = tiles_of(b);
+      }
+    }
+    // Where sequence z's tiles start: a scan of the tile counts over the
+    // CTA, after those of the earlier chunks (s_carry).
+    int x = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+      int w = s_warp[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      s_warp[lane] = w;
+    }
+    __syncthreads();
+    const int incl = x + (warp > 0 ? s_warp[warp - 1] : 0);
+    s_b[tid] = b;
+    s_n[tid] = n;
+    s_start[tid] = s_carry + incl - n;
+    __syncthreads();
+    // The previous kernel may still read the workspace (a no-op when
+    // already waited for).
+    dev::pdl_wait();
+    // A warp per sequence writes its tiles, a lane per tile.
+    const int cnt = min(kOrderThreads, num_seqs - base);
+    for (int i = warp; i < cnt; i += kOrderThreads / 32) {
+      const int nb = s_n[i], st = s_start[i], sb = s_b[i];
+      for (int t = lane; t < nb; t += 32)
+        if (st + t < cap) tiles[st + t] = make_int2(sb, nb - 1 - t);
+    }
+    __syncthreads();  // every thread has read s_carry and the chunk's rows
+    if (tid == kOrderThreads - 1) s_carry += incl;
+    __syncthreads();
+  }
+  dev::pdl_wait();
+  const int total = s_carry;
+  if (total > cap) bad = true;
+  for (int i = total + tid; i < cap; i += kOrderThreads)
+    tiles[i] = make_int2(-1, 0);
+  if (bad) dev::set_error(dev_err, PA_ERR_DEVICE_OOB);
 }
 
-size_t prefill_workspace_bytes(const pa_prefill_desc* d) {
+// New tokens per query tile (tile rows / query group) and the tile map's
+// capacity: the map holds sum over sequences of ceil(q_len / tok) tiles,
+// which is at most total_q / tok + num_seqs when the sequences' rows do not
+// overlap, and at most num_seqs * ceil(max_q_len / tok) as the plan kernel
+// drops a sequence above max_q_len.
+int tile_tokens(const pa_prefill_desc* d) {
+  return kRows / (d->num_q_heads / d->num_kv_heads);
+}
+int64_t tile_cap(const pa_prefill_desc* d) {
+  const int tok = tile_tokens(d);
+  return std::min(static_cast<int64_t>(d->total_q) / tok + d->num_seqs,
+                  static_cast<int64_t>(d->num_seqs) *
+                      ((static_cast<int64_t>(d->max_q_len) + tok - 1) / tok));
+}
+
+// The sequence order (num_seqs int32), then the tile map (int2 entries),
+// each rounded up to 16 bytes.
+size_t order_bytes(const pa_prefill_desc* d) {
   return (static_cast<size_t>(d->num_seqs) * sizeof(int32_t) + 15) &
          ~size_t(15);
+}
+size_t prefill_workspace_bytes(const pa_prefill_desc* d) {
+  const size_t order = order_bytes(d);
+  const int G = d->num_kv_heads > 0 ? d->num_q_heads / d->num_kv_heads : 0;
+  if (d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->total_q < 0 ||
+      d->max_q_len < 0 || d->num_q_heads % d->num_kv_heads || G <= 0 ||
+      G > kRows)
+    return order;  // the call rejects this shape
+  return order + ((static_cast<size_t>(tile_cap(d)) * sizeof(int2) + 15) &
+                  ~size_t(15));
 }
 
 template <typename T, int BS, int G, int D, int RQ>
@@ -1041,10 +1183,8 @@ pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
   if (e != cudaSuccess)
     return fail(PA_ERR_CUDA, "pa_prefill: cudaFuncSetAttribute(%zu): %s",
                 smem, cudaGetErrorString(e));
-  constexpr int kTok = kRows / G;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim =
-      dim3(d->num_kv_heads, (d->max_q_len + kTok - 1) / kTok, d->num_seqs);
+  cfg.gridDim = dim3(static_cast<unsigned>(tile_cap(d) * d->num_kv_heads));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -1135,6 +1275,12 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
       !pagedkv::aligned16(k_cache) || !pagedkv::aligned16(v_cache))
     return fail(PA_ERR_INVALID_ARG,
                 "pa_prefill: out, q and the caches must be 16-byte aligned");
+  // One CTA per (tile-map entry, KV head) in a one-dimensional grid.
+  if (pagedkv::tile_cap(d) * d->num_kv_heads > 0x7fffffffLL)
+    return fail(PA_ERR_UNSUPPORTED,
+                "pa_prefill: %lld query tiles x %d KV heads exceed the grid",
+                static_cast<long long>(pagedkv::tile_cap(d)),
+                d->num_kv_heads);
   const size_t need = pagedkv::prefill_workspace_bytes(d);
   if (!workspace || workspace_bytes < need || !pagedkv::aligned16(workspace))
     return fail(PA_ERR_WORKSPACE,
@@ -1142,10 +1288,6 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
                 "got %zu at %p", need, workspace_bytes, workspace);
   if (d->num_blocks == 0 || d->num_seqs > 65535 || d->num_kv_heads > 65535)
     return fail(PA_ERR_INVALID_ARG, "pa_prefill: bad pool or batch size");
-  if ((d->max_q_len + pagedkv::kRows / G - 1) / (pagedkv::kRows / G) > 65535)
-    return fail(PA_ERR_UNSUPPORTED,
-                "pa_prefill: max_q_len %d needs more than 65535 query tiles",
-                d->max_q_len);
   if (static_cast<int64_t>(d->num_blocks) * d->num_kv_heads * d->block_size >
       0x7fffffffLL)
     return fail(PA_ERR_UNSUPPORTED, "pa_prefill: pool exceeds 2^31 rows");
@@ -1170,7 +1312,9 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
     return fail(PA_ERR_CUDA, "pa_prefill: cuTensorMapEncodeTiled failed");
   pagedkv::PrefillArgs a;
   a.out = out;
-  a.order = static_cast<const int32_t*>(workspace);
+  int2* tiles = reinterpret_cast<int2*>(static_cast<uint8_t*>(workspace) +
+                                        pagedkv::order_bytes(d));
+  a.tiles = tiles;
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.query_start = query_start;
@@ -1185,13 +1329,24 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
   a.out_f32 = d->out_fp32;
   a.pv_split = d->pv;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  pagedkv::prefill_order_kernel<<<1, pagedkv::kOrderThreads, 0, s>>>(
-      context_lens, d->num_seqs, pagedkv::order_shift(max_ctx),
-      static_cast<int32_t*>(workspace));
+  cudaLaunchConfig_t pcfg = {};
+  pcfg.gridDim = dim3(1);
+  pcfg.blockDim = dim3(pagedkv::kOrderThreads);
+  pcfg.stream = s;
+  cudaLaunchAttribute pattr[1];
+  pattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pattr[0].val.programmaticStreamSerializationAllowed = 1;
+  pcfg.attrs = pattr;
+  pcfg.numAttrs = 1;
+  cudaError_t oe = cudaLaunchKernelEx(
+      &pcfg, pagedkv::prefill_plan_kernel, context_lens, query_start,
+      d->num_seqs, d->total_q, d->max_q_len, pagedkv::order_shift(max_ctx),
+      pagedkv::tile_tokens(d), static_cast<int>(pagedkv::tile_cap(d)),
+      static_cast<int32_t*>(workspace), tiles, dev_err);
   pagedkv::count_launch();
-  const cudaError_t oe = cudaGetLastError();
+  if (oe == cudaSuccess) oe = cudaGetLastError();
   if (oe != cudaSuccess)
-    return fail(PA_ERR_CUDA, "pa_prefill: order launch failed: %s",
+    return fail(PA_ERR_CUDA, "pa_prefill: plan launch failed: %s",
                 cudaGetErrorString(oe));
   if (rq == 8)
     return d->dtype == PA_BF16

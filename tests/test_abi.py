@@ -126,11 +126,13 @@ def test_prefill_needs_its_order_workspace(pkv):
                              head_dim=128, block_size=16,
                              max_blocks_per_seq=4, num_blocks=16, dtype=1,
                              total_q=20, max_q_len=4, max_context_len=64)
-    # the sequence order: 5 int32, rounded up to 16 bytes
-    assert lib.pa_prefill_workspace_bytes(ctypes.byref(d)) == 32
+    # the sequence order (5 int32 -> 32 bytes) and the tile map: G = 4, so
+    # 32 new tokens per tile, room for 20 // 32 + 5 = 5 tiles of 8 bytes
+    # (-> 48)
+    assert lib.pa_prefill_workspace_bytes(ctypes.byref(d)) == 80
     fake = 0x1000
     args = [fake] * 7 + [ctypes.c_float(1.0), ctypes.byref(d)]
-    for ws, nbytes in ((None, 32), (fake, 16), (fake + 4, 32)):
+    for ws, nbytes in ((None, 80), (fake, 32), (fake + 4, 80)):
         st = lib.pa_prefill(*args, ws, nbytes, None, None)
         assert st == _lib.PA_ERR_WORKSPACE, (ws, nbytes)
         assert b"workspace" in lib.pa_last_error()
@@ -144,12 +146,14 @@ def test_prefill_needs_its_order_workspace(pkv):
 def test_prefill_refuses_more_query_tiles_than_the_grid_holds(pkv):
     from paged_kv_cache_383_b200 import _lib
     lib = _lib.load()
-    # G = 1: 128 new tokens per tile, 65535 tiles at most
-    d = _lib.pa_prefill_desc(num_seqs=1, num_q_heads=2, num_kv_heads=2,
+    # G = 1: 128 new tokens per tile; one CTA per (tile, KV head) in a
+    # one-dimensional grid of at most 2^31 - 1: (2^31 - 1) // 128 + 1 tiles
+    # x 256 KV heads is over
+    d = _lib.pa_prefill_desc(num_seqs=1, num_q_heads=256, num_kv_heads=256,
                              head_dim=128, block_size=16,
                              max_blocks_per_seq=1 << 20, num_blocks=1 << 20,
-                             dtype=1, total_q=128 * 65535 + 1,
-                             max_q_len=128 * 65535 + 1)
+                             dtype=1, total_q=(1 << 31) - 1,
+                             max_q_len=(1 << 31) - 1)
     fake = 0x1000
     st = lib.pa_prefill(*([fake] * 7), ctypes.c_float(1.0), ctypes.byref(d),
                         fake, 16, None, None)

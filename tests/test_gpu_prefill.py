@@ -104,6 +104,29 @@ def test_bad_block_id_is_flagged(pkv):
     _check(pin, out, "other sequences intact", seqs=[0, 2])
 
 
+@pytest.mark.parametrize("q_lens,max_q", [((40, 10, 90), 40), ((3, 8, 2), 4)])
+def test_sequence_above_max_q_len_is_flagged(pkv, q_lens, max_q):
+    """A sequence with more new tokens than max_q_len gets no query tiles
+    and sets PA_ERR_DEVICE_OOB; the other sequences' rows are still computed
+    (the tile layout, and with max_q_len 4 the few-row layout)."""
+    w = wl.Workload("over_max_q", 91, 3, 16, 4, 128, 16, "bfloat16", "fixed",
+                    fixed_lengths=(300, 200, 90))
+    pin = wl.make_prefill(w, q_lens, device="cuda")
+    inp = pin.paged
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.full_like(pin.q, float("nan"))
+    out32 = prefill_both(pkv, out, pin.q, inp.k_cache, inp.v_cache,
+                         torch.from_numpy(inp.block_tables).cuda(),
+                         torch.from_numpy(inp.lengths.astype(np.int32)).cuda(),
+                         torch.from_numpy(pin.query_start).cuda(),
+                         w.softmax_scale, max_q_len=max_q,
+                         max_context_len=int(inp.lengths.max()), dev_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 5
+    ok = [b for b in range(3) if pin.q_lens[b] <= max_q]
+    _check(pin, (out, out32), "sequences within max_q_len", seqs=ok)
+
+
 @pytest.mark.parametrize("bs", [16, 32])
 @pytest.mark.parametrize("head_dim", [64, 128])
 def test_unwritten_slots_hold_nan(pkv, bs, head_dim):
