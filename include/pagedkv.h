@@ -287,10 +287,10 @@ typedef struct {
 } pa_prefill_desc;
 
 /* Bytes of device workspace pa_prefill needs for this shape: the sequence
- * order (num_seqs int32) and the map of query tiles (8 bytes per tile, room
- * for min(total_q / T + num_seqs, num_seqs * ceil(max_q_len / T)) tiles of
- * T = 128 / G new tokens, G = num_q_heads / num_kv_heads), each rounded up
- * to 16. */
+ * order (num_seqs int32, rounded up to 16), a 16-byte work counter, and the
+ * map of query tiles (8 bytes per tile, room for min(total_q / T + num_seqs,
+ * num_seqs * ceil(max_q_len / T)) tiles of T = 128 / G new tokens,
+ * G = num_q_heads / num_kv_heads, rounded up to 16). */
 size_t pa_prefill_workspace_bytes(const pa_prefill_desc* desc);
 
 /* workspace: pa_prefill_workspace_bytes(desc) bytes of caller-owned device
@@ -299,10 +299,12 @@ size_t pa_prefill_workspace_bytes(const pa_prefill_desc* desc);
  * launches a one-CTA kernel that orders the sequences longest context
  * first and lists their query tiles (128 / G new tokens each) in that
  * order, each sequence's last tile (the one that sees the most keys)
- * first; then the prefill, one CTA per listed tile and KV head, chained by
- * programmatic launch.  So a long sequence never starts last, and no CTA is
- * spent on tiles past a shorter sequence's new tokens.  PA_ERR_UNSUPPORTED
- * when that grid would exceed 2^31 - 1 CTAs.  The first kernel is itself
+ * first; then the prefill, chained by programmatic launch: a persistent
+ * grid (two CTAs per SM) whose CTAs take (listed tile, KV head) work items
+ * from the counter in that order.  So a long sequence never starts last, no
+ * work is spent on tiles past a shorter sequence's new tokens, and a CTA
+ * loads its next item while it computes the current one.
+ * PA_ERR_UNSUPPORTED when the items would exceed 2^31 - 1.  The first kernel is itself
  * launched programmatically: it reads context_lens and query_start before
  * it waits for the kernel launched just before the call, so that kernel,
  * if it lets its dependents start early, must not be the one that writes

@@ -62,6 +62,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -169,14 +170,18 @@ struct PrefillArgs {
   int total_q;
   int out_f32;  // 1: out is float32 (the value before the cast to T)
   int pv_split;  // pa_prefill_pv: 0 per tile as needed, 1 always, 2 never
+  int* counter;   // next work item (zeroed by the plan kernel)
+  int num_items;  // tile-map entries x KV heads
 };
 
 // barriers: q_full, k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
-// s_full, s_free, p_full, o_ready, done, then the tensor-memory base address
-// word and the residual vote.
+// s_full, s_free, p_full, o_ready, done, q_empty, item_full[2],
+// item_empty[2]; then the tensor-memory base address word, the residual vote
+// and (16 bytes on) two work-item slots.
 template <int KS, int VS> __host__ __device__ constexpr int num_bars() {
-  return 1 + 2 * KS + 2 * VS + 4 + 1;
+  return 1 + 2 * KS + 2 * VS + 4 + 1 + 1 + 4;
 }
+constexpr int kItemWords = 8;  // one published work item
 constexpr int kTileHalf = kKeys * 128;  // 8 KB: 64 keys x 64 dims (128 B)
 
 // Shared memory for head_dim D (offsets from a 1024-byte aligned base): the
@@ -193,9 +198,10 @@ struct Layout {
   static constexpr int kOffV = kOffK + KS * kKVTile;
   static constexpr int kOffBars = kOffV + VS * kKVTile;
   // 1024 bytes of slack for aligning the base, then the layout above; after
-  // the barriers, the tensor-memory address word and two residual votes.
+  // the barriers, the tensor-memory address word and the residual vote (16
+  // bytes with padding) and two work-item slots.
   static constexpr size_t kSmemBytes =
-      1024 + kOffBars + num_bars<KS, VS>() * 8 + 32;
+      1024 + kOffBars + num_bars<KS, VS>() * 8 + 16 + 2 * kItemWords * 4;
 };
 template <int D, int RQ>
 using LayoutFor = Layout<D, q_rows<RQ>(), k_stages<RQ>(), v_stages<RQ>()>;
@@ -232,15 +238,23 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t k_empty0 = k_full0 + kKStages * 8;
   const uint32_t v_full0 = k_empty0 + kKStages * 8;
   const uint32_t v_empty0 = v_full0 + kVStages * 8;
-  // S, P and P.V barriers, one each: tile t completes phase t (waited on
-  // with parity t & 1).  s_full: S(t) is in tensor memory; s_free: the
-  // softmax warps have S(t) in registers; p_full: P(t) is in tensor memory;
-  // o_ready: P(t).V has completed (O is current, the P buffer is free).
+  // S, P and P.V barriers, one each: the CTA's tile t (counted over all its
+  // work items) completes phase t (waited on with parity t & 1).  s_full:
+  // S(t) is in tensor memory; s_free: the softmax warps have S(t) in
+  // registers; p_full: P(t) is in tensor memory; o_ready: P(t).V has
+  // completed (O is current, the P buffer is free).
   const uint32_t s_full = v_empty0 + kVStages * 8;
   const uint32_t s_free = s_full + 8;
   const uint32_t p_full = s_free + 8;
   const uint32_t o_ready = p_full + 8;
   const uint32_t done = o_ready + 8;
+  // q_empty: an item's S MMAs are done with the Q buffer (one phase per
+  // computed item).  item_full[s] / item_empty[s]: work-item slot s was
+  // published / read by all five consumers (the MMA thread and the four
+  // softmax warps).
+  const uint32_t q_empty = done + 8;
+  const uint32_t item_full0 = q_empty + 8;
+  const uint32_t item_empty0 = item_full0 + 16;
   uint32_t* tmem_slot =
       reinterpret_cast<uint32_t*>(smem + kOffBars + kNumBars * 8);
   // Residual vote: a softmax warp whose rows need P's residual in tile t
@@ -248,54 +262,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   // issuer reads it after that barrier; a stale word holds t or less, so it
   // never needs clearing.
   volatile uint32_t* pv_vote = tmem_slot + 1;
+  volatile int* item_s = reinterpret_cast<volatile int*>(tmem_slot + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // One CTA per (tile-map entry, KV head), the KV head varying fastest.  The
-  // map (written by the plan kernel, which this grid follows by programmatic
-  // launch) lists the sequences longest context first and each sequence's
-  // query tiles from its last one, which sees the most keys (the causal
-  // triangle): the grid's tail is short work even when a few long sequences
-  // or whole prompts dominate, and no CTA is spent on a tile past a shorter
-  // sequence's new tokens.  Entries past the last tile are (-1, 0).
-  const int kvh = static_cast<int>(blockIdx.x % a.num_kv_heads);
-  const int entry = static_cast<int>(blockIdx.x / a.num_kv_heads);
   dev::pdl_trigger();  // the next call's plan kernel may start its reads
-  dev::pdl_wait();
-  const int2 tile = a.tiles[entry];
-  if (tile.x < 0) return;
-  const int b = tile.x;
-  const int qt = tile.y;
-  const int L = a.context_lens[b];
-  const int q0 = a.query_start[b];
-  const int q_len = a.query_start[b + 1] - q0;
-  if (L < 0 || L > a.max_blocks_per_seq * BS || L > a.max_context_len ||
-      q_len < 0 || q_len > L || q0 < 0 || q0 + q_len > a.total_q) {
-    if (qt == 0 && kvh == 0 && tid == 0)
-      dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
-    return;
-  }
-  const int tok0 = qt * kTok;
-  if (RQ > 0 && q_len * G > 4 * RQ) {
-    // max_q_len was below this sequence's new-token count: the few-row
-    // layout misses rows, which are left unwritten.
-    if (kvh == 0 && tid == 0) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
-  }
-  if (tok0 >= q_len) return;
-  const int n_q = min(kTok, q_len - tok0);
-  const int kv_end = L - q_len + tok0 + n_q;     // keys this tile may see
-  const int n_tiles = (kv_end + kKeys - 1) / kKeys;
-  const int n_pages = (kv_end + BS - 1) / BS;
-
-  // Block ids of the pages the tile reads; every one is checked here, and
-  // the producer reads them again (from L2) a tile ahead of its loads, so
-  // shared memory does not grow with the context.
-  int bad = 0;
-  const int32_t* row = a.block_tables +
-                       static_cast<int64_t>(b) * a.max_blocks_per_seq;
-  for (int i = tid; i < n_pages; i += kThreads) {
-    const int32_t p = row[i];
-    bad |= (p < 0 || p >= a.num_blocks);
-  }
   if (tid == 0) {
     dev::mbar_init(q_full, 1);
     for (int s = 0; s < kKStages; ++s) {
@@ -311,13 +281,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     dev::mbar_init(p_full, 4);
     dev::mbar_init(o_ready, 1);
     dev::mbar_init(done, 4);
+    dev::mbar_init(q_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      dev::mbar_init(item_full0 + 8 * s, 1);
+      dev::mbar_init(item_empty0 + 8 * s, 5);
+    }
     dev::fence_mbar_init();
     pv_vote[0] = 0u;
-  }
-  bad = __syncthreads_or(bad);
-  if (bad) {
-    if (tid == 0) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
-    return;
   }
   if (warp == 1) {  // the whole warp allocates tensor memory
     dev::tmem_alloc(dev::smem_u32(tmem_slot), kTmemCols);
@@ -329,60 +299,98 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t tbase = *tmem_slot;
   // S: columns [0, 64); P: columns [64, 128) (rounded part in the first 32,
   // residual in the next 32, two 16-bit values per column); O: columns
-  // [128, 256).  S and P have buffers of their own, so S(j+1) can be
-  // computed as soon as the softmax warps hold S(j) in registers, without
-  // waiting for P(j).V (which only P's buffer holds up).
+  // [128, 256).  S and P have buffers of their own, so S(t+1) can be
+  // computed as soon as the softmax warps hold S(t) in registers, without
+  // waiting for P(t).V (which only P's buffer holds up).
   const uint32_t s_tmem = tbase;
   const uint32_t p_tmem = tbase + kKeys;
   const uint32_t o_tmem = tbase + 128;
+  // The tile map and the item counter come from the plan kernel, which this
+  // grid follows by programmatic launch.
+  dev::pdl_wait();
+
+  // The grid is persistent: two CTAs per SM, each taking work items from a
+  // counter in the workspace.  Item i is KV head i % num_kv_heads of tile-
+  // map entry i / num_kv_heads; the map lists the sequences longest context
+  // first and each sequence's query tiles from its last one, which sees the
+  // most keys (the causal triangle), so items are taken heaviest first and
+  // the CTAs end together whatever the mix of tile lengths.  The producer
+  // takes each item and publishes it to the other warps through a two-slot
+  // ring; the next item's Q tile, first K tiles and first S are in flight
+  // while the current item's last tiles and output are computed.
+  struct Item {
+    int state;  // kWork, kSkip (invalid input, flagged) or kEnd
+    int b, kvh, qt, L, q0, q_len;
+  };
+  constexpr int kWork = 0, kSkip = 1, kEnd = 2;
+  // What an item computes: new tokens tok0 .. tok0 + n_q - 1 of its
+  // sequence, over keys [0, kv_end) in n_tiles tiles of 64.
+  struct Span {
+    int tok0, n_q, kv_end, n_tiles;
+  };
+  auto span_of = [](const Item& it) {
+    Span sp;
+    sp.tok0 = it.qt * kTok;
+    sp.n_q = min(kTok, it.q_len - sp.tok0);
+    sp.kv_end = it.L - it.q_len + sp.tok0 + sp.n_q;
+    sp.n_tiles = (sp.kv_end + kKeys - 1) / kKeys;
+    return sp;
+  };
+  // Consumers read item n from slot n & 1 once it is published (the
+  // barrier's acquire orders the reads after the producer's writes).
+  auto read_item = [&](int n, Item& it) -> bool {
+    const int slot = n & 1;
+    if (!dev::mbar_wait(item_full0 + 8 * slot, (n >> 1) & 1)) return false;
+    const volatile int* d = item_s + kItemWords * slot;
+    it.state = d[0];
+    it.b = d[1];
+    it.kvh = d[2];
+    it.qt = d[3];
+    it.L = d[4];
+    it.q0 = d[5];
+    it.q_len = d[6];
+    return true;
+  };
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- work items and TMA producer ----------------
     if (lane == 0) {
       dev::prefetch_tmap(&qmap);
       dev::prefetch_tmap(&kmap);
       dev::prefetch_tmap(&vmap);
-      if constexpr (RQ > 0) {
-        // Few query rows: RQ/G tokens of G heads (RQ rows) into the first RQ
-        // of each 16-row quarter of the 64-row A operand (the rest is
-        // padding).  With M = 64 the tensor cores put row 16q + i of S and O
-        // in tensor-memory lane 32q + i, and read P's row 16q + i from that
-        // lane: the same lanes the softmax warps use.
-        constexpr int kQTok = RQ / G;
-        dev::mbar_arrive_expect_tx(q_full, 4 * kHalves * RQ * 128);
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq)
-#pragma unroll
-          for (int h = 0; h < kHalves; ++h)
-            dev::tma_load_3d(q_s + h * kHalfQ + qq * 16 * 128, &qmap, 64 * h,
-                             kvh * G, q0 + tok0 + qq * kQTok, q_full);
-      } else {
-        dev::mbar_arrive_expect_tx(q_full, kQBytes);
-#pragma unroll
-        for (int h = 0; h < kHalves; ++h)
-          dev::tma_load_3d(q_s + h * kHalfQ, &qmap, 64 * h, kvh * G,
-                           q0 + tok0, q_full);
-      }
-      // Block ids of a tile's pages; pages past the sequence are masked, so
-      // they read the first page instead.
-      const int32_t first = row[0];
-      auto fetch = [&](int j, int32_t (&ids)[kPagesPerTile]) {
-#pragma unroll
-        for (int p = 0; p < kPagesPerTile; ++p) {
-          const int page = j * kPagesPerTile + p;
-          ids[p] = page < n_pages ? __ldg(row + page) : first;
-        }
+      // Take item n: past the map's last tile (or its end) there is no more
+      // work.  A sequence outside the table or the rows, or with more new
+      // tokens than the few-row layout holds, is flagged and skipped.
+      auto draw = [&](Item& it) {
+        it = Item{kEnd, 0, 0, 0, 0, 0, 0};
+        const int i = atomicAdd(a.counter, 1);
+        if (i >= a.num_items) return;
+        const int2 e = a.tiles[i / a.num_kv_heads];
+        if (e.x < 0) return;
+        it.b = e.x;
+        it.qt = e.y;
+        it.kvh = i % a.num_kv_heads;
+        it.L = a.context_lens[it.b];
+        it.q0 = a.query_start[it.b];
+        it.q_len = a.query_start[it.b + 1] - it.q0;
+        const bool bad =
+            it.L < 0 || it.L > a.max_blocks_per_seq * BS ||
+            it.L > a.max_context_len || it.q_len < 0 || it.q_len > it.L ||
+            it.q0 < 0 || it.q0 + it.q_len > a.total_q ||
+            it.qt * kTok >= it.q_len || (RQ > 0 && it.q_len * G > 4 * RQ);
+        if (bad) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
+        it.state = bad ? kSkip : kWork;
       };
-      int32_t cur[kPagesPerTile], nxt[kPagesPerTile], prv[kPagesPerTile];
-      fetch(0, nxt);
-      // K tile j and V tile j-1 per step: a K stage is free once S(j) has
-      // read it, a V stage once P(j).V has, and V is needed a tile later.
-      auto load = [&](int j, bool is_v,
+      // K tile t and V tile t-1 per step (t counted over the CTA's items): a
+      // K stage is free once S(t) has read it, a V stage once P(t).V has,
+      // and V is needed a tile later.
+      auto load = [&](uint32_t t, bool is_v, int kvh,
                       const int32_t (&ids)[kPagesPerTile]) -> bool {
         const int ns = is_v ? kVStages : kKStages;
-        const int s = j % ns;
+        const int s = t % ns;
         const uint32_t empty = (is_v ? v_empty0 : k_empty0) + 8 * s;
-        if (j >= ns && !dev::mbar_wait(empty, ((j / ns) - 1) & 1))
+        if (t >= static_cast<uint32_t>(ns) &&
+            !dev::mbar_wait(empty, ((t / ns) - 1) & 1))
           return false;
         const uint32_t full = (is_v ? v_full0 : k_full0) + 8 * s;
         dev::mbar_arrive_expect_tx(full, kKVTile);
@@ -398,28 +406,108 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         return true;
       };
-      for (int t = 0; t <= n_tiles; ++t) {
-        if (t < n_tiles) {
-#pragma unroll
-          for (int p = 0; p < kPagesPerTile; ++p) cur[p] = nxt[p];
-          if (t + 1 < n_tiles) fetch(t + 1, nxt);  // in flight meanwhile
-        }
-        if ((t < n_tiles && !load(t, false, cur)) ||
-            (t >= 1 && !load(t - 1, true, prv))) {
-          dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
+      uint32_t g = 0;  // tiles of this CTA's earlier items
+      int v = 0;       // items computed so far
+      bool ok = true;
+      for (int n = 0; ok; ++n) {
+        Item it;
+        draw(it);
+        const int slot = n & 1;
+        if (n >= 2 &&
+            !dev::mbar_wait(item_empty0 + 8 * slot, ((n >> 1) - 1) & 1)) {
+          ok = false;
           break;
         }
+        volatile int* d = item_s + kItemWords * slot;
+        d[0] = it.state;
+        d[1] = it.b;
+        d[2] = it.kvh;
+        d[3] = it.qt;
+        d[4] = it.L;
+        d[5] = it.q0;
+        d[6] = it.q_len;
+        dev::mbar_arrive(item_full0 + 8 * slot);
+        if (it.state == kEnd) break;
+        if (it.state == kSkip) continue;
+        const Span sp = span_of(it);
+        const int kvh = it.kvh;
+        // The Q buffer is free once the previous item's S MMAs are done.
+        if (v >= 1 && !dev::mbar_wait(q_empty, (v - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        if constexpr (RQ > 0) {
+          // Few query rows: RQ/G tokens of G heads (RQ rows) into the first
+          // RQ of each 16-row quarter of the 64-row A operand (the rest is
+          // padding).  With M = 64 the tensor cores put row 16q + i of S and
+          // O in tensor-memory lane 32q + i, and read P's row 16q + i from
+          // that lane: the same lanes the softmax warps use.
+          constexpr int kQTok = RQ / G;
+          dev::mbar_arrive_expect_tx(q_full, 4 * kHalves * RQ * 128);
 #pragma unroll
-        for (int p = 0; p < kPagesPerTile; ++p) prv[p] = cur[p];
+          for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+            for (int h = 0; h < kHalves; ++h)
+              dev::tma_load_3d(q_s + h * kHalfQ + qq * 16 * 128, &qmap,
+                               64 * h, kvh * G, it.q0 + sp.tok0 + qq * kQTok,
+                               q_full);
+        } else {
+          dev::mbar_arrive_expect_tx(q_full, kQBytes);
+#pragma unroll
+          for (int h = 0; h < kHalves; ++h)
+            dev::tma_load_3d(q_s + h * kHalfQ, &qmap, 64 * h, kvh * G,
+                             it.q0 + sp.tok0, q_full);
+        }
+        // Block ids of a tile's pages, read a tile ahead of its loads and
+        // checked there: an id outside the pool sets PA_ERR_DEVICE_OOB and
+        // reads page 0 instead (the item's rows are then unspecified).
+        // Pages past the sequence are masked, so they read its first page.
+        const int32_t* row = a.block_tables +
+                             static_cast<int64_t>(it.b) * a.max_blocks_per_seq;
+        const int n_pages = (sp.kv_end + BS - 1) / BS;
+        bool bad_id = false;
+        auto valid_id = [&](int32_t id) {
+          const bool bad = id < 0 || id >= a.num_blocks;
+          bad_id |= bad;
+          return bad ? 0 : id;
+        };
+        const int32_t first = valid_id(__ldg(row));
+        auto fetch = [&](int j, int32_t (&ids)[kPagesPerTile]) {
+#pragma unroll
+          for (int p = 0; p < kPagesPerTile; ++p) {
+            const int page = j * kPagesPerTile + p;
+            ids[p] = page < n_pages ? valid_id(__ldg(row + page)) : first;
+          }
+        };
+        int32_t cur[kPagesPerTile], nxt[kPagesPerTile], prv[kPagesPerTile];
+        fetch(0, nxt);
+        for (int t = 0; t <= sp.n_tiles; ++t) {
+          if (t < sp.n_tiles) {
+#pragma unroll
+            for (int p = 0; p < kPagesPerTile; ++p) cur[p] = nxt[p];
+            if (t + 1 < sp.n_tiles) fetch(t + 1, nxt);  // in flight meanwhile
+          }
+          if ((t < sp.n_tiles && !load(g + t, false, kvh, cur)) ||
+              (t >= 1 && !load(g + t - 1, true, kvh, prv))) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int p = 0; p < kPagesPerTile; ++p) prv[p] = cur[p];
+        }
+        if (bad_id) dev::set_error(a.dev_err, PA_ERR_DEVICE_OOB);
+        g += sp.n_tiles;
+        ++v;
       }
+      if (!ok) dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
     }
     return;
   }
 
   if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    bool ok = true;
     if (lane == 0) {
+      bool ok = true;
       // M = 128 query rows per MMA, or 64 in the few-row layouts (at most 16
       // real rows per lane quarter): half the tensor work per tile.
       constexpr int kMmaM = RQ > 0 ? 64 : kRows;
@@ -427,18 +515,16 @@ __global__ void __launch_bounds__(kThreads, 2)
                                                         false, false);
       constexpr uint32_t idesc_pv = dev::umma_idesc_f16(kBf16, kMmaM, D,
                                                         false, true);
-      auto issue_pv = [&](int t) -> bool {
+      // O += P(t).V for the CTA's tile t; an item's first tile overwrites O.
+      auto issue_pv = [&](uint32_t t, bool first) -> bool {
         if (!dev::mbar_wait(p_full, t & 1) ||
             !dev::mbar_wait(v_full0 + 8 * (t % kVStages), (t / kVStages) & 1))
           return false;
         dev::tc_fence_after();
         const uint32_t vt = vring + (t % kVStages) * kKVTile;
         const int parts =
-            a.pv_split == 1 ||
-                    (a.pv_split == 0 &&
-                     pv_vote[0] == static_cast<uint32_t>(t) + 1u)
-                ? 2
-                : 1;
+            a.pv_split == 1 || (a.pv_split == 0 && pv_vote[0] == t + 1u) ? 2
+                                                                         : 1;
         for (int part = 0; part < parts; ++part) {  // P rounded, residual
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk) {
@@ -448,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 dev::sw128_desc(vt + kk * 2048, kTileHalf, 1024);
             dev::umma_f16_ts(o_tmem, p_tmem + part * (kKeys / 2) + kk * 8,
                              bd, idesc_pv,
-                             (t > 0 || part > 0 || kk > 0) ? 1u : 0u);
+                             (!first || part > 0 || kk > 0) ? 1u : 0u);
           }
         }
         dev::umma_commit(o_ready);
@@ -456,8 +542,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         return true;
       };
       // S(t) = Q K(t)^T, once K(t) has landed and the softmax warps hold
-      // S(t-1) in registers.
-      auto issue_s = [&](int t) -> bool {
+      // S(t-1) in registers; after an item's last S the Q buffer is free.
+      auto issue_s = [&](uint32_t t, bool last) -> bool {
         const int s = t % kKStages;
         if (!dev::mbar_wait(k_full0 + 8 * s, (t / kKStages) & 1) ||
             (t >= 1 && !dev::mbar_wait(s_free, (t - 1) & 1)))
@@ -475,27 +561,81 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         dev::umma_commit(s_full);
         dev::umma_commit(k_empty0 + 8 * s);
+        if (last) dev::umma_commit(q_empty);
         return true;
       };
-      // S(j+1) is issued while the softmax works on tile j, before P(j).V,
-      // which waits for the softmax.
-      ok = dev::mbar_wait(q_full, 0) && issue_s(0);
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles) ok = issue_s(j + 1);
-        if (ok) ok = issue_pv(j);
+      uint32_t g = 0;  // tiles of this CTA's earlier items
+      int v = 0;       // items computed so far
+      for (int n = 0; ok; ++n) {
+        Item it;
+        if (!read_item(n, it)) {
+          ok = false;
+          break;
+        }
+        dev::mbar_arrive(item_empty0 + 8 * (n & 1));
+        if (it.state == kEnd) break;
+        if (it.state == kSkip) continue;
+        const int nt = span_of(it).n_tiles;
+        // S(j+1) is issued while the softmax works on tile j, before
+        // P(j).V, which waits for the softmax.
+        ok = dev::mbar_wait(q_full, v & 1) && issue_s(g, nt == 1);
+        for (int j = 0; ok && j < nt; ++j) {
+          if (j + 1 < nt) ok = issue_s(g + j + 1, j + 2 == nt);
+          if (ok) ok = issue_pv(g + j, j == 0);
+        }
+        g += nt;
+        ++v;
       }
-      const int last = n_tiles - 1;
-      if (ok) ok = dev::mbar_wait(o_ready, last & 1);
+      if (ok && g > 0) ok = dev::mbar_wait(o_ready, (g - 1) & 1);
       if (!ok) dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
-      // Release tensor memory only after the softmax warps are done with it.
-      if (!dev::mbar_wait(done, 0)) dev::set_error(a.dev_err,
-                                                   PA_ERR_DEVICE_TIMEOUT);
+      // Release tensor memory only after the softmax warps are done with it
+      // (they arrive after their last item's output).
+      if (!dev::mbar_wait(done, 0))
+        dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
     }
     __syncwarp();
     dev::tc_fence_after();
     dev::tmem_dealloc(tbase, kTmemCols);
     return;
   }
+
+  // Softmax warps: each reads every item in turn, like the MMA thread, and
+  // writes back its share of the item's output.  Wait results are made
+  // warp-uniform: the tcgen05 loads and stores are warp-collective.
+  const int quarter = warp & 3;  // tensor-memory lane quarter of this warp
+  const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+  const float c = a.scale_log2;
+  auto wait_pv = [&](uint32_t t) {  // P(t).V has completed
+    return __all_sync(0xffffffffu, dev::mbar_wait(o_ready, t & 1));
+  };
+  auto next_item = [&](int n, Item& it) -> bool {
+    if (!__all_sync(0xffffffffu, read_item(n, it))) return false;
+    __syncwarp();
+    if (lane == 0) dev::mbar_arrive(item_empty0 + 8 * (n & 1));
+    return true;
+  };
+  // Keys past the context get P = 0, but 0 * NaN is NaN in the MMA: in the
+  // last tile (k0 + 64 > L), clear the V rows of slots the sequence never
+  // wrote (and of pages past it).  Warp q clears rows 16q .. 16q+15, once
+  // the tile has landed (P(t).V, the stage's next reader, waits for p_full).
+  auto clear_v_tail = [&](uint32_t t, int k0, int L) -> bool {
+    if (!__all_sync(0xffffffffu,
+                    dev::mbar_wait(v_full0 + 8 * (t % kVStages),
+                                   (t / kVStages) & 1)))
+      return false;
+    const uint32_t vt = vring + (t % kVStages) * kKVTile;
+    for (int idx = lane; idx < 16 * 8 * kHalves; idx += 32) {
+      const int krow = quarter * 16 + idx / (8 * kHalves);
+      const int ch = idx % (8 * kHalves);
+      if (k0 + krow >= L)
+        dev::st_shared_zero16(vt + (ch >> 3) * kTileHalf + krow * 128 +
+                              (ch & 7) * 16);
+    }
+    dev::fence_proxy_async_smem();  // visible to the tensor cores' P.V
+    return true;
+  };
+  bool ok = true;
+  uint32_t g = 0;  // tiles of this CTA's earlier items
 
   if constexpr (RQ > 0) {
     // ------ softmax warps, few query rows (<= 4 * RQ real, RQ per quarter) --
@@ -506,128 +646,189 @@ __global__ void __launch_bounds__(kThreads, 2)
     // being padding, two rows when RQ = 16).  Lanes RQ .. 31 of every
     // quarter are padding: never read back.
     constexpr int kR = RQ / 8;  // rows per thread
-    const int quarter = warp & 3;
     const int c4 = lane & 3;  // this thread's key pairs
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    int t_loc[kR], hq[kR], qpos[kR];
-    bool valid[kR];
+    int t_loc[kR], hq[kR];
 #pragma unroll
     for (int x = 0; x < kR; ++x) {
       const int rr = quarter * RQ + (lane >> 2) + 8 * x;  // query row
       t_loc[x] = rr / G;
       hq[x] = rr - t_loc[x] * G;
-      valid[x] = t_loc[x] < n_q;
-      qpos[x] = valid[x] ? L - q_len + tok0 + t_loc[x] : kv_end - 1;
     }
-    const bool idle = quarter * RQ >= n_q * G;  // no real row in this warp
-    const float c = a.scale_log2;
-    float m_ref[kR], l[kR];  // l: this thread's keys only
-#pragma unroll
-    for (int x = 0; x < kR; ++x) {
-      m_ref[x] = -INFINITY;
-      l[x] = 0.f;
-    }
-    bool ok = true;
-    auto wait_pv = [&](int t) {
-      return __all_sync(0xffffffffu, dev::mbar_wait(o_ready, t & 1));
-    };
-    for (int j = 0; j < n_tiles && ok; ++j) {
-      ok = __all_sync(0xffffffffu, dev::mbar_wait(s_full, j & 1));
-      if (!ok) break;
-      float sa[32];
-      if (!idle) {
-        dev::tc_fence_after();
-        tmem_ld16x256_x8(s_tmem + lane_off, sa);
-        dev::tmem_ld_wait();
-        dev::tc_fence_before();
-      }
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive(s_free);
-      const int k0 = j * kKeys;
-      if (k0 + kKeys > L) {
-        // As below: clear the V rows past the context in the last tile.
-        ok = __all_sync(0xffffffffu,
-                        dev::mbar_wait(v_full0 + 8 * (j % kVStages),
-                                       (j / kVStages) & 1));
-        if (!ok) break;
-        const uint32_t vt = vring + (j % kVStages) * kKVTile;
-        for (int idx = lane; idx < 16 * 8 * kHalves; idx += 32) {
-          const int krow = quarter * 16 + idx / (8 * kHalves);
-          const int ch = idx % (8 * kHalves);
-          if (k0 + krow >= L)
-            dev::st_shared_zero16(vt + (ch >> 3) * kTileHalf + krow * 128 +
-                                  (ch & 7) * 16);
-        }
-        dev::fence_proxy_async_smem();
-      }
-      if (idle) {
-        // Like the other warps, arrive for tile j only once P(j-1).V is done:
-        // a warp that ran a tile ahead would have its arrival counted toward
-        // tile j-1 on the single p_full barrier.
-        if (j >= 1 && !wait_pv(j - 1)) {
-          ok = false;
-          break;
-        }
-        __syncwarp();
-        if (lane == 0) dev::mbar_arrive(p_full);
-        continue;
-      }
-      // sa[4k + 2x + e]: row x, key 8k + 2 c4 + e.
-      float sv[kR][16];
-      float factor[kR];
-      bool grow = false, want = false;
+    for (int n = 0; ok; ++n) {
+      Item it;
+      ok = next_item(n, it);
+      if (!ok || it.state == kEnd) break;
+      if (it.state == kSkip) continue;
+      const Span sp = span_of(it);
+      const int L = it.L;
+      int qpos[kR];
+      bool valid[kR];
 #pragma unroll
       for (int x = 0; x < kR; ++x) {
+        valid[x] = t_loc[x] < sp.n_q;
+        qpos[x] = valid[x] ? L - it.q_len + sp.tok0 + t_loc[x]
+                           : sp.kv_end - 1;
+      }
+      const bool idle = quarter * RQ >= sp.n_q * G;  // no real row here
+      float m_ref[kR], l[kR];  // l: this thread's keys only
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          sv[x][2 * k] = sa[4 * k + 2 * x];
-          sv[x][2 * k + 1] = sa[4 * k + 2 * x + 1];
+      for (int x = 0; x < kR; ++x) {
+        m_ref[x] = -INFINITY;
+        l[x] = 0.f;
+      }
+      for (int j = 0; j < sp.n_tiles && ok; ++j) {
+        const uint32_t t = g + j;
+        ok = __all_sync(0xffffffffu, dev::mbar_wait(s_full, t & 1));
+        if (!ok) break;
+        float sa[32];
+        if (!idle) {
+          dev::tc_fence_after();
+          tmem_ld16x256_x8(s_tmem + lane_off, sa);
+          dev::tmem_ld_wait();
+          dev::tc_fence_before();
         }
-        const int lim = qpos[x] - k0;
-        if (lim < kKeys - 1) {
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(s_free);
+        const int k0 = j * kKeys;
+        if (k0 + kKeys > L && !(ok = clear_v_tail(t, k0, L))) break;
+        if (idle) {
+          // Like the other warps, arrive for tile t only once P(t-1).V is
+          // done: a warp that ran a tile ahead would have its arrival
+          // counted toward tile t-1 on the single p_full barrier.
+          if (t >= 1 && !wait_pv(t - 1)) {
+            ok = false;
+            break;
+          }
+          __syncwarp();
+          if (lane == 0) dev::mbar_arrive(p_full);
+          continue;
+        }
+        // sa[4k + 2x + e]: row x, key 8k + 2 c4 + e.
+        float sv[kR][16];
+        float factor[kR];
+        bool grow = false, want = false;
+#pragma unroll
+        for (int x = 0; x < kR; ++x) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            sv[x][2 * k] = sa[4 * k + 2 * x];
+            sv[x][2 * k + 1] = sa[4 * k + 2 * x + 1];
+          }
+          const int lim = qpos[x] - k0;
+          if (lim < kKeys - 1) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+#pragma unroll
+              for (int e = 0; e < 2; ++e)
+                if (8 * k + 2 * c4 + e > lim) sv[x][2 * k + e] = -INFINITY;
+          }
+          float m4[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) m4[u] = fmaxf(sv[x][u], sv[x][u + 4]);
+#pragma unroll
+          for (int k = 8; k < 16; ++k) m4[k & 3] = fmaxf(m4[k & 3], sv[x][k]);
+          float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          mx *= c;
+          factor[x] = 1.f;
+          if (j == 0) {
+            m_ref[x] = mx;
+          } else if (mx > m_ref[x] + kRescaleLog2) {
+            factor[x] = dev::fast_exp2(m_ref[x] - mx);
+            m_ref[x] = mx;
+            l[x] *= factor[x];
+            grow = true;
+          }
+          float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            sv[x][k] = dev::fast_exp2(fmaf(sv[x][k], c, -m_ref[x]));
+            l4[k & 3] += sv[x][k];
+          }
+          l[x] += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+          // Residual vote, as in the one-row-per-thread layout: the row's
+          // sum so far is spread over its four threads.
+          if (a.pv_split == 0) {
+            float lr = l[x] + __shfl_xor_sync(0xffffffffu, l[x], 1);
+            lr += __shfl_xor_sync(0xffffffffu, lr, 2);
+            want |=
+                valid[x] && dev::fast_exp2(mx - m_ref[x]) * kSplitInv > lr;
+          }
+        }
+        const bool split = __any_sync(0xffffffffu, want || a.pv_split == 1);
+        if (__any_sync(0xffffffffu, grow)) {
+          ok = wait_pv(t - 1);
+          if (!ok) break;
+          dev::tc_fence_after();
+#pragma unroll
+          for (int col = 0; col < D; col += 32) {
+            float ov[16];
+            tmem_ld16x256_x4(o_tmem + lane_off + col, ov);
+            dev::tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+              for (int x = 0; x < kR; ++x) {
+                ov[4 * k + 2 * x] *= factor[x];
+                ov[4 * k + 2 * x + 1] *= factor[x];
+              }
+            tmem_st16x256_x4(o_tmem + lane_off + col, ov);
+          }
+          dev::tmem_st_wait();
+        }
+        // P(t) into its buffer: column 4k + c4 of each half holds keys
+        // 8k + 2 c4 and 8k + 2 c4 + 1 of row x in lane t/4 + 8x; a padding
+        // lane gets zeros.
+        {
+          uint32_t hw[16], lw[16];
 #pragma unroll
           for (int k = 0; k < 8; ++k)
 #pragma unroll
-            for (int e = 0; e < 2; ++e)
-              if (8 * k + 2 * c4 + e > lim) sv[x][2 * k + e] = -INFINITY;
+            for (int x = 0; x < 2; ++x) {
+              if (x < kR) {
+                const uint32_t w = M::pack(sv[x][2 * k], sv[x][2 * k + 1]);
+                hw[2 * k + x] = w;
+                if (split) {
+                  const float2 hf = M::unpack(w);
+                  lw[2 * k + x] =
+                      M::pack(sv[x][2 * k] - hf.x, sv[x][2 * k + 1] - hf.y);
+                } else {
+                  lw[2 * k + x] = 0u;
+                }
+              } else {
+                hw[2 * k + x] = 0u;
+                lw[2 * k + x] = 0u;
+              }
+            }
+          // P(t-1).V must have read the P buffer before it is overwritten.
+          if (t >= 1 && !wait_pv(t - 1)) {
+            ok = false;
+            break;
+          }
+          dev::tc_fence_after();
+          const uint32_t pa = p_tmem + lane_off;
+          tmem_st16x128_x8(pa, hw);
+          if (a.pv_split != 2) tmem_st16x128_x8(pa + kKeys / 2, lw);
+          dev::tmem_st_wait();
         }
-        float m4[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) m4[u] = fmaxf(sv[x][u], sv[x][u + 4]);
-#pragma unroll
-        for (int k = 8; k < 16; ++k) m4[k & 3] = fmaxf(m4[k & 3], sv[x][k]);
-        float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        mx *= c;
-        factor[x] = 1.f;
-        if (j == 0) {
-          m_ref[x] = mx;
-        } else if (mx > m_ref[x] + kRescaleLog2) {
-          factor[x] = dev::fast_exp2(m_ref[x] - mx);
-          m_ref[x] = mx;
-          l[x] *= factor[x];
-          grow = true;
-        }
-        float l4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          sv[x][k] = dev::fast_exp2(fmaf(sv[x][k], c, -m_ref[x]));
-          l4[k & 3] += sv[x][k];
-        }
-        l[x] += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-        // Residual vote, as in the one-row-per-thread layout: the row's sum
-        // so far is spread over its four threads.
-        if (a.pv_split == 0) {
-          float lr = l[x] + __shfl_xor_sync(0xffffffffu, l[x], 1);
-          lr += __shfl_xor_sync(0xffffffffu, lr, 2);
-          want |= valid[x] && dev::fast_exp2(mx - m_ref[x]) * kSplitInv > lr;
+        dev::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (split) pv_vote[0] = t + 1u;
+          dev::mbar_arrive(p_full);
         }
       }
-      const bool split = __any_sync(0xffffffffu, want || a.pv_split == 1);
-      if (__any_sync(0xffffffffu, grow)) {
-        ok = wait_pv(j - 1);
-        if (!ok) break;
+      // The item's output: the row sums over the four threads, O / l -> out.
+      float inv[kR];
+#pragma unroll
+      for (int x = 0; x < kR; ++x) {
+        l[x] += __shfl_xor_sync(0xffffffffu, l[x], 1);
+        l[x] += __shfl_xor_sync(0xffffffffu, l[x], 2);
+        inv[x] = l[x] > 0.f ? 1.f / l[x] : 0.f;
+      }
+      if (ok && !idle) ok = wait_pv(g + sp.n_tiles - 1);
+      if (ok && !idle) {
         dev::tc_fence_after();
 #pragma unroll
         for (int col = 0; col < D; col += 32) {
@@ -635,97 +836,30 @@ __global__ void __launch_bounds__(kThreads, 2)
           tmem_ld16x256_x4(o_tmem + lane_off + col, ov);
           dev::tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
+          for (int x = 0; x < kR; ++x) {
+            if (!valid[x]) continue;
+            const int64_t idx =
+                (static_cast<int64_t>(it.q0 + sp.tok0 + t_loc[x]) *
+                     a.num_q_heads +
+                 it.kvh * G + hq[x]) * D + 2 * c4 + col;
 #pragma unroll
-            for (int x = 0; x < kR; ++x) {
-              ov[4 * k + 2 * x] *= factor[x];
-              ov[4 * k + 2 * x + 1] *= factor[x];
-            }
-          tmem_st16x256_x4(o_tmem + lane_off + col, ov);
-        }
-        dev::tmem_st_wait();
-      }
-      // P(j) into its buffer: column 4k + c4 of each half holds keys
-      // 8k + 2 c4 and 8k + 2 c4 + 1 of row x in lane t/4 + 8x; a padding
-      // lane gets zeros.
-      {
-        uint32_t hw[16], lw[16];
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            if (x < kR) {
-              const uint32_t w = M::pack(sv[x][2 * k], sv[x][2 * k + 1]);
-              hw[2 * k + x] = w;
-              if (split) {
-                const float2 hf = M::unpack(w);
-                lw[2 * k + x] =
-                    M::pack(sv[x][2 * k] - hf.x, sv[x][2 * k + 1] - hf.y);
-              } else {
-                lw[2 * k + x] = 0u;
-              }
-            } else {
-              hw[2 * k + x] = 0u;
-              lw[2 * k + x] = 0u;
+            for (int k = 0; k < 4; ++k) {
+              const int64_t e = idx + 8 * k;  // dims e, e + 1
+              const float v0 = ov[4 * k + 2 * x] * inv[x];
+              const float v1 = ov[4 * k + 2 * x + 1] * inv[x];
+              if (a.out_f32)
+                *reinterpret_cast<float2*>(static_cast<float*>(a.out) + e) =
+                    make_float2(v0, v1);
+              else
+                *reinterpret_cast<uint32_t*>(static_cast<T*>(a.out) + e) =
+                    M::pack(v0, v1);
             }
           }
-        // P(j-1).V must have read the P buffer before it is overwritten.
-        if (j >= 1 && !wait_pv(j - 1)) {
-          ok = false;
-          break;
-        }
-        dev::tc_fence_after();
-        const uint32_t pa = p_tmem + lane_off;
-        tmem_st16x128_x8(pa, hw);
-        if (a.pv_split != 2) tmem_st16x128_x8(pa + kKeys / 2, lw);
-        dev::tmem_st_wait();
-      }
-      dev::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (split) pv_vote[0] = static_cast<uint32_t>(j) + 1u;
-        dev::mbar_arrive(p_full);
-      }
-    }
-    // Epilogue: the row sums over the four threads, O / l -> out.
-    float inv[kR];
-#pragma unroll
-    for (int x = 0; x < kR; ++x) {
-      l[x] += __shfl_xor_sync(0xffffffffu, l[x], 1);
-      l[x] += __shfl_xor_sync(0xffffffffu, l[x], 2);
-      inv[x] = l[x] > 0.f ? 1.f / l[x] : 0.f;
-    }
-    if (ok && !idle) ok = wait_pv(n_tiles - 1);
-    if (ok && !idle) {
-      dev::tc_fence_after();
-#pragma unroll
-      for (int col = 0; col < D; col += 32) {
-        float ov[16];
-        tmem_ld16x256_x4(o_tmem + lane_off + col, ov);
-        dev::tmem_ld_wait();
-#pragma unroll
-        for (int x = 0; x < kR; ++x) {
-          if (!valid[x]) continue;
-          const int64_t idx =
-              (static_cast<int64_t>(q0 + tok0 + t_loc[x]) * a.num_q_heads +
-               kvh * G + hq[x]) * D + 2 * c4 + col;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int64_t e = idx + 8 * k;  // dims e, e + 1
-            const float v0 = ov[4 * k + 2 * x] * inv[x];
-            const float v1 = ov[4 * k + 2 * x + 1] * inv[x];
-            if (a.out_f32)
-              *reinterpret_cast<float2*>(static_cast<float*>(a.out) + e) =
-                  make_float2(v0, v1);
-            else
-              *reinterpret_cast<uint32_t*>(static_cast<T*>(a.out) + e) =
-                  M::pack(v0, v1);
-          }
         }
       }
-    } else if (!ok) {
-      dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
+      g += sp.n_tiles;
     }
+    if (!ok) dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
     dev::tc_fence_before();
     __syncwarp();
     if (lane == 0) dev::mbar_arrive(done);
@@ -733,233 +867,217 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 
   // ---------------- softmax warps (thread = query row) ----------------
-  const int quarter = warp & 3;  // tensor-memory lane quarter of this warp
   const int r = quarter * 32 + lane;
-  const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
   const int t_loc = r / G;
-  const int g = r - t_loc * G;
-  const int tok = tok0 + t_loc;
-  const bool valid = t_loc < n_q;
-  // Padding rows (no query) see every key the tile loads; never stored.
-  const int qpos = valid ? L - q_len + tok : kv_end - 1;
-  const float c = a.scale_log2;
-  // A warp whose 32 rows are all padding (few new tokens: 4 drafts x 8 heads
-  // fill one warp's rows of 128) computes nothing: it keeps the barrier
-  // protocol (including the wait for P(j-1).V before it arrives for tile j)
-  // and its share of the V clearing only.  Its rows of P hold stale values,
-  // which reach only its own (never stored) rows of O.
-  const bool idle = quarter * 32 >= n_q * G;
-  float m_ref = -INFINITY, l = 0.f;
-  bool ok = true;
+  const int hg = r - t_loc * G;  // query head within the group
   // The residual columns of this warp's rows hold something other than
   // zeros (tensor memory starts undefined).
   bool res_dirty = true;
-  // Wait results are made warp-uniform: the tcgen05 loads and stores below
-  // are warp-collective.
-  auto wait_pv = [&](int t) {  // P(t).V has completed
-    return __all_sync(0xffffffffu, dev::mbar_wait(o_ready, t & 1));
-  };
-  for (int j = 0; j < n_tiles && ok; ++j) {
-    ok = __all_sync(0xffffffffu, dev::mbar_wait(s_full, j & 1));
-    if (!ok) break;
-    float sv[kKeys];
-    if (!idle) {
-      dev::tc_fence_after();
-      const uint32_t sa = s_tmem + lane_off;
-      float (&lo)[32] = *reinterpret_cast<float(*)[32]>(sv);
-      float (&hi)[32] = *reinterpret_cast<float(*)[32]>(sv + 32);
-      dev::tmem_ld32(sa, lo);
-      dev::tmem_ld32(sa + 32, hi);
-      dev::tmem_ld_wait();
-      dev::tc_fence_before();
-    }
-    __syncwarp();
-    if (lane == 0) dev::mbar_arrive(s_free);
-    const int k0 = j * kKeys;
-    if (k0 + kKeys > L) {
-      // Keys past the context get P = 0, but 0 * NaN is NaN in the MMA:
-      // clear the V rows of slots the sequence never wrote (and of pages
-      // past it).  Warp q clears rows 16q .. 16q+15 of the last tile, once
-      // it has landed (P(j).V, the stage's next reader, waits for p_full).
-      ok = __all_sync(0xffffffffu,
-                      dev::mbar_wait(v_full0 + 8 * (j % kVStages),
-                                     (j / kVStages) & 1));
+  for (int n = 0; ok; ++n) {
+    Item it;
+    ok = next_item(n, it);
+    if (!ok || it.state == kEnd) break;
+    if (it.state == kSkip) continue;
+    const Span sp = span_of(it);
+    const int L = it.L;
+    const int tok = sp.tok0 + t_loc;
+    const bool valid = t_loc < sp.n_q;
+    // Padding rows (no query) see every key the tile loads; never stored.
+    const int qpos = valid ? L - it.q_len + tok : sp.kv_end - 1;
+    // A warp whose 32 rows are all padding (few new tokens: 4 drafts x 8
+    // heads fill one warp's rows of 128) computes nothing: it keeps the
+    // barrier protocol (including the wait for P(t-1).V before it arrives
+    // for tile t) and its share of the V clearing only.  Its rows of P hold
+    // stale values, which reach only its own (never stored) rows of O.
+    const bool idle = quarter * 32 >= sp.n_q * G;
+    float m_ref = -INFINITY, l = 0.f;
+    for (int j = 0; j < sp.n_tiles && ok; ++j) {
+      const uint32_t t = g + j;
+      ok = __all_sync(0xffffffffu, dev::mbar_wait(s_full, t & 1));
       if (!ok) break;
-      const uint32_t vt = vring + (j % kVStages) * kKVTile;
-      for (int idx = lane; idx < 16 * 8 * kHalves; idx += 32) {
-        const int krow = quarter * 16 + idx / (8 * kHalves);
-        const int ch = idx % (8 * kHalves);
-        if (k0 + krow >= L)
-          dev::st_shared_zero16(vt + (ch >> 3) * kTileHalf + krow * 128 +
-                                (ch & 7) * 16);
-      }
-      dev::fence_proxy_async_smem();  // visible to the tensor cores' P.V
-    }
-    if (idle) {
-      // Like the other warps, arrive for tile j only once P(j-1).V is done:
-      // a warp that ran a tile ahead would have its arrival counted toward
-      // tile j-1 on the single p_full barrier.
-      if (j >= 1 && !wait_pv(j - 1)) {
-        ok = false;
-        break;
+      float sv[kKeys];
+      if (!idle) {
+        dev::tc_fence_after();
+        const uint32_t sa = s_tmem + lane_off;
+        float (&lo)[32] = *reinterpret_cast<float(*)[32]>(sv);
+        float (&hi)[32] = *reinterpret_cast<float(*)[32]>(sv + 32);
+        dev::tmem_ld32(sa, lo);
+        dev::tmem_ld32(sa + 32, hi);
+        dev::tmem_ld_wait();
+        dev::tc_fence_before();
       }
       __syncwarp();
-      if (lane == 0) dev::mbar_arrive(p_full);
-      continue;
-    }
-    // Causal mask: only tiles that reach past this row's position.
-    const int lim = qpos - k0;
-    if (lim < kKeys - 1) {
+      if (lane == 0) dev::mbar_arrive(s_free);
+      const int k0 = j * kKeys;
+      if (k0 + kKeys > L && !(ok = clear_v_tail(t, k0, L))) break;
+      if (idle) {
+        // Like the other warps, arrive for tile t only once P(t-1).V is done:
+        // a warp that ran a tile ahead would have its arrival counted toward
+        // tile t-1 on the single p_full barrier.
+        if (t >= 1 && !wait_pv(t - 1)) {
+          ok = false;
+          break;
+        }
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(p_full);
+        continue;
+      }
+      // Causal mask: only tiles that reach past this row's position.
+      const int lim = qpos - k0;
+      if (lim < kKeys - 1) {
 #pragma unroll
-      for (int k = 0; k < kKeys; ++k)
-        if (k > lim) sv[k] = -INFINITY;
-    }
-    // Eight independent partial maxima of eight keys each (and eight partial
-    // sums below), three inputs per max instruction: a 64-long serial chain
-    // of dependent instructions would stall the warp on each step.
-    float m8[8];
+        for (int k = 0; k < kKeys; ++k)
+          if (k > lim) sv[k] = -INFINITY;
+      }
+      // Eight independent partial maxima of eight keys each (and eight partial
+      // sums below), three inputs per max instruction: a 64-long serial chain
+      // of dependent instructions would stall the warp on each step.
+      float m8[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
-      m8[u] = dev::fmax3(dev::fmax3(sv[u], sv[u + 8], sv[u + 16]),
-                         dev::fmax3(sv[u + 24], sv[u + 32], sv[u + 40]),
-                         fmaxf(sv[u + 48], sv[u + 56]));
-    float mx = dev::fmax3(dev::fmax3(m8[0], m8[1], m8[2]),
-                          dev::fmax3(m8[3], m8[4], m8[5]),
-                          fmaxf(m8[6], m8[7]));
-    mx *= c;  // the scale is positive: max commutes with it
-    float factor = 1.f;
-    if (j == 0) {
-      m_ref = mx;  // O is still empty: the first P.V overwrites it
-    } else if (mx > m_ref + kRescaleLog2) {
-      factor = dev::fast_exp2(m_ref - mx);
-      m_ref = mx;
-      l *= factor;
+      for (int u = 0; u < 8; ++u)
+        m8[u] = dev::fmax3(dev::fmax3(sv[u], sv[u + 8], sv[u + 16]),
+                           dev::fmax3(sv[u + 24], sv[u + 32], sv[u + 40]),
+                           fmaxf(sv[u + 48], sv[u + 56]));
+      float mx = dev::fmax3(dev::fmax3(m8[0], m8[1], m8[2]),
+                            dev::fmax3(m8[3], m8[4], m8[5]),
+                            fmaxf(m8[6], m8[7]));
+      mx *= c;  // the scale is positive: max commutes with it
+      float factor = 1.f;
+      if (j == 0) {
+        m_ref = mx;  // O is still empty: the first P.V overwrites it
+      } else if (mx > m_ref + kRescaleLog2) {
+        factor = dev::fast_exp2(m_ref - mx);
+        m_ref = mx;
+        l *= factor;
+      }
+      if (__any_sync(0xffffffffu, factor != 1.f)) {
+        // O must hold P(t-1).V before it is rescaled (P(t).V is not issued
+        // until this warp arrives on p_full below).
+        ok = wait_pv(t - 1);
+        if (!ok) break;
+        dev::tc_fence_after();
+#pragma unroll
+        for (int col = 0; col < D; col += 32) {
+          float ov[32];
+          dev::tmem_ld32(o_tmem + lane_off + col, ov);
+          dev::tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] *= factor;
+          dev::tmem_st32(o_tmem + lane_off + col, ov);
+        }
+        dev::tmem_st_wait();
+      }
+      // P = 2^(s * c - m_ref) in two halves of 32 keys, two keys per
+      // instruction for the exponents and the sums.  Each half's rounded part
+      // goes to tensor memory as soon as it is packed (once P(j-1).V has read
+      // the buffer), so the store of the first half overlaps the exponentials
+      // of the second.
+      uint32_t hw[kKeys / 2];
+      {
+        const float2 c2 = make_float2(c, c);
+        const float2 nm2 = make_float2(-m_ref, -m_ref);
+        float2 l4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int e = 16 * h; e < 16 * h + 16; ++e) {
+            const float2 x =
+                dev::ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), c2, nm2);
+            sv[2 * e] = dev::fast_exp2(x.x);
+            sv[2 * e + 1] = dev::fast_exp2(x.y);
+            l4[e & 3] =
+                dev::fadd2(l4[e & 3], make_float2(sv[2 * e], sv[2 * e + 1]));
+            hw[e] = M::pack(sv[2 * e], sv[2 * e + 1]);
+          }
+          if (h == 0) {
+            // P(t-1).V must have read the P buffer before it is overwritten.
+            if (t >= 1 && !wait_pv(t - 1)) ok = false;
+            if (!ok) break;
+            dev::tc_fence_after();
+          }
+          dev::tmem_st16u(
+              p_tmem + lane_off + 16 * h,
+              *reinterpret_cast<const uint32_t(*)[16]>(hw + 16 * h));
+        }
+        if (!ok) break;
+        const float2 la = dev::fadd2(l4[0], l4[1]);
+        const float2 lb = dev::fadd2(l4[2], l4[3]);
+        l += (la.x + la.y) + (lb.x + lb.y);
+      }
+      // Does a key of this tile need P's residual?  Its p is at most
+      // 2^(mx - m_ref); it needs it if that can exceed l / kSplitInv.
+      const bool split = __any_sync(
+          0xffffffffu,
+          a.pv_split == 1 ||
+              (a.pv_split == 0 && valid &&
+               dev::fast_exp2(mx - m_ref) * kSplitInv > l));
+      // The residual P - hi.  When this warp's rows need none, its residual
+      // columns must read as zeros (another warp's rows may make the MMA add
+      // them): they are cleared once after a tile that wrote a residual, not
+      // every tile.
+      if (a.pv_split != 2 && (split || res_dirty)) {
+        uint32_t lw[kKeys / 2];
+        if (split) {
+          const float2 m1 = make_float2(-1.f, -1.f);
+#pragma unroll
+          for (int e = 0; e < kKeys / 2; ++e) {
+            const float2 r = dev::ffma2(M::unpack(hw[e]), m1,
+                                        make_float2(sv[2 * e], sv[2 * e + 1]));
+            lw[e] = M::pack(r.x, r.y);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < kKeys / 2; ++e) lw[e] = 0u;
+        }
+        dev::tmem_st32u(p_tmem + lane_off + kKeys / 2, lw);
+      }
+      res_dirty = split;
+      dev::tmem_st_wait();
+      dev::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (split) pv_vote[0] = t + 1u;
+        dev::mbar_arrive(p_full);
+      }
     }
-    if (__any_sync(0xffffffffu, factor != 1.f)) {
-      // O must hold P(j-1).V before it is rescaled (P(j).V is not issued
-      // until this warp arrives on p_full below).
-      ok = wait_pv(j - 1);
-      if (!ok) break;
+    // The item's output: O / l -> out[token, query head].
+    if (ok && !idle) ok = wait_pv(g + sp.n_tiles - 1);
+    if (ok && !idle) {
       dev::tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const int64_t idx =
+          (static_cast<int64_t>(it.q0 + tok) * a.num_q_heads + it.kvh * G +
+           hg) * D;
+      T* dst = static_cast<T*>(a.out) + idx;
+      float* dst32 = static_cast<float*>(a.out) + idx;  // out_f32 only
 #pragma unroll
       for (int col = 0; col < D; col += 32) {
         float ov[32];
         dev::tmem_ld32(o_tmem + lane_off + col, ov);
         dev::tmem_ld_wait();
+        if (valid && a.out_f32) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) ov[e] *= factor;
-        dev::tmem_st32(o_tmem + lane_off + col, ov);
-      }
-      dev::tmem_st_wait();
-    }
-    // P = 2^(s * c - m_ref) in two halves of 32 keys, two keys per
-    // instruction for the exponents and the sums.  Each half's rounded part
-    // goes to tensor memory as soon as it is packed (once P(j-1).V has read
-    // the buffer), so the store of the first half overlaps the exponentials
-    // of the second.
-    uint32_t hw[kKeys / 2];
-    {
-      const float2 c2 = make_float2(c, c);
-      const float2 nm2 = make_float2(-m_ref, -m_ref);
-      float2 l4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                      make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst32 + col + e) =
+                make_float4(ov[e] * inv, ov[e + 1] * inv, ov[e + 2] * inv,
+                            ov[e + 3] * inv);
+        } else if (valid) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int e = 16 * h; e < 16 * h + 16; ++e) {
-          const float2 x =
-              dev::ffma2(make_float2(sv[2 * e], sv[2 * e + 1]), c2, nm2);
-          sv[2 * e] = dev::fast_exp2(x.x);
-          sv[2 * e + 1] = dev::fast_exp2(x.y);
-          l4[e & 3] =
-              dev::fadd2(l4[e & 3], make_float2(sv[2 * e], sv[2 * e + 1]));
-          hw[e] = M::pack(sv[2 * e], sv[2 * e + 1]);
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w;
+            w.x = M::pack(ov[e] * inv, ov[e + 1] * inv);
+            w.y = M::pack(ov[e + 2] * inv, ov[e + 3] * inv);
+            w.z = M::pack(ov[e + 4] * inv, ov[e + 5] * inv);
+            w.w = M::pack(ov[e + 6] * inv, ov[e + 7] * inv);
+            *reinterpret_cast<uint4*>(dst + col + e) = w;
+          }
         }
-        if (h == 0) {
-          // P(j-1).V must have read the P buffer before it is overwritten.
-          if (j >= 1 && !wait_pv(j - 1)) ok = false;
-          if (!ok) break;
-          dev::tc_fence_after();
-        }
-        dev::tmem_st16u(p_tmem + lane_off + 16 * h,
-                        *reinterpret_cast<const uint32_t(*)[16]>(hw + 16 * h));
       }
-      if (!ok) break;
-      const float2 la = dev::fadd2(l4[0], l4[1]);
-      const float2 lb = dev::fadd2(l4[2], l4[3]);
-      l += (la.x + la.y) + (lb.x + lb.y);
     }
-    // Does a key of this tile need P's residual?  Its p is at most
-    // 2^(mx - m_ref); it needs it if that can exceed l / kSplitInv.
-    const bool split = __any_sync(
-        0xffffffffu,
-        a.pv_split == 1 ||
-            (a.pv_split == 0 && valid &&
-             dev::fast_exp2(mx - m_ref) * kSplitInv > l));
-    // The residual P - hi.  When this warp's rows need none, its residual
-    // columns must read as zeros (another warp's rows may make the MMA add
-    // them): they are cleared once after a tile that wrote a residual, not
-    // every tile.
-    if (a.pv_split != 2 && (split || res_dirty)) {
-      uint32_t lw[kKeys / 2];
-      if (split) {
-        const float2 m1 = make_float2(-1.f, -1.f);
-#pragma unroll
-        for (int e = 0; e < kKeys / 2; ++e) {
-          const float2 r = dev::ffma2(M::unpack(hw[e]), m1,
-                                      make_float2(sv[2 * e], sv[2 * e + 1]));
-          lw[e] = M::pack(r.x, r.y);
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < kKeys / 2; ++e) lw[e] = 0u;
-      }
-      dev::tmem_st32u(p_tmem + lane_off + kKeys / 2, lw);
-    }
-    res_dirty = split;
-    dev::tmem_st_wait();
-    dev::tc_fence_before();
-    __syncwarp();
-    if (lane == 0) {
-      if (split) pv_vote[0] = static_cast<uint32_t>(j) + 1u;
-      dev::mbar_arrive(p_full);
-    }
+    g += sp.n_tiles;
   }
-  // Epilogue: O / l -> out[token, query head].
-  if (ok && !idle) ok = wait_pv(n_tiles - 1);
-  if (ok && !idle) {
-    dev::tc_fence_after();
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    const int64_t idx =
-        (static_cast<int64_t>(q0 + tok) * a.num_q_heads + kvh * G + g) * D;
-    T* dst = static_cast<T*>(a.out) + idx;
-    float* dst32 = static_cast<float*>(a.out) + idx;  // out_f32 only
-#pragma unroll
-    for (int col = 0; col < D; col += 32) {
-      float ov[32];
-      dev::tmem_ld32(o_tmem + lane_off + col, ov);
-      dev::tmem_ld_wait();
-      if (valid && a.out_f32) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dst32 + col + e) =
-              make_float4(ov[e] * inv, ov[e + 1] * inv, ov[e + 2] * inv,
-                          ov[e + 3] * inv);
-      } else if (valid) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint4 w;
-          w.x = M::pack(ov[e] * inv, ov[e + 1] * inv);
-          w.y = M::pack(ov[e + 2] * inv, ov[e + 3] * inv);
-          w.z = M::pack(ov[e + 4] * inv, ov[e + 5] * inv);
-          w.w = M::pack(ov[e + 6] * inv, ov[e + 7] * inv);
-          *reinterpret_cast<uint4*>(dst + col + e) = w;
-        }
-      }
-    }
-  } else if (!ok) {
-    dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
-  }
+  if (!ok) dev::set_error(a.dev_err, PA_ERR_DEVICE_TIMEOUT);
   dev::tc_fence_before();
   __syncwarp();
   if (lane == 0) dev::mbar_arrive(done);
@@ -1037,7 +1155,8 @@ __global__ void __launch_bounds__(kOrderThreads)
                         const int32_t* __restrict__ query_start, int num_seqs,
                         int total_q, int max_q_len, int shift, int tok,
                         int cap, int32_t* __restrict__ order,
-                        int2* __restrict__ tiles, int32_t* dev_err) {
+                        int2* __restrict__ tiles, int* counter,
+                        int32_t* dev_err) {
   dev::pdl_trigger();
   __shared__ int s_b[kOrderThreads], s_n[kOrderThreads];
   __shared__ int s_start[kOrderThreads];
@@ -1136,6 +1255,7 @@ __global__ void __launch_bounds__(kOrderThreads)
   if (total > cap) bad = true;
   for (int i = total + tid; i < cap; i += kOrderThreads)
     tiles[i] = make_int2(-1, 0);
+  if (tid == 0) *counter = 0;  // the prefill's work items start at 0
   if (bad) dev::set_error(dev_err, PA_ERR_DEVICE_OOB);
 }
 
@@ -1154,12 +1274,13 @@ int64_t tile_cap(const pa_prefill_desc* d) {
                       ((static_cast<int64_t>(d->max_q_len) + tok - 1) / tok));
 }
 
-// The sequence order (num_seqs int32), then the tile map (int2 entries),
-// each rounded up to 16 bytes.
+// The sequence order (num_seqs int32, rounded up to 16 bytes), the work
+// counter (16 bytes), then the tile map (int2 entries, rounded up to 16).
 size_t order_bytes(const pa_prefill_desc* d) {
   return (static_cast<size_t>(d->num_seqs) * sizeof(int32_t) + 15) &
          ~size_t(15);
 }
+constexpr size_t kCounterBytes = 16;
 size_t prefill_workspace_bytes(const pa_prefill_desc* d) {
   const size_t order = order_bytes(d);
   const int G = d->num_kv_heads > 0 ? d->num_q_heads / d->num_kv_heads : 0;
@@ -1167,8 +1288,26 @@ size_t prefill_workspace_bytes(const pa_prefill_desc* d) {
       d->max_q_len < 0 || d->num_q_heads % d->num_kv_heads || G <= 0 ||
       G > kRows)
     return order;  // the call rejects this shape
-  return order + ((static_cast<size_t>(tile_cap(d)) * sizeof(int2) + 15) &
-                  ~size_t(15));
+  return order + kCounterBytes +
+         ((static_cast<size_t>(tile_cap(d)) * sizeof(int2) + 15) &
+          ~size_t(15));
+}
+
+// SMs of the current device (cached per device ordinal).
+int sm_count() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
+      cudaSuccess)
+    return 0;
+  if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
+  return n;
 }
 
 template <typename T, int BS, int G, int D, int RQ>
@@ -1184,7 +1323,11 @@ pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
     return fail(PA_ERR_CUDA, "pa_prefill: cudaFuncSetAttribute(%zu): %s",
                 smem, cudaGetErrorString(e));
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(tile_cap(d) * d->num_kv_heads));
+  // Persistent: two CTAs per SM (shared and tensor memory allow no more),
+  // fewer when there are fewer work items.
+  const int64_t slots = 2LL * std::max(sm_count(), 1);
+  cfg.gridDim =
+      dim3(static_cast<unsigned>(std::min<int64_t>(a.num_items, slots)));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
@@ -1275,10 +1418,11 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
       !pagedkv::aligned16(k_cache) || !pagedkv::aligned16(v_cache))
     return fail(PA_ERR_INVALID_ARG,
                 "pa_prefill: out, q and the caches must be 16-byte aligned");
-  // One CTA per (tile-map entry, KV head) in a one-dimensional grid.
+  // Work items (tile-map entry, KV head) are counted in an int.
   if (pagedkv::tile_cap(d) * d->num_kv_heads > 0x7fffffffLL)
     return fail(PA_ERR_UNSUPPORTED,
-                "pa_prefill: %lld query tiles x %d KV heads exceed the grid",
+                "pa_prefill: %lld query tiles x %d KV heads exceed 2^31 - 1 "
+                "work items",
                 static_cast<long long>(pagedkv::tile_cap(d)),
                 d->num_kv_heads);
   const size_t need = pagedkv::prefill_workspace_bytes(d);
@@ -1312,9 +1456,13 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
     return fail(PA_ERR_CUDA, "pa_prefill: cuTensorMapEncodeTiled failed");
   pagedkv::PrefillArgs a;
   a.out = out;
-  int2* tiles = reinterpret_cast<int2*>(static_cast<uint8_t*>(workspace) +
-                                        pagedkv::order_bytes(d));
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* counter = reinterpret_cast<int*>(ws + pagedkv::order_bytes(d));
+  int2* tiles = reinterpret_cast<int2*>(ws + pagedkv::order_bytes(d) +
+                                        pagedkv::kCounterBytes);
   a.tiles = tiles;
+  a.counter = counter;
+  a.num_items = static_cast<int>(pagedkv::tile_cap(d) * d->num_kv_heads);
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.query_start = query_start;
@@ -1342,7 +1490,7 @@ extern "C" pa_status pa_prefill(void* out, const void* q, const void* k_cache,
       &pcfg, pagedkv::prefill_plan_kernel, context_lens, query_start,
       d->num_seqs, d->total_q, d->max_q_len, pagedkv::order_shift(max_ctx),
       pagedkv::tile_tokens(d), static_cast<int>(pagedkv::tile_cap(d)),
-      static_cast<int32_t*>(workspace), tiles, dev_err);
+      static_cast<int32_t*>(workspace), tiles, counter, dev_err);
   pagedkv::count_launch();
   if (oe == cudaSuccess) oe = cudaGetLastError();
   if (oe != cudaSuccess)

@@ -126,13 +126,13 @@ def test_prefill_needs_its_order_workspace(pkv):
                              head_dim=128, block_size=16,
                              max_blocks_per_seq=4, num_blocks=16, dtype=1,
                              total_q=20, max_q_len=4, max_context_len=64)
-    # the sequence order (5 int32 -> 32 bytes) and the tile map: G = 4, so
-    # 32 new tokens per tile, room for 20 // 32 + 5 = 5 tiles of 8 bytes
-    # (-> 48)
-    assert lib.pa_prefill_workspace_bytes(ctypes.byref(d)) == 80
+    # the sequence order (5 int32 -> 32 bytes), the work counter (16) and
+    # the tile map: G = 4, so 32 new tokens per tile, room for
+    # min(20 // 32 + 5, 5 * 1) = 5 tiles of 8 bytes (-> 48)
+    assert lib.pa_prefill_workspace_bytes(ctypes.byref(d)) == 96
     fake = 0x1000
     args = [fake] * 7 + [ctypes.c_float(1.0), ctypes.byref(d)]
-    for ws, nbytes in ((None, 80), (fake, 32), (fake + 4, 80)):
+    for ws, nbytes in ((None, 96), (fake, 80), (fake + 4, 96)):
         st = lib.pa_prefill(*args, ws, nbytes, None, None)
         assert st == _lib.PA_ERR_WORKSPACE, (ws, nbytes)
         assert b"workspace" in lib.pa_last_error()
