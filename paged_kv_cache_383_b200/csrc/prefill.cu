@@ -12,11 +12,19 @@
 // [KV-cache chapter] "Common misconception..." describes serving kernels
 // doing: FlashAttention-style tiles over paged memory.
 //
-// B200 design.  Work unit = (tile of 128 query rows, KV head, sequence); a
+// B200 design.  Work item = (tile of 128 query rows, KV head, sequence); a
 // row is a (new token, query head of this KV head) pair, so with G query heads
 // per KV head a tile holds 128/G tokens and each K/V byte serves all G heads.
-//   * Warp 0, lane 0 loads the Q tile with one 3-D TMA box per half of
-//     head_dim, then streams 64-key K and V tiles page by page (2-D TMA boxes
+//   * A one-CTA plan kernel sorts the sequences longest context first and
+//     lists their query tiles in that order (each sequence's last tile, the
+//     one that sees the most keys, first).  The prefill grid is persistent,
+//     two CTAs per SM: each takes (listed tile, KV head) items from a
+//     counter, heaviest first, so the CTAs end together.
+//   * Warp 0, lane 0 takes the items and publishes each to the other warps
+//     through a two-slot ring in shared memory.  It loads an item's Q tile
+//     with one 3-D TMA box per half of head_dim (once the previous item's S
+//     MMAs are done with the buffer), then streams 64-key K and V tiles page
+//     by page (2-D TMA boxes
 //     of block_size rows x 128 B, 128-byte swizzle, no multicast) into
 //     separate 2-stage K and V rings: a K stage is free again once S(j) has
 //     read it, a V stage once P(j).V has, and V tile j is loaded after K
@@ -52,6 +60,10 @@
 //     from global memory a tile ahead) and tensor memory 256 columns, so two
 //     CTAs share an SM at any context length: one CTA's softmax runs while
 //     the other's tiles are on the tensor cores.
+//   * Barrier phases count a CTA's tiles over all its items, so the next
+//     item's Q, first K tiles and first S are in flight while the current
+//     item's last tiles and output are computed: the CTA start and the gap
+//     between CTAs are paid once per SM slot, not once per query tile.
 //   * Every wait is bounded (1 s) and reports PA_ERR_DEVICE_TIMEOUT; tensor
 //     memory is always released.  A barrier that is waited on by parity is
 //     never allowed to run two phases ahead of its waiter: each double
