@@ -104,6 +104,31 @@ def test_bad_block_id_is_flagged(pkv):
     _check(pin, out, "other sequences intact", seqs=[0, 2])
 
 
+@pytest.mark.parametrize("q_lens", [(30, 30, 30), (2, 2, 2)])
+def test_bad_context_length_is_skipped_and_flagged(pkv, q_lens):
+    """A sequence whose context length runs past its block table is flagged
+    (PA_ERR_DEVICE_OOB) and its work items are skipped by every warp of the
+    persistent grid; the other sequences' rows are still exact (tile and
+    few-row layouts)."""
+    w = wl.Workload("prefillbadlen", 17, 3, 16, 8, 128, 16, "bfloat16",
+                    "fixed", fixed_lengths=(90, 90, 90))
+    pin = wl.make_prefill(w, q_lens, device="cuda")
+    inp = pin.paged
+    lens = inp.lengths.astype(np.int32).copy()
+    lens[1] = inp.block_tables.shape[1] * w.block_size + 5
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.full_like(pin.q, float("nan"))
+    out32 = prefill_both(pkv, out, pin.q, inp.k_cache, inp.v_cache,
+                         torch.from_numpy(inp.block_tables).cuda(),
+                         torch.from_numpy(lens).cuda(),
+                         torch.from_numpy(pin.query_start).cuda(),
+                         w.softmax_scale, max_q_len=max(q_lens),
+                         max_context_len=int(lens.max()), dev_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 5
+    _check(pin, (out, out32), "other sequences intact", seqs=[0, 2])
+
+
 @pytest.mark.parametrize("q_lens,max_q", [((40, 10, 90), 40), ((3, 8, 2), 4)])
 def test_sequence_above_max_q_len_is_flagged(pkv, q_lens, max_q):
     """A sequence with more new tokens than max_q_len gets no query tiles
