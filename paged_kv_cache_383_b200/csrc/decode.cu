@@ -49,7 +49,6 @@
 
 #include <cmath>
 #include <cstdint>
-#include <atomic>
 #include <mutex>
 
 #include "device_utils.cuh"
@@ -1003,36 +1002,6 @@ __global__ void __launch_bounds__(kReduceWarps * 32)
 
 // ---------------------------------------------------------------------------
 // Host side.
-
-// SM count of the current device, looked up once per device ordinal (the
-// launch path asks on every call).
-int device_sm_count() {
-  static std::atomic<int> cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev >= 0 && dev < 64) {
-    const int c = cached[dev].load(std::memory_order_relaxed);
-    if (c > 0) return c;
-  }
-  int count = 148;
-  cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
-  if (dev >= 0 && dev < 64) cached[dev].store(count, std::memory_order_relaxed);
-  return count;
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
-                                         cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
 
 // The cache viewed as a 2-D tensor of rows (block, kv head, slot) x head_dim;
 // one TMA box is block_size rows x 64 elements (128 bytes), swizzled.

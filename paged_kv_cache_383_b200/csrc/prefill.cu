@@ -74,7 +74,6 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <atomic>
 #include <cmath>
 #include <cstdint>
 
@@ -1098,20 +1097,6 @@ __global__ void __launch_bounds__(kThreads, 2)
 // ---------------------------------------------------------------------------
 // Host side.
 
-PFN_cuTensorMapEncodeTiled_v12000 encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
-                                         cudaEnableDefault,
-                                         &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
 CUtensorMapDataType tma_type(pa_dtype t) {
   return t == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -1120,7 +1105,7 @@ CUtensorMapDataType tma_type(pa_dtype t) {
 // q [total_q, Hq, D] as a 3-D tensor; box = 64 dims x G heads x tokens.
 bool encode_q(CUtensorMap* m, const void* q, int total_q, int hq, int hd,
               int g, int tok, pa_dtype dt) {
-  auto enc = encoder();
+  auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(hd),
                         static_cast<cuuint64_t>(hq),
@@ -1138,7 +1123,7 @@ bool encode_q(CUtensorMap* m, const void* q, int total_q, int hq, int hd,
 
 bool encode_cache(CUtensorMap* m, const void* cache, uint64_t rows, int hd,
                   int bs, pa_dtype dt) {
-  auto enc = encoder();
+  auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(hd), rows};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(hd) * 2};
@@ -1305,23 +1290,6 @@ size_t prefill_workspace_bytes(const pa_prefill_desc* d) {
           ~size_t(15));
 }
 
-// SMs of the current device (cached per device ordinal).
-int sm_count() {
-  static std::atomic<int> cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev >= 0 && dev < 64) {
-    const int c = cached[dev].load(std::memory_order_relaxed);
-    if (c > 0) return c;
-  }
-  int n = 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
-      cudaSuccess)
-    return 0;
-  if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
-  return n;
-}
-
 template <typename T, int BS, int G, int D, int RQ>
 pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
                  const CUtensorMap& qm, const CUtensorMap& km,
@@ -1337,7 +1305,7 @@ pa_status launch(const pa_prefill_desc* d, const PrefillArgs& a,
   cudaLaunchConfig_t cfg = {};
   // Persistent: two CTAs per SM (shared and tensor memory allow no more),
   // fewer when there are fewer work items.
-  const int64_t slots = 2LL * std::max(sm_count(), 1);
+  const int64_t slots = 2LL * std::max(device_sm_count(), 1);
   cfg.gridDim =
       dim3(static_cast<unsigned>(std::min<int64_t>(a.num_items, slots)));
   cfg.blockDim = dim3(kThreads);

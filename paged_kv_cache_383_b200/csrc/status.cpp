@@ -1,5 +1,8 @@
-// Version, status strings and the thread-local error text of the C ABI.
+// Version, status strings and the thread-local error text of the C ABI;
+// the launch count and the device queries the launch paths share.
 #include "status.h"
+
+#include <cuda_runtime.h>
 
 #include <atomic>
 #include <cstdio>
@@ -24,6 +27,38 @@ pa_status fail(pa_status s, const char* fmt, ...) {
 void clear_error() { g_last_error[0] = 0; }
 
 const char* last_error() { return g_last_error; }
+
+int device_sm_count() {
+  static std::atomic<int> cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int count = 148;
+  cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
+  if (dev >= 0 && dev < 64) cached[dev].store(count, std::memory_order_relaxed);
+  return count;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> cached{nullptr};
+  PFN_cuTensorMapEncodeTiled_v12000 fn =
+      cached.load(std::memory_order_acquire);
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                         cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+      cached.store(fn, std::memory_order_release);
+    }
+  }
+  return fn;
+}
 
 }  // namespace pagedkv
 
