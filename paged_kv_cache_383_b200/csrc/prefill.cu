@@ -374,8 +374,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       // tokens than the few-row layout holds, is flagged and skipped.
       auto draw = [&](Item& it) {
         it = Item{kEnd, 0, 0, 0, 0, 0, 0};
-        const int i = atomicAdd(a.counter, 1);
-        if (i >= a.num_items) return;
+        // Unsigned: each CTA draws once past the last item, which must not
+        // wrap to a negative index however close num_items is to 2^31.
+        const unsigned u =
+            atomicAdd(reinterpret_cast<unsigned*>(a.counter), 1u);
+        if (u >= static_cast<unsigned>(a.num_items)) return;
+        const int i = static_cast<int>(u);
         const int2 e = a.tiles[i / a.num_kv_heads];
         if (e.x < 0) return;
         it.b = e.x;
