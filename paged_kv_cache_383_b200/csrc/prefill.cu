@@ -1159,20 +1159,22 @@ __global__ void __launch_bounds__(kOrderThreads)
                         int2* __restrict__ tiles, int* counter,
                         int32_t* dev_err) {
   dev::pdl_trigger();
-  __shared__ int s_b[kOrderThreads], s_n[kOrderThreads];
-  __shared__ int s_start[kOrderThreads];
-  __shared__ int s_warp[kOrderThreads / 32];
-  __shared__ int s_carry;
+  // Tile counts and their running sum in 64 bits: sequences whose rows
+  // overlap (each range valid on its own) may list more than 2^31 tiles.
+  __shared__ int s_b[kOrderThreads];
+  __shared__ long long s_n[kOrderThreads], s_start[kOrderThreads];
+  __shared__ long long s_warp[kOrderThreads / 32];
+  __shared__ long long s_carry;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   bool bad = false;
-  auto tiles_of = [&](int b) {  // 0 (and flagged) for invalid rows
+  auto tiles_of = [&](int b) -> long long {  // 0 (flagged) if invalid
     const int q0 = query_start[b], q1 = query_start[b + 1];
     if (q0 < 0 || q1 < q0 || q1 > total_q || q1 - q0 > context_lens[b] ||
         q1 - q0 > max_q_len) {
       bad = true;
       return 0;
     }
-    return (q1 - q0 + tok - 1) / tok;
+    return (static_cast<long long>(q1 - q0) + tok - 1) / tok;
   };
   // Up to kOrderThreads sequences, one per thread: a sequence's tile count
   // is loaded with its length and the sort places both at its rank in
@@ -1180,7 +1182,7 @@ __global__ void __launch_bounds__(kOrderThreads)
   // there too, so after the wait for the previous kernel only the map's
   // stores are left.  More sequences go through `order` in global memory.
   const bool one_pass = num_seqs <= kOrderThreads;
-  const int my_n = one_pass && tid < num_seqs ? tiles_of(tid) : 0;
+  const long long my_n = one_pass && tid < num_seqs ? tiles_of(tid) : 0;
   auto key = [&](int i) {
     const int L = context_lens[i];
     return L <= 0 ? 0 : (L >> shift);
@@ -1202,7 +1204,8 @@ __global__ void __launch_bounds__(kOrderThreads)
   __syncthreads();  // the placed ranks (and the order, for more sequences)
   for (int base = 0; base < num_seqs; base += kOrderThreads) {
     const int z = base + tid;
-    int b = -1, n = 0;
+    int b = -1;
+    long long n = 0;
     if (z < num_seqs) {
       if (one_pass) {
         b = s_b[z];
@@ -1214,25 +1217,25 @@ __global__ void __launch_bounds__(kOrderThreads)
     }
     // Where sequence z's tiles start: a scan of the tile counts over the
     // CTA, after those of the earlier chunks (s_carry).
-    int x = n;
+    long long x = n;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      const long long y = __shfl_up_sync(0xffffffffu, x, o);
       if (lane >= o) x += y;
     }
     if (lane == 31) s_warp[warp] = x;
     __syncthreads();
     if (warp == 0) {
-      int w = s_warp[lane];
+      long long w = s_warp[lane];
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, w, o);
+        const long long y = __shfl_up_sync(0xffffffffu, w, o);
         if (lane >= o) w += y;
       }
       s_warp[lane] = w;
     }
     __syncthreads();
-    const int incl = x + (warp > 0 ? s_warp[warp - 1] : 0);
+    const long long incl = x + (warp > 0 ? s_warp[warp - 1] : 0);
     s_b[tid] = b;
     s_n[tid] = n;
     s_start[tid] = s_carry + incl - n;
@@ -1243,18 +1246,21 @@ __global__ void __launch_bounds__(kOrderThreads)
     // A warp per sequence writes its tiles, a lane per tile.
     const int cnt = min(kOrderThreads, num_seqs - base);
     for (int i = warp; i < cnt; i += kOrderThreads / 32) {
-      const int nb = s_n[i], st = s_start[i], sb = s_b[i];
-      for (int t = lane; t < nb; t += 32)
-        if (st + t < cap) tiles[st + t] = make_int2(sb, nb - 1 - t);
+      const long long st = s_start[i];
+      const int sb = s_b[i];
+      // Only the tiles that fit the map: slots st .. min(st + n, cap) - 1.
+      const long long end = min(st + s_n[i], static_cast<long long>(cap));
+      for (long long slot = st + lane; slot < end; slot += 32)
+        tiles[slot] = make_int2(sb, static_cast<int>(st + s_n[i] - 1 - slot));
     }
     __syncthreads();  // every thread has read s_carry and the chunk's rows
     if (tid == kOrderThreads - 1) s_carry += incl;
     __syncthreads();
   }
   dev::pdl_wait();
-  const int total = s_carry;
+  const long long total = s_carry;
   if (total > cap) bad = true;
-  for (int i = total + tid; i < cap; i += kOrderThreads)
+  for (long long i = total + tid; i < cap; i += kOrderThreads)
     tiles[i] = make_int2(-1, 0);
   if (tid == 0) *counter = 0;  // the prefill's work items start at 0
   if (bad) dev::set_error(dev_err, PA_ERR_DEVICE_OOB);

@@ -129,6 +129,30 @@ def test_bad_context_length_is_skipped_and_flagged(pkv, q_lens):
     _check(pin, (out, out32), "other sequences intact", seqs=[0, 2])
 
 
+def test_overlapping_rows_overflow_the_tile_map_and_are_flagged(pkv):
+    """Sequences 0 and 2 both given query rows [0, 64) (each range valid on
+    its own; sequence 1's runs backwards, 64 -> 0, and is flagged) list 8
+    tiles of 16 tokens where the map holds min(64 / 16 + 3, 3 * 4) = 7: the
+    plan kernel cuts the map at its capacity and flags PA_ERR_DEVICE_OOB;
+    the call writes only rows of out and ends without a timeout."""
+    w = wl.Workload("overlap", 19, 3, 64, 8, 128, 16, "bfloat16", "fixed",
+                    fixed_lengths=(200, 200, 200))
+    pin = wl.make_prefill(w, (64, 0, 0), device="cuda")
+    inp = pin.paged
+    q = pin.q[:64].contiguous()
+    qs = torch.tensor([0, 64, 0, 64], dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.zeros_like(q)
+    pkv.pa_prefill(out, q, inp.k_cache, inp.v_cache,
+                   torch.from_numpy(inp.block_tables).cuda(),
+                   torch.from_numpy(inp.lengths.astype(np.int32)).cuda(), qs,
+                   w.softmax_scale, max_q_len=64, max_context_len=200,
+                   dev_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 5
+    assert torch.isfinite(out.float()).all()
+
+
 @pytest.mark.parametrize("q_lens,max_q", [((40, 10, 90), 40), ((3, 8, 2), 4)])
 def test_sequence_above_max_q_len_is_flagged(pkv, q_lens, max_q):
     """A sequence with more new tokens than max_q_len gets no query tiles
