@@ -119,6 +119,33 @@ def test_zero_sized_calls_are_noops(pkv):
                               1, None, None) == _lib.PA_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("seqs,hq,hkv,total_q,max_q", [
+    (8, 64, 8, 33166, 8192),    # whole prompts: T = 16, bound by total_q
+    (16, 64, 8, 8192, 512),     # 512-token chunks: 32 tiles each, exact
+    (256, 64, 8, 1024, 4),      # 4 drafts: one tile per sequence
+    (3, 8, 8, 1000, 700),       # G = 1: T = 128
+    (5, 32, 8, 7, 7),           # fewer rows than tiles' worth
+])
+def test_prefill_workspace_formula(pkv, seqs, hq, hkv, total_q, max_q):
+    """pa_prefill_workspace_bytes is the header's formula: the order
+    (num_seqs int32) rounded up to 16, a 16-byte work counter, and 8 bytes
+    per tile-map entry for min(total_q // T + num_seqs,
+    num_seqs * ceil(max_q_len / T)) entries of T = 128 / G new tokens,
+    rounded up to 16."""
+    from paged_kv_cache_383_b200 import _lib
+    lib = _lib.load()
+    d = _lib.pa_prefill_desc(num_seqs=seqs, num_q_heads=hq, num_kv_heads=hkv,
+                             head_dim=128, block_size=16,
+                             max_blocks_per_seq=512, num_blocks=4096, dtype=1,
+                             total_q=total_q, max_q_len=max_q,
+                             max_context_len=8192)
+    t = 128 // (hq // hkv)
+    cap = min(total_q // t + seqs, seqs * -(-max_q // t))
+    up16 = lambda n: (n + 15) // 16 * 16
+    assert (lib.pa_prefill_workspace_bytes(ctypes.byref(d)) ==
+            up16(4 * seqs) + 16 + up16(8 * cap))
+
+
 def test_prefill_needs_its_order_workspace(pkv):
     from paged_kv_cache_383_b200 import _lib
     lib = _lib.load()
